@@ -1,0 +1,257 @@
+"""CPU oracle for the quantization hot path -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The CUDA
+library never does, and this package never touches it: the two share no code.
+
+The arithmetic lives in ``wq_oracle.c`` (plain single-threaded C11, built with
+``-O2 -fno-fast-math -ffp-contract=off`` so that every fp32 operation is one
+IEEE-754 operation with round-to-nearest-even).  This module only marshals
+numpy arrays in and out of it; each wrapper names the passage of the source
+pages that the C routine follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "wq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+CFLAGS = ["-std=c11", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared",
+          "-Wall", "-Wextra"]
+
+
+def build(force: bool = False) -> str:
+    """Compile ``wq_oracle.c`` into ``liboracle.so`` (gcc) if it is missing or stale."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        _declare(_lib)
+        if not _lib.orc_rounding_mode_is_nearest():
+            raise RuntimeError("oracle requires the FE_TONEAREST rounding mode")
+    return _lib
+
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+def _declare(L):
+    L.orc_half_to_float.argtypes = [ctypes.c_uint16]
+    L.orc_half_to_float.restype = ctypes.c_float
+    L.orc_float_to_half.argtypes = [ctypes.c_float]
+    L.orc_float_to_half.restype = ctypes.c_uint16
+    L.orc_rounding_mode_is_nearest.restype = _I
+    L.orc_quantize_group_int4.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P]
+    L.orc_quantize_group_int4.restype = _I
+    L.orc_dequant_int4.argtypes = [_P, _P, _P, _I, _I, _I, _P]
+    L.orc_dequant_int4.restype = None
+    L.orc_quantize_sym_rows.argtypes = [_P, _I, _I, _P, _I, _I, _P, _P]
+    L.orc_quantize_sym_rows.restype = _I
+    L.orc_smooth.argtypes = [_P, _I, _P, _I, _I, ctypes.c_double, _P]
+    L.orc_smooth.restype = _I
+    L.orc_matmul_w4a16_ref.argtypes = [_P, _I, _P, _P, _P, _I, _I, _I, _P, _I, _P, _P]
+    L.orc_matmul_w4a16_ref.restype = None
+    L.orc_matmul_w8a16_ref.argtypes = [_P, _I, _P, _P, _I, _I, _P, _I, _P, _P]
+    L.orc_matmul_w8a16_ref.restype = None
+    L.orc_gemm_w8a8_ref.argtypes = [_P, _P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _P]
+    L.orc_gemm_w8a8_ref.restype = _I
+
+
+def _ptr(a: np.ndarray | None):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a: np.ndarray, dtype) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _f16_bits(a: np.ndarray) -> np.ndarray:
+    a = np.asarray(a)
+    if a.dtype == np.float16:
+        return np.ascontiguousarray(a).view(np.uint16)
+    if a.dtype == np.uint16:
+        return np.ascontiguousarray(a)
+    raise TypeError(f"expected float16 (or its uint16 bits), got {a.dtype}")
+
+
+# --------------------------------------------------------------------------
+# binary16 conversions (IEEE 754 definition)
+# --------------------------------------------------------------------------
+def half_to_float(bits: int) -> float:
+    return float(lib().orc_half_to_float(int(bits)))
+
+
+def float_to_half(x: float) -> int:
+    return int(lib().orc_float_to_half(float(np.float32(x))))
+
+
+# --------------------------------------------------------------------------
+# INT4 asymmetric per-group ("Quantization Explained", Scale and Zero-Point;
+# "Quantization from Scratch", round-to-nearest quantize())
+# --------------------------------------------------------------------------
+def quantize_group_int4(w: np.ndarray, group_size: int = 128):
+    """Returns (qweight u32 [N, K/8], scales fp16 [N, K/g], qzeros u32 [N, ceil(K/g/8)])."""
+    w = np.asarray(w)
+    if w.ndim != 2:
+        raise ValueError("w must be 2-D [N, K]")
+    N, K = w.shape
+    if w.dtype == np.float32:
+        src, is16 = _c(w, np.float32), 0
+    else:
+        src, is16 = _f16_bits(w), 1
+    G = K // group_size
+    qw = np.zeros((N, K // 8), np.uint32)
+    sc = np.zeros((N, G), np.uint16)
+    qz = np.zeros((N, (G + 7) // 8), np.uint32)
+    rc = lib().orc_quantize_group_int4(_ptr(src), is16, N, K, group_size, _ptr(qw), _ptr(sc), _ptr(qz))
+    if rc != 0:
+        raise ValueError(f"orc_quantize_group_int4: bad arguments N={N} K={K} g={group_size}")
+    return qw, sc.view(np.float16), qz
+
+
+def dequant_int4(qweight, scales, qzeros, K: int, group_size: int = 128) -> np.ndarray:
+    """w^ = s (q - z) in fp64, [N, K] ("Quantization from Scratch", Scale and zero-point)."""
+    qw = _c(qweight, np.uint32)
+    sc = _f16_bits(scales)
+    qz = _c(qzeros, np.uint32)
+    N = qw.shape[0]
+    out = np.zeros((N, K), np.float64)
+    lib().orc_dequant_int4(_ptr(qw), _ptr(sc), _ptr(qz), N, K, group_size, _ptr(out))
+    return out
+
+
+def unpack_int4_codes(qweight, K: int) -> np.ndarray:
+    """Codes q[n, k] in [0, 15] from the packed layout (nibble k mod 8 of word k/8)."""
+    qw = _c(qweight, np.uint32)
+    shifts = (4 * np.arange(8, dtype=np.uint32))
+    codes = (qw[:, :, None] >> shifts[None, None, :]) & 0xF
+    return codes.reshape(qw.shape[0], K).astype(np.int32)
+
+
+def unpack_int4_zeros(qzeros, G: int) -> np.ndarray:
+    qz = _c(qzeros, np.uint32)
+    shifts = (4 * np.arange(8, dtype=np.uint32))
+    z = (qz[:, :, None] >> shifts[None, None, :]) & 0xF
+    return z.reshape(qz.shape[0], -1)[:, :G].astype(np.int32)
+
+
+# --------------------------------------------------------------------------
+# INT8 symmetric per row ("How quantization works": math, quant.py, q8_per_row,
+# SmoothQuant Xs = X / s, Ws = W * s)
+# --------------------------------------------------------------------------
+def quantize_int8_per_channel(w: np.ndarray, smooth: np.ndarray | None = None):
+    """Weights [N, K] fp16 -> (int8 [N, K], fp32 scales [N]); w*s_j first if smooth."""
+    return quantize_sym_rows(w, smooth, 1, 8)
+
+
+def quantize_int8_per_token(x: np.ndarray, smooth: np.ndarray | None = None):
+    """Activations [M, K] fp16 -> (int8 [M, K], fp32 scales [M]); x/s_j first if smooth."""
+    return quantize_sym_rows(x, smooth, 2, 8)
+
+
+def quantize_sym_rows(a, smooth=None, mode: int = 0, bits: int = 8):
+    """Symmetric b-bit quantization, one scale per row of ``a`` (fp16 [R, K]).
+    mode 1 multiplies column k by smooth[k] first, mode 2 divides by it."""
+    bits16 = _f16_bits(a)
+    R, K = bits16.shape
+    sm = None if smooth is None else _c(smooth, np.float32)
+    if sm is not None and sm.shape != (K,):
+        raise ValueError("smooth must have shape [K]")
+    q = np.zeros((R, K), np.int8)
+    s = np.zeros(R, np.float32)
+    rc = lib().orc_quantize_sym_rows(_ptr(bits16), R, K, _ptr(sm), mode if sm is not None else 0,
+                                     int(bits), _ptr(q), _ptr(s))
+    if rc != 0:
+        raise ValueError("orc_quantize_sym_rows: bad arguments")
+    return q, s
+
+
+def smooth_factors(x: np.ndarray, w: np.ndarray, alpha: float = 0.5) -> np.ndarray:
+    """s_j = max|X_j|^a / max|W_j|^(1-a) ("How quantization works", SmoothQuant)."""
+    xb, wb = _f16_bits(x), _f16_bits(w)
+    M, K = xb.shape
+    N, K2 = wb.shape
+    if K != K2:
+        raise ValueError("X and W must share K")
+    s = np.zeros(K, np.float32)
+    rc = lib().orc_smooth(_ptr(xb), M, _ptr(wb), N, K, float(alpha), _ptr(s))
+    if rc != 0:
+        raise ValueError("orc_smooth: bad arguments")
+    return s
+
+
+# --------------------------------------------------------------------------
+# fp64 matmul references
+# --------------------------------------------------------------------------
+def _rows_arg(rows, N):
+    if rows is None:
+        return None, N
+    r = _c(rows, np.int32)
+    if r.size and (r.min() < 0 or r.max() >= N):
+        raise ValueError("row index out of range")
+    return r, int(r.size)
+
+
+def matmul_w4a16_ref(x, qweight, scales, qzeros, K: int, group_size: int = 128, rows=None):
+    """(y [B, nrows], bound [B, nrows]) in fp64: y = sum_k s(q-z) x, bound = sum_k |s(q-z) x|."""
+    xb = _f16_bits(np.atleast_2d(x))
+    B = xb.shape[0]
+    qw = _c(qweight, np.uint32)
+    sc = _f16_bits(scales)
+    qz = _c(qzeros, np.uint32)
+    N = qw.shape[0]
+    r, nr = _rows_arg(rows, N)
+    y = np.zeros((B, nr), np.float64)
+    bd = np.zeros((B, nr), np.float64)
+    lib().orc_matmul_w4a16_ref(_ptr(xb), B, _ptr(qw), _ptr(sc), _ptr(qz), N, K, group_size,
+                               _ptr(r), nr, _ptr(y), _ptr(bd))
+    return y, bd
+
+
+def matmul_w8a16_ref(x, wq, sw, rows=None):
+    xb = _f16_bits(np.atleast_2d(x))
+    B, K = xb.shape
+    q = _c(wq, np.int8)
+    s = _c(sw, np.float32)
+    N = q.shape[0]
+    r, nr = _rows_arg(rows, N)
+    y = np.zeros((B, nr), np.float64)
+    bd = np.zeros((B, nr), np.float64)
+    lib().orc_matmul_w8a16_ref(_ptr(xb), B, _ptr(q), _ptr(s), N, K, _ptr(r), nr, _ptr(y), _ptr(bd))
+    return y, bd
+
+
+def gemm_w8a8_ref(xq, sx, wq, sw, ms=None, ns=None):
+    """(acc int64 [nm, nn], y fp64, bound fp64) on the selected rows of X (ms) and of W (ns)."""
+    a = _c(xq, np.int8)
+    b = _c(wq, np.int8)
+    M, K = a.shape
+    N = b.shape[0]
+    sxa = _c(sx, np.float32)
+    swa = _c(sw, np.float32)
+    m_arr, nm = _rows_arg(ms, M)
+    n_arr, nn = _rows_arg(ns, N)
+    acc = np.zeros((nm, nn), np.int64)
+    y = np.zeros((nm, nn), np.float64)
+    bd = np.zeros((nm, nn), np.float64)
+    rc = lib().orc_gemm_w8a8_ref(_ptr(a), _ptr(sxa), _ptr(b), _ptr(swa), M, N, K, _ptr(m_arr), nm,
+                                 _ptr(n_arr), nn, _ptr(acc), _ptr(y), _ptr(bd))
+    if rc == -2:
+        raise OverflowError("an int8 accumulator left the int32 range")
+    return acc, y, bd

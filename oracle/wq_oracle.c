@@ -1,0 +1,355 @@
+/*
+ * wq_oracle.c -- plain, slow, single-threaded CPU oracle for the quantization
+ * hot path.  TEST INFRASTRUCTURE ONLY: the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg are the only callers.  It shares no code with
+ * the CUDA library (no headers, helpers or tables) and never calls it.
+ *
+ * Every routine is the plain definition from the source pages, written as
+ * scalar loops in the order the pages state the steps:
+ *
+ *   [P1] "How quantization works" (AI-infra handbook): section "The math of
+ *        quantization" (symmetric s = max|x|/(2^(b-1)-1), q = clamp(round(x/s)),
+ *        x^ = q*s), the quant.py listing (absmax clamped at 1e-8), section
+ *        "Activation quantization and outliers" (per-row INT8, SmoothQuant
+ *        s_j = max|X_j|^a / max|W_j|^(1-a) with 1e-5 clamps, X/s and W*s),
+ *        exercise 2 (fp16 scale + 4-bit zero point per group of 128).
+ *   [P2] "Quantization" (engine-room ch. 15), section "The Mathematics":
+ *        SmoothQuant Y = (X diag(s)^-1)(diag(s) W).
+ *   [P3] "Quantization from Scratch: Scale, Zero-Point, GPTQ and AWQ":
+ *        section "Scale and zero-point" (w^ = (q - z) s) and the round-to-
+ *        nearest quantize() in "Measured on two real layers" (scale 0 -> 1).
+ *   [P4] "Quantization: Smaller Weights, Same Answers (Mostly)": section
+ *        "How does quantized matrix multiplication actually run on the GPU?"
+ *        (integer products summed exactly in a 32-bit accumulator).
+ *   [P5] "Quantization Explained: INT8, INT4, GPTQ and AWQ for LLMs":
+ *        "Uniform Affine Quantization" (x_q = round(x/s) + z,
+ *        x^ = s (x_q - z)), "Scale and Zero-Point" (s = (max-min)/(2^b-1),
+ *        z = round(-min/s)), "Manual Group-Wise Quantizer" (clamp to [0,15]).
+ *
+ * Readings where the pages are silent (each also listed in the design notes):
+ *   - round() is round-half-to-even (the pages' code uses torch/np.round);
+ *     here nearbyint() in the default FE_TONEAREST mode.
+ *   - x/s is an IEEE fp32 division (no reciprocal, no fused multiply-add);
+ *     build with -ffp-contract=off -fno-fast-math.
+ *   - the INT4 group scale is rounded to fp16 (the stored format) BEFORE z
+ *     and the codes are computed, so quantizer and dequantizer share one grid.
+ *   - the INT4 group range is widened to contain 0 (lo = min(min,0),
+ *     hi = max(max,0)) so that z lands in [0,15] and 0 maps to an exact code.
+ *   - INT4 codes: element k of a row is nibble (k mod 8) of word k/8; the
+ *     zero point of group j is nibble (j mod 8) of zero word j/8.
+ *   - INT8 scales are fp32; smoothing never rounds X/s or W*s to fp16.
+ *   - inputs must be finite.
+ *
+ * Floating-point matmul references are computed in fp64.
+ */
+#include <fenv.h>
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+/* ------------------------------------------------------------------------ */
+/* IEEE 754 binary16, written from the format definition:                    */
+/*   normal:    (-1)^s * 2^(e-15) * (1 + m/1024),  1 <= e <= 30              */
+/*   subnormal: (-1)^s * 2^(-14)  * (m/1024),      e == 0                    */
+/* ------------------------------------------------------------------------ */
+
+float orc_half_to_float(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);                 /* 2^-14 * m/1024 */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(1024 + m), e - 25);     /* 2^(e-15) * (1024+m)/1024 */
+    return (float)(sign ? -v : v);
+}
+
+/* Nearest binary16 value, ties to even mantissa; overflow to infinity. */
+uint16_t orc_float_to_half(float f)
+{
+    uint16_t sign = signbit(f) ? 0x8000 : 0;
+    double a = fabs((double)f);
+    if (isnan(f))
+        return 0x7e00;
+    /* 65520 is the midpoint between 65504 (largest finite) and 2^16; it and
+       everything above round to infinity. */
+    if (a >= 65520.0)
+        return sign | 0x7c00;
+    if (a < ldexp(1.0, -14)) {
+        /* subnormal grid: multiples of 2^-24 */
+        double m = nearbyint(a / ldexp(1.0, -24));
+        return sign | (uint16_t)m;                 /* m == 1024 is the smallest normal */
+    }
+    int E;
+    frexp(a, &E);                                  /* a = f * 2^E, f in [0.5, 1) */
+    int e = E - 1;                                 /* a in [2^e, 2^(e+1)) */
+    double m = nearbyint(a / ldexp(1.0, e - 10));  /* in [1024, 2048] */
+    if (m == 2048.0) {
+        m = 1024.0;
+        e += 1;
+    }
+    return sign | (uint16_t)(((e + 15) << 10) | ((int)m - 1024));
+}
+
+static int rne_to_int(float v)
+{
+    return (int)nearbyintf(v);                     /* FE_TONEAREST: half to even */
+}
+
+static int clampi(int v, int lo, int hi)
+{
+    return v < lo ? lo : (v > hi ? hi : v);
+}
+
+int orc_rounding_mode_is_nearest(void)
+{
+    return fegetround() == FE_TONEAREST;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Asymmetric INT4 per-group quantizer  ([P5] "Scale and Zero-Point",        */
+/* [P3] quantize(), [P1] exercise 2 for the stored format).                  */
+/* w: [N][K] fp32 (w_is_f16 == 0) or fp16 bits (w_is_f16 == 1), row-major.   */
+/* Outputs: qweight [N][K/8], scales fp16 bits [N][K/g],                     */
+/*          qzeros [N][ceil(K/g/8)].  Returns 0, or -1 on bad arguments.     */
+/* ------------------------------------------------------------------------ */
+static float load_w(const void *w, int w_is_f16, size_t idx)
+{
+    return w_is_f16 ? orc_half_to_float(((const uint16_t *)w)[idx]) : ((const float *)w)[idx];
+}
+
+int orc_quantize_group_int4(const void *w, int w_is_f16, int N, int K, int g,
+                            uint32_t *qweight, uint16_t *scales, uint32_t *qzeros)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || K % 8 != 0)
+        return -1;
+    const int G = K / g;
+    const int ZW = (G + 7) / 8;
+    memset(qweight, 0, sizeof(uint32_t) * (size_t)N * (K / 8));
+    memset(qzeros, 0, sizeof(uint32_t) * (size_t)N * ZW);
+    for (int n = 0; n < N; ++n) {
+        for (int j = 0; j < G; ++j) {
+            const size_t base = (size_t)n * K + (size_t)j * g;
+            /* range of the group, widened to contain 0 */
+            float lo = 0.0f, hi = 0.0f;
+            for (int t = 0; t < g; ++t) {
+                float v = load_w(w, w_is_f16, base + t);
+                if (v < lo) lo = v;
+                if (v > hi) hi = v;
+            }
+            /* s = (max - min) / (2^4 - 1), stored as fp16; a zero scale becomes 1 */
+            float s32 = (hi - lo) / 15.0f;
+            uint16_t s16 = orc_float_to_half(s32);
+            if (s16 == 0)
+                s16 = 0x3c00;                       /* 1.0 */
+            float s = orc_half_to_float(s16);
+            /* z = round(-min / s), kept in the 4-bit range */
+            int z = clampi(rne_to_int(-lo / s), 0, 15);
+            scales[(size_t)n * G + j] = s16;
+            qzeros[(size_t)n * ZW + j / 8] |= (uint32_t)z << (4 * (j % 8));
+            /* q = clamp(round(w / s) + z, 0, 15) */
+            for (int t = 0; t < g; ++t) {
+                int k = j * g + t;
+                float v = load_w(w, w_is_f16, base + t);
+                int q = clampi(rne_to_int(v / s) + z, 0, 15);
+                qweight[(size_t)n * (K / 8) + k / 8] |= (uint32_t)q << (4 * (k % 8));
+            }
+        }
+    }
+    return 0;
+}
+
+/* Unpack helpers for the stored INT4 layout. */
+int orc_int4_code(const uint32_t *qweight, int K, int n, int k)
+{
+    return (int)((qweight[(size_t)n * (K / 8) + k / 8] >> (4 * (k % 8))) & 0xf);
+}
+
+int orc_int4_zero(const uint32_t *qzeros, int K, int g, int n, int j)
+{
+    const int ZW = (K / g + 7) / 8;
+    return (int)((qzeros[(size_t)n * ZW + j / 8] >> (4 * (j % 8))) & 0xf);
+}
+
+/* w^[n][k] = s * (q - z) in fp64  ([P3] "Scale and zero-point", [P5]). */
+void orc_dequant_int4(const uint32_t *qweight, const uint16_t *scales,
+                      const uint32_t *qzeros, int N, int K, int g, double *what)
+{
+    const int G = K / g;
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            int j = k / g;
+            double s = (double)orc_half_to_float(scales[(size_t)n * G + j]);
+            int q = orc_int4_code(qweight, K, n, k);
+            int z = orc_int4_zero(qzeros, K, g, n, j);
+            what[(size_t)n * K + k] = s * (double)(q - z);
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Symmetric b-bit per row ([P1] "The math of quantization", quant.py       */
+/* fake_quant_int, q8_per_row; SmoothQuant's Xs = X / s, Ws = W * s first).  */
+/* x: fp16 bits [R][K].  mode 0: no smoothing; 1: multiply column k by       */
+/* smooth[k] (weights, diag(s) W); 2: divide column k by smooth[k]           */
+/* (activations, X diag(s)^-1).  bits in [2, 8]: s = max|x| / (2^(b-1) - 1), */
+/* codes clamped to [-2^(b-1), 2^(b-1) - 1].  Outputs q [R][K] int8 and      */
+/* scales [R] fp32.  INT8 per channel / per token is bits == 8.              */
+/* ------------------------------------------------------------------------ */
+static float smoothed(float v, const float *smooth, int mode, int k)
+{
+    if (mode == 1) return v * smooth[k];
+    if (mode == 2) return v / smooth[k];
+    return v;
+}
+
+int orc_quantize_sym_rows(const uint16_t *x, int R, int K, const float *smooth, int mode,
+                          int bits, int8_t *q, float *scales)
+{
+    if (R <= 0 || K <= 0 || mode < 0 || mode > 2 || (mode != 0 && !smooth) || bits < 2 || bits > 8)
+        return -1;
+    const int qmax = (1 << (bits - 1)) - 1;
+    for (int r = 0; r < R; ++r) {
+        const uint16_t *row = x + (size_t)r * K;
+        float a = 0.0f;
+        for (int k = 0; k < K; ++k) {
+            float v = fabsf(smoothed(orc_half_to_float(row[k]), smooth, mode, k));
+            if (v > a) a = v;
+        }
+        if (a < 1e-8f) a = 1e-8f;                   /* absmax.clamp(min=1e-8) */
+        float s = a / (float)qmax;                  /* s = max|x| / (2^(b-1) - 1) */
+        scales[r] = s;
+        for (int k = 0; k < K; ++k) {
+            float v = smoothed(orc_half_to_float(row[k]), smooth, mode, k);
+            q[(size_t)r * K + k] = (int8_t)clampi(rne_to_int(v / s), -qmax - 1, qmax);
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* SmoothQuant factors ([P1] "Activation quantization and outliers",         */
+/* [P2] "The Mathematics"): s_j = max|X_j|^a / max|W_j|^(1-a), both maxima   */
+/* clamped at 1e-5, X: fp16 [M][K], W: fp16 [N][K] (nn.Linear layout, so    */
+/* column j of both is input channel j).  For a == 0.5 the powers are        */
+/* square roots (correctly rounded); otherwise pow() in fp64 rounded to fp32.*/
+/* ------------------------------------------------------------------------ */
+int orc_smooth(const uint16_t *X, int M, const uint16_t *W, int N, int K,
+               double alpha, float *s)
+{
+    if (M <= 0 || N <= 0 || K <= 0)
+        return -1;
+    for (int j = 0; j < K; ++j) {
+        float ax = 0.0f, aw = 0.0f;
+        for (int m = 0; m < M; ++m) {
+            float v = fabsf(orc_half_to_float(X[(size_t)m * K + j]));
+            if (v > ax) ax = v;
+        }
+        for (int n = 0; n < N; ++n) {
+            float v = fabsf(orc_half_to_float(W[(size_t)n * K + j]));
+            if (v > aw) aw = v;
+        }
+        if (ax < 1e-5f) ax = 1e-5f;
+        if (aw < 1e-5f) aw = 1e-5f;
+        float num, den;
+        if (alpha == 0.5) {
+            num = sqrtf(ax);
+            den = sqrtf(aw);
+        } else {
+            num = (float)pow((double)ax, alpha);
+            den = (float)pow((double)aw, 1.0 - alpha);
+        }
+        s[j] = num / den;
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* W4A16 matmul reference in fp64 ([P1] "Inference view": weights unpacked,  */
+/* multiplied by their scales and accumulated): y[b][n] = sum_k w^[n][k]     */
+/* x[b][k], plus bound[b][n] = sum_k |w^[n][k] x[b][k]|.  rows (nullable)    */
+/* selects output rows; results are [B][nrows].                              */
+/* ------------------------------------------------------------------------ */
+void orc_matmul_w4a16_ref(const uint16_t *x, int B, const uint32_t *qweight,
+                          const uint16_t *scales, const uint32_t *qzeros, int N, int K,
+                          int g, const int *rows, int nrows, double *y, double *bound)
+{
+    const int G = K / g;
+    if (!rows) nrows = N;
+    for (int i = 0; i < nrows; ++i) {
+        int n = rows ? rows[i] : i;
+        for (int b = 0; b < B; ++b) {
+            double acc = 0.0, bnd = 0.0;
+            for (int k = 0; k < K; ++k) {
+                int j = k / g;
+                double s = (double)orc_half_to_float(scales[(size_t)n * G + j]);
+                int q = orc_int4_code(qweight, K, n, k);
+                int z = orc_int4_zero(qzeros, K, g, n, j);
+                double t = s * (double)(q - z) * (double)orc_half_to_float(x[(size_t)b * K + k]);
+                acc += t;
+                bnd += fabs(t);
+            }
+            y[(size_t)b * nrows + i] = acc;
+            bound[(size_t)b * nrows + i] = bnd;
+        }
+    }
+}
+
+/* W8A16 reference: w^[n][k] = sw[n] * q[n][k] ([P1] per-channel INT8). */
+void orc_matmul_w8a16_ref(const uint16_t *x, int B, const int8_t *wq, const float *sw,
+                          int N, int K, const int *rows, int nrows, double *y, double *bound)
+{
+    if (!rows) nrows = N;
+    for (int i = 0; i < nrows; ++i) {
+        int n = rows ? rows[i] : i;
+        for (int b = 0; b < B; ++b) {
+            double acc = 0.0, bnd = 0.0;
+            for (int k = 0; k < K; ++k) {
+                double t = (double)sw[n] * (double)wq[(size_t)n * K + k] *
+                           (double)orc_half_to_float(x[(size_t)b * K + k]);
+                acc += t;
+                bnd += fabs(t);
+            }
+            y[(size_t)b * nrows + i] = acc;
+            bound[(size_t)b * nrows + i] = bnd;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* W8A8 reference ([P4] quantized matmul on the GPU; [P1] W8A8 scheme):      */
+/* acc[m][n] = sum_k xq[m][k] wq[n][k] exactly (int64, checked to fit int32),*/
+/* y = acc * sx[m] * sw[n] in fp64, bound = sx sw sum |xq wq|.               */
+/* ms/ns select rows of X and rows of W (columns of y); results [nm][nn].    */
+/* Returns 0, or -2 if an accumulator leaves the int32 range.                */
+/* ------------------------------------------------------------------------ */
+int orc_gemm_w8a8_ref(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                      int M, int N, int K, const int *ms, int nm, const int *ns, int nn,
+                      int64_t *acc, double *y, double *bound)
+{
+    int rc = 0;
+    if (!ms) nm = M;
+    if (!ns) nn = N;
+    for (int a = 0; a < nm; ++a) {
+        int m = ms ? ms[a] : a;
+        for (int c = 0; c < nn; ++c) {
+            int n = ns ? ns[c] : c;
+            int64_t s = 0, sa = 0;
+            for (int k = 0; k < K; ++k) {
+                int64_t p = (int64_t)xq[(size_t)m * K + k] * (int64_t)wq[(size_t)n * K + k];
+                s += p;
+                sa += p < 0 ? -p : p;
+            }
+            if (s > INT32_MAX || s < INT32_MIN)
+                rc = -2;
+            acc[(size_t)a * nn + c] = s;
+            y[(size_t)a * nn + c] = (double)s * (double)sx[m] * (double)sw[n];
+            bound[(size_t)a * nn + c] = (double)sa * (double)sx[m] * (double)sw[n];
+        }
+    }
+    return rc;
+}

@@ -1,0 +1,388 @@
+"""Pins for the CPU oracle: page-printed values, closed forms, invariants, special
+cases that reduce to library routines, and brute force on tiny inputs.
+
+Each check is chosen so that a plausible slip in the oracle (a dropped term, a
+wrong sign or index, a transposed operand, a wrong rounding mode) fails one of
+them.  These run without a GPU.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------
+# binary16 conversion against numpy's independent implementation
+# --------------------------------------------------------------------------
+def test_half_to_float_all_bit_patterns():
+    L = oracle.lib()
+    bits = np.arange(65536, dtype=np.uint32)
+    ours = np.array([L.orc_half_to_float(int(b)) for b in bits], np.float32)
+    ref = bits.astype(np.uint16).view(np.float16).astype(np.float32)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+
+
+def test_float_to_half_matches_numpy_rne():
+    L = oracle.lib()
+    g = np.random.default_rng(1)
+    # random bit patterns over the whole fp16-relevant exponent range, plus edges
+    mant = g.integers(0, 1 << 23, 40000, dtype=np.uint32)
+    expo = g.integers(127 - 27, 127 + 17, 40000, dtype=np.uint32)
+    sign = g.integers(0, 2, 40000, dtype=np.uint32)
+    f = ((sign << 31) | (expo << 23) | mant).view(np.float32)
+    edges = np.array([0.0, -0.0, 65504.0, 65519.99, 65520.0, 70000.0, 2 ** -24, 2 ** -25,
+                      3 * 2 ** -25, 2 ** -14, 2 ** -14 - 2 ** -25, 1.0 + 2 ** -11,
+                      1.0 + 3 * 2 ** -11, 0.1, 0.128, 0.052, 1e-8, -2 ** -26], np.float32)
+    f = np.concatenate([f, edges, -edges])
+    with np.errstate(over="ignore"):
+        ref = f.astype(np.float16).view(np.uint16)
+    ours = np.array([L.orc_float_to_half(float(v)) for v in f], np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# --------------------------------------------------------------------------
+# INT4 asymmetric: the pages' worked examples
+# --------------------------------------------------------------------------
+def test_int4_six_weight_worked_example():
+    d = gold("int4_worked_six_weights.json")
+    w = np.zeros((1, d["pad_with_zeros_to"]), np.float32)
+    w[0, :6] = d["weights"]
+    qw, sc, qz = oracle.quantize_group_int4(w, group_size=8)
+    codes = oracle.unpack_int4_codes(qw, 8)[0]
+    z = oracle.unpack_int4_zeros(qz, 1)[0, 0]
+    s = float(sc[0, 0])
+    assert round(s, 3) == d["scale"]
+    assert z == d["zero_point"]
+    assert list(codes[:6]) == d["codes"]
+    assert list(codes[6:]) == [z, z]                  # the exact zeros land on z
+    back = oracle.dequant_int4(qw, sc, qz, 8, 8)[0, :6]
+    assert [round(v, 3) for v in back] == d["dequantized_3dp"]
+    err = np.abs(back - np.asarray(d["weights"]))
+    assert round(err.max(), 3) == d["max_abs_error"]
+    assert err.max() <= s / 2 and round(s / 2, 3) == d["half_step"]
+
+
+def test_int4_eight_weight_worked_example():
+    d = gold("int4_worked_eight_weights.json")
+    w = np.asarray([d["weights"]], np.float32)
+    qw, sc, qz = oracle.quantize_group_int4(w, group_size=8)
+    assert round(float(sc[0, 0]), 4) == d["scale_4dp"]
+    assert oracle.unpack_int4_zeros(qz, 1)[0, 0] == d["zero_point"]
+    assert list(oracle.unpack_int4_codes(qw, 8)[0]) == d["codes"]
+    back = oracle.dequant_int4(qw, sc, qz, 8, 8)[0]
+    assert [round(v, 3) + 0.0 for v in back] == d["dequantized_3dp"]
+
+
+def test_int4_fp16_input_path_matches_fp32_path():
+    # The same values given as fp16 and as the fp32 of those fp16 values quantize identically.
+    g = np.random.default_rng(2)
+    w16 = (g.standard_normal((8, 256)) * 0.02).astype(np.float16)
+    a = oracle.quantize_group_int4(w16, 128)
+    b = oracle.quantize_group_int4(w16.astype(np.float32), 128)
+    for x, y in zip(a, b):
+        assert np.array_equal(np.asarray(x).view(np.uint8), np.asarray(y).view(np.uint8))
+
+
+# --------------------------------------------------------------------------
+# INT4 invariants: error bound s/2, exact zero, range coverage, packing layout
+# --------------------------------------------------------------------------
+def _int4_case(seed=3, N=64, K=1024, g=128):
+    r = np.random.default_rng(seed)
+    w = (r.standard_normal((N, K)) * 0.02).astype(np.float32)
+    w.reshape(-1)[96::97] *= 20                        # outliers, as in the tiny workload
+    w[:, 5::37] = 0.0                                  # exact zeros
+    w[3, :128] = 0.0                                   # an all-zero group
+    w[4, 128:256] = 0.25                               # a constant group
+    w[5, 256:384] = np.abs(w[5, 256:384]) + 0.01       # an all-positive group
+    w[6, 384:512] = -np.abs(w[6, 384:512]) - 0.01      # an all-negative group
+    return w, oracle.quantize_group_int4(w, g)
+
+
+def test_int4_error_bound_half_step():
+    w, (qw, sc, qz) = _int4_case()
+    N, K = w.shape
+    s = np.repeat(sc.astype(np.float64), 128, axis=1)
+    z = np.repeat(oracle.unpack_int4_zeros(qz, K // 128), 128, axis=1)
+    back = oracle.dequant_int4(qw, sc, qz, K)
+    pre = np.rint(w / s) + z                           # pre-clamp code (float reading)
+    inside = (pre >= 0) & (pre <= 15)
+    err = np.abs(back - w)
+    slack = np.spacing(np.abs(w).astype(np.float32)).astype(np.float64) + 2 ** -40
+    assert np.all(err[inside] <= s[inside] / 2 + slack[inside] + s[inside] * 2 ** -22)
+    # with the range widened to contain 0 and the fp16 scale, clipping is at most one step
+    assert np.all(err <= 1.5 * s)
+
+
+def test_int4_zero_maps_exactly():
+    w, (qw, sc, qz) = _int4_case()
+    back = oracle.dequant_int4(qw, sc, qz, w.shape[1])
+    assert np.all(back[w == 0.0] == 0.0)
+    assert np.all(back[3, :128] == 0.0) and sc[3, 0] == np.float16(1.0)
+
+
+def test_int4_constant_and_one_signed_groups():
+    w, (qw, sc, qz) = _int4_case()
+    K = w.shape[1]
+    z = oracle.unpack_int4_zeros(qz, K // 128)
+    codes = oracle.unpack_int4_codes(qw, K)
+    # constant 0.25: range [0, 0.25] -> s = fp16(0.25/15), z = 0, codes 15
+    assert sc[4, 1] == np.float16(np.float32(0.25) / np.float32(15))
+    assert z[4, 1] == 0 and np.all(codes[4, 128:256] == 15)
+    # all-positive group: z = 0, the maximum gets code 15; all-negative: z = 15
+    assert z[5, 2] == 0 and codes[5, 256:384].max() == 15
+    assert z[6, 3] == 15 and codes[6, 384:512].min() == 0
+
+
+def test_int4_packing_order_nibbles():
+    # values (c - 7) * 0.125 for c = 0..15 give s = 0.125 exactly, z = 7 and codes c; read back
+    # through the documented layout: element k -> nibble (k mod 8) of word k // 8.
+    K = 1024
+    base = (np.arange(16, dtype=np.float32) - 7) * np.float32(0.125)
+    w = np.tile(base, K // 16)[None, :].copy()
+    qw, sc, qz = oracle.quantize_group_int4(w, 128)
+    codes = oracle.unpack_int4_codes(qw, K)[0]
+    assert np.array_equal(codes, np.tile(np.arange(16), K // 16))
+    word0 = int(qw[0, 0])
+    assert [(word0 >> (4 * i)) & 0xF for i in range(8)] == list(range(8))
+    assert qz.shape == (1, 1) and int(qz[0, 0]) == 0x77777777 and np.all(sc == np.float16(0.125))
+
+
+def test_storage_overhead_and_70b_estimate():
+    d = gold("storage_overhead.json")
+    N, K, g = 256, 8192, d["group"]
+    w = np.zeros((N, K), np.float16)
+    qw, sc, qz = oracle.quantize_group_int4(w, g)
+    bits_per_weight_overhead = 8 * (sc.nbytes + qz.nbytes) / (N * K)
+    assert bits_per_weight_overhead == d["overhead_bits_per_weight"]
+    bytes_per_param = (qw.nbytes + sc.nbytes + qz.nbytes) / (N * K)
+    assert bytes_per_param == d["bytes_per_param"]
+    assert round(d["params"] * bytes_per_param / 1e9, 1) == d["total_gb_1dp"]
+
+
+# --------------------------------------------------------------------------
+# Symmetric quantization: the pages' INT8 and INT4 examples
+# --------------------------------------------------------------------------
+def test_int8_worked_example_with_outlier():
+    d = gold("int8_worked_outlier.json")
+    w = np.asarray([d["weights"]], np.float16)
+    q, s = oracle.quantize_int8_per_channel(w)
+    assert q[0, 1] == d["code_of_0.12"]
+    back = q.astype(np.float64) * s[0]
+    assert np.all(np.abs(back - w.astype(np.float64)) <= s[0] / 2 + 1e-12)   # half a step
+    w2 = np.asarray([d["weights"] + [d["outlier"]]], np.float16)
+    q2, s2 = oracle.quantize_int8_per_channel(w2)
+    assert round(float(s2[0] / s[0]), 1) == d["step_ratio_with_outlier"]
+    assert q2[0, 0] == d["code_of_0.04_with_outlier"]
+    lost = 1 - q2[0, 1] * float(s2[0]) / float(w2[0, 1])
+    assert round(100 * lost) == d["loss_of_0.12_with_outlier_percent"]
+
+
+def test_symmetric_int4_exercises():
+    d = gold("symmetric_int4_exercises.json")
+    e = d["exercise_step"]
+    q, s = oracle.quantize_sym_rows(np.asarray([e["group"]], np.float16), bits=4)
+    assert round(float(s[0]), 4) == e["scale_4dp"] and q[0, 1] == e["code_of_0.05"]
+    o = d["outlier_group"]
+    q, s = oracle.quantize_sym_rows(np.asarray([o["group"]], np.float16), bits=4)
+    assert round(float(s[0]), 2) == o["scale_2dp"]
+    small = [i for i, v in enumerate(o["group"]) if abs(v) < 1]
+    assert np.all(q[0, small] == o["small_codes"]) and q[0, 4] == 7
+
+
+def test_int8_codes_range_and_bound():
+    g = np.random.default_rng(4)
+    x = (g.standard_normal((32, 512)) * 3).astype(np.float16)
+    x[:, 7] *= 50
+    x[5] = 0                                            # all-zero row: scale clamp 1e-8/127
+    q, s = oracle.quantize_int8_per_token(x)
+    assert s[5] == np.float32(1e-8) / np.float32(127) and np.all(q[5] == 0)
+    assert q.min() >= -127 and q.max() <= 127           # absmax row scale never needs -128
+    assert np.all(np.abs(q).max(axis=1)[np.arange(32) != 5] == 127)
+    back = q.astype(np.float64) * s[:, None].astype(np.float64)
+    err = np.abs(back - x.astype(np.float64))
+    assert np.all(err <= s[:, None] / 2 * (1 + 2 ** -20) + 1e-30)
+
+
+def test_int8_smoothing_direction():
+    # mode 1 multiplies by s_j, mode 2 divides: x = s (exactly representable) -> x/s = 1, w*s = s^2
+    s = np.asarray([2.0, 4.0, 0.5, 8.0], np.float32)
+    x = np.asarray([[2.0, 4.0, 0.5, 8.0]], np.float16)
+    qx, sx = oracle.quantize_int8_per_token(x, s)
+    assert np.all(qx == 127)                            # x / s == 1 everywhere
+    qw, sw = oracle.quantize_int8_per_channel(x, s)
+    assert sw[0] == np.float32(64.0) / np.float32(127)  # max of w*s is 8*8
+    assert qw[0, 3] == 127 and qw[0, 2] == round(0.25 / (64 / 127))
+
+
+# --------------------------------------------------------------------------
+# SmoothQuant factors
+# --------------------------------------------------------------------------
+def test_smooth_closed_forms():
+    X = np.zeros((3, 5), np.float16)
+    W = np.zeros((4, 5), np.float16)
+    X[1, 0], W[2, 0] = -4.0, 1.0        # sqrt(4)/sqrt(1) = 2
+    X[0, 1], W[3, 1] = 9.0, -0.25       # 3 / 0.5 = 6
+    X[2, 2], W[0, 2] = 0.25, 16.0       # 0.5 / 4 = 0.125
+    W[1, 3] = 4.0                       # X column all zero -> clamp 1e-5
+    # column 4 all zero in both -> 1
+    s = oracle.smooth_factors(X, W, 0.5)
+    assert s[0] == 2.0 and s[1] == 6.0 and s[2] == 0.125
+    assert s[3] == np.float32(np.sqrt(np.float32(1e-5))) / np.float32(2.0)
+    assert s[4] == 1.0
+    # alpha = 1: s = max|X_j| ; alpha = 0: s = 1 / max|W_j|
+    s1 = oracle.smooth_factors(X, W, 1.0)
+    assert s1[0] == 4.0 and s1[1] == 9.0 and s1[2] == 0.25
+    s0 = oracle.smooth_factors(X, W, 0.0)
+    assert s0[0] == 1.0 and s0[1] == 4.0 and s0[2] == np.float32(1 / 16)
+
+
+def test_smooth_balances_columns_and_orientation():
+    # alpha = 0.5 equalizes max|X_j / s_j| and max|W_j * s_j| (= sqrt(ax*aw)); non-square
+    # shapes catch a max taken over the wrong axis of W [out, in].
+    g = np.random.default_rng(5)
+    X = g.standard_normal((48, 96)).astype(np.float16)
+    X[:, [3, 17, 60]] *= 40
+    W = (g.standard_normal((80, 96)) * 0.05).astype(np.float16)
+    s = oracle.smooth_factors(X, W, 0.5).astype(np.float64)
+    mx = np.abs(X.astype(np.float64) / s).max(axis=0)
+    mw = np.abs(W.astype(np.float64) * s).max(axis=0)
+    assert np.allclose(mx, mw, rtol=1e-6)
+    # and the factor tracks the activation outliers
+    assert np.all(s[[3, 17, 60]] > 4 * np.median(s))
+
+
+def test_smoothquant_equivalence_exact_in_fp64():
+    # (X diag(s)^-1)(diag(s) W)^T = X W^T  ("How quantization works", SmoothQuant; the
+    # engine-room chapter's Y = (X diag(s)^-1)(diag(s) W))
+    g = np.random.default_rng(6)
+    X = g.standard_normal((16, 64)).astype(np.float16)
+    W = (g.standard_normal((24, 64)) * 0.02).astype(np.float16)
+    s = oracle.smooth_factors(X, W, 0.5).astype(np.float64)
+    Y = X.astype(np.float64) @ W.astype(np.float64).T
+    Ys = (X.astype(np.float64) / s) @ (W.astype(np.float64) * s).T
+    assert np.max(np.abs(Ys - Y)) <= 1e-12 * np.max(np.abs(Y))
+
+
+# --------------------------------------------------------------------------
+# matmul references: special cases that reduce to library routines / closed forms
+# --------------------------------------------------------------------------
+def test_w4a16_ref_reduces_to_dequant_and_numpy_matmul():
+    w, (qw, sc, qz) = _int4_case(seed=7, N=24, K=256)
+    K = 256
+    what = oracle.dequant_int4(qw, sc, qz, K)
+    g = np.random.default_rng(8)
+    x = g.standard_normal((3, K)).astype(np.float16)
+    y, bound = oracle.matmul_w4a16_ref(x, qw, sc, qz, K)
+    ref = x.astype(np.float64) @ what.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-15)
+    assert np.allclose(bound, np.abs(x.astype(np.float64)) @ np.abs(what).T, rtol=1e-12)
+    # one-hot activations pick out single dequantized weights (catches a transposed operand)
+    e = np.zeros((2, K), np.float16)
+    e[0, 17], e[1, 200] = 1.0, 1.0
+    y1, _ = oracle.matmul_w4a16_ref(e, qw, sc, qz, K)
+    assert np.array_equal(y1[0], what[:, 17]) and np.array_equal(y1[1], what[:, 200])
+    # selected rows agree with the full result
+    ys, _ = oracle.matmul_w4a16_ref(x, qw, sc, qz, K, rows=[5, 0, 23])
+    assert np.array_equal(ys, y[:, [5, 0, 23]])
+
+
+def test_w8a8_ref_is_exact_integer_matmul():
+    g = np.random.default_rng(9)
+    xq = g.integers(-128, 128, (7, 48), dtype=np.int8)
+    wq = g.integers(-128, 128, (9, 48), dtype=np.int8)
+    sx = g.random(7, dtype=np.float32) + 0.5
+    sw = g.random(9, dtype=np.float32) + 0.5
+    acc, y, bound = oracle.gemm_w8a8_ref(xq, sx, wq, sw)
+    ref = xq.astype(np.int64) @ wq.astype(np.int64).T
+    assert np.array_equal(acc, ref)
+    assert np.allclose(y, ref * sx[:, None].astype(np.float64) * sw[None, :].astype(np.float64),
+                       rtol=1e-15)
+    # every pair of int8 codes (K = 1): the products themselves
+    a = np.arange(-128, 128, dtype=np.int8)[:, None]
+    acc1, _, _ = oracle.gemm_w8a8_ref(a, np.ones(256, np.float32), a, np.ones(256, np.float32))
+    assert np.array_equal(acc1, np.outer(np.arange(-128, 128), np.arange(-128, 128)))
+    # the worst case for K = 8192 stays inside int32 (|acc| <= 128^2 * 8192 = 2^27)
+    big = np.full((1, 8192), -128, np.int8)
+    acc2, _, _ = oracle.gemm_w8a8_ref(big, np.ones(1, np.float32), big, np.ones(1, np.float32))
+    assert acc2[0, 0] == 128 * 128 * 8192
+
+
+def test_w8a16_ref_reduces_to_numpy():
+    g = np.random.default_rng(10)
+    wq = g.integers(-127, 128, (12, 96), dtype=np.int8)
+    sw = (g.random(12, dtype=np.float32) + 0.1) * 0.01
+    x = g.standard_normal((2, 96)).astype(np.float16)
+    y, b = oracle.matmul_w8a16_ref(x, wq, sw)
+    what = wq.astype(np.float64) * sw[:, None].astype(np.float64)
+    assert np.allclose(y, x.astype(np.float64) @ what.T, rtol=1e-12, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# direction-only statistics the pages assert (finer granularity -> less error,
+# SmoothQuant between weight-only and plain W8A8)
+# --------------------------------------------------------------------------
+def _rel(a, b):
+    return np.linalg.norm(a - b) / np.linalg.norm(b)
+
+
+def test_granularity_orderings():
+    g = np.random.default_rng(11)
+    W = (g.standard_normal((64, 1024)) * np.exp(g.normal(np.log(0.02), 0.5, (64, 1)))).astype(np.float16)
+    W.reshape(-1)[g.random(W.size) < 0.001] *= 30
+    Wd = W.astype(np.float64)
+    q, s = oracle.quantize_sym_rows(W.reshape(1, -1), bits=8)          # per tensor
+    e_t = _rel((q.astype(np.float64) * s[0]).reshape(W.shape), Wd)
+    q, s = oracle.quantize_int8_per_channel(W)                          # per channel
+    e_c = _rel(q.astype(np.float64) * s[:, None], Wd)
+    assert e_c < e_t
+    qw, sc, qz = oracle.quantize_group_int4(W, 1024)                   # INT4 per channel
+    e4c = _rel(oracle.dequant_int4(qw, sc, qz, 1024, 1024), Wd)
+    qw, sc, qz = oracle.quantize_group_int4(W, 128)                    # INT4 per group
+    e4g = _rel(oracle.dequant_int4(qw, sc, qz, 1024, 128), Wd)
+    assert e4g < e4c and e_c < e4g
+
+
+def test_smoothquant_error_ordering():
+    g = np.random.default_rng(12)
+    X = g.standard_normal((128, 256)).astype(np.float32)
+    X[:, [4, 77, 150, 201]] *= 40
+    X = X.astype(np.float16)
+    W = (g.standard_normal((192, 256)) * 0.02).astype(np.float16)
+    Xd, Wd = X.astype(np.float64), W.astype(np.float64)
+    Y = Xd @ Wd.T
+    qw, sw = oracle.quantize_int8_per_channel(W)
+    Wq = qw * sw[:, None].astype(np.float64)
+    err_w8 = _rel(Xd @ Wq.T, Y)
+    qx, sx = oracle.quantize_sym_rows(X.reshape(1, -1), bits=8)        # per-tensor X as on the page
+    Xq = (qx.astype(np.float64) * sx[0]).reshape(X.shape)
+    err_w8a8 = _rel(Xq @ Wq.T, Y)
+    s = oracle.smooth_factors(X, W, 0.5)
+    qws, sws = oracle.quantize_int8_per_channel(W, s)
+    Xs = (X.astype(np.float32) / s).astype(np.float32)
+    qxs = np.rint(Xs / (np.abs(Xs).max() / np.float32(127)))           # per tensor, for the ordering
+    Xsq = qxs.astype(np.float64) * float(np.abs(Xs).max() / np.float32(127))
+    err_sq = _rel(Xsq @ (qws * sws[:, None].astype(np.float64)).T, Y)
+    assert err_w8 < err_sq < err_w8a8
+    # per-token on the smoothed activations (the path's granularity) is better still
+    qxt, sxt = oracle.quantize_int8_per_token(X, s)
+    err_sq_tok = _rel((qxt * sxt[:, None].astype(np.float64)) @ (qws * sws[:, None].astype(np.float64)).T, Y)
+    assert err_sq_tok < err_w8a8
+
+
+def test_bad_arguments_rejected():
+    with pytest.raises(ValueError):
+        oracle.quantize_group_int4(np.zeros((2, 100), np.float16), 128)
+    with pytest.raises(ValueError):
+        oracle.quantize_sym_rows(np.zeros((2, 8), np.float16), bits=9)
