@@ -1,0 +1,251 @@
+"""Python binding of ``libwq.so``, the sm_100a weight/activation quantization library.
+
+Argument marshalling only: every function checks tensor devices, dtypes and
+shapes, allocates outputs with PyTorch (PyTorch owns device memory and streams
+here), and calls the C entry point of the same name on the current CUDA stream.
+All arithmetic runs in the library's kernels.  There is no CPU fallback: if
+``libwq.so`` is missing the import fails.
+
+Packed INT4 tensors are carried as ``torch.int32`` (bit-identical to the
+library's ``uint32`` words) and fp16 as ``torch.float16``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = ["WQError", "lib", "quantize_group_int4", "quantize_int8_per_channel", "quantize_int8_per_token",
+           "smooth", "smooth_workspace_bytes", "gemv_w4a16", "gemm_w4a16", "gemm_w8a8", "gemv_w8a16",
+           "matmul_w4a16", "device_status", "set_wait_limit", "LIB_PATH"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwq.so")
+
+WQ_OK, WQ_ERR_INVALID_ARG, WQ_ERR_ALIGNMENT, WQ_ERR_UNSUPPORTED, WQ_ERR_CUDA, WQ_ERR_TIMEOUT = range(6)
+WQ_F32, WQ_F16 = 0, 1
+_STATUS = {0: "WQ_OK", 1: "WQ_ERR_INVALID_ARG", 2: "WQ_ERR_ALIGNMENT", 3: "WQ_ERR_UNSUPPORTED",
+           4: "WQ_ERR_CUDA", 5: "WQ_ERR_TIMEOUT"}
+
+
+class WQError(RuntimeError):
+    def __init__(self, status: int, where: str, message: str):
+        super().__init__(f"{where}: {_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python bit_gemv_gemm_group_b200/build.py`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+_P, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+_SIGS = {
+    "wq_quantize_group_int4": [_P, _I, _I, _I, _I, _P, _P, _P, _P],
+    "wq_quantize_int8_per_channel": [_P, _I, _I, _P, _P, _P, _P],
+    "wq_quantize_int8_per_token": [_P, _I, _I, _P, _P, _P, _P],
+    "wq_smooth": [_P, _I, _P, _I, _I, _F, _P, _P, _P],
+    "wq_gemv_w4a16": [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P],
+    "wq_gemm_w4a16": [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P],
+    "wq_gemm_w8a8": [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P],
+    "wq_gemv_w8a16": [_P, _I, _P, _P, _I, _I, _P, _P],
+    "wq_device_status": [_P],
+}
+for _name, _args in _SIGS.items():
+    _fn = getattr(lib, _name)
+    _fn.argtypes = _args
+    _fn.restype = ctypes.c_int
+lib.wq_last_error.argtypes = []
+lib.wq_last_error.restype = ctypes.c_char_p
+lib.wq_smooth_workspace_bytes.argtypes = [_I]
+lib.wq_smooth_workspace_bytes.restype = ctypes.c_size_t
+lib.wq_set_wait_limit.argtypes = [ctypes.c_uint64]
+lib.wq_set_wait_limit.restype = None
+
+
+def _check(status: int, where: str):
+    if status != WQ_OK:
+        raise WQError(status, where, lib.wq_last_error().decode(errors="replace"))
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _cuda(t: torch.Tensor, name: str, dtypes, ndim=None) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-D, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _empty(shape, dtype, like: torch.Tensor) -> torch.Tensor:
+    return torch.empty(shape, dtype=dtype, device=like.device)
+
+
+# --------------------------------------------------------------------------
+# quantizers
+# --------------------------------------------------------------------------
+def quantize_group_int4(w: torch.Tensor, group_size: int = 128, stream=None):
+    """Asymmetric INT4 per group -> (qweight int32 [N, K/8], scales fp16 [N, K/g], qzeros int32 [N, ceil(K/g/8)])."""
+    _cuda(w, "w", (torch.float16, torch.float32), 2)
+    N, K = w.shape
+    G = K // group_size if group_size > 0 else 0
+    qw = _empty((N, K // 8), torch.int32, w)
+    sc = _empty((N, G), torch.float16, w)
+    qz = _empty((N, (G + 7) // 8), torch.int32, w)
+    dt = WQ_F16 if w.dtype == torch.float16 else WQ_F32
+    _check(lib.wq_quantize_group_int4(_ptr(w), dt, N, K, group_size, _ptr(qw), _ptr(sc), _ptr(qz),
+                                      _P(_stream(stream))), "wq_quantize_group_int4")
+    return qw, sc, qz
+
+
+def _q8(fn, name, a, smooth_vec, stream):
+    _cuda(a, "input", (torch.float16,), 2)
+    R, K = a.shape
+    if smooth_vec is not None:
+        _cuda(smooth_vec, "smooth", (torch.float32,), 1)
+        if smooth_vec.numel() != K:
+            raise ValueError("smooth must have K elements")
+    q = _empty((R, K), torch.int8, a)
+    s = _empty((R,), torch.float32, a)
+    _check(fn(_ptr(a), R, K, _ptr(smooth_vec), _ptr(q), _ptr(s), _P(_stream(stream))), name)
+    return q, s
+
+
+def quantize_int8_per_channel(w: torch.Tensor, smooth_vec: torch.Tensor | None = None, stream=None):
+    """Symmetric INT8 per row of weights (w * s_j first when smoothing) -> (int8 [N, K], fp32 [N])."""
+    return _q8(lib.wq_quantize_int8_per_channel, "wq_quantize_int8_per_channel", w, smooth_vec, stream)
+
+
+def quantize_int8_per_token(x: torch.Tensor, smooth_vec: torch.Tensor | None = None, stream=None):
+    """Symmetric INT8 per activation row (x / s_j first when smoothing) -> (int8 [M, K], fp32 [M])."""
+    return _q8(lib.wq_quantize_int8_per_token, "wq_quantize_int8_per_token", x, smooth_vec, stream)
+
+
+def smooth_workspace_bytes(K: int) -> int:
+    return int(lib.wq_smooth_workspace_bytes(int(K)))
+
+
+def smooth(x: torch.Tensor, w: torch.Tensor, alpha: float = 0.5, workspace: torch.Tensor | None = None,
+           stream=None) -> torch.Tensor:
+    """SmoothQuant factors s_j = max|X_j|^alpha / max|W_j|^(1-alpha) -> fp32 [K]."""
+    _cuda(x, "x", (torch.float16,), 2)
+    _cuda(w, "w", (torch.float16,), 2)
+    M, K = x.shape
+    N, K2 = w.shape
+    if K != K2:
+        raise ValueError("x and w must share K")
+    s = _empty((K,), torch.float32, x)
+    if workspace is None:
+        workspace = _empty((max(1, smooth_workspace_bytes(K)),), torch.uint8, x)
+    _cuda(workspace, "workspace", (torch.uint8,), 1)
+    if workspace.numel() < smooth_workspace_bytes(K):
+        raise ValueError("workspace too small")
+    _check(lib.wq_smooth(_ptr(x), M, _ptr(w), N, K, float(alpha), _ptr(s), _ptr(workspace), _P(_stream(stream))),
+           "wq_smooth")
+    return s
+
+
+# --------------------------------------------------------------------------
+# matmuls
+# --------------------------------------------------------------------------
+def _w4_args(x, qweight, scales, qzeros, group_size):
+    _cuda(x, "x", (torch.float16,), 2)
+    _cuda(qweight, "qweight", (torch.int32,), 2)
+    _cuda(scales, "scales", (torch.float16,), 2)
+    _cuda(qzeros, "qzeros", (torch.int32,), 2)
+    B, K = x.shape
+    N = qweight.shape[0]
+    if qweight.shape[1] * 8 != K:
+        raise ValueError("qweight must be [N, K/8]")
+    if group_size <= 0 or K % group_size or tuple(scales.shape) != (N, K // group_size):
+        raise ValueError("scales must be [N, K/group_size]")
+    if tuple(qzeros.shape) != (N, (K // group_size + 7) // 8):
+        raise ValueError("qzeros must be [N, ceil(K/group_size/8)]")
+    return B, N, K
+
+
+def gemv_w4a16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stream=None):
+    """y [B, N] fp16 = x [B, K] @ dequant(W)^T for B = 1..8 (fused dequant GEMV)."""
+    B, N, K = _w4_args(x, qweight, scales, qzeros, group_size)
+    y = out if out is not None else _empty((B, N), torch.float16, x)
+    _cuda(y, "out", (torch.float16,), 2)
+    _check(lib.wq_gemv_w4a16(_ptr(x), B, _ptr(qweight), _ptr(scales), _ptr(qzeros), N, K, group_size, _ptr(y),
+                             _P(_stream(stream))), "wq_gemv_w4a16")
+    return y
+
+
+def gemm_w4a16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stream=None):
+    """y [M, N] fp16 = x [M, K] @ dequant(W)^T for M >= 16 on the tensor cores."""
+    M, N, K = _w4_args(x, qweight, scales, qzeros, group_size)
+    y = out if out is not None else _empty((M, N), torch.float16, x)
+    _cuda(y, "out", (torch.float16,), 2)
+    _check(lib.wq_gemm_w4a16(_ptr(x), M, _ptr(qweight), _ptr(scales), _ptr(qzeros), N, K, group_size, _ptr(y),
+                             _P(_stream(stream))), "wq_gemm_w4a16")
+    return y
+
+
+def matmul_w4a16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stream=None):
+    """GEMV for up to 8 activation rows, tensor-core GEMM above (the caller's choice made for it)."""
+    if x.shape[0] <= 8:
+        return gemv_w4a16(x, qweight, scales, qzeros, group_size, out, stream)
+    return gemm_w4a16(x, qweight, scales, qzeros, group_size, out, stream)
+
+
+def gemm_w8a8(xq, sx, wq, sw, out=None, return_acc: bool = False, acc_out=None, stream=None):
+    """y [M, N] fp16 = fp16((xq @ wq^T) * sx[m] * sw[n]); optionally also the int32 accumulators."""
+    _cuda(xq, "xq", (torch.int8,), 2)
+    _cuda(wq, "wq", (torch.int8,), 2)
+    _cuda(sx, "sx", (torch.float32,), 1)
+    _cuda(sw, "sw", (torch.float32,), 1)
+    M, K = xq.shape
+    N, K2 = wq.shape
+    if K != K2 or sx.numel() != M or sw.numel() != N:
+        raise ValueError("shape mismatch: xq [M,K], wq [N,K], sx [M], sw [N]")
+    y = out if out is not None else _empty((M, N), torch.float16, xq)
+    _cuda(y, "out", (torch.float16,), 2)
+    acc = acc_out
+    if acc is None and return_acc:
+        acc = _empty((M, N), torch.int32, xq)
+    if acc is not None:
+        _cuda(acc, "acc_out", (torch.int32,), 2)
+    _check(lib.wq_gemm_w8a8(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), M, N, K, _ptr(y), _ptr(acc),
+                            _P(_stream(stream))), "wq_gemm_w8a8")
+    return (y, acc) if (return_acc or acc_out is not None) else y
+
+
+def gemv_w8a16(x, wq, sw, out=None, stream=None):
+    """y [B, N] fp16 = fp16(sw[n] * (x @ wq^T)) for B = 1..8."""
+    _cuda(x, "x", (torch.float16,), 2)
+    _cuda(wq, "wq", (torch.int8,), 2)
+    _cuda(sw, "sw", (torch.float32,), 1)
+    B, K = x.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K or sw.numel() != N:
+        raise ValueError("shape mismatch: x [B,K], wq [N,K], sw [N]")
+    y = out if out is not None else _empty((B, N), torch.float16, x)
+    _cuda(y, "out", (torch.float16,), 2)
+    _check(lib.wq_gemv_w8a16(_ptr(x), B, _ptr(wq), _ptr(sw), N, K, _ptr(y), _P(_stream(stream))), "wq_gemv_w8a16")
+    return y
+
+
+def device_status(stream=None) -> int:
+    """Synchronizes the stream and returns (and clears) the device status word (0 = WQ_OK)."""
+    return int(lib.wq_device_status(_P(_stream(stream))))
+
+
+def set_wait_limit(polls: int) -> None:
+    lib.wq_set_wait_limit(int(polls))

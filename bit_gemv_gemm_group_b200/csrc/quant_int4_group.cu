@@ -1,0 +1,168 @@
+// Asymmetric INT4 per-group quantizer: per-group min/max reduction with warp
+// shuffles -> fp16 scale and 4-bit zero point -> round/clamp -> 8 codes per
+// uint32.
+//
+// Source: "Quantization Explained: INT8, INT4, GPTQ and AWQ for LLMs",
+// sections "Uniform Affine Quantization", "Scale and Zero-Point" and "Manual
+// Group-Wise Quantizer"; "Quantization from Scratch", section "Scale and
+// zero-point" and its round-to-nearest quantize() (zero scale -> 1); "How
+// quantization works", section "Granularity" and exercise 2 (fp16 scale and
+// 4-bit zero point per 128 weights).
+//
+// Work decomposition: one warp per (row, zero word) = 8 consecutive groups of
+// one row.  Each lane owns 8 consecutive elements (one 16-byte load for fp16),
+// so a group of G elements is handled by G/8 lanes and a warp covers 256/G
+// groups per iteration.  All of a warp's loads are issued before any
+// arithmetic (G/32 x 16 B in flight per lane) to keep HBM busy.  HBM bytes per
+// weight: 2 (fp16 in) + 0.5 + 2.5/G (out).
+#include "wq_device.cuh"
+#include "wq_host.h"
+
+namespace wq {
+namespace {
+
+template <typename TIn>
+struct Loader;
+
+template <>
+struct Loader<__half> {
+    // 8 fp16 elements -> 8 floats
+    static __device__ __forceinline__ void load8(const __half *p, float (&v)[8]) {
+        uint4 r = ld_stream_u4(p);
+        float2 a = half2_bits_to_float2(r.x), b = half2_bits_to_float2(r.y);
+        float2 c = half2_bits_to_float2(r.z), d = half2_bits_to_float2(r.w);
+        v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+        v[4] = c.x; v[5] = c.y; v[6] = d.x; v[7] = d.y;
+    }
+};
+
+template <>
+struct Loader<float> {
+    static __device__ __forceinline__ void load8(const float *p, float (&v)[8]) {
+        uint4 r0 = ld_stream_u4(p), r1 = ld_stream_u4(p + 4);
+        v[0] = __uint_as_float(r0.x); v[1] = __uint_as_float(r0.y);
+        v[2] = __uint_as_float(r0.z); v[3] = __uint_as_float(r0.w);
+        v[4] = __uint_as_float(r1.x); v[5] = __uint_as_float(r1.y);
+        v[6] = __uint_as_float(r1.z); v[7] = __uint_as_float(r1.w);
+    }
+};
+
+template <typename TIn, int G>
+__global__ void __launch_bounds__(256) quant_int4_group_kernel(const TIn *__restrict__ w, int N, int K,
+                                                                uint32_t *__restrict__ qweight,
+                                                                uint16_t *__restrict__ scales,
+                                                                uint32_t *__restrict__ qzeros) {
+    constexpr int LPG = G / 8;       // lanes per group
+    constexpr int GPI = 32 / LPG;    // groups per warp iteration
+    constexpr int ITERS = 8 / GPI;   // iterations per zero word (8 groups)
+    const int groups = K / G;
+    const int zwords = (groups + 7) / 8;
+    const int lane = threadIdx.x & 31;
+    const long long unit = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (unit >= (long long)N * zwords) return;
+    const int n = (int)(unit / zwords);
+    const int zw = (int)(unit % zwords);
+    const int sub = lane / LPG;  // group slot within an iteration
+    const int li = lane % LPG;   // lane within the group
+
+    // Issue every load of this warp first.
+    float v[ITERS][8];
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int j = zw * 8 + it * GPI + sub;
+        if (j < groups) {
+            Loader<TIn>::load8(w + (size_t)n * K + (size_t)j * G + li * 8, v[it]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[it][e] = 0.0f;
+        }
+    }
+
+    uint32_t zacc = 0;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int j = zw * 8 + it * GPI + sub;
+        // Range of the group, widened to contain 0.
+        float lo = 0.0f, hi = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            lo = fminf(lo, v[it][e]);
+            hi = fmaxf(hi, v[it][e]);
+        }
+#pragma unroll
+        for (int off = LPG / 2; off >= 1; off >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        }
+        // s = fp16((hi - lo) / 15); a zero scale becomes 1.
+        uint16_t s16 = float_to_half_bits_rn(__fdiv_rn(hi - lo, 15.0f));
+        if (s16 == 0) s16 = 0x3c00;
+        const float s = half_bits_to_float(s16);
+        // z = round(-lo / s) in [0, 15]
+        const int z = clampi(__float2int_rn(__fdiv_rn(-lo, s)), 0, 15);
+        if (j < groups) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int q = clampi(__float2int_rn(__fdiv_rn(v[it][e], s)) + z, 0, 15);
+                word |= (uint32_t)q << (4 * e);
+            }
+            qweight[(size_t)n * (K / 8) + (size_t)j * (G / 8) + li] = word;
+            if (li == 0) {
+                scales[(size_t)n * groups + j] = s16;
+                zacc |= (uint32_t)z << (4 * (j & 7));
+            }
+        }
+    }
+    const uint32_t zword = __reduce_or_sync(0xffffffffu, zacc);
+    if (lane == 0) qzeros[(size_t)n * zwords + zw] = zword;
+}
+
+template <typename TIn, int G>
+cudaError_t launch(const void *w, int N, int K, uint32_t *qweight, uint16_t *scales, uint32_t *qzeros,
+                   cudaStream_t stream) {
+    const int zwords = (K / G + 7) / 8;
+    const long long units = (long long)N * zwords;
+    const int warps_per_block = 8;
+    const long long blocks = (units + warps_per_block - 1) / warps_per_block;
+    quant_int4_group_kernel<TIn, G><<<(unsigned)blocks, warps_per_block * 32, 0, stream>>>(
+        static_cast<const TIn *>(w), N, K, qweight, scales, qzeros);
+    return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace wq
+
+extern "C" wq_status wq_quantize_group_int4(const void *w, wq_dtype w_dtype, int N, int K, int group_size,
+                                            uint32_t *qweight, uint16_t *scales, uint32_t *qzeros,
+                                            void *stream) {
+    WQ_REQUIRE_PTR(w, "w");
+    WQ_REQUIRE_PTR(qweight, "qweight");
+    WQ_REQUIRE_PTR(scales, "scales");
+    WQ_REQUIRE_PTR(qzeros, "qzeros");
+    WQ_REQUIRE(N > 0 && K > 0, WQ_ERR_INVALID_ARG, "N and K must be positive (N=%d K=%d)", N, K);
+    WQ_REQUIRE(w_dtype == WQ_F32 || w_dtype == WQ_F16, WQ_ERR_INVALID_ARG, "unknown w_dtype %d",
+               (int)w_dtype);
+    WQ_REQUIRE(group_size == 32 || group_size == 64 || group_size == 128 || group_size == 256,
+               WQ_ERR_UNSUPPORTED, "group_size must be 32, 64, 128 or 256 (got %d)", group_size);
+    WQ_REQUIRE(K % group_size == 0, WQ_ERR_INVALID_ARG, "K (%d) must be a multiple of group_size (%d)", K,
+               group_size);
+    const long long units = (long long)N * ((K / group_size + 7) / 8);
+    WQ_REQUIRE(units / 8 < (1ll << 31), WQ_ERR_UNSUPPORTED, "matrix too large");
+    cudaStream_t st = wq::as_stream(stream);
+    cudaError_t e;
+    const bool f16 = w_dtype == WQ_F16;
+    switch (group_size) {
+        case 32: e = f16 ? wq::launch<__half, 32>(w, N, K, qweight, scales, qzeros, st)
+                         : wq::launch<float, 32>(w, N, K, qweight, scales, qzeros, st); break;
+        case 64: e = f16 ? wq::launch<__half, 64>(w, N, K, qweight, scales, qzeros, st)
+                         : wq::launch<float, 64>(w, N, K, qweight, scales, qzeros, st); break;
+        case 128: e = f16 ? wq::launch<__half, 128>(w, N, K, qweight, scales, qzeros, st)
+                          : wq::launch<float, 128>(w, N, K, qweight, scales, qzeros, st); break;
+        default: e = f16 ? wq::launch<__half, 256>(w, N, K, qweight, scales, qzeros, st)
+                         : wq::launch<float, 256>(w, N, K, qweight, scales, qzeros, st); break;
+    }
+    if (e != cudaSuccess)
+        return wq::fail(WQ_ERR_CUDA, "wq_quantize_group_int4: launch failed: %s", cudaGetErrorString(e));
+    return WQ_OK;
+}

@@ -1,0 +1,175 @@
+// Symmetric INT8 row quantizers: per output channel (weights, optional
+// SmoothQuant W * s) and per token (activations, optional X / s).
+//
+// Source: "How quantization works", sections "The math of quantization"
+// (s = max|x| / (2^(b-1) - 1), q = clamp(round(x/s), -2^(b-1), 2^(b-1)-1)),
+// the quant.py listing (absmax clamped at 1e-8), q8_per_row and SmoothQuant's
+// "Xs, Ws = X / s, W * s" in "Activation quantization and outliers";
+// "Quantization: Smaller Weights, Same Answers (Mostly)", Quick Reference
+// (per-token dynamic activation scales).
+//
+// One CTA of 256 threads per row.  Each thread owns 16-byte chunks of 8 fp16
+// values; for K <= 16384 the (smoothed) row stays in registers between the
+// absmax pass and the quantize pass, so HBM sees 2 B read + 1 B written per
+// element.  Longer rows are read twice (the second read hits L2).
+#include "wq_device.cuh"
+#include "wq_host.h"
+
+namespace wq {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kChunk = 8;                         // fp16 elements per 16-byte chunk
+constexpr int kRowStep = kThreads * kChunk;       // elements per pass over the CTA
+
+enum Mode { kPlain = 0, kMul = 1, kDiv = 2 };
+
+template <int MODE>
+__device__ __forceinline__ void smooth8(float (&v)[8], const float *__restrict__ smooth, int k) {
+    if (MODE == kPlain) return;
+    const float4 a = __ldg(reinterpret_cast<const float4 *>(smooth + k));
+    const float4 b = __ldg(reinterpret_cast<const float4 *>(smooth + k + 4));
+    const float s[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] = (MODE == kMul) ? __fmul_rn(v[e], s[e]) : __fdiv_rn(v[e], s[e]);
+}
+
+__device__ __forceinline__ void load8(const uint16_t *p, float (&v)[8]) {
+    const uint4 r = ld_stream_u4(p);
+    const float2 a = half2_bits_to_float2(r.x), b = half2_bits_to_float2(r.y);
+    const float2 c = half2_bits_to_float2(r.z), d = half2_bits_to_float2(r.w);
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+    v[4] = c.x; v[5] = c.y; v[6] = d.x; v[7] = d.y;
+}
+
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s) {
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int q0 = clampi(__float2int_rn(__fdiv_rn(v[e], s)), -128, 127);
+        const int q1 = clampi(__float2int_rn(__fdiv_rn(v[e + 4], s)), -128, 127);
+        lo |= (uint32_t)(q0 & 0xff) << (8 * e);
+        hi |= (uint32_t)(q1 & 0xff) << (8 * e);
+    }
+    return make_uint2(lo, hi);
+}
+
+__device__ __forceinline__ float block_max(float a, float *red) {
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
+    const int warp = threadIdx.x >> 5;
+    if ((threadIdx.x & 31) == 0) red[warp] = a;
+    __syncthreads();
+    float m = red[0];
+#pragma unroll
+    for (int i = 1; i < kThreads / 32; ++i) m = fmaxf(m, red[i]);
+    return m;
+}
+
+// NCH > 0: the row is kept in registers (K <= NCH * 2048).  NCH == 0: two passes.
+template <int NCH, int MODE>
+__global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_t *__restrict__ x, int K,
+                                                                   const float *__restrict__ smooth,
+                                                                   int8_t *__restrict__ q,
+                                                                   float *__restrict__ scales) {
+    __shared__ float red[kThreads / 32];
+    const size_t row = blockIdx.x;
+    const uint16_t *xr = x + row * K;
+    int8_t *qr = q + row * K;
+    const int t0 = threadIdx.x * kChunk;
+    float amax = 0.0f;
+    if (NCH > 0) {
+        float v[NCH > 0 ? NCH : 1][8];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int k = c * kRowStep + t0;
+            if (k < K) {
+                load8(xr + k, v[c]);
+                smooth8<MODE>(v[c], smooth, k);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[c][e]));
+            }
+        }
+        const float a = fmaxf(block_max(amax, red), 1e-8f);
+        const float s = __fdiv_rn(a, 127.0f);
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int k = c * kRowStep + t0;
+            if (k < K) *reinterpret_cast<uint2 *>(qr + k) = quant8(v[c], s);
+        }
+        if (threadIdx.x == 0) scales[row] = s;
+    } else {
+        for (int k = t0; k < K; k += kRowStep) {
+            float v[8];
+            load8(xr + k, v);
+            smooth8<MODE>(v, smooth, k);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+        }
+        const float a = fmaxf(block_max(amax, red), 1e-8f);
+        const float s = __fdiv_rn(a, 127.0f);
+        for (int k = t0; k < K; k += kRowStep) {
+            float v[8];
+            const uint4 r = *reinterpret_cast<const uint4 *>(xr + k);  // L2-resident re-read
+            const float2 a0 = half2_bits_to_float2(r.x), a1 = half2_bits_to_float2(r.y);
+            const float2 a2 = half2_bits_to_float2(r.z), a3 = half2_bits_to_float2(r.w);
+            v[0] = a0.x; v[1] = a0.y; v[2] = a1.x; v[3] = a1.y;
+            v[4] = a2.x; v[5] = a2.y; v[6] = a3.x; v[7] = a3.y;
+            smooth8<MODE>(v, smooth, k);
+            *reinterpret_cast<uint2 *>(qr + k) = quant8(v, s);
+        }
+        if (threadIdx.x == 0) scales[row] = s;
+    }
+}
+
+template <int MODE>
+cudaError_t launch_mode(const uint16_t *x, int R, int K, const float *smooth, int8_t *q, float *scales,
+                        cudaStream_t st) {
+    const int nch = (K + kRowStep - 1) / kRowStep;
+    dim3 grid(R), block(kThreads);
+    if (nch <= 1)
+        quant_int8_rows_kernel<1, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+    else if (nch <= 2)
+        quant_int8_rows_kernel<2, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+    else if (nch <= 4)
+        quant_int8_rows_kernel<4, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+    else if (nch <= 8)
+        quant_int8_rows_kernel<8, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+    else
+        quant_int8_rows_kernel<0, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+    return cudaGetLastError();
+}
+
+wq_status quantize_rows(const char *name, const uint16_t *x, int R, int K, const float *smooth, int mode,
+                        int8_t *q, float *scales, void *stream) {
+    WQ_REQUIRE_PTR(x, "input");
+    WQ_REQUIRE_PTR(q, "q");
+    WQ_REQUIRE_PTR(scales, "scales");
+    if (smooth) WQ_REQUIRE(aligned16(smooth), WQ_ERR_ALIGNMENT, "smooth is not 16-byte aligned");
+    WQ_REQUIRE(R > 0 && K > 0, WQ_ERR_INVALID_ARG, "%s: sizes must be positive (rows=%d K=%d)", name, R, K);
+    WQ_REQUIRE(K % 16 == 0, WQ_ERR_UNSUPPORTED, "%s: K (%d) must be a multiple of 16", name, K);
+    WQ_REQUIRE(R < (1 << 30), WQ_ERR_UNSUPPORTED, "%s: too many rows", name);
+    cudaStream_t st = as_stream(stream);
+    cudaError_t e;
+    if (!smooth)
+        e = launch_mode<kPlain>(x, R, K, nullptr, q, scales, st);
+    else if (mode == kMul)
+        e = launch_mode<kMul>(x, R, K, smooth, q, scales, st);
+    else
+        e = launch_mode<kDiv>(x, R, K, smooth, q, scales, st);
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "%s: launch failed: %s", name, cudaGetErrorString(e));
+    return WQ_OK;
+}
+
+}  // namespace
+}  // namespace wq
+
+extern "C" wq_status wq_quantize_int8_per_channel(const uint16_t *w, int N, int K, const float *smooth,
+                                                  int8_t *q, float *scales, void *stream) {
+    return wq::quantize_rows("wq_quantize_int8_per_channel", w, N, K, smooth, wq::kMul, q, scales, stream);
+}
+
+extern "C" wq_status wq_quantize_int8_per_token(const uint16_t *x, int M, int K, const float *smooth,
+                                                int8_t *q, float *scales, void *stream) {
+    return wq::quantize_rows("wq_quantize_int8_per_token", x, M, K, smooth, wq::kDiv, q, scales, stream);
+}

@@ -1,0 +1,207 @@
+/*
+ * wq.h -- C ABI of the B200 (sm_100a) weight/activation quantization library.
+ *
+ * The library implements the data-parallel hot path of LLM post-training
+ * quantization as described in five web pages on the subject:
+ *
+ *   [P1] "How quantization works" (AI-infra handbook)
+ *   [P2] "Quantization" (engine-room, chapter 15)
+ *   [P3] "Quantization from Scratch: Scale, Zero-Point, GPTQ and AWQ"
+ *   [P4] "Quantization: Smaller Weights, Same Answers (Mostly)"
+ *   [P5] "Quantization Explained: INT8, INT4, GPTQ and AWQ for LLMs"
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument is a DEVICE pointer to memory owned by the caller
+ *    (allocate it however you like; the library never allocates, frees or
+ *    keeps a pointer after the call returns).  Every base address must be
+ *    16-byte aligned (WQ_ERR_ALIGNMENT otherwise).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Each call only validates its arguments on the host and
+ *    enqueues kernels on `stream`; it never synchronizes the device.
+ *  - Matrices are row-major.  Weights are [N out][K in] (nn.Linear layout),
+ *    activations are [B or M][K], outputs are [B or M][N].
+ *  - fp16 data is passed as uint16_t bit patterns (IEEE 754 binary16).
+ *  - Rounding is round-half-to-even everywhere; every division is an IEEE
+ *    fp32 division; the library is built without fast-math.
+ *  - On a precondition violation the call returns an error status, launches
+ *    nothing and records a message readable with wq_last_error() (per host
+ *    thread).  Launch failures return WQ_ERR_CUDA.
+ *  - Kernels that wait on asynchronous copies or tensor-core operations bound
+ *    every wait; a wait that runs out records WQ_ERR_TIMEOUT in a device
+ *    status word that wq_device_status() reads.
+ *
+ * Packed INT4 layout (written by wq_quantize_group_int4, read by the W4A16
+ * matmuls):
+ *  - qweight uint32 [N][K/8]: element k of row n is nibble (k mod 8), i.e.
+ *    bits [4(k mod 8), 4(k mod 8)+4), of word k/8.
+ *  - scales  fp16   [N][K/g]: the step of group j = k / g.
+ *  - qzeros  uint32 [N][ceil((K/g)/8)]: the zero point of group j is nibble
+ *    (j mod 8) of word j/8; unused nibbles of the last word are 0.
+ *  Storage is 0.5 + 2.5/g bytes per weight: 0.15625 bit/weight of overhead
+ *  at g = 128 ([P3] "Where to put the scales", [P1] exercise 2).
+ */
+#ifndef WQ_H
+#define WQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WQ_OK = 0,
+    WQ_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, inconsistent sizes */
+    WQ_ERR_ALIGNMENT = 2,   /* a base address is not 16-byte aligned */
+    WQ_ERR_UNSUPPORTED = 3, /* a size outside what the kernels implement */
+    WQ_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed */
+    WQ_ERR_TIMEOUT = 5      /* a bounded wait inside a kernel ran out */
+} wq_status;
+
+typedef enum { WQ_F32 = 0, WQ_F16 = 1 } wq_dtype;
+
+/*
+ * Asymmetric INT4 per-group quantization.
+ * Source: [P5] "Uniform Affine Quantization" and "Scale and Zero-Point"
+ * (s = (max - min) / (2^b - 1), z = round(-min / s), x_q = round(x/s) + z,
+ * clamp to [0, 15]); [P3] "Scale and zero-point" and its round-to-nearest
+ * quantize() (a zero scale becomes 1); [P1] "Granularity" (one scale per g
+ * consecutive weights of a row) and exercise 2 (fp16 scale, 4-bit zero).
+ * Per (row n, group j), in fp32:
+ *   lo = min(0, min w), hi = max(0, max w)      (range widened to contain 0)
+ *   s  = fp16_rn((hi - lo) / 15); if s == 0 then s = 1
+ *   z  = clamp(rne(-lo / s), 0, 15)
+ *   q  = clamp(rne(w / s) + z, 0, 15)          (s is the stored fp16 value)
+ * w:        [N][K], fp32 (w_dtype WQ_F32) or fp16 bits (WQ_F16).
+ * qweight:  out, uint32 [N][K/8];  scales: out, fp16 [N][K/g];
+ * qzeros:   out, uint32 [N][ceil(K/g/8)]  (layout above).
+ * group_size in {32, 64, 128, 256}, K % group_size == 0.  Inputs must be
+ * finite and (hi - lo)/15 must fit fp16 (|w| below ~4.9e5).
+ */
+wq_status wq_quantize_group_int4(const void *w, wq_dtype w_dtype, int N, int K, int group_size,
+                                 uint32_t *qweight, uint16_t *scales, uint32_t *qzeros,
+                                 void *stream);
+
+/*
+ * Symmetric INT8 per output channel (one fp32 scale per weight row).
+ * Source: [P1] "The math of quantization" (s = max|x| / (2^(b-1) - 1),
+ * q = clamp(round(x/s), -2^(b-1), 2^(b-1) - 1)), the quant.py listing
+ * (absmax clamped at 1e-8), q8_per_row, and SmoothQuant's Ws = W * s in
+ * "Activation quantization and outliers".  Per row n, in fp32:
+ *   w'_k = smooth ? w_k * smooth[k] : w_k
+ *   a = max(max_k |w'_k|, 1e-8);  scales[n] = a / 127
+ *   q[n][k] = clamp(rne(w'_k / scales[n]), -128, 127)
+ * w: fp16 [N][K];  smooth: nullable fp32 [K];  q: out int8 [N][K];
+ * scales: out fp32 [N].  K % 16 == 0.
+ */
+wq_status wq_quantize_int8_per_channel(const uint16_t *w, int N, int K, const float *smooth,
+                                       int8_t *q, float *scales, void *stream);
+
+/*
+ * Symmetric INT8 per token (one fp32 scale per activation row, computed at
+ * run time).  Source: as above, with SmoothQuant's Xs = X / s ([P1]) and
+ * per-token dynamic activation scales ([P4] "Quick Reference").  Per row m:
+ *   x'_k = smooth ? x_k / smooth[k] : x_k       (IEEE fp32 division)
+ *   a = max(max_k |x'_k|, 1e-8);  scales[m] = a / 127
+ *   q[m][k] = clamp(rne(x'_k / scales[m]), -128, 127)
+ * x: fp16 [M][K];  smooth: nullable fp32 [K];  q: out int8 [M][K];
+ * scales: out fp32 [M].  K % 16 == 0.
+ */
+wq_status wq_quantize_int8_per_token(const uint16_t *x, int M, int K, const float *smooth,
+                                     int8_t *q, float *scales, void *stream);
+
+/*
+ * SmoothQuant smoothing factors.  Source: [P1] "Activation quantization and
+ * outliers" (s = X.abs().amax(0).clamp(1e-5)^a / W.abs().amax(0).clamp(1e-5)^(1-a))
+ * and [P2] "The Mathematics" (s_j = max|X_j|^a / max|W_j|^(1-a)).
+ *   ax_j = max(max_m |x[m][j]|, 1e-5),  aw_j = max(max_n |w[n][j]|, 1e-5)
+ *   s[j] = alpha == 0.5 ? sqrt(ax_j) / sqrt(aw_j)          (correctly rounded)
+ *                       : (float)pow(ax_j, alpha) / (float)pow(aw_j, 1 - alpha)
+ *                         (pow in fp64)
+ * x: fp16 [M][K] (calibration activations), w: fp16 [N][K];  s: out fp32 [K].
+ * workspace: caller-owned scratch of wq_smooth_workspace_bytes(K) bytes,
+ * 16-byte aligned; its contents on entry do not matter (the call clears
+ * it) and calls that share one workspace must not overlap on the GPU.
+ * K % 8 == 0.  0 <= alpha <= 1.
+ */
+size_t wq_smooth_workspace_bytes(int K);
+wq_status wq_smooth(const uint16_t *x, int M, const uint16_t *w, int N, int K, float alpha,
+                    float *s, void *workspace, void *stream);
+
+/*
+ * Fused dequantize + GEMV, W4A16, for decode batches B = 1..8.  Source: [P1]
+ * "Inference view" (weights unpacked in registers, multiplied by their
+ * scales), [P3] "Scale and zero-point" (w^ = (q - z) s), [P5] "Why It Is
+ * Faster" (decode streams the weights).
+ *   y[b][n] = fp16_rn( sum_k s[n][k/g] * (q[n][k] - z[n][k/g]) * x[b][k] )
+ * accumulated in fp32 (order unspecified).
+ * x: fp16 [B][K];  qweight/scales/qzeros: the packed layout above;
+ * y: out fp16 [B][N].  group_size in {32, 64, 128, 256}; K % group_size == 0;
+ * K % 32 == 0.
+ */
+wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qweight, const uint16_t *scales,
+                        const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y,
+                        void *stream);
+
+/*
+ * W4A16 GEMM on the tensor cores for M >= 16 rows of activations: tiles of
+ * packed weights are dequantized into shared memory and fed to tcgen05 MMAs
+ * with fp32 accumulation in tensor memory ([P1] "Inference view").  Same
+ * arithmetic and layouts as wq_gemv_w4a16 (each dequantized weight is
+ * rounded to fp16 before the MMA); M in [16, 256]; group_size == 128;
+ * K % 128 == 0.
+ */
+wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
+                        const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y,
+                        void *stream);
+
+/*
+ * W8A8 INT8 GEMM on the tensor cores with a fused dequantization epilogue.
+ * Source: [P4] "How does quantized matrix multiplication actually run on the
+ * GPU?" (int8 operands, exact 32-bit accumulation; symmetric scales make the
+ * zero-point terms vanish) and [P1] "Mainstream schemes" (W8A8 INT8).
+ *   acc[m][n] = sum_k xq[m][k] * wq[n][k]      (int32, exact)
+ *   y[m][n]   = fp16_rn( (float)acc * sx[m] * sw[n] )     (fp32 products)
+ * xq: int8 [M][K], sx: fp32 [M], wq: int8 [N][K], sw: fp32 [N];
+ * y: out fp16 [M][N];  acc_out: nullable, out int32 [M][N] (raw accumulators).
+ * K % 16 == 0, K <= 131072 (so |acc| < 2^31).
+ */
+wq_status wq_gemm_w8a8(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                       int M, int N, int K, uint16_t *y, int32_t *acc_out, void *stream);
+
+/*
+ * W8A16 GEMV (INT8 per-channel weights, fp16 activations), B = 1..8.
+ * Source: [P1] "Mainstream schemes" (W8A16) and the per-channel INT8 above.
+ *   y[b][n] = fp16_rn( sw[n] * sum_k q[n][k] * x[b][k] )   (fp32 accumulation)
+ * x: fp16 [B][K];  wq: int8 [N][K];  sw: fp32 [N];  y: out fp16 [B][N].
+ * K % 16 == 0.
+ */
+wq_status wq_gemv_w8a16(const uint16_t *x, int B, const int8_t *wq, const float *sw, int N, int K,
+                        uint16_t *y, void *stream);
+
+/* Message describing the last error status returned on this host thread. */
+const char *wq_last_error(void);
+
+/*
+ * Synchronizes `stream`, then reads and clears the library's device status
+ * word: WQ_OK, or WQ_ERR_TIMEOUT if a bounded wait ran out in a kernel since
+ * the last call (or WQ_ERR_CUDA if synchronization failed).
+ */
+wq_status wq_device_status(void *stream);
+
+/*
+ * Wall-clock limit, in nanoseconds, of each bounded wait inside the
+ * tensor-core kernels (default 2e9, two seconds; 0 restores the default).
+ * Applies to launches made after the call.  Small values exist so that tests
+ * can make a wait run out on purpose; the kernel then stops, drains its own
+ * in-flight copies and tensor-core operations, releases its tensor memory and
+ * records WQ_ERR_TIMEOUT for wq_device_status().
+ */
+void wq_set_wait_limit(uint64_t nanoseconds);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WQ_H */

@@ -1,0 +1,297 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on seeded inputs.
+
+Codes, scales, zero points, INT8 codes/scales and smoothing factors must be
+bit-exact; matmul outputs must satisfy |y - y_ref| <= 2e-3 * sum_k |w^ x| + 1e-5
+per element (y_ref and the bound in fp64 from the oracle).  Small cases span
+several tiles and ragged tails; the full-size workloads are checked on sampled
+rows the oracle computes one by one.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+RTOL_BOUND, ATOL = 2e-3, 1e-5
+
+
+@pytest.fixture(scope="module")
+def wq():
+    import bit_gemv_gemm_group_b200 as m
+    return m
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host(t, dtype=None):
+    a = t.cpu().numpy()
+    return a.view(dtype) if dtype is not None else a
+
+
+def assert_within_bound(y, y_ref, bound, what=""):
+    y = np.asarray(y, np.float64)
+    err = np.abs(y - y_ref)
+    lim = RTOL_BOUND * bound + ATOL
+    bad = err > lim
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} outside tolerance; worst excess "
+                           f"{(err - lim).max():.3e} at {np.unravel_index(np.argmax(err - lim), err.shape)}")
+
+
+def sample_rows(N, k=256, seed=0):
+    if N <= k:
+        return np.arange(N)
+    r = np.random.default_rng(seed).choice(N, size=k - 2, replace=False)
+    return np.unique(np.concatenate([r, [0, N - 1]])).astype(np.int32)
+
+
+# --------------------------------------------------------------------------
+# INT4 group quantizer
+# --------------------------------------------------------------------------
+def _special_weights(N, K, seed, dtype=np.float16):
+    g = np.random.default_rng(seed)
+    w = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    w.reshape(-1)[96::97] *= 20
+    if N > 8 and K >= 512:
+        w[1, :128] = 0.0
+        w[2, 128:256] = 0.25
+        w[3, 256:384] = np.abs(w[3, 256:384]) + 0.01
+        w[4, 384:512] = -np.abs(w[4, 384:512]) - 0.01
+        w[5, ::7] = 0.0
+    return w.astype(dtype)
+
+
+SMALL_INT4 = [  # (N, K, g, dtype)
+    (1, 128, 128, np.float16), (17, 384, 128, np.float16), (33, 1024, 128, np.float16),
+    (64, 1536, 128, np.float16), (9, 96, 32, np.float16), (40, 640, 64, np.float16),
+    (13, 2048, 256, np.float16), (24, 512, 128, np.float32), (300, 4096, 128, np.float16),
+]
+
+
+@pytest.mark.parametrize("N,K,g,dtype", SMALL_INT4)
+def test_int4_quantizer_bit_exact_small(wq, N, K, g, dtype):
+    w = _special_weights(N, K, seed=N * 7 + K, dtype=dtype)
+    qw, sc, qz = wq.quantize_group_int4(dev(w), g)
+    torch.cuda.synchronize()
+    rqw, rsc, rqz = oracle.quantize_group_int4(w, g)
+    assert np.array_equal(host(qw, np.uint32), rqw)
+    assert np.array_equal(host(sc).view(np.uint16), rsc.view(np.uint16))
+    assert np.array_equal(host(qz, np.uint32), rqz)
+
+
+@pytest.mark.parametrize("cfg,shape_index", [(1, 0), (2, 0), (3, 0), (3, 1)])
+def test_int4_quantizer_bit_exact_configs(wq, cfg, shape_index):
+    w = workloads.config_weight(cfg, shape_index)
+    qw, sc, qz = wq.quantize_group_int4(dev(w), 128)
+    torch.cuda.synchronize()
+    rows = sample_rows(w.shape[0], 512, seed=cfg)
+    rqw, rsc, rqz = oracle.quantize_group_int4(w[rows], 128)
+    assert np.array_equal(host(qw, np.uint32)[rows], rqw)
+    assert np.array_equal(host(sc).view(np.uint16)[rows], rsc.view(np.uint16))
+    assert np.array_equal(host(qz, np.uint32)[rows], rqz)
+
+
+# --------------------------------------------------------------------------
+# W4A16 GEMV
+# --------------------------------------------------------------------------
+GEMV_SMALL = [  # (N, K, g, B)
+    (1, 128, 128, 1), (17, 384, 128, 1), (33, 1024, 128, 3), (64, 1536, 128, 8),
+    (9, 96, 32, 2), (40, 640, 64, 4), (13, 2048, 256, 5), (300, 4096, 128, 1),
+    (3000, 2048, 128, 1), (3000, 2048, 128, 8), (2500, 512, 128, 6), (129, 7168, 128, 7),
+]
+
+
+@pytest.mark.parametrize("N,K,g,B", GEMV_SMALL)
+def test_gemv_w4a16_small(wq, N, K, g, B):
+    w = _special_weights(N, K, seed=N + 3 * K)
+    rqw, rsc, rqz = oracle.quantize_group_int4(w, g)
+    x = workloads.activations(B, K, 0.01, 50.0, seed=N, tensor_id=K)
+    x[0, :3] = 0.0
+    y = wq.gemv_w4a16(dev(x), dev(rqw.view(np.int32)), dev(rsc), dev(rqz.view(np.int32)), g)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.matmul_w4a16_ref(x, rqw, rsc, rqz, K, g)
+    assert_within_bound(host(y).astype(np.float64), y_ref, bound, f"gemv N={N} K={K} B={B}")
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_gemv_w4a16_configs(wq, cfg):
+    c = workloads.CONFIGS[cfg]
+    for si, (N, K) in enumerate(c.shapes):
+        w = workloads.config_weight(cfg, si)
+        qw, sc, qz = wq.quantize_group_int4(dev(w), 128)
+        rows = sample_rows(N, 384, seed=si)
+        hqw, hsc, hqz = host(qw, np.uint32), host(sc), host(qz, np.uint32)
+        for B in [b for b in c.batches if b <= 8]:
+            x = workloads.config_activations(cfg, B, K)
+            y = wq.gemv_w4a16(dev(x), qw, sc, qz, 128)
+            torch.cuda.synchronize()
+            y_ref, bound = oracle.matmul_w4a16_ref(x, hqw, hsc, hqz, K, 128, rows=rows)
+            assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"cfg{cfg} {N}x{K} B={B}")
+
+
+# --------------------------------------------------------------------------
+# INT8 quantizers and smoothing
+# --------------------------------------------------------------------------
+INT8_SMALL = [(1, 16), (7, 48), (33, 2048), (5, 2064), (64, 4096), (3, 16384), (2, 16400), (4, 40960)]
+
+
+@pytest.mark.parametrize("R,K", INT8_SMALL)
+@pytest.mark.parametrize("smoothing", [False, True])
+def test_int8_quantizers_bit_exact_small(wq, R, K, smoothing):
+    g = np.random.default_rng(R * K)
+    a = (g.standard_normal((R, K)) * 2).astype(np.float32)
+    a[:, g.choice(K, size=max(1, K // 100), replace=False)] *= 40
+    if R > 2:
+        a[1] = 0.0
+    a = a.astype(np.float16)
+    s = (np.exp(g.normal(0, 1, K)) + 0.05).astype(np.float32) if smoothing else None
+    sd = dev(s) if smoothing else None
+    qc, sc = wq.quantize_int8_per_channel(dev(a), sd)
+    qt, st = wq.quantize_int8_per_token(dev(a), sd)
+    torch.cuda.synchronize()
+    rqc, rsc = oracle.quantize_int8_per_channel(a, s)
+    rqt, rst = oracle.quantize_int8_per_token(a, s)
+    assert np.array_equal(host(qc), rqc) and np.array_equal(host(sc).view(np.uint32), rsc.view(np.uint32))
+    assert np.array_equal(host(qt), rqt) and np.array_equal(host(st).view(np.uint32), rst.view(np.uint32))
+
+
+SMOOTH_SMALL = [(1, 1, 8), (3, 5, 24), (37, 300, 520), (256, 257, 256), (600, 90, 1032)]
+
+
+@pytest.mark.parametrize("M,N,K", SMOOTH_SMALL)
+@pytest.mark.parametrize("alpha", [0.5, 0.75, 0.0, 1.0])
+def test_smooth_small(wq, M, N, K, alpha):
+    g = np.random.default_rng(M + N + K)
+    X = g.standard_normal((M, K)).astype(np.float32)
+    X[:, g.choice(K, size=max(1, K // 50), replace=False)] *= 60
+    X[:, 0] = 0.0                                   # an all-zero column hits the 1e-5 clamp
+    X = X.astype(np.float16)
+    W = (g.standard_normal((N, K)) * 0.02).astype(np.float16)
+    s = host(wq.smooth(dev(X), dev(W), alpha))
+    ref = oracle.smooth_factors(X, W, alpha)
+    if alpha in (0.5, 1.0, 0.0):
+        # 0.5: correctly rounded square roots; 1.0 / 0.0: pow(x, 1) and pow(x, 0) are exact
+        assert np.array_equal(s.view(np.uint32), ref.view(np.uint32))
+    else:
+        # fp64 pow rounded to fp32 on both sides: at most 1 ulp apart
+        ulps = np.abs(s.view(np.int32).astype(np.int64) - ref.view(np.int32).astype(np.int64))
+        assert ulps.max() <= 1
+
+
+def test_smooth_reuses_dirty_workspace(wq):
+    g = np.random.default_rng(5)
+    X = g.standard_normal((64, 512)).astype(np.float16)
+    W = (g.standard_normal((96, 512)) * 0.02).astype(np.float16)
+    ws = torch.full((wq.smooth_workspace_bytes(512),), 0x7f, dtype=torch.uint8, device="cuda")
+    s1 = host(wq.smooth(dev(X), dev(W), 0.5, workspace=ws))
+    s2 = host(wq.smooth(dev(X), dev(W), 0.5, workspace=ws))
+    ref = oracle.smooth_factors(X, W, 0.5)
+    assert np.array_equal(s1, ref) and np.array_equal(s2, ref)
+
+
+# --------------------------------------------------------------------------
+# W8A16 GEMV
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("N,K,B", [(1, 16, 1), (17, 48, 2), (300, 4096, 1), (3000, 2048, 8), (129, 7168, 5)])
+def test_gemv_w8a16_small(wq, N, K, B):
+    g = np.random.default_rng(N + K + B)
+    w = (g.standard_normal((N, K)) * 0.02).astype(np.float16)
+    q, s = oracle.quantize_int8_per_channel(w)
+    x = workloads.activations(B, K, 0.01, 50.0, seed=N, tensor_id=B)
+    y = host(wq.gemv_w8a16(dev(x), dev(q), dev(s)))
+    y_ref, bound = oracle.matmul_w8a16_ref(x, q, s)
+    assert_within_bound(y.astype(np.float64), y_ref, bound, f"w8a16 N={N} K={K} B={B}")
+
+
+def test_w8a16_config3(wq):
+    c = workloads.CONFIGS[3]
+    for si, (N, K) in enumerate(c.shapes):
+        w = workloads.config_weight(3, si)
+        q, s = wq.quantize_int8_per_channel(dev(w))
+        rows = sample_rows(N, 256, seed=si)
+        rq, rs = oracle.quantize_int8_per_channel(w[rows])
+        hq, hs = host(q), host(s)
+        assert np.array_equal(hq[rows], rq) and np.array_equal(hs[rows].view(np.uint32), rs.view(np.uint32))
+        for B in (1, 8):
+            x = workloads.config_activations(3, B, K)
+            y = host(wq.gemv_w8a16(dev(x), q, s))
+            y_ref, bound = oracle.matmul_w8a16_ref(x, hq, hs, rows=rows)
+            assert_within_bound(y.astype(np.float64)[:, rows], y_ref, bound, f"w8a16 cfg3 {N}x{K} B={B}")
+
+
+# --------------------------------------------------------------------------
+# W8A8 INT8 tensor-core GEMM
+# --------------------------------------------------------------------------
+def _gemm_check(wq, xq, sx, wq8, sw, ms=None, ns=None):
+    y, acc = wq.gemm_w8a8(dev(xq), dev(sx), dev(wq8), dev(sw), return_acc=True)
+    torch.cuda.synchronize()
+    racc, ry, rb = oracle.gemm_w8a8_ref(xq, sx, wq8, sw, ms, ns)
+    hy, hacc = host(y).astype(np.float64), host(acc).astype(np.int64)
+    if ms is not None:
+        hy, hacc = hy[np.ix_(ms, ns)], hacc[np.ix_(ms, ns)]
+    assert np.array_equal(hacc, racc)
+    assert_within_bound(hy, ry, rb, "w8a8")
+
+
+W8A8_SMALL = [(1, 1, 16), (128, 256, 128), (130, 300, 144), (64, 40, 1040), (257, 513, 256), (300, 1000, 2000),
+              (512, 1024, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", W8A8_SMALL)
+def test_gemm_w8a8_small(wq, M, N, K):
+    g = np.random.default_rng(M * N + K)
+    xq = g.integers(-128, 128, (M, K), dtype=np.int8)
+    wq8 = g.integers(-128, 128, (N, K), dtype=np.int8)
+    sx = (g.random(M, dtype=np.float32) + 0.01) * 0.05
+    sw = (g.random(N, dtype=np.float32) + 0.01) * 0.01
+    _gemm_check(wq, xq, sx, wq8, sw)
+
+
+def test_gemm_w8a8_every_code_pair(wq):
+    # acc[m][n] = (m - 128) * (n - 128): all 256 x 256 int8 products through the tensor cores
+    codes = np.arange(-128, 128, dtype=np.int8)
+    xq = np.zeros((256, 16), np.int8)
+    xq[:, 0] = codes
+    wq8 = np.zeros((256, 16), np.int8)
+    wq8[:, 5] = codes
+    wq8[:, 0] = codes
+    _gemm_check(wq, xq, np.ones(256, np.float32), wq8, np.ones(256, np.float32) * np.float32(2 ** -16))
+
+
+def test_gemm_w8a8_extreme_accumulators(wq):
+    K = 8192
+    xq = np.full((130, K), -128, np.int8)
+    xq[1] = 127
+    wq8 = np.full((260, K), -128, np.int8)
+    wq8[3, ::2] = 127
+    _gemm_check(wq, xq, np.full(130, 1e-6, np.float32), wq8, np.full(260, 1e-4, np.float32))
+
+
+def test_w8a8_smoothquant_pipeline_full_size(wq):
+    # Config 5: smoothing -> per-channel(W * s) -> per-token(X / s) -> INT8 GEMM, in the
+    # launch configuration the benchmark times; sampled rows checked one by one.
+    M, N, K = 2048, 8192, 8192
+    X = workloads.config_activations(5, M, K)
+    W = workloads.config_weight(5)
+    Xd, Wd = dev(X), dev(W)
+    s = wq.smooth(Xd, Wd, 0.5)
+    wq8, sw = wq.quantize_int8_per_channel(Wd, s)
+    xq8, sx = wq.quantize_int8_per_token(Xd, s)
+    y, acc = wq.gemm_w8a8(xq8, sx, wq8, sw, return_acc=True)
+    torch.cuda.synchronize()
+    rs = oracle.smooth_factors(X, W, 0.5)
+    assert np.array_equal(host(s).view(np.uint32), rs.view(np.uint32))
+    ms = sample_rows(M, 96, seed=1)
+    ns = sample_rows(N, 160, seed=2)
+    rxq, rsx = oracle.quantize_int8_per_token(X[ms], rs)
+    rwq, rsw = oracle.quantize_int8_per_channel(W[ns], rs)
+    assert np.array_equal(host(xq8)[ms], rxq) and np.array_equal(host(sx)[ms], rsx)
+    assert np.array_equal(host(wq8)[ns], rwq) and np.array_equal(host(sw)[ns], rsw)
+    racc, ry, rb = oracle.gemm_w8a8_ref(rxq, rsx, rwq, rsw)
+    assert np.array_equal(host(acc)[np.ix_(ms, ns)].astype(np.int64), racc)
+    assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, "w8a8 config 5")
+    assert wq.device_status() == 0
