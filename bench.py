@@ -1,0 +1,464 @@
+#!/usr/bin/env python
+"""Benchmark of the quantization hot path on B200: one JSON line on stdout.
+
+A *step* is one pass of every hot-path kernel over the 70B-class W4A16 layer
+(28672x8192 up and 8192x28672 down fp16 weights, N(0, 0.015), activations with
+0.5% outlier channels x100) and the W8A8 SmoothQuant layer (X [2048, 8192] with
+64 outlier channels x60, W [8192, 8192]):
+
+  INT4 group quantizer on both weights          (fresh outputs)
+  W4A16 GEMV, batch 1, on both weights          (the headline: HBM GB/s)
+  W4A16 tensor-core GEMM, batch 16 and 64, on both weights
+  INT8 per-channel quantizer on both weights + W8A16 GEMV, batch 1
+  SmoothQuant factors, INT8 per-channel (W*s) and per-token (X/s) quantizers
+  W8A8 INT8 tensor-core GEMM                    (the second headline: TOPS)
+
+Every input lives in HBM before the timed region; the matmuls read packed
+weights that no kernel of the step has touched since the previous step, and
+the step streams several GB, so no kernel reads its operands from L2.  Kernel
+times come from CUDA events on the launching stream.  `value` is the batch-1
+W4A16 GEMV's algorithmic bytes / its device time over all ranks; the W8A8
+GEMM's INT8 TOPS ride along in `w8a8`.
+
+--impl reference times the CPU oracle (single-threaded C) on a bounded sample
+of the same workload instead.  With torchrun (N > 1) every rank runs an
+independent replica (the path has no exchange step); rank 0 prints.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "W4A16 GEMV achieved HBM GB/s (% of peak) + W8A8 GEMM INT8 TOPS (% of peak)"
+WORKLOAD = "llama70b_class_w4a16_layer+w8a8_smoothquant_2048x8192x8192"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+UP, DOWN = (28672, 8192), (8192, 28672)
+W8A8_SHAPE = (2048, 8192, 8192)
+
+
+# ----------------------------------------------------------------------------- peaks
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+def packed_bytes(N, K, g=128):
+    return N * K // 2 + 2 * N * (K // g) + 4 * N * ((K // g + 7) // 8)
+
+
+def work_table():
+    """Algorithmic bytes (HBM) and ops per launch of each kernel in a step."""
+    t = {}
+    for tag, (N, K) in (("up", UP), ("down", DOWN)):
+        t[f"quant_int4_{tag}"] = {"bytes": 2 * N * K + packed_bytes(N, K), "ops": 0}
+        t[f"gemv_w4a16_b1_{tag}"] = {"bytes": packed_bytes(N, K) + 2 * K + 2 * N, "ops": 2 * N * K}
+        for M in (16, 64):
+            t[f"gemm_w4a16_m{M}_{tag}"] = {"bytes": packed_bytes(N, K) + 2 * M * K + 2 * M * N, "ops": 2 * M * N * K}
+        t[f"quant_int8_pc_{tag}"] = {"bytes": 3 * N * K + 4 * N, "ops": 0}
+        t[f"gemv_w8a16_b1_{tag}"] = {"bytes": N * K + 4 * N + 2 * K + 2 * N, "ops": 2 * N * K}
+    M, N, K = W8A8_SHAPE
+    t["smooth"] = {"bytes": 2 * (M + N) * K + 4 * K, "ops": 0}
+    t["quant_int8_pc_smooth"] = {"bytes": 3 * N * K + 4 * N + 4 * K, "ops": 0}
+    t["quant_int8_pt_smooth"] = {"bytes": 3 * M * K + 4 * M + 4 * K, "ops": 0}
+    t["gemm_w8a8"] = {"bytes": M * K + N * K + 4 * (M + N) + 2 * M * N, "ops": 2 * M * N * K}
+    return t
+
+
+def roofline_for(name, us, work, peaks):
+    """Achieved rate against the kernel's binding roofline (measured peaks)."""
+    hbm = peaks["hbm_gbs"]
+    int8 = 2.0 * peaks["bf16_tflops"]          # INT8 dense = 2 x bf16 (nominal ratio)
+    f16 = peaks["bf16_tflops"]                 # fp16 dense = bf16
+    b, ops = work["bytes"], work["ops"]
+    if name == "gemm_w8a8":
+        ach = ops / (us * 1e-6) / 1e12
+        return {"bound": "tensor", "achieved": ach, "peak": int8, "unit": "TOPS", "frac": ach / int8}
+    if name.startswith("gemm_w4a16"):
+        t_mem, t_tc = b / (hbm * 1e9), ops / (f16 * 1e12)
+        if t_tc > t_mem:
+            ach = ops / (us * 1e-6) / 1e12
+            return {"bound": "tensor", "achieved": ach, "peak": f16, "unit": "TFLOP/s", "frac": ach / f16}
+    ach = b / (us * 1e-6) / 1e9
+    return {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm}
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index, period_ms=20):
+        self.index, self.period_ms, self.rows, self.proc = index, period_ms, [], None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", str(self.period_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [c.strip() for c in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        rows = [r for (t, r) in self.rows if t0 - 0.05 <= t <= t1 + 0.05 and len(r) >= 9]
+        if not rows:
+            rows = [r for (_, r) in self.rows if len(r) >= 9]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def reduce_max(values, world, device=None):
+    """Element-wise max over ranks (identity for world == 1)."""
+    if world == 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def aggregate_value(bytes_per_rank_step, steps, world, max_time_s):
+    """Whole-job GB/s: units all ranks processed / max-over-ranks time."""
+    return bytes_per_rank_step * steps * world / max_time_s / 1e9
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def make_inputs(torch, dev):
+    import workloads
+    ins = {}
+    for tag, (N, K), si in (("up", UP, 0), ("down", DOWN, 1)):
+        w = workloads.config_weight(4, si)
+        ins[f"w_{tag}"] = torch.from_numpy(w).to(dev)
+        del w
+        for B in (1, 16, 64):
+            ins[f"x{B}_{tag}"] = torch.from_numpy(workloads.config_activations(4, B, K)).to(dev)
+    M, N, K = W8A8_SHAPE
+    ins["X5"] = torch.from_numpy(workloads.config_activations(5, M, K)).to(dev)
+    ins["W5"] = torch.from_numpy(workloads.config_weight(5)).to(dev)
+    return ins
+
+
+class Step:
+    """Buffers and launches of one hot-path step, with per-kernel CUDA events."""
+
+    def __init__(self, torch, wq, ins):
+        self.torch, self.wq, self.ins = torch, wq, ins
+        self.names = []
+        # read-side packed weights (previous "model state"), never written inside a step
+        self.qB = {t: wq.quantize_group_int4(ins[f"w_{t}"], 128) for t in ("up", "down")}
+        self.q8B = {t: wq.quantize_int8_per_channel(ins[f"w_{t}"]) for t in ("up", "down")}
+        torch.cuda.synchronize()
+        self.ws = torch.empty(wq.smooth_workspace_bytes(W8A8_SHAPE[2]), dtype=torch.uint8, device=ins["X5"].device)
+        self.out = {}
+
+    def launches(self):
+        wq, ins, qB, q8B = self.wq, self.ins, self.qB, self.q8B
+        L = []
+        for t in ("up", "down"):
+            L.append((f"quant_int4_{t}", lambda t=t: wq.quantize_group_int4(ins[f"w_{t}"], 128)))
+        for t in ("up", "down"):
+            L.append((f"gemv_w4a16_b1_{t}", lambda t=t: wq.gemv_w4a16(ins[f"x1_{t}"], *qB[t], 128)))
+        for M in (16, 64):
+            for t in ("up", "down"):
+                L.append((f"gemm_w4a16_m{M}_{t}", lambda t=t, M=M: wq.gemm_w4a16(ins[f"x{M}_{t}"], *qB[t], 128)))
+        for t in ("up", "down"):
+            L.append((f"quant_int8_pc_{t}", lambda t=t: wq.quantize_int8_per_channel(ins[f"w_{t}"])))
+        for t in ("up", "down"):
+            L.append((f"gemv_w8a16_b1_{t}", lambda t=t: wq.gemv_w8a16(ins[f"x1_{t}"], *q8B[t])))
+
+        def smooth():
+            self.out["s"] = wq.smooth(ins["X5"], ins["W5"], 0.5, workspace=self.ws)
+
+        def q_w():
+            self.out["wq5"] = wq.quantize_int8_per_channel(ins["W5"], self.out["s"])
+
+        def q_x():
+            self.out["xq5"] = wq.quantize_int8_per_token(ins["X5"], self.out["s"])
+
+        def w8a8():
+            xq, sx = self.out["xq5"]
+            w8, sw = self.out["wq5"]
+            self.out["y5"] = wq.gemm_w8a8(xq, sx, w8, sw)
+
+        L += [("smooth", smooth), ("quant_int8_pc_smooth", q_w), ("quant_int8_pt_smooth", q_x), ("gemm_w8a8", w8a8)]
+        return L
+
+
+def run_gpu(args):
+    import torch
+    import bit_gemv_gemm_group_b200 as wq
+
+    rank, world, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    ins = make_inputs(torch, dev)
+    step = Step(torch, wq, ins)
+    launches = step.launches()
+    names = [n for n, _ in launches]
+    work = work_table()
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier(device_ids=[dev.index])
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        for _, fn in launches:
+            fn()
+    barrier()
+    if wq.device_status() != 0:
+        raise RuntimeError("a kernel reported a wait timeout during warm-up")
+
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in launches]
+           for _ in range(args.steps)]
+    sampler = ClockSampler(dev.index)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    t_wall0 = time.time()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(args.steps):
+        for (name, fn), (e0, e1) in zip(launches, evs[k]):
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+    end.record(stream)
+    barrier()
+    t_wall1 = time.time()
+    sampler.stop()
+    if wq.device_status() != 0:
+        raise RuntimeError("a kernel reported a wait timeout in the timed region")
+    total_ms = start.elapsed_time(end)
+    per_kernel_us = {n: [] for n in names}
+    for k in range(args.steps):
+        for n, (e0, e1) in zip(names, evs[k]):
+            per_kernel_us[n].append(e0.elapsed_time(e1) * 1e3)
+    mean_us = {n: sum(v) / len(v) for n, v in per_kernel_us.items()}
+
+    # max over ranks of the timed region and of each kernel's summed time
+    red = reduce_max([total_ms] + [sum(per_kernel_us[n]) for n in names], world, dev)
+    total_ms_max, kernel_tot_us_max = red[0], dict(zip(names, red[1:]))
+
+    gemv = [n for n in names if n.startswith("gemv_w4a16_b1")]
+    gemv_bytes = sum(work[n]["bytes"] for n in gemv)
+    gemv_time_s = sum(kernel_tot_us_max[n] for n in gemv) * 1e-6
+    value = aggregate_value(gemv_bytes, args.steps, world, gemv_time_s)
+    w8a8_s = kernel_tot_us_max["gemm_w8a8"] * 1e-6
+    w8a8_tops = work["gemm_w8a8"]["ops"] * args.steps * world / w8a8_s / 1e12
+
+    kernels = []
+    for n in names:
+        r = roofline_for(n, mean_us[n], work[n], peaks)
+        kernels.append({"name": n, "us": round(mean_us[n], 2), "achieved": round(r["achieved"], 1),
+                        "unit": r["unit"], "bound": r["bound"], "frac": round(r["frac"], 4)})
+    # dominant kernel of the step (largest device time); traffic comes from a committed ncu capture
+    dom = max(names, key=lambda n: mean_us[n])
+    rdom = roofline_for(dom, mean_us[dom], work[dom], peaks)
+    traffic = load_traffic(dom)
+    gemv_roof = roofline_for("gemv_w4a16_b1_up", 1.0, {"bytes": 1, "ops": 0}, peaks)
+
+    # e2e: the GEMV through the public API with the activations copied in from pinned host
+    # memory and the result read back, every step
+    e2e = run_e2e(torch, wq, step, args.steps, stream)
+
+    clocks = sampler.summary(t_wall0, t_wall1)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(total_ms_max / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int4 weights x fp16 activations; int8 x int8",
+        "data": "synthetic (seeded; shapes and outlier structure of the pages' workloads)",
+        "config": {"workload": WORKLOAD, "w4a16_shapes": [list(UP), list(DOWN)], "gemv_batch": 1,
+                   "gemm_batches": [16, 64], "group_size": 128, "w8a8": list(W8A8_SHAPE), "alpha": 0.5,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2; matmul operands untouched since the previous step"},
+        "value_frac_of_hbm_peak": round(value / world / peaks["hbm_gbs"], 4),
+        "w8a8": {"value": round(w8a8_tops, 1), "unit": "TOPS", "peak": 2.0 * peaks["bf16_tflops"],
+                 "frac": round(w8a8_tops / world / (2.0 * peaks["bf16_tflops"]), 4),
+                 "peak_note": "INT8 dense = 2 x measured bf16 burst (nominal ratio)"},
+        "roofline": {"kernel": dom, "bound": rdom["bound"], "achieved": round(rdom["achieved"], 1),
+                     "peak": rdom["peak"], "unit": rdom["unit"], "frac": round(rdom["frac"], 4),
+                     "traffic": traffic, "peak_source": peaks["source"]},
+        "gemv_roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": gemv_roof["peak"],
+                          "unit": "GB/s", "frac": round(value / world / gemv_roof["peak"], 4)},
+        "kernels": kernels,
+        "e2e": e2e,
+        "gpu_launches": len(launches) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[dev.index])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(torch, wq, step, steps, stream):
+    ins, qB = step.ins, step.qB
+    hx = {t: ins[f"x1_{t}"].cpu().pin_memory() for t in ("up", "down")}
+    hy = {t: torch.empty((1, (UP if t == "up" else DOWN)[0]), dtype=torch.float16).pin_memory()
+          for t in ("up", "down")}
+    dx = {t: torch.empty_like(ins[f"x1_{t}"]) for t in ("up", "down")}
+    dy = {t: torch.empty((1, (UP if t == "up" else DOWN)[0]), dtype=torch.float16, device=ins["X5"].device)
+          for t in ("up", "down")}
+
+    def one():
+        for t in ("up", "down"):
+            dx[t].copy_(hx[t], non_blocking=True)
+            wq.gemv_w4a16(dx[t], *qB[t], 128, out=dy[t])
+            hy[t].copy_(dy[t], non_blocking=True)
+
+    for _ in range(3):
+        one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        one()
+    e.record(stream)
+    torch.cuda.synchronize()
+    t = s.elapsed_time(e) * 1e-3
+    w = work_table()
+    byts = w["gemv_w4a16_b1_up"]["bytes"] + w["gemv_w4a16_b1_down"]["bytes"]
+    h2d = sum(hx[t].numel() * 2 for t in hx)
+    d2h = sum(hy[t].numel() * 2 for t in hy)
+    return {"value": round(byts * steps / t / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "what": "batch-1 W4A16 GEMV on both weights via the Python/C API, "
+                                              "x copied from pinned host memory and y read back each step"}
+
+
+def load_traffic(kernel):
+    """Per-launch DRAM bytes for `kernel` from the committed ncu summary, if any."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    return None if e is None else e.get("bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(seconds=12.0, steps=None):
+    """The oracle's fp64 W4A16 GEMV on a bounded sample of the workload's rows (one core)."""
+    import oracle
+    import workloads
+    w = workloads.config_weight(4, 0, shape=(4096, UP[1]))  # the first rows of the up-projection
+    qw, sc, qz = oracle.quantize_group_int4(w, 128)
+    x = workloads.config_activations(4, 1, UP[1])
+    K = UP[1]
+    # calibrate on 64 rows, then size the sample to ~`seconds`
+    t0 = time.perf_counter()
+    oracle.matmul_w4a16_ref(x, qw[:64], sc[:64], qz[:64], K, 128)
+    per_row = (time.perf_counter() - t0) / 64
+    rows = int(max(64, min(qw.shape[0], seconds / max(per_row, 1e-9))))
+    t0 = time.perf_counter()
+    oracle.matmul_w4a16_ref(x, qw[:rows], sc[:rows], qz[:rows], K, 128)
+    dt = time.perf_counter() - t0
+    byts = packed_bytes(rows, K) + 2 * K + 2 * rows
+    return {"value": round(byts / dt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"fp64 oracle W4A16 GEMV, batch 1, first {rows} rows of the 28672x8192 up-projection "
+                      f"({dt:.1f} s)", "host_cores_total": os.cpu_count()}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        cpu_baseline(min(1.0, per_step))
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(per_step))
+    dt = time.perf_counter() - t0
+    v = statistics.median([b["value"] for b in vals])
+    line = {"metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp64 (oracle)", "data": "synthetic (seeded)",
+            "config": {"workload": WORKLOAD, "sample": vals[-1]["sample"]}, "impl": "reference",
+            "cpu_baseline": {"value": v, "unit": "GB/s", "kind": "oracle", "cores": 1, "sample": vals[-1]["sample"]},
+            "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["wq", "reference"], default="wq")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="size of the CPU oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,7 +1,455 @@
-// W4A16 tensor-core GEMM (placeholder until the tcgen05 kernel lands).
+// W4A16 GEMM on the tensor cores (tcgen05, kind::f16) for M >= 16 activation
+// rows: packed INT4 tiles are dequantized into shared memory and fed to MMAs
+// with fp32 accumulation in tensor memory.
+//
+// Source: "How quantization works", section "Inference view" (quantized
+// weights are unpacked, multiplied by their scales and fed to the Tensor Cores
+// inside the kernel); "Quantization from Scratch", sections "Scale and
+// zero-point" (w^ = (q - z) s) and "What it buys at decode" (a batch of B
+// sequences reads every weight once and does 2 FLOPs per weight per sequence).
+//
+//   y[m][n] = fp16_rn( sum_k fp16_rn(s[n][k/128] * (q[n][k] - z[n][k/128])) * x[m][k] )
+//
+// Swap-AB: the MMA's M dimension is 128 weight rows (TMEM lanes) and its N
+// dimension is the activation tile (16..128 rows of x), so small batches still
+// use full 128-row MMAs.  Per CTA (480 threads):
+//   warp 0      TMA: packed weight tiles (128 rows x 32 bytes = 64 codes) into
+//               a 12-deep ring
+//   warp 1      TMA: x tiles (MT rows x 64 fp16, 128-byte swizzle)
+//   warp 2      TMEM allocation and tcgen05.mma issue (4 x K=16 per stage)
+//   warps 3-10  dequantize: each thread turns 32 codes of one row into fp16
+//               with PRMT/LOP3 (code -> 1024 + q), one exact fp16x2 fma
+//               (-> q - z) and one fp16x2 multiply by the scale, and stores
+//               them into the 128-byte-swizzled K-major A tile
+//   warps 11-14 epilogue: tcgen05.ld of the 128 x MT fp32 accumulator
+// K is split over the S CTAs of a thread-block cluster when the weight tiles
+// alone would leave SMs idle; their fp32 partial tiles are summed in the
+// leading CTA's shared memory through distributed shared memory, so the
+// kernel needs no global scratch.  No multicast of any kind.
+#include "sm100.cuh"
+#include "wq_device.cuh"
 #include "wq_host.h"
 
-extern "C" wq_status wq_gemm_w4a16(const uint16_t *, int, const uint32_t *, const uint16_t *, const uint32_t *, int,
-                                   int, int, uint16_t *, void *) {
-    return wq::fail(WQ_ERR_UNSUPPORTED, "wq_gemm_w4a16: not built yet");
+#include <algorithm>
+
+namespace wq {
+namespace {
+
+using namespace sm100;
+
+constexpr int BMW = 128;                    // weight rows per tile (MMA M)
+constexpr int BK = 64;                      // k per stage: one 128-byte fp16 row
+constexpr int STAGES = 4;                   // A/B stages
+constexpr int PSTAGES = 12;                 // packed-tile ring
+constexpr uint32_t A_BYTES = BMW * BK * 2;  // 16 KB
+constexpr uint32_t P_BYTES = BMW * BK / 2;  // 4 KB of packed codes
+constexpr int THREADS = 480;
+constexpr int DQ_THREADS = 256;
+constexpr uint64_t DRAIN_NS = 2000000000ull;
+constexpr unsigned SITE_PRODUCER = 0x201, SITE_MMA = 0x202, SITE_DEQUANT = 0x204, SITE_EPILOGUE = 0x208,
+                   SITE_DRAIN = 0x210;
+
+template <int MT>
+struct Layout {
+    static constexpr uint32_t B_BYTES = MT * 128;
+    static constexpr uint32_t OFF_A = 0;
+    static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr uint32_t OFF_P = OFF_B + STAGES * B_BYTES;
+    static constexpr uint32_t PIPE_BYTES = OFF_P + PSTAGES * P_BYTES;  // reused for split-K partials
+    static constexpr size_t SMEM = 1024 + PIPE_BYTES + 512;  // alignment slack + barriers
+};
+
+struct Bars {
+    uint64_t pk_full[PSTAGES];
+    uint64_t pk_empty[PSTAGES];
+    uint64_t a_full[STAGES];   // dequantized weight tile written (256 arrivals)
+    uint64_t x_full[STAGES];   // activation tile landed (TMA transaction count)
+    uint64_t st_empty[STAGES];
+    uint64_t tmem_full;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// fp16x2 constant (-(1024 + z), -(64 + z)) for zero point z.
+__device__ __forceinline__ uint32_t zero_consts(uint32_t z) { return 0xD400E400u + z * 0x00100001u; }
+
+// One word of 8 codes (k .. k+7) -> 8 fp16 weights fp16_rn(s (q - z)) in k order.
+// Byte i holds codes 2i (low nibble) and 2i+1 (high nibble); PRMT copies it into
+// both halves, LOP3 keeps the low nibble in the low half (1024 + q) and the high
+// nibble in bits 4..7 of the high half (1024 + 16 q); one fma with (1, 1/16) and
+// (-(1024+z), -(64+z)) gives q - z exactly, one multiply applies the scale.
+__device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t zc, uint32_t s2) {
+    const uint32_t c1 = 0x2C003C00u;  // (1.0, 0.0625)
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t y = prmt(w, 0u, 0x4040u + 0x0101u * i);
+        const uint32_t h = (y & 0x00F0000Fu) | 0x64006400u;
+        o[i] = hmul2(hfma2(h, c1, zc), s2);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <int MT, bool SB>
+__global__ void __launch_bounds__(THREADS, 1)
+    gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
+                      const uint16_t *__restrict__ scales, const uint32_t *__restrict__ qzeros,
+                      uint16_t *__restrict__ y, int M, int N, int K, int splits, unsigned int *status,
+                      uint64_t limit_ns) {
+    using L = Layout<MT>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars *bar = reinterpret_cast<Bars *>(base + L::PIPE_BYTES);
+    const uint32_t sA = smem_u32(base + L::OFF_A), sB = smem_u32(base + L::OFF_B), sP = smem_u32(base + L::OFF_P);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rank = (int)blockIdx.x;  // cluster dims (splits, 1, 1)
+    const int n0 = blockIdx.y * BMW, m0 = blockIdx.z * MT;
+    const int kb_total = K / BK;
+    const int nkb = kb_total / splits;
+    const int kb0 = rank * nkb;
+    const int groups = K / 128, zwords = (groups + 7) / 8;
+    constexpr uint32_t IDESC = make_idesc(/*f32*/ 1, /*f16*/ 0, /*f16*/ 0, BMW, MT);
+    constexpr uint32_t TMEM_COLS = MT < 32 ? 32 : MT;
+
+    if (threadIdx.x == 0) {
+        for (int p = 0; p < PSTAGES; ++p) {
+            mbar_init(smem_u32(&bar->pk_full[p]), 1);
+            mbar_init(smem_u32(&bar->pk_empty[p]), DQ_THREADS);
+        }
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&bar->a_full[s]), DQ_THREADS);
+            mbar_init(smem_u32(&bar->x_full[s]), 1);
+            mbar_init(smem_u32(&bar->st_empty[s]), 1);
+        }
+        mbar_init(smem_u32(&bar->tmem_full), 1);
+        mbar_init(smem_u32(&bar->drain), 1);
+        bar->abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmap_q);
+        prefetch_tmap(&tmap_x);
+    }
+    if (warp == 2) {
+        tmem_alloc(smem_u32(&bar->tmem_base), TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = bar->tmem_base;
+    const WaitCtl ctl{&bar->abort, status, limit_ns};
+
+    if (warp == 0) {
+        if (lane == 0) {  // ------------------------------------------------ packed-code producer
+            int i = 0;
+            for (; i < nkb; ++i) {
+                const int p = i % PSTAGES, up = i / PSTAGES;
+                if (!wait_parity(smem_u32(&bar->pk_empty[p]), (up & 1) ^ 1, ctl, SITE_PRODUCER)) break;
+                const uint32_t fb = smem_u32(&bar->pk_full[p]);
+                mbar_arrive_expect_tx(fb, P_BYTES);
+                tma_load_2d(sP + p * P_BYTES, &tmap_q, fb, (kb0 + i) * (BK / 2), n0);
+            }
+            for (int p = 0; p < PSTAGES; ++p) {
+                const int issued = i > p ? (i - p - 1) / PSTAGES + 1 : 0;
+                if (issued) drain_parity(smem_u32(&bar->pk_full[p]), (issued - 1) & 1, DRAIN_NS, status, SITE_DRAIN);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {  // ------------------------------------------------ activation producer
+            int i = 0;
+            for (; i < nkb; ++i) {
+                const int s = i % STAGES, u = i / STAGES;
+                if (!wait_parity(smem_u32(&bar->st_empty[s]), (u & 1) ^ 1, ctl, SITE_PRODUCER)) break;
+                const uint32_t fb = smem_u32(&bar->x_full[s]);
+                mbar_arrive_expect_tx(fb, L::B_BYTES);
+                tma_load_2d(sB + s * L::B_BYTES, &tmap_x, fb, (kb0 + i) * BK, m0);
+            }
+            for (int s = 0; s < STAGES; ++s) {
+                const int issued = i > s ? (i - s - 1) / STAGES + 1 : 0;
+                if (issued) drain_parity(smem_u32(&bar->x_full[s]), (issued - 1) & 1, DRAIN_NS, status, SITE_DRAIN);
+            }
+        }
+    } else if (warp == 2) {
+        if (lane == 0) {  // ------------------------------------------------ MMA issuer
+            bool ok = true;
+            for (int i = 0; i < nkb; ++i) {
+                const int s = i % STAGES, u = i / STAGES;
+                if (!wait_parity(smem_u32(&bar->x_full[s]), u & 1, ctl, SITE_MMA) ||
+                    !wait_parity(smem_u32(&bar->a_full[s]), u & 1, ctl, SITE_MMA)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = sA + s * A_BYTES, b_addr = sB + s * L::B_BYTES;
+#pragma unroll
+                for (int kk = 0; kk < BK / 16; ++kk)
+                    mma_f16(tmem_base, umma_desc_sw128_kmajor(a_addr + kk * 32), umma_desc_sw128_kmajor(b_addr + kk * 32),
+                            IDESC, (i | kk) != 0);
+                tc_commit(smem_u32(&bar->st_empty[s]));
+            }
+            if (ok) tc_commit(smem_u32(&bar->tmem_full));
+            tc_commit(smem_u32(&bar->drain));
+            drain_parity(smem_u32(&bar->drain), 0, DRAIN_NS, status, SITE_DRAIN);
+        }
+        __syncwarp();
+    } else if (warp < 11) {
+        // -------------------------------------------------------------------- dequantizers
+        const int d = threadIdx.x - 96;
+        const int row = d & (BMW - 1), half = d >> 7;
+        const int n = min(n0 + row, N - 1);
+        const uint32_t a_row = sA + row * 128;
+        const int sw = row & 7;
+        const uint16_t *srow = scales + (size_t)n * groups;
+        const uint32_t *zrow = qzeros + (size_t)n * zwords;
+        bool ok = true;
+        auto stage = [&](int i, uint32_t zc, uint32_t s2) -> bool {
+            const int p = i % PSTAGES, up = i / PSTAGES;
+            const int s = i % STAGES, u = i / STAGES;
+            if (!wait_parity(smem_u32(&bar->pk_full[p]), up & 1, ctl, SITE_DEQUANT)) return false;
+            uint4 w;
+            asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                         : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                         : "r"(sP + p * P_BYTES + row * 32 + half * 16));
+            mbar_arrive(smem_u32(&bar->pk_empty[p]));
+            if (!wait_parity(smem_u32(&bar->st_empty[s]), (u & 1) ^ 1, ctl, SITE_DEQUANT)) return false;
+            const uint32_t dst = a_row + s * A_BYTES;
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const uint4 o = dequant_word(ws[j], zc, s2);
+                const int chunk = half * 4 + j;
+                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst + ((chunk ^ sw) << 4)), "r"(o.x),
+                             "r"(o.y), "r"(o.z), "r"(o.w)
+                             : "memory");
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(smem_u32(&bar->a_full[s]));
+            return true;
+        };
+        if (SB) {
+            // Scales and zero points of 8 groups (1024 codes) at a time, fetched one
+            // such block ahead so their latency hides behind 16 stages of work.
+            const int sb0 = kb0 / 16, nsb = nkb / 16;
+            uint4 cs = __ldg(reinterpret_cast<const uint4 *>(srow) + sb0);
+            uint32_t cz = __ldg(zrow + sb0);
+            for (int b = 0; b < nsb && ok; ++b) {
+                uint4 ns = cs;
+                uint32_t nz = cz;
+                if (b + 1 < nsb) {
+                    ns = __ldg(reinterpret_cast<const uint4 *>(srow) + sb0 + b + 1);
+                    nz = __ldg(zrow + sb0 + b + 1);
+                }
+                const uint32_t sv[4] = {cs.x, cs.y, cs.z, cs.w};
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const uint32_t s2 = prmt(sv[g >> 1], 0u, (g & 1) ? 0x3232u : 0x1010u);
+                    const uint32_t zc = zero_consts((cz >> (4 * g)) & 0xFu);
+                    if (!stage(b * 16 + 2 * g, zc, s2) || !stage(b * 16 + 2 * g + 1, zc, s2)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                cs = ns;
+                cz = nz;
+            }
+        } else {
+            for (int i = 0; i < nkb && ok; i += 2) {
+                const int g = (kb0 + i) >> 1;
+                const uint32_t sh = __ldg(srow + g);
+                const uint32_t s2 = sh | (sh << 16);
+                const uint32_t zc = zero_consts((__ldg(zrow + (g >> 3)) >> (4 * (g & 7))) & 0xFu);
+                ok = stage(i, zc, s2) && (i + 1 >= nkb || stage(i + 1, zc, s2));
+            }
+        }
+    }
+
+    // ------------------------------------------------------------------------ epilogue
+    const bool epi = warp >= 11;
+    const int q = warp & 3;
+    const int erow = q * 32 + lane;
+    const int n = n0 + erow;
+    bool have_acc = false;
+    if (epi) {
+        have_acc = wait_parity(smem_u32(&bar->tmem_full), 0, ctl, SITE_EPILOGUE);
+        have_acc = __all_sync(0xffffffffu, have_acc);
+        tc_fence_after();
+    }
+    const uint32_t t_row = tmem_base + ((uint32_t)(q * 32) << 16);
+    if (splits == 1) {
+        if (epi && have_acc) {
+#pragma unroll 1
+            for (int c = 0; c < MT; c += 16) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(t_row + c, r);
+                tmem_ld_wait();
+                if (n < N) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (m0 + c + j < M)
+                            y[(size_t)(m0 + c + j) * N + n] = float_to_half_bits_rn(__uint_as_float(r[j]));
+                }
+            }
+        }
+    } else {
+        // Split-K: partial tiles of CTAs 1..S-1 go to CTA 0's shared memory (the
+        // pipeline buffers, idle by now), CTA 0 adds them in rank order.
+        cluster_sync();  // every CTA of the cluster is past its main loop
+        const uint32_t red = smem_u32(base);
+        if (epi && rank != 0) {
+            const uint32_t slot = mapa_shared(red, 0) + (uint32_t)((rank - 1) * BMW + erow) * MT * 4;
+#pragma unroll 1
+            for (int c = 0; c < MT; c += 16) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(t_row + c, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; j += 4)
+                    st_cluster_v4(slot + (c + j) * 4, __uint_as_float(r[j]), __uint_as_float(r[j + 1]),
+                                  __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
+            }
+        }
+        cluster_sync();  // partials have landed
+        if (epi && rank == 0) {
+            const float *redp = reinterpret_cast<const float *>(base);
+#pragma unroll 1
+            for (int c = 0; c < MT; c += 16) {
+                uint32_t r[16];
+                tmem_ld_32x32b_x16(t_row + c, r);
+                tmem_ld_wait();
+                float acc[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[j] = __uint_as_float(r[j]);
+                for (int sl = 0; sl < splits - 1; ++sl) {
+                    const float *pp = redp + (size_t)(sl * BMW + erow) * MT + c;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) acc[j] += pp[j];
+                }
+                if (n < N && have_acc) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (m0 + c + j < M) y[(size_t)(m0 + c + j) * N + n] = float_to_half_bits_rn(acc[j]);
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+template <int MT, bool SB>
+wq_status launch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t *scales, const uint32_t *qzeros,
+                 uint16_t *y, int M, int N, int K, int splits, unsigned int *status, cudaStream_t st) {
+    auto kern = gemm_w4a16_kernel<MT, SB>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Layout<MT>::SMEM);
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(splits, (N + BMW - 1) / BMW, (M + MT - 1) / MT);
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = Layout<MT>::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, tq, tx, scales, qzeros, y, M, N, K, splits, status, wait_limit());
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: launch failed: %s", cudaGetErrorString(e));
+    return WQ_OK;
+}
+
+// Number of CTAs sharing one weight tile's K range: a divisor of the stage
+// count (a multiple of 16 stages each on the fast path), at most 8, whose
+// partial tiles fit the leading CTA's pipeline buffers, chosen to fill the
+// SMs in as few, as full waves as possible.
+int choose_splits(int tiles, int K, int MT, bool fast, size_t pipe_bytes, int sms) {
+    const int kb = K / BK;
+    int best = 1;
+    double best_eff = -1.0;
+    for (int s = 1; s <= 8; ++s) {
+        if (kb % s) continue;
+        if (fast && (kb / s) % 16) continue;
+        if (!fast && s > 1) continue;
+        if ((size_t)(s - 1) * BMW * MT * 4 > pipe_bytes) continue;
+        const double waves = (double)tiles * s / sms;
+        const double eff = waves / std::ceil(waves);
+        if (eff > best_eff + 0.02) {
+            best_eff = eff;
+            best = s;
+        }
+    }
+    return best;
+}
+
+template <int MT>
+wq_status dispatch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t *scales, const uint32_t *qzeros,
+                   uint16_t *y, int M, int N, int K, unsigned int *status, cudaStream_t st) {
+    const bool fast = (K % 1024) == 0;
+    const int tiles = ((N + BMW - 1) / BMW) * ((M + MT - 1) / MT);
+    const int splits = choose_splits(tiles, K, MT, fast, Layout<MT>::PIPE_BYTES, num_sms());
+    if (fast && (K / BK / splits) % 16 == 0)
+        return launch<MT, true>(tq, tx, scales, qzeros, y, M, N, K, splits, status, st);
+    return launch<MT, false>(tq, tx, scales, qzeros, y, M, N, K, splits, status, st);
+}
+
+}  // namespace
+}  // namespace wq
+
+extern "C" wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
+                                   const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y, void *stream) {
+    using namespace wq;
+    WQ_REQUIRE_PTR(x, "x");
+    WQ_REQUIRE_PTR(qweight, "qweight");
+    WQ_REQUIRE_PTR(scales, "scales");
+    WQ_REQUIRE_PTR(qzeros, "qzeros");
+    WQ_REQUIRE_PTR(y, "y");
+    WQ_REQUIRE(M > 0 && N > 0 && K > 0, WQ_ERR_INVALID_ARG, "wq_gemm_w4a16: sizes must be positive (M=%d N=%d K=%d)",
+               M, N, K);
+    WQ_REQUIRE(group_size == 128, WQ_ERR_UNSUPPORTED, "wq_gemm_w4a16: group_size must be 128 (got %d)", group_size);
+    WQ_REQUIRE(K % 128 == 0, WQ_ERR_INVALID_ARG, "wq_gemm_w4a16: K (%d) must be a multiple of 128", K);
+    WQ_REQUIRE(M >= 16, WQ_ERR_UNSUPPORTED, "wq_gemm_w4a16: M (%d) below 16: use wq_gemv_w4a16", M);
+    unsigned int *status = device_status_word();
+    if (!status) return WQ_ERR_CUDA;
+    const int MT = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    CUtensorMap tq, tx;
+    if (!encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qweight, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
+                        BK / 2, BMW, CU_TENSOR_MAP_SWIZZLE_NONE))
+        return WQ_ERR_CUDA;
+    if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK,
+                        MT, CU_TENSOR_MAP_SWIZZLE_128B))
+        return WQ_ERR_CUDA;
+    cudaStream_t st = as_stream(stream);
+    switch (MT) {
+        case 16: return dispatch<16>(tq, tx, scales, qzeros, y, M, N, K, status, st);
+        case 32: return dispatch<32>(tq, tx, scales, qzeros, y, M, N, K, status, st);
+        case 64: return dispatch<64>(tq, tx, scales, qzeros, y, M, N, K, status, st);
+        default: return dispatch<128>(tq, tx, scales, qzeros, y, M, N, K, status, st);
+    }
 }

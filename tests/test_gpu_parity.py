@@ -295,3 +295,43 @@ def test_w8a8_smoothquant_pipeline_full_size(wq):
     assert np.array_equal(host(acc)[np.ix_(ms, ns)].astype(np.int64), racc)
     assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, "w8a8 config 5")
     assert wq.device_status() == 0
+
+
+# --------------------------------------------------------------------------
+# W4A16 tensor-core GEMM
+# --------------------------------------------------------------------------
+GEMM_W4_SMALL = [  # (M, N, K): ragged M/N, K on and off the 1024-code fast path, split-K clusters
+    (16, 128, 128), (16, 300, 1024), (20, 256, 2048), (64, 1000, 4096), (33, 129, 1152),
+    (128, 512, 8192), (100, 384, 3072), (16, 4096, 14336), (48, 640, 16384), (17, 130, 640),
+]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_W4_SMALL)
+def test_gemm_w4a16_small(wq, M, N, K):
+    w = _special_weights(N, K, seed=M + N + K)
+    rqw, rsc, rqz = oracle.quantize_group_int4(w, 128)
+    x = workloads.activations(M, K, 0.01, 50.0, seed=M, tensor_id=N)
+    y = wq.gemm_w4a16(dev(x), dev(rqw.view(np.int32)), dev(rsc), dev(rqz.view(np.int32)), 128)
+    torch.cuda.synchronize()
+    rows = sample_rows(N, 300, seed=K)
+    y_ref, bound = oracle.matmul_w4a16_ref(x, rqw, rsc, rqz, K, 128, rows=rows)
+    assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"gemm_w4a16 M={M} N={N} K={K}")
+    assert wq.device_status() == 0
+
+
+@pytest.mark.parametrize("cfg", [3, 4])
+def test_gemm_w4a16_configs(wq, cfg):
+    c = workloads.CONFIGS[cfg]
+    for si, (N, K) in enumerate(c.shapes):
+        w = workloads.config_weight(cfg, si)
+        qw, sc, qz = wq.quantize_group_int4(dev(w), 128)
+        del w
+        rows = sample_rows(N, 128, seed=si + 10)
+        hqw, hsc, hqz = host(qw, np.uint32), host(sc), host(qz, np.uint32)
+        for B in c.batches:
+            x = workloads.config_activations(cfg, B, K)
+            y = wq.matmul_w4a16(dev(x), qw, sc, qz, 128)
+            torch.cuda.synchronize()
+            y_ref, bound = oracle.matmul_w4a16_ref(x, hqw[rows], hsc[rows], hqz[rows], K, 128)
+            assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"cfg{cfg} {N}x{K} B={B}")
+    assert wq.device_status() == 0
