@@ -201,19 +201,13 @@ class Step:
         self.out = {}
 
     def launches(self):
+        """The step's kernels, ordered so that no matmul finds its operands in L2: the batch-1
+        GEMVs run after the 470 MB INT8 weight stream of the W8A16 GEMVs (clean lines), and
+        every packed weight read was last touched a full step earlier or before that stream."""
         wq, ins, qB, q8B = self.wq, self.ins, self.qB, self.q8B
         L = []
         for t in ("up", "down"):
             L.append((f"quant_int4_{t}", lambda t=t: wq.quantize_group_int4(ins[f"w_{t}"], 128)))
-        for t in ("up", "down"):
-            L.append((f"gemv_w4a16_b1_{t}", lambda t=t: wq.gemv_w4a16(ins[f"x1_{t}"], *qB[t], 128)))
-        for M in (16, 64):
-            for t in ("up", "down"):
-                L.append((f"gemm_w4a16_m{M}_{t}", lambda t=t, M=M: wq.gemm_w4a16(ins[f"x{M}_{t}"], *qB[t], 128)))
-        for t in ("up", "down"):
-            L.append((f"quant_int8_pc_{t}", lambda t=t: wq.quantize_int8_per_channel(ins[f"w_{t}"])))
-        for t in ("up", "down"):
-            L.append((f"gemv_w8a16_b1_{t}", lambda t=t: wq.gemv_w8a16(ins[f"x1_{t}"], *q8B[t])))
 
         def smooth():
             self.out["s"] = wq.smooth(ins["X5"], ins["W5"], 0.5, workspace=self.ws)
@@ -230,6 +224,15 @@ class Step:
             self.out["y5"] = wq.gemm_w8a8(xq, sx, w8, sw)
 
         L += [("smooth", smooth), ("quant_int8_pc_smooth", q_w), ("quant_int8_pt_smooth", q_x), ("gemm_w8a8", w8a8)]
+        for t in ("up", "down"):
+            L.append((f"quant_int8_pc_{t}", lambda t=t: wq.quantize_int8_per_channel(ins[f"w_{t}"])))
+        for M in (16, 64):
+            for t in ("up", "down"):
+                L.append((f"gemm_w4a16_m{M}_{t}", lambda t=t, M=M: wq.gemm_w4a16(ins[f"x{M}_{t}"], *qB[t], 128)))
+        for t in ("up", "down"):
+            L.append((f"gemv_w8a16_b1_{t}", lambda t=t: wq.gemv_w8a16(ins[f"x1_{t}"], *q8B[t])))
+        for t in ("up", "down"):
+            L.append((f"gemv_w4a16_b1_{t}", lambda t=t: wq.gemv_w4a16(ins[f"x1_{t}"], *qB[t], 128)))
         return L
 
 

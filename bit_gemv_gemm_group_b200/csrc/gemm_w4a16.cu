@@ -39,7 +39,7 @@ using namespace sm100;
 
 constexpr int BMW = 128;                    // weight rows per tile (MMA M)
 constexpr int BK = 64;                      // k per stage: one 128-byte fp16 row
-constexpr int STAGES = 4;                   // A/B stages
+constexpr int STAGES = 4;                   // dequantized A stages
 constexpr int PSTAGES = 12;                 // packed-tile ring
 constexpr uint32_t A_BYTES = BMW * BK * 2;  // 16 KB
 constexpr uint32_t P_BYTES = BMW * BK / 2;  // 4 KB of packed codes
@@ -52,19 +52,24 @@ constexpr unsigned SITE_PRODUCER = 0x201, SITE_MMA = 0x202, SITE_DEQUANT = 0x204
 template <int MT>
 struct Layout {
     static constexpr uint32_t B_BYTES = MT * 128;
+    // activation tiles get their own ring, deep enough that a tile is requested
+    // well before the MMA needs it (x comes from L2; its latency would otherwise
+    // stall the MMA warp every few stages)
+    static constexpr int XSTAGES = MT <= 32 ? 12 : MT <= 64 ? 8 : 4;
     static constexpr uint32_t OFF_A = 0;
     static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
-    static constexpr uint32_t OFF_P = OFF_B + STAGES * B_BYTES;
+    static constexpr uint32_t OFF_P = OFF_B + XSTAGES * B_BYTES;
     static constexpr uint32_t PIPE_BYTES = OFF_P + PSTAGES * P_BYTES;  // reused for split-K partials
-    static constexpr size_t SMEM = 1024 + PIPE_BYTES + 512;  // alignment slack + barriers
+    static constexpr size_t SMEM = 1024 + PIPE_BYTES + 1024;  // alignment slack + barriers
 };
 
 struct Bars {
     uint64_t pk_full[PSTAGES];
     uint64_t pk_empty[PSTAGES];
     uint64_t a_full[STAGES];   // dequantized weight tile written (256 arrivals)
-    uint64_t x_full[STAGES];   // activation tile landed (TMA transaction count)
-    uint64_t st_empty[STAGES];
+    uint64_t st_empty[STAGES]; // A stage consumed by the MMAs
+    uint64_t x_full[12];       // activation tile landed (TMA transaction count)
+    uint64_t x_empty[12];      // activation tile consumed by the MMAs
     uint64_t tmem_full;
     uint64_t drain;
     uint32_t tmem_base;
@@ -138,8 +143,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(&bar->a_full[s]), DQ_THREADS);
-            mbar_init(smem_u32(&bar->x_full[s]), 1);
             mbar_init(smem_u32(&bar->st_empty[s]), 1);
+        }
+        for (int s = 0; s < L::XSTAGES; ++s) {
+            mbar_init(smem_u32(&bar->x_full[s]), 1);
+            mbar_init(smem_u32(&bar->x_empty[s]), 1);
         }
         mbar_init(smem_u32(&bar->tmem_full), 1);
         mbar_init(smem_u32(&bar->drain), 1);
@@ -179,14 +187,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {  // ------------------------------------------------ activation producer
             int i = 0;
             for (; i < nkb; ++i) {
-                const int s = i % STAGES, u = i / STAGES;
-                if (!wait_parity(smem_u32(&bar->st_empty[s]), (u & 1) ^ 1, ctl, SITE_PRODUCER)) break;
+                const int s = i % L::XSTAGES, u = i / L::XSTAGES;
+                if (!wait_parity(smem_u32(&bar->x_empty[s]), (u & 1) ^ 1, ctl, SITE_PRODUCER)) break;
                 const uint32_t fb = smem_u32(&bar->x_full[s]);
                 mbar_arrive_expect_tx(fb, L::B_BYTES);
                 tma_load_2d(sB + s * L::B_BYTES, &tmap_x, fb, (kb0 + i) * BK, m0);
             }
-            for (int s = 0; s < STAGES; ++s) {
-                const int issued = i > s ? (i - s - 1) / STAGES + 1 : 0;
+            for (int s = 0; s < L::XSTAGES; ++s) {
+                const int issued = i > s ? (i - s - 1) / L::XSTAGES + 1 : 0;
                 if (issued) drain_parity(smem_u32(&bar->x_full[s]), (issued - 1) & 1, DRAIN_NS, status, SITE_DRAIN);
             }
         }
@@ -195,18 +203,20 @@ __global__ void __launch_bounds__(THREADS, 1)
             bool ok = true;
             for (int i = 0; i < nkb; ++i) {
                 const int s = i % STAGES, u = i / STAGES;
-                if (!wait_parity(smem_u32(&bar->x_full[s]), u & 1, ctl, SITE_MMA) ||
+                const int xs = i % L::XSTAGES, xu = i / L::XSTAGES;
+                if (!wait_parity(smem_u32(&bar->x_full[xs]), xu & 1, ctl, SITE_MMA) ||
                     !wait_parity(smem_u32(&bar->a_full[s]), u & 1, ctl, SITE_MMA)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a_addr = sA + s * A_BYTES, b_addr = sB + s * L::B_BYTES;
+                const uint32_t a_addr = sA + s * A_BYTES, b_addr = sB + xs * L::B_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
                     mma_f16(tmem_base, umma_desc_sw128_kmajor(a_addr + kk * 32), umma_desc_sw128_kmajor(b_addr + kk * 32),
                             IDESC, (i | kk) != 0);
                 tc_commit(smem_u32(&bar->st_empty[s]));
+                tc_commit(smem_u32(&bar->x_empty[xs]));
             }
             if (ok) tc_commit(smem_u32(&bar->tmem_full));
             tc_commit(smem_u32(&bar->drain));

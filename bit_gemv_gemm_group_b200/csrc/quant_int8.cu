@@ -42,12 +42,13 @@ __device__ __forceinline__ void load8(const uint16_t *p, float (&v)[8]) {
     v[4] = c.x; v[5] = c.y; v[6] = d.x; v[7] = d.y;
 }
 
-__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s) {
+// |v / s| <= 127 (1 + 2^-23) < 2^8 (E = 7): codes via rne_quotient, identical to rne(fl(v / s)).
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s, float rs) {
     uint32_t lo = 0, hi = 0;
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const int q0 = clampi(__float2int_rn(__fdiv_rn(v[e], s)), -128, 127);
-        const int q1 = clampi(__float2int_rn(__fdiv_rn(v[e + 4], s)), -128, 127);
+        const int q0 = clampi(rne_quotient<7>(v[e], s, rs), -128, 127);
+        const int q1 = clampi(rne_quotient<7>(v[e + 4], s, rs), -128, 127);
         lo |= (uint32_t)(q0 & 0xff) << (8 * e);
         hi |= (uint32_t)(q1 & 0xff) << (8 * e);
     }
@@ -92,10 +93,11 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
         }
         const float a = fmaxf(block_max(amax, red), 1e-8f);
         const float s = __fdiv_rn(a, 127.0f);
+        const float rs = __frcp_rn(s);
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
             const int k = c * kRowStep + t0;
-            if (k < K) *reinterpret_cast<uint2 *>(qr + k) = quant8(v[c], s);
+            if (k < K) *reinterpret_cast<uint2 *>(qr + k) = quant8(v[c], s, rs);
         }
         if (threadIdx.x == 0) scales[row] = s;
     } else {
@@ -108,6 +110,7 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
         }
         const float a = fmaxf(block_max(amax, red), 1e-8f);
         const float s = __fdiv_rn(a, 127.0f);
+        const float rs = __frcp_rn(s);
         for (int k = t0; k < K; k += kRowStep) {
             float v[8];
             const uint4 r = *reinterpret_cast<const uint4 *>(xr + k);  // L2-resident re-read
@@ -116,7 +119,7 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
             v[0] = a0.x; v[1] = a0.y; v[2] = a1.x; v[3] = a1.y;
             v[4] = a2.x; v[5] = a2.y; v[6] = a3.x; v[7] = a3.y;
             smooth8<MODE>(v, smooth, k);
-            *reinterpret_cast<uint2 *>(qr + k) = quant8(v, s);
+            *reinterpret_cast<uint2 *>(qr + k) = quant8(v, s, rs);
         }
         if (threadIdx.x == 0) scales[row] = s;
     }

@@ -45,4 +45,21 @@ __device__ __forceinline__ uint16_t float_to_half_bits_rn(float f) {
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return min(max(v, lo), hi); }
 
+// rne(fl(a / b)) -- the integer that rounding the IEEE fp32 quotient to the
+// nearest (ties to even) gives -- for |a / b| < 2^(E+1), with y = RN(1/b).
+// q = RN(a * y) has relative error below 2^-23 + 2^-48, so |q - a/b| <
+// 2^(E-22) and |fl(a/b) - a/b| <= 2^(E-24); both lie on the same side of every
+// half-integer that q is more than `guard` = 2^(E-21) away from, and then
+// round to the same integer.  Otherwise (a near-tie, rare) the correctly
+// rounded quotient decides.  q - rint(q) and its distance to 0.5 are exact
+// (Sterbenz), so the test itself does not round.
+template <int E>
+__device__ __forceinline__ int rne_quotient(float a, float b, float y) {
+    constexpr float guard = E >= 21 ? 1.0f : 1.0f / (float)(1u << (21 - E));
+    const float q = __fmul_rn(a, y);
+    const float n = rintf(q);
+    if (fabsf(fabsf(__fsub_rn(q, n)) - 0.5f) <= guard) return __float2int_rn(__fdiv_rn(a, b));
+    return __float2int_rn(n);
+}
+
 }  // namespace wq
