@@ -346,56 +346,58 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_w4a16_mma_kernel(const ui
 }
 
 // ---------------------------------------------------------------------------
-// Streaming variant of the MMA GEMV for K % 1024 == 0 (the decode shapes).
-// Small per-group loads of scales, zero points and x through L1 leave warps
-// waiting on long scoreboards, and register prefetching keeps too few weight
-// bytes in flight; here one producer warp per CTA streams everything through
-// shared memory, so ~90 KB per CTA are in flight and the consumer warps only
-// read shared memory:
-//   - per group (128 codes): the CTA tile's codes (2-D TMA, ROWS x 64 B) and
-//     x rows 0..7 (2-D TMA, 8 x 128 fp16; rows >= B arrive zero-filled, which
-//     is exactly the MMA's padding), into a kGRing-deep ring;
-//   - per block of 8 groups: the tile's fp16 scales (2-D TMA, ROWS x 16 B)
-//     and zero-point words (cp.async, 4 B per row), double-buffered.
-// All 8 consumer warps walk the same groups, each owning RT*16 rows, so no
-// cross-warp reduction is needed.  When the tiles alone would leave SMs idle,
-// K is split across the CTAs of a thread-block cluster and the fp32 partial
-// results are summed in the leading CTA through distributed shared memory.
-// A consumer makes its shared-memory reads visible to the async proxy
-// (fence.proxy.async) before releasing a stage for the next TMA write.
+// Streaming GEMV for K % 256 == 0 (the decode shapes).
+//
+// Memory side: one producer warp per CTA streams the CTA tile's codes through
+// a shared-memory ring (2-D TMA, one ROWS x 64-byte plane per group, GPS
+// groups per stage).  The same warp turns x into the MMA's B fragments once
+// per CTA: each producer lane loads the 32 x values that consumer lane
+// `lane` needs for a group, permutes them into fragment order and stores them
+// lane-major (conflict-free 16-byte loads for every consumer warp), and adds
+// them up into the group sum X_g of its batch row.  The consumers fetch the
+// fp16 scales and zero-point words of their own rows from global memory one
+// block of 8 groups ahead; the CTA's shared memory is the ring alone, so two
+// CTAs fit on an SM and two consumer warps share each SM sub-partition.
+//
+// Compute side (warp-level mma.sync m16n8k16, batch = N): the codes go into
+// the A fragment as fp16 *subnormals*.  Masking a word with 0x000F000F leaves
+// two nibbles in the mantissa bits of two fp16 lanes, i.e. exactly q * 2^-24
+// (and 0x00F000F0 gives q * 2^-20), one LOP3 per pair and no conversion or
+// subtraction; the MMA multiplies them exactly.  The x lanes that meet the
+// 2^-20 codes are pre-scaled by 2^-4 (exact for |x| >= 2^-10, below that the
+// rounding is far inside the tolerance), so one MMA chain accumulates
+// D = 2^-24 sum_k q x in fp32, and the zero point enters per group through
+// X_g:  y += s (2^24 D - z X_g).
+// Each consumer warp owns RT m-tiles (RT independent MMA chains).  K is split
+// over a thread-block cluster (DSMEM reduction into the leading CTA) when the
+// tiles alone would leave SMs idle.  A consumer makes its shared-memory reads
+// visible to the async proxy (fence.proxy.async) before releasing a stage for
+// the next TMA write.
 // ---------------------------------------------------------------------------
-constexpr int kConsumerWarps = 8;
-constexpr int kGRing = 5;
+constexpr uint32_t kStreamRingBudget = 110 * 1024;  // two CTAs per SM (228 KB, 1 KB reserved per CTA)
 
-template <int RT>
+template <int CW, int RT, int GPS>
 struct StreamLayout {
-    static constexpr int ROWS = kConsumerWarps * RT * 16;
-    static constexpr uint32_t W_BYTES = ROWS * 64;
-    static constexpr uint32_t X_BYTES = 8 * 128 * 2;
-    static constexpr uint32_t STAGE = W_BYTES + X_BYTES;
-    static constexpr uint32_t S_BYTES = ROWS * 16;
-    static constexpr uint32_t Z_BYTES = ROWS * 4;
-    static constexpr uint32_t OFF_S = kGRing * STAGE;
-    static constexpr uint32_t OFF_Z = OFF_S + 2 * S_BYTES;
-    static constexpr uint32_t OFF_BAR = OFF_Z + 2 * Z_BYTES;
+    static_assert(GPS == 2, "the consumers fetch the scales of a stage as one 32-bit word");
+    static constexpr int ROWS = CW * RT * 16;          // <= 256 (TMA box)
+    static constexpr uint32_t PLANE = ROWS * 64;       // codes of one group
+    static constexpr uint32_t W_BYTES = PLANE * GPS;
+    static constexpr uint32_t XF_BYTES = 32 * 64;      // B fragments of one group: [4][32 lanes][16 B]
+    static constexpr uint32_t OFF_XF = W_BYTES;
+    static constexpr uint32_t OFF_XS = OFF_XF + XF_BYTES * GPS;  // X_g: [GPS][8] fp32
+    static constexpr uint32_t STAGE = (OFF_XS + 32 * GPS + 127) / 128 * 128;  // TMA destinations 128-byte aligned
+    static constexpr int RING = (kStreamRingBudget / STAGE) < 3 ? 3
+                                : (kStreamRingBudget / STAGE) > 8 ? 8 : (kStreamRingBudget / STAGE);
+    static constexpr uint32_t OFF_BAR = RING * STAGE;
     static constexpr size_t SMEM = 128 + OFF_BAR + 256;
+    static constexpr int THREADS = (CW + 1) * 32;
 };
 
 struct StreamBars {
-    uint64_t wfull[kGRing];
-    uint64_t wempty[kGRing];
-    uint64_t sfull[2];
-    uint64_t sempty[2];
+    uint64_t full[8];
+    uint64_t empty[8];
     int abort;
 };
-
-__device__ __forceinline__ void cp_async_4(uint32_t dst, const void *src) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
 
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
@@ -403,20 +405,33 @@ __device__ __forceinline__ uint4 lds128(uint32_t a) {
     return v;
 }
 
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+__device__ __forceinline__ float2 lds64f(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
     return v;
 }
 
-template <int RT>
-__global__ void __launch_bounds__((kConsumerWarps + 1) * 32)
-    gemv_w4a16_stream_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
-                             const __grid_constant__ CUtensorMap tmap_s, const uint32_t *__restrict__ qzeros, int N,
-                             int K, int B, int splits, uint16_t *__restrict__ y, unsigned int *status,
-                             uint64_t limit_ns) {
+__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+
+__device__ __forceinline__ void sts32f(uint32_t a, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+template <int CW, int RT, int GPS>
+__global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
+    gemv_w4a16_stream_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restrict__ x,
+                             const uint16_t *__restrict__ scales, const uint32_t *__restrict__ qzeros, int N, int K,
+                             int B, int splits, uint16_t *__restrict__ y, unsigned int *status, uint64_t limit_ns) {
     using namespace sm100;
-    using L = StreamLayout<RT>;
+    using L = StreamLayout<CW, RT, GPS>;
     extern __shared__ uint8_t stream_smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(stream_smem_raw) + 127) & ~uintptr_t(127));
     StreamBars *bar = reinterpret_cast<StreamBars *>(base + L::OFF_BAR);
@@ -425,25 +440,18 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32)
     const int rank = (int)blockIdx.x;
     const int n0 = blockIdx.y * L::ROWS;
     const int groups = K >> 7, zwords = (groups + 7) >> 3;
-    const int ng = groups / splits, g_begin = rank * ng, nsb = ng >> 3;
+    const int nst = groups / (splits * GPS);  // stages of this CTA
+    const int g_begin = rank * nst * GPS;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kGRing; ++s) {
-            mbar_init(smem_u32(&bar->wfull[s]), 1);
-            mbar_init(smem_u32(&bar->wempty[s]), kConsumerWarps);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(smem_u32(&bar->sfull[b]), 1 + 32);
-            mbar_init(smem_u32(&bar->sempty[b]), kConsumerWarps);
+        for (int s = 0; s < L::RING; ++s) {
+            mbar_init(smem_u32(&bar->full[s]), 1 + 32);  // TMA transaction + the producer lanes' fragment stores
+            mbar_init(smem_u32(&bar->empty[s]), CW);
         }
         bar->abort = 0;
         fence_mbar_init();
     }
-    if (threadIdx.x == kConsumerWarps * 32) {
-        prefetch_tmap(&tmap_w);
-        prefetch_tmap(&tmap_x);
-        prefetch_tmap(&tmap_s);
-    }
+    if (threadIdx.x == CW * 32) prefetch_tmap(&tmap_w);
     __syncthreads();
     const WaitCtl ctl{&bar->abort, status, limit_ns};
 
@@ -452,131 +460,180 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32)
     for (int i = 0; i < RT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
     const int t = lane & 3, r = lane >> 2;
 
-    if (warp == kConsumerWarps) {
+    if (warp == CW) {
         // ------------------------------------------------------------------ producer warp
-        int issued = 0, sblocks = 0;
-        bool ok = true;
-        for (int sb = 0; sb < nsb && ok; ++sb) {
-            const int b = sb & 1;
-            ok = __all_sync(0xffffffffu, wait_parity(smem_u32(&bar->sempty[b]), ((sb >> 1) & 1) ^ 1, ctl, 0x401));
-            if (!ok) break;
-            const int blk = (g_begin >> 3) + sb;
+        // Lane (r, t) prepares consumer lane (r, t)'s fragment: batch row r, the
+        // 32 values k = 32t .. 32t+31 of each group (the codes of the same k sit
+        // in that lane's 16 code bytes).
+        const bool has_row = r < B;
+        const uint16_t *xrow = x + (size_t)(has_row ? r : 0) * K + 32 * t;
+        uint4 xr[GPS][4];
+#pragma unroll
+        for (int q = 0; q < GPS; ++q)
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+                xr[q][v] = has_row ? __ldg(reinterpret_cast<const uint4 *>(xrow + (size_t)(g_begin + q) * 128 + 8 * v))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+        int issued = 0;
+        for (int i = 0; i < nst; ++i) {
+            const int s = i % L::RING, u = i / L::RING;
+            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&bar->empty[s]), (u & 1) ^ 1, ctl, 0x402))) break;
+            const uint32_t fb = smem_u32(&bar->full[s]);
+            const uint32_t st = sbase + s * L::STAGE;
+            const int g = g_begin + i * GPS;
             if (lane == 0) {
-                mbar_arrive_expect_tx(smem_u32(&bar->sfull[b]), L::S_BYTES);
-                tma_load_2d(sbase + L::OFF_S + b * L::S_BYTES, &tmap_s, smem_u32(&bar->sfull[b]), blk * 8, n0);
+                mbar_arrive_expect_tx(fb, L::W_BYTES);
+                // one 64-byte-pitch plane per group keeps the consumers' 16-byte loads conflict-free
+#pragma unroll
+                for (int q = 0; q < GPS; ++q) tma_load_2d(st + q * L::PLANE, &tmap_w, fb, (g + q) * 64, n0);
             }
-            for (int row = lane; row < L::ROWS; row += 32)
-                cp_async_4(sbase + L::OFF_Z + b * L::Z_BYTES + row * 4,
-                           qzeros + (size_t)min(n0 + row, N - 1) * zwords + blk);
-            cp_async_arrive_noinc(smem_u32(&bar->sfull[b]));
-            ++sblocks;
-            for (int gg = 0; gg < 8; ++gg) {
-                const int i = sb * 8 + gg, s = i % kGRing, u = i / kGRing;
-                if (lane == 0) {
-                    if (!wait_parity(smem_u32(&bar->wempty[s]), (u & 1) ^ 1, ctl, 0x402)) {
-                        ok = false;
-                    } else {
-                        const uint32_t fb = smem_u32(&bar->wfull[s]);
-                        mbar_arrive_expect_tx(fb, L::STAGE);
-                        tma_load_2d(sbase + s * L::STAGE, &tmap_w, fb, (g_begin + i) * 64, n0);
-                        tma_load_2d(sbase + s * L::STAGE + L::W_BYTES, &tmap_x, fb, (g_begin + i) * 128, 0);
-                        ++issued;
-                    }
+            ++issued;
+#pragma unroll
+            for (int q = 0; q < GPS; ++q) {
+                // fragment k-step 2j: (x0,x4) and 2^-4 (x1,x5) of chunk j; k-step 2j+1: (x2,x6) and 2^-4 (x3,x7)
+                float sum0 = 0.0f, sum1 = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 c = xr[q][j];
+                    sts128(st + L::OFF_XF + q * L::XF_BYTES + j * 512 + lane * 16, prmt_u(c.x, c.z, 0x5410u),
+                           hmul2_u(prmt_u(c.x, c.z, 0x7632u), 0x2C002C00u), prmt_u(c.y, c.w, 0x5410u),
+                           hmul2_u(prmt_u(c.y, c.w, 0x7632u), 0x2C002C00u));
+                    const float2 f0 = half2_bits_to_float2(c.x), f1 = half2_bits_to_float2(c.y);
+                    const float2 f2 = half2_bits_to_float2(c.z), f3 = half2_bits_to_float2(c.w);
+                    sum0 += (f0.x + f1.x) + (f2.x + f3.x);
+                    sum1 += (f0.y + f1.y) + (f2.y + f3.y);
                 }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok) break;
+                float xg = sum0 + sum1;
+                xg += __shfl_xor_sync(0xffffffffu, xg, 1);
+                xg += __shfl_xor_sync(0xffffffffu, xg, 2);
+                if (t == 0) sts32f(st + L::OFF_XS + q * 32 + r * 4, xg);  // X_g of batch r
+            }
+            mbar_arrive(fb);  // release: the fragments are visible to the consumers' acquire
+            if (i + 1 < nst) {  // the next stage's x, in flight while this warp waits for a free slot
+                const int gn = g + GPS;
+#pragma unroll
+                for (int q = 0; q < GPS; ++q)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        xr[q][v] = has_row
+                                       ? __ldg(reinterpret_cast<const uint4 *>(xrow + (size_t)(gn + q) * 128 + 8 * v))
+                                       : make_uint4(0u, 0u, 0u, 0u);
             }
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");
         if (lane == 0 && bar->abort) {
-            for (int s = 0; s < kGRing; ++s) {
-                const int uses = issued > s ? (issued - s - 1) / kGRing + 1 : 0;
-                if (uses) drain_parity(smem_u32(&bar->wfull[s]), (uses - 1) & 1, 2000000000ull, status, 0x410);
-            }
-            for (int b = 0; b < 2; ++b) {
-                const int uses = sblocks > b ? (sblocks - b - 1) / 2 + 1 : 0;
-                if (uses) drain_parity(smem_u32(&bar->sfull[b]), (uses - 1) & 1, 2000000000ull, status, 0x410);
+            for (int s = 0; s < L::RING; ++s) {
+                const int uses = issued > s ? (issued - s - 1) / L::RING + 1 : 0;
+                if (uses) drain_parity(smem_u32(&bar->full[s]), (uses - 1) & 1, 2000000000ull, status, 0x410);
             }
         }
     } else {
         // ------------------------------------------------------------------ consumer warps
         const int wrow = warp * RT * 16;
-        bool ok = true;
-        for (int sb = 0; sb < nsb && ok; ++sb) {
-            const int b = sb & 1;
-            ok = __all_sync(0xffffffffu, wait_parity(smem_u32(&bar->sfull[b]), (sb >> 1) & 1, ctl, 0x404));
-            if (!ok) break;
-            uint4 sreg[RT][2];
-            uint32_t zreg[RT][2];
+        // this lane's rows are nl + 8 (2i + h); rows past N read no scales and are never stored
+        const int nl = n0 + wrow + r;
+        const uint16_t *srow = scales + (size_t)min(nl, N - 1) * groups;
+        const uint32_t *zrow = qzeros + (size_t)min(nl, N - 1) * zwords;
+        const size_t sstep = (size_t)8 * groups, zstep = (size_t)8 * zwords;
+        // Scales and zero-point words travel per block of 4 stages (8 groups, one
+        // zero word per row): lane t of a row quad holds the scale pair of the
+        // block's stage t and hands it to its quad by shuffle, so a warp reads each
+        // row's 16 scale bytes with one sector request.  The next block's words are
+        // in flight while the current block is processed.
+        const int nblk = (nst + 3) >> 2;
+        uint32_t sw[RT][2], zw[RT][2], swn[RT][2], zwn[RT][2];
+        auto fetch = [&](int blk, uint32_t (&sv)[RT][2], uint32_t (&zv)[RT][2]) {
+            const int g0 = g_begin + blk * 8;
+            const int gs = min(g0 + 2 * t, g_begin + 2 * (nst - 1));  // stage t of the block, clamped
 #pragma unroll
             for (int i = 0; i < RT; ++i)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int row = wrow + 16 * i + r + 8 * h;
-                    sreg[i][h] = lds128(sbase + L::OFF_S + b * L::S_BYTES + row * 16);
-                    zreg[i][h] = lds32(sbase + L::OFF_Z + b * L::Z_BYTES + row * 4);
+                    const bool in = nl + 16 * i + 8 * h < N;
+                    sv[i][h] = in ? __ldg(reinterpret_cast<const uint32_t *>(srow + (2 * i + h) * sstep + gs)) : 0u;
+                    zv[i][h] = in ? __ldg(zrow + (2 * i + h) * zstep + (g0 >> 3)) : 0u;
                 }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bar->sempty[b]));
-#pragma unroll
-            for (int gg = 0; gg < 8; ++gg) {
-                const int i_st = sb * 8 + gg, s = i_st % kGRing, u = i_st / kGRing;
-                ok = __all_sync(0xffffffffu, wait_parity(smem_u32(&bar->wfull[s]), u & 1, ctl, 0x408));
-                if (!ok) break;
-                const uint32_t st = sbase + s * L::STAGE;
-                uint4 xv[4];
-#pragma unroll
-                for (int v = 0; v < 4; ++v) xv[v] = lds128(st + L::W_BYTES + r * 256 + t * 64 + v * 16);
-                uint4 wv[RT][2];
+        };
+        fetch(0, sw, zw);
+        bool ok = true;
+#pragma unroll 1
+        for (int blk = 0; blk < nblk && ok; ++blk) {
+            fetch(blk + 1 < nblk ? blk + 1 : blk, swn, zwn);
+#pragma unroll 1
+            for (int gs = 0; gs < 4; ++gs) {
+                const int it = blk * 4 + gs;
+                if (it >= nst) break;
+                const int s = it % L::RING, u = it / L::RING;
+                const int g = g_begin + it * GPS;
+                uint32_t scw[RT][2];
 #pragma unroll
                 for (int i = 0; i < RT; ++i)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) wv[i][h] = lds128(st + (wrow + 16 * i + r + 8 * h) * 64 + t * 16);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_u32(&bar->wempty[s]));
-                uint32_t bf[8][2];
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    bf[2 * j][0] = prmt_u(xv[j].x, xv[j].z, 0x5410u);
-                    bf[2 * j][1] = prmt_u(xv[j].x, xv[j].z, 0x7632u);
-                    bf[2 * j + 1][0] = prmt_u(xv[j].y, xv[j].w, 0x5410u);
-                    bf[2 * j + 1][1] = prmt_u(xv[j].y, xv[j].w, 0x7632u);
+                    for (int h = 0; h < 2; ++h) scw[i][h] = __shfl_sync(0xffffffffu, sw[i][h], (lane & ~3) | gs);
+                if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&bar->full[s]), u & 1, ctl, 0x408))) {
+                    ok = false;
+                    break;
                 }
+                const uint32_t st = sbase + s * L::STAGE;
+                const int zsh = 4 * (g & 7);
+                // one group at a time (half the live fragments); the stage is released
+                // once the last group's operands are in registers
 #pragma unroll
-                for (int i = 0; i < RT; ++i) {
-                    const uint32_t z0 = (zreg[i][0] >> (4 * gg)) & 0xFu, z1 = (zreg[i][1] >> (4 * gg)) & 0xFu;
-                    const uint32_t zlo0 = 0xE400E400u + z0 * 0x00010001u, zhi0 = 0xD400D400u + z0 * 0x00100010u;
-                    const uint32_t zlo1 = 0xE400E400u + z1 * 0x00010001u, zhi1 = 0xD400D400u + z1 * 0x00100010u;
-                    float ce[4] = {0.0f, 0.0f, 0.0f, 0.0f}, co[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                    const uint32_t wa[4] = {wv[i][0].x, wv[i][0].y, wv[i][0].z, wv[i][0].w};
-                    const uint32_t wb[4] = {wv[i][1].x, wv[i][1].y, wv[i][1].z, wv[i][1].w};
+                for (int q = 0; q < GPS; ++q) {
+                    uint4 xv[4];
+                    uint4 wv[RT][2];
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        uint32_t pa[4], pb[4];
-                        dequant_pairs(wa[j], zlo0, zhi0, pa);
-                        dequant_pairs(wb[j], zlo1, zhi1, pb);
-                        const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
-                        const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
-                        mma_16816(ce, a0, bf[2 * j][0], bf[2 * j][1]);
-                        mma_16816(co, a1, bf[2 * j + 1][0], bf[2 * j + 1][1]);
+                    for (int v = 0; v < 4; ++v) xv[v] = lds128(st + L::OFF_XF + q * L::XF_BYTES + v * 512 + lane * 16);
+                    const float2 xg = lds64f(st + L::OFF_XS + q * 32 + t * 8);  // X_g of batches 2t, 2t+1
+#pragma unroll
+                    for (int i = 0; i < RT; ++i)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            wv[i][h] = lds128(st + q * L::PLANE + (wrow + 16 * i + r + 8 * h) * 64 + t * 16);
+                    if (q == GPS - 1) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(smem_u32(&bar->empty[s]));
                     }
-                    const uint32_t sw0 = gg < 2 ? sreg[i][0].x : gg < 4 ? sreg[i][0].y : gg < 6 ? sreg[i][0].z : sreg[i][0].w;
-                    const uint32_t sw1 = gg < 2 ? sreg[i][1].x : gg < 4 ? sreg[i][1].y : gg < 6 ? sreg[i][1].z : sreg[i][1].w;
-                    const float s0 = half_bits_to_float((uint16_t)((gg & 1) ? (sw0 >> 16) : (sw0 & 0xFFFFu)));
-                    const float s1 = half_bits_to_float((uint16_t)((gg & 1) ? (sw1 >> 16) : (sw1 & 0xFFFFu)));
-                    acc[i][0] = fmaf(s0, ce[0] + co[0], acc[i][0]);
-                    acc[i][1] = fmaf(s0, ce[1] + co[1], acc[i][1]);
-                    acc[i][2] = fmaf(s1, ce[2] + co[2], acc[i][2]);
-                    acc[i][3] = fmaf(s1, ce[3] + co[3], acc[i][3]);
+#pragma unroll
+                    for (int i = 0; i < RT; ++i) {
+                        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+                        const uint32_t wa[4] = {wv[i][0].x, wv[i][0].y, wv[i][0].z, wv[i][0].w};
+                        const uint32_t wb[4] = {wv[i][1].x, wv[i][1].y, wv[i][1].z, wv[i][1].w};
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint32_t a8 = wa[j] >> 8, b8 = wb[j] >> 8;
+                            const uint32_t a0[4] = {wa[j] & 0x000F000Fu, wb[j] & 0x000F000Fu, wa[j] & 0x00F000F0u,
+                                                    wb[j] & 0x00F000F0u};
+                            const uint32_t a1[4] = {a8 & 0x000F000Fu, b8 & 0x000F000Fu, a8 & 0x00F000F0u,
+                                                    b8 & 0x00F000F0u};
+                            mma_16816(d, a0, xv[j].x, xv[j].y);
+                            mma_16816(d, a1, xv[j].z, xv[j].w);
+                        }
+                        const float s0 = half_bits_to_float((uint16_t)(scw[i][0] >> (16 * q)));
+                        const float s1 = half_bits_to_float((uint16_t)(scw[i][1] >> (16 * q)));
+                        const float z0 = (float)((zw[i][0] >> (zsh + 4 * q)) & 0xFu);
+                        const float z1 = (float)((zw[i][1] >> (zsh + 4 * q)) & 0xFu);
+                        const float a0s = s0 * 16777216.0f, a1s = s1 * 16777216.0f;  // exact: times 2^24
+                        const float b0s = -s0 * z0, b1s = -s1 * z1;                  // exact: fp16 x 4-bit integer
+                        acc[i][0] = fmaf(a0s, d[0], fmaf(b0s, xg.x, acc[i][0]));
+                        acc[i][1] = fmaf(a0s, d[1], fmaf(b0s, xg.y, acc[i][1]));
+                        acc[i][2] = fmaf(a1s, d[2], fmaf(b1s, xg.x, acc[i][2]));
+                        acc[i][3] = fmaf(a1s, d[3], fmaf(b1s, xg.y, acc[i][3]));
+                    }
                 }
             }
+#pragma unroll
+            for (int i = 0; i < RT; ++i)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    sw[i][h] = swn[i][h];
+                    zw[i][h] = zwn[i][h];
+                }
         }
     }
 
     // ---------------------------------------------------------------------- results
-    const bool cons = warp < kConsumerWarps;
+    const bool cons = warp < CW;
     const int wrow = warp * RT * 16;
     if (splits == 1) {
         if (cons && !bar->abort) {
@@ -629,26 +686,22 @@ __global__ void __launch_bounds__((kConsumerWarps + 1) * 32)
     }
 }
 
-template <int RT>
+template <int CW, int RT, int GPS>
 wq_status launch_stream(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
                         int K, int splits, uint16_t *y, cudaStream_t st) {
-    using L = StreamLayout<RT>;
+    using L = StreamLayout<CW, RT, GPS>;
     unsigned int *status = device_status_word();
     if (!status) return WQ_ERR_CUDA;
-    CUtensorMap tw, tx, ts;
+    CUtensorMap tw;
     if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qw, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 64,
-                        L::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, (uint64_t)K, (uint64_t)B, (uint64_t)K * 2, 128, 8,
-                        CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !encode_tmap_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, sc, (uint64_t)K / 128, (uint64_t)N,
-                        (uint64_t)K / 64, 8, L::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
+                        L::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
         return WQ_ERR_CUDA;
-    auto kern = gemv_w4a16_stream_kernel<RT>;
+    auto kern = gemv_w4a16_stream_kernel<CW, RT, GPS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
     if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_gemv_w4a16: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(splits, (N + L::ROWS - 1) / L::ROWS, 1);
-    cfg.blockDim = dim3((kConsumerWarps + 1) * 32);
+    cfg.blockDim = dim3(L::THREADS);
     cfg.dynamicSmemBytes = L::SMEM;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -658,42 +711,46 @@ wq_status launch_stream(const uint16_t *x, int B, const uint32_t *qw, const uint
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, tw, tx, ts, qz, N, K, B, splits, y, status, wait_limit());
+    e = cudaLaunchKernelEx(&cfg, kern, tw, x, sc, qz, N, K, B, splits, y, status, wait_limit());
     if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_gemv_w4a16: launch failed: %s", cudaGetErrorString(e));
     return WQ_OK;
 }
 
-// Tile height (RT) and K split of the streaming GEMV: the cluster size divides
-// K/1024 (whole blocks of 8 groups per CTA), at most 8, and the partial results
-// fit the leading CTA's ring; the choice fills the SMs' CTA slots in the fewest,
-// fullest waves, preferring the taller tile (fewer x fragments per weight).
-wq_status gemv_stream(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
-                      int K, uint16_t *y, cudaStream_t st) {
-    const int blocks8 = K / 1024;
-    const int sms = num_sms();
-    int best_rt = 1, best_s = 1;
-    double best = -1.0;
-    for (int rt = 2; rt >= 1; --rt) {
-        const int rows = kConsumerWarps * rt * 16;
-        const size_t smem = rt == 2 ? StreamLayout<2>::SMEM : StreamLayout<1>::SMEM;
-        const size_t ring = rt == 2 ? (size_t)StreamLayout<2>::OFF_S : (size_t)StreamLayout<1>::OFF_S;
-        const int per_sm = (int)std::min<size_t>(2048 / ((kConsumerWarps + 1) * 32), 227 * 1024 / smem);
-        const int tiles = (N + rows - 1) / rows;
-        for (int s = 1; s <= 8; ++s) {
-            if (blocks8 % s) continue;
-            if ((size_t)(s - 1) * rows * 8 * 4 > ring) continue;
-            const double waves = (double)tiles * s / ((double)sms * per_sm);
-            double score = waves / std::ceil(waves) + (rt == 2 ? 0.03 : 0.0) - 0.002 * s;
-            if (waves < 0.5) score -= 1.0;  // leaves most SMs idle
-            if (score > best) {
-                best = score;
-                best_rt = rt;
-                best_s = s;
-            }
+// Tile height and K split of the streaming GEMV.  Two CTAs are resident per
+// SM; the split (cluster size, at most 8, dividing the stage count, partials
+// fitting the leading CTA's ring) is the smallest one that reaches the best
+// fill of those slots over whole waves.  The 256-row tile (4 consumer warps x
+// 4 m-tiles) is the fastest on B200; the 128-row tile serves matrices with too
+// few 256-row tiles.
+template <typename L>
+int stream_splits(int N, int K, int sms) {
+    const int tiles = (N + L::ROWS - 1) / L::ROWS;
+    const long long slots = 2ll * sms;
+    int best = 1;
+    double best_fill = 0.0;
+    for (int s = 1; s <= 8; ++s) {
+        if (s > 1 && (K / 128) % (8 * s)) continue;  // every CTA starts on a zero-point word
+        if ((size_t)(s - 1) * L::ROWS * 8 * 4 > L::OFF_BAR) continue;
+        const long long ctas = (long long)tiles * s;
+        const long long waves = (ctas + slots - 1) / slots;
+        const double fill = (double)ctas / (double)(waves * slots);
+        if (fill > best_fill + 1e-9) {
+            best_fill = fill;
+            best = s;
         }
     }
-    return best_rt == 2 ? launch_stream<2>(x, B, qw, sc, qz, N, K, best_s, y, st)
-                        : launch_stream<1>(x, B, qw, sc, qz, N, K, best_s, y, st);
+    return best;
+}
+
+wq_status gemv_stream(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
+                      int K, uint16_t *y, cudaStream_t st) {
+    const int sms = num_sms();
+    using Big = StreamLayout<4, 4, 2>;
+    using Small = StreamLayout<4, 2, 2>;
+    const int tiles_big = (N + Big::ROWS - 1) / Big::ROWS;
+    if (tiles_big * 8 >= 2 * sms)
+        return launch_stream<4, 4, 2>(x, B, qw, sc, qz, N, K, stream_splits<Big>(N, K, sms), y, st);
+    return launch_stream<4, 2, 2>(x, B, qw, sc, qz, N, K, stream_splits<Small>(N, K, sms), y, st);
 }
 
 template <int RT>
@@ -741,7 +798,7 @@ extern "C" wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qwe
                "wq_gemv_w4a16: K (%d) must be a multiple of group_size (%d)", K, group_size);
     cudaStream_t st = wq::as_stream(stream);
     cudaError_t e;
-    if (group_size == 128 && K % 1024 == 0) return wq::gemv_stream(x, B, qweight, scales, qzeros, N, K, y, st);
+    if (group_size == 128 && K % 256 == 0) return wq::gemv_stream(x, B, qweight, scales, qzeros, N, K, y, st);
     if (group_size == 128) {
         // Two 16-row MMA tiles per CTA when that still gives every SM several CTAs.
         const long long blocks2 = (N + 31) / 32;

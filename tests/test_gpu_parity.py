@@ -102,6 +102,7 @@ GEMV_SMALL = [  # (N, K, g, B)
     (1, 128, 128, 1), (17, 384, 128, 1), (33, 1024, 128, 3), (64, 1536, 128, 8),
     (9, 96, 32, 2), (40, 640, 64, 4), (13, 2048, 256, 5), (300, 4096, 128, 1),
     (3000, 2048, 128, 1), (3000, 2048, 128, 8), (2500, 512, 128, 6), (129, 7168, 128, 7),
+    (77, 256, 128, 4), (520, 1280, 128, 2), (4100, 768, 128, 8), (1000, 3328, 128, 3),
 ]
 
 
