@@ -17,7 +17,7 @@ import os
 import torch
 
 __all__ = ["WQError", "lib", "quantize_group_int4", "quantize_int8_per_channel", "quantize_int8_per_token",
-           "smooth", "smooth_workspace_bytes", "gemv_w4a16", "gemm_w4a16", "gemm_w8a8", "gemv_w8a16",
+           "smooth", "smooth_workspace_bytes", "smooth_noalloc", "gemv_w4a16", "gemm_w4a16", "gemm_w8a8", "gemv_w8a16",
            "matmul_w4a16", "device_status", "set_wait_limit", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwq.so")
@@ -45,6 +45,7 @@ _SIGS = {
     "wq_quantize_int8_per_channel": [_P, _I, _I, _P, _P, _P, _P],
     "wq_quantize_int8_per_token": [_P, _I, _I, _P, _P, _P, _P],
     "wq_smooth": [_P, _I, _P, _I, _I, _F, _P, _P, _P],
+    "wq_smooth_noalloc": [_P, _I, _P, _I, _I, _F, _P, _P],
     "wq_gemv_w4a16": [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P],
     "wq_gemm_w4a16": [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P],
     "wq_gemm_w8a8": [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P],
@@ -156,6 +157,32 @@ def smooth(x: torch.Tensor, w: torch.Tensor, alpha: float = 0.5, workspace: torc
         raise ValueError("workspace too small")
     _check(lib.wq_smooth(_ptr(x), M, _ptr(w), N, K, float(alpha), _ptr(s), _ptr(workspace), _P(_stream(stream))),
            "wq_smooth")
+    return s
+
+
+SMOOTH_NOALLOC_MAX_K = 65536
+
+
+def smooth_noalloc(x: torch.Tensor, w: torch.Tensor, alpha: float = 0.5, s: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """`smooth` through the entry point that allocates no device memory in the library call.
+
+    The workspace is the library's built-in device array (K <= SMOOTH_NOALLOC_MAX_K); pass `s`
+    (fp32 [K], on x's device) to keep this wrapper allocation-free as well.  Calls that overlap
+    on the GPU share that array and race."""
+    _cuda(x, "x", (torch.float16,), 2)
+    _cuda(w, "w", (torch.float16,), 2)
+    M, K = x.shape
+    N, K2 = w.shape
+    if K != K2:
+        raise ValueError("x and w must share K")
+    if s is None:
+        s = _empty((K,), torch.float32, x)
+    _cuda(s, "s", (torch.float32,), 1)
+    if s.numel() != K:
+        raise ValueError("s must have K elements")
+    _check(lib.wq_smooth_noalloc(_ptr(x), M, _ptr(w), N, K, float(alpha), _ptr(s), _P(_stream(stream))),
+           "wq_smooth_noalloc")
     return s
 
 

@@ -147,3 +147,64 @@ extern "C" wq_status wq_smooth(const uint16_t *x, int M, const uint16_t *w, int 
                                                       total);
     return wq::check_launch("wq_smooth");
 }
+
+// ---------------------------------------------------------------------------
+// Allocation-free smoothing.
+//
+// Some callers cannot allocate device memory for the workspace: a plug-in that
+// runs inside a host engine which owns all device memory and exposes no
+// allocator, or a latency-critical path where cudaMalloc's implicit device
+// synchronization is not allowed.  wq_smooth_noalloc gives them the same
+// computation with the workspace in a fixed-size array that the library keeps
+// in device memory (every GPU that loads the library holds it until the
+// process exits).  Host code cannot use the array's name as a device address,
+// so the device address is looked up once per device with cudaGetSymbolAddress
+// (on the first call made while that device is current) and cached.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace wq {
+namespace {
+
+constexpr size_t kNoAllocWords = 2 * (size_t)WQ_SMOOTH_NOALLOC_MAX_K + 4;  // ax | aw | ticket, K padded to 4
+static __device__ __align__(256) unsigned int g_smooth_scratch[kNoAllocWords];
+
+constexpr int kScratchDevices = 64;
+std::mutex g_scratch_mu;
+unsigned int *g_scratch_ptr[kScratchDevices];
+
+unsigned int *smooth_scratch() {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= kScratchDevices) {
+        fail(WQ_ERR_CUDA, "wq_smooth_noalloc: cudaGetDevice failed");
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_smooth_scratch);
+        if (e != cudaSuccess) {
+            fail(WQ_ERR_CUDA, "wq_smooth_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+            return nullptr;
+        }
+        g_scratch_ptr[dev] = static_cast<unsigned int *>(p);
+    }
+    return g_scratch_ptr[dev];
+}
+
+}  // namespace
+}  // namespace wq
+
+extern "C" wq_status wq_smooth_noalloc(const uint16_t *x, int M, const uint16_t *w, int N, int K, float alpha,
+                                       float *s, void *stream) {
+    WQ_REQUIRE(K <= WQ_SMOOTH_NOALLOC_MAX_K, WQ_ERR_UNSUPPORTED,
+               "wq_smooth_noalloc: K (%d) exceeds the built-in workspace (K <= %d); use wq_smooth with a "
+               "caller-owned workspace",
+               K, WQ_SMOOTH_NOALLOC_MAX_K);
+    WQ_REQUIRE(K > 0, WQ_ERR_INVALID_ARG, "wq_smooth_noalloc: K must be positive (K=%d)", K);
+    unsigned int *scratch = wq::smooth_scratch();
+    if (!scratch) return WQ_ERR_CUDA;
+    // wq_smooth clears the part of the workspace that must start at zero.
+    return wq_smooth(x, M, w, N, K, alpha, s, scratch, stream);
+}

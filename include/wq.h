@@ -131,6 +131,30 @@ wq_status wq_smooth(const uint16_t *x, int M, const uint16_t *w, int N, int K, f
                     float *s, void *workspace, void *stream);
 
 /*
+ * wq_smooth without a caller-provided workspace.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory themselves (a plug-in inside a host engine that owns all
+ * device memory and offers no allocator, or a latency-critical path that may
+ * not call cudaMalloc because of its implicit device synchronization).
+ * Same arguments, result and restrictions as wq_smooth, plus K <=
+ * WQ_SMOOTH_NOALLOC_MAX_K (larger K returns WQ_ERR_UNSUPPORTED and launches
+ * nothing).
+ * The workspace is a fixed array of 2 * WQ_SMOOTH_NOALLOC_MAX_K + 4 words
+ * (512 KiB) held in the device memory of every GPU that loads the library,
+ * until the process exits.  The call allocates nothing: no cudaMalloc, no
+ * cudaFree, no allocating library routine.  The first call on a device (made
+ * while that device is current) looks up the array's device address with
+ * cudaGetSymbolAddress and caches it; make that first call before any stream
+ * capture.  All calls on a device share the one array, which keeps the last
+ * call's contents (each call clears what must start at zero), so calls that
+ * overlap on the GPU (concurrent streams, several host threads) race and
+ * give wrong results: order them on one stream or with events.
+ */
+#define WQ_SMOOTH_NOALLOC_MAX_K 65536
+wq_status wq_smooth_noalloc(const uint16_t *x, int M, const uint16_t *w, int N, int K, float alpha,
+                            float *s, void *stream);
+
+/*
  * Fused dequantize + GEMV, W4A16, for decode batches B = 1..8.  Source: [P1]
  * "Inference view" (weights unpacked in registers, multiplied by their
  * scales), [P3] "Scale and zero-point" (w^ = (q - z) s), [P5] "Why It Is
