@@ -357,19 +357,23 @@ def run_gpu(args):
 
 
 def run_e2e(torch, wq, step, steps, stream):
+    """Both batch-1 GEMVs through the public API, with the step's activations copied in from
+    pinned host memory (one copy) and both results read back (one copy) every step."""
     ins, qB = step.ins, step.qB
-    hx = {t: ins[f"x1_{t}"].cpu().pin_memory() for t in ("up", "down")}
-    hy = {t: torch.empty((1, (UP if t == "up" else DOWN)[0]), dtype=torch.float16).pin_memory()
-          for t in ("up", "down")}
-    dx = {t: torch.empty_like(ins[f"x1_{t}"]) for t in ("up", "down")}
-    dy = {t: torch.empty((1, (UP if t == "up" else DOWN)[0]), dtype=torch.float16, device=ins["X5"].device)
-          for t in ("up", "down")}
+    kx = {"up": UP[1], "down": DOWN[1]}
+    ny = {"up": UP[0], "down": DOWN[0]}
+    hx = torch.cat([ins["x1_up"].reshape(-1), ins["x1_down"].reshape(-1)]).cpu().pin_memory()
+    hy = torch.empty(ny["up"] + ny["down"], dtype=torch.float16).pin_memory()
+    dx = torch.empty_like(hx, device=ins["X5"].device)
+    dy = torch.empty(hy.numel(), dtype=torch.float16, device=ins["X5"].device)
+    xv = {"up": dx[:kx["up"]].view(1, -1), "down": dx[kx["up"]:].view(1, -1)}
+    yv = {"up": dy[:ny["up"]].view(1, -1), "down": dy[ny["up"]:].view(1, -1)}
 
     def one():
+        dx.copy_(hx, non_blocking=True)
         for t in ("up", "down"):
-            dx[t].copy_(hx[t], non_blocking=True)
-            wq.gemv_w4a16(dx[t], *qB[t], 128, out=dy[t])
-            hy[t].copy_(dy[t], non_blocking=True)
+            wq.gemv_w4a16(xv[t], *qB[t], 128, out=yv[t])
+        hy.copy_(dy, non_blocking=True)
 
     for _ in range(3):
         one()
@@ -383,11 +387,10 @@ def run_e2e(torch, wq, step, steps, stream):
     t = s.elapsed_time(e) * 1e-3
     w = work_table()
     byts = w["gemv_w4a16_b1_up"]["bytes"] + w["gemv_w4a16_b1_down"]["bytes"]
-    h2d = sum(hx[t].numel() * 2 for t in hx)
-    d2h = sum(hy[t].numel() * 2 for t in hy)
-    return {"value": round(byts * steps / t / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "what": "batch-1 W4A16 GEMV on both weights via the Python/C API, "
-                                              "x copied from pinned host memory and y read back each step"}
+    return {"value": round(byts * steps / t / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": hx.numel() * 2,
+            "d2h_bytes_per_step": hy.numel() * 2,
+            "what": "batch-1 W4A16 GEMV on both weights via the Python/C API, x copied from pinned host memory "
+                    "and y read back each step (one copy each way)"}
 
 
 def load_traffic(kernel):
@@ -459,6 +462,29 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_profile_case(args):
+    """Runs one named kernel of the step `--profile-launches` times on the step's inputs and
+    prints nothing: the command that ncu captures for the per-kernel summaries."""
+    import torch
+    import bit_gemv_gemm_group_b200 as wq
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    step = Step(torch, wq, make_inputs(torch, dev))
+    launches = dict(step.launches())
+    if args.profile_case not in launches:
+        raise SystemExit(f"unknown kernel {args.profile_case!r}; one of {sorted(launches)}")
+    for name in ("smooth", "quant_int8_pc_smooth", "quant_int8_pt_smooth"):  # producers of the W8A8 operands
+        if args.profile_case in ("quant_int8_pc_smooth", "quant_int8_pt_smooth", "gemm_w8a8") and name != args.profile_case:
+            launches[name]()
+    torch.cuda.synchronize()
+    for _ in range(args.profile_launches):
+        launches[args.profile_case]()
+    torch.cuda.synchronize()
+    if wq.device_status() != 0:
+        raise RuntimeError("a kernel reported a wait timeout")
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -467,7 +493,13 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["wq", "reference"], default="wq")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="size of the CPU oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-case", default=None,
+                    help="run only this kernel of the step (e.g. gemv_w4a16_b1_up) for an ncu capture; no output")
+    ap.add_argument("--profile-launches", type=int, default=3)
     args = ap.parse_args(argv)
+    if args.profile_case:
+        run_profile_case(args)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     if args.impl == "reference":

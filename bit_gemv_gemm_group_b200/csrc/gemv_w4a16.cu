@@ -346,18 +346,18 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_w4a16_mma_kernel(const ui
 }
 
 // ---------------------------------------------------------------------------
-// Streaming GEMV for K % 256 == 0 (the decode shapes).
+// Streaming GEMV for K % 256 == 0 (the decode shapes), batch 1..8*NT.
 //
 // Memory side: one producer warp per CTA streams the CTA tile's codes through
-// a shared-memory ring (2-D TMA, one ROWS x 64-byte plane per group, GPS
+// a shared-memory ring (2-D TMA, one ROWS x 64-byte plane per group, two
 // groups per stage).  The same warp turns x into the MMA's B fragments once
-// per CTA: each producer lane loads the 32 x values that consumer lane
-// `lane` needs for a group, permutes them into fragment order and stores them
-// lane-major (conflict-free 16-byte loads for every consumer warp), and adds
-// them up into the group sum X_g of its batch row.  The consumers fetch the
-// fp16 scales and zero-point words of their own rows from global memory one
-// block of 8 groups ahead; the CTA's shared memory is the ring alone, so two
-// CTAs fit on an SM and two consumer warps share each SM sub-partition.
+// per CTA: each producer lane loads the 32 x values that consumer lane `lane`
+// needs for a group (per n-tile of 8 batch rows), permutes them into fragment
+// order and stores them lane-major (conflict-free 16-byte loads for every
+// consumer warp), and adds them up into the group sum X_g of its batch row.
+// The consumers fetch the fp16 scales and zero-point words of their own rows
+// from global memory one block of 8 groups ahead; the CTA's shared memory is
+// the ring alone, so two CTAs fit on an SM.
 //
 // Compute side (warp-level mma.sync m16n8k16, batch = N): the codes go into
 // the A fragment as fp16 *subnormals*.  Masking a word with 0x000F000F leaves
@@ -366,31 +366,33 @@ __global__ void __launch_bounds__(kMmaWarps * 32) gemv_w4a16_mma_kernel(const ui
 // subtraction; the MMA multiplies them exactly.  The x lanes that meet the
 // 2^-20 codes are pre-scaled by 2^-4 (exact for |x| >= 2^-10, below that the
 // rounding is far inside the tolerance), so one MMA chain accumulates
-// D = 2^-24 sum_k q x in fp32, and the zero point enters per group through
-// X_g:  y += s (2^24 D - z X_g).
-// Each consumer warp owns RT m-tiles (RT independent MMA chains).  K is split
-// over a thread-block cluster (DSMEM reduction into the leading CTA) when the
-// tiles alone would leave SMs idle.  A consumer makes its shared-memory reads
-// visible to the async proxy (fence.proxy.async) before releasing a stage for
-// the next TMA write.
+// D = 2^-24 sum_k q x in fp32.  With X'_g = 2^-24 X_g (scaled by the
+// producer) a group adds s (D - z X'_g) to the accumulator, and the result is
+// scaled by 2^24 once at the end: y = 2^24 sum_g s_g (D_g - z_g X'_g).
+// Each consumer warp owns RT m-tiles and NT n-tiles (RT*NT independent MMA
+// chains, interleaved).  K is split over a thread-block cluster (DSMEM
+// reduction into the leading CTA) when the tiles alone would leave SMs idle.
+// A consumer makes its shared-memory reads visible to the async proxy
+// (fence.proxy.async) before releasing a stage for the next TMA write.
 // ---------------------------------------------------------------------------
 constexpr uint32_t kStreamRingBudget = 110 * 1024;  // two CTAs per SM (228 KB, 1 KB reserved per CTA)
+constexpr int kGPS = 2;                              // groups per stage (scales fetched as one 32-bit pair)
 
-template <int CW, int RT, int GPS>
+template <int CW, int RT, int NT>
 struct StreamLayout {
-    static_assert(GPS == 2, "the consumers fetch the scales of a stage as one 32-bit word");
     static constexpr int ROWS = CW * RT * 16;          // <= 256 (TMA box)
     static constexpr uint32_t PLANE = ROWS * 64;       // codes of one group
-    static constexpr uint32_t W_BYTES = PLANE * GPS;
-    static constexpr uint32_t XF_BYTES = 32 * 64;      // B fragments of one group: [4][32 lanes][16 B]
+    static constexpr uint32_t W_BYTES = PLANE * kGPS;
+    static constexpr uint32_t XF_BYTES = NT * 32 * 64; // B fragments of one group: [NT][4][32 lanes][16 B]
     static constexpr uint32_t OFF_XF = W_BYTES;
-    static constexpr uint32_t OFF_XS = OFF_XF + XF_BYTES * GPS;  // X_g: [GPS][8] fp32
-    static constexpr uint32_t STAGE = (OFF_XS + 32 * GPS + 127) / 128 * 128;  // TMA destinations 128-byte aligned
+    static constexpr uint32_t OFF_XS = OFF_XF + XF_BYTES * kGPS;  // X'_g: [kGPS][8 * NT] fp32
+    static constexpr uint32_t STAGE = (OFF_XS + 32 * NT * kGPS + 127) / 128 * 128;  // 128-byte aligned TMA
     static constexpr int RING = (kStreamRingBudget / STAGE) < 3 ? 3
                                 : (kStreamRingBudget / STAGE) > 8 ? 8 : (kStreamRingBudget / STAGE);
     static constexpr uint32_t OFF_BAR = RING * STAGE;
     static constexpr size_t SMEM = 128 + OFF_BAR + 256;
     static constexpr int THREADS = (CW + 1) * 32;
+    static constexpr int MAX_B = 8 * NT;
 };
 
 struct StreamBars {
@@ -398,6 +400,20 @@ struct StreamBars {
     uint64_t empty[8];
     int abort;
 };
+
+// Read-only global loads kept where they are written (volatile): a prefetch that the compiler
+// sank next to its use would expose the full memory latency.
+__device__ __forceinline__ uint32_t ldg_nc_u32(const void *p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint4 ldg_nc_u4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
 
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
@@ -425,13 +441,14 @@ __device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
     return d;
 }
 
-template <int CW, int RT, int GPS>
-__global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
+template <int CW, int RT, int NT>
+__global__ void __launch_bounds__(StreamLayout<CW, RT, NT>::THREADS, 2)
     gemv_w4a16_stream_kernel(const __grid_constant__ CUtensorMap tmap_w, const uint16_t *__restrict__ x,
                              const uint16_t *__restrict__ scales, const uint32_t *__restrict__ qzeros, int N, int K,
                              int B, int splits, uint16_t *__restrict__ y, unsigned int *status, uint64_t limit_ns) {
     using namespace sm100;
-    using L = StreamLayout<CW, RT, GPS>;
+    using L = StreamLayout<CW, RT, NT>;
+    constexpr int GPS = kGPS;
     extern __shared__ uint8_t stream_smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(stream_smem_raw) + 127) & ~uintptr_t(127));
     StreamBars *bar = reinterpret_cast<StreamBars *>(base + L::OFF_BAR);
@@ -455,29 +472,37 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
     __syncthreads();
     const WaitCtl ctl{&bar->abort, status, limit_ns};
 
-    float acc[RT][4];
+    float acc[RT][NT][4];
 #pragma unroll
-    for (int i = 0; i < RT; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+    for (int i = 0; i < RT; ++i)
+#pragma unroll
+        for (int n = 0; n < NT; ++n) acc[i][n][0] = acc[i][n][1] = acc[i][n][2] = acc[i][n][3] = 0.0f;
     const int t = lane & 3, r = lane >> 2;
 
     if (warp == CW) {
         // ------------------------------------------------------------------ producer warp
-        // Lane (r, t) prepares consumer lane (r, t)'s fragment: batch row r, the
-        // 32 values k = 32t .. 32t+31 of each group (the codes of the same k sit
-        // in that lane's 16 code bytes).
-        const bool has_row = r < B;
-        const uint16_t *xrow = x + (size_t)(has_row ? r : 0) * K + 32 * t;
-        uint4 xr[GPS][4];
+        // Lane (r, t) prepares consumer lane (r, t)'s fragments: batch rows r + 8n,
+        // the 32 values k = 32t .. 32t+31 of each group (the codes of the same k
+        // sit in that lane's 16 code bytes).
+        const uint16_t *xrow = x + (size_t)r * K + 32 * t;
+        // One n-tile: x of stage i lives in xa (even i) or xb (odd i); each buffer is
+        // refilled for stage i + 2 right after stage i's fragments are stored, so the
+        // loads have a whole stage to arrive.
+        auto load_x = [&](int i, uint4 (&xr)[NT][GPS][4]) {
+            const int g = g_begin + i * GPS;
 #pragma unroll
-        for (int q = 0; q < GPS; ++q)
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-                xr[q][v] = has_row ? __ldg(reinterpret_cast<const uint4 *>(xrow + (size_t)(g_begin + q) * 128 + 8 * v))
-                                   : make_uint4(0u, 0u, 0u, 0u);
+                for (int q = 0; q < GPS; ++q)
+#pragma unroll
+                    for (int v = 0; v < 4; ++v)
+                        xr[n][q][v] = r + 8 * n < B ? ldg_nc_u4(xrow + (size_t)(8 * n) * K + (size_t)(g + q) * 128 + 8 * v)
+                                                    : make_uint4(0u, 0u, 0u, 0u);
+        };
         int issued = 0;
-        for (int i = 0; i < nst; ++i) {
+        auto produce = [&](int i, const uint4 (&xr)[NT][GPS][4]) -> bool {
             const int s = i % L::RING, u = i / L::RING;
-            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&bar->empty[s]), (u & 1) ^ 1, ctl, 0x402))) break;
+            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&bar->empty[s]), (u & 1) ^ 1, ctl, 0x402))) return false;
             const uint32_t fb = smem_u32(&bar->full[s]);
             const uint32_t st = sbase + s * L::STAGE;
             const int g = g_begin + i * GPS;
@@ -489,35 +514,48 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
             }
             ++issued;
 #pragma unroll
-            for (int q = 0; q < GPS; ++q) {
-                // fragment k-step 2j: (x0,x4) and 2^-4 (x1,x5) of chunk j; k-step 2j+1: (x2,x6) and 2^-4 (x3,x7)
-                float sum0 = 0.0f, sum1 = 0.0f;
+            for (int n = 0; n < NT; ++n)
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 c = xr[q][j];
-                    sts128(st + L::OFF_XF + q * L::XF_BYTES + j * 512 + lane * 16, prmt_u(c.x, c.z, 0x5410u),
-                           hmul2_u(prmt_u(c.x, c.z, 0x7632u), 0x2C002C00u), prmt_u(c.y, c.w, 0x5410u),
-                           hmul2_u(prmt_u(c.y, c.w, 0x7632u), 0x2C002C00u));
-                    const float2 f0 = half2_bits_to_float2(c.x), f1 = half2_bits_to_float2(c.y);
-                    const float2 f2 = half2_bits_to_float2(c.z), f3 = half2_bits_to_float2(c.w);
-                    sum0 += (f0.x + f1.x) + (f2.x + f3.x);
-                    sum1 += (f0.y + f1.y) + (f2.y + f3.y);
+                for (int q = 0; q < GPS; ++q) {
+                    // fragment k-step 2j: (x0,x4) and 2^-4 (x1,x5) of chunk j; 2j+1: (x2,x6) and 2^-4 (x3,x7)
+                    float sum0 = 0.0f, sum1 = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 c = xr[n][q][j];
+                        sts128(st + L::OFF_XF + q * L::XF_BYTES + (n * 4 + j) * 512 + lane * 16,
+                               prmt_u(c.x, c.z, 0x5410u), hmul2_u(prmt_u(c.x, c.z, 0x7632u), 0x2C002C00u),
+                               prmt_u(c.y, c.w, 0x5410u), hmul2_u(prmt_u(c.y, c.w, 0x7632u), 0x2C002C00u));
+                        const float2 f0 = half2_bits_to_float2(c.x), f1 = half2_bits_to_float2(c.y);
+                        const float2 f2 = half2_bits_to_float2(c.z), f3 = half2_bits_to_float2(c.w);
+                        sum0 += (f0.x + f1.x) + (f2.x + f3.x);
+                        sum1 += (f0.y + f1.y) + (f2.y + f3.y);
+                    }
+                    float xg = sum0 + sum1;
+                    xg += __shfl_xor_sync(0xffffffffu, xg, 1);
+                    xg += __shfl_xor_sync(0xffffffffu, xg, 2);
+                    // -2^-24 X_g of batch row r + 8n (exact scaling)
+                    if (t == 0) sts32f(st + L::OFF_XS + (q * NT + n) * 32 + r * 4, xg * -5.9604644775390625e-8f);
                 }
-                float xg = sum0 + sum1;
-                xg += __shfl_xor_sync(0xffffffffu, xg, 1);
-                xg += __shfl_xor_sync(0xffffffffu, xg, 2);
-                if (t == 0) sts32f(st + L::OFF_XS + q * 32 + r * 4, xg);  // X_g of batch r
-            }
             mbar_arrive(fb);  // release: the fragments are visible to the consumers' acquire
-            if (i + 1 < nst) {  // the next stage's x, in flight while this warp waits for a free slot
-                const int gn = g + GPS;
-#pragma unroll
-                for (int q = 0; q < GPS; ++q)
-#pragma unroll
-                    for (int v = 0; v < 4; ++v)
-                        xr[q][v] = has_row
-                                       ? __ldg(reinterpret_cast<const uint4 *>(xrow + (size_t)(gn + q) * 128 + 8 * v))
-                                       : make_uint4(0u, 0u, 0u, 0u);
+            return true;
+        };
+        if (NT == 1) {
+            uint4 xa[NT][GPS][4], xb[NT][GPS][4];
+            load_x(0, xa);
+            if (nst > 1) load_x(1, xb);
+            for (int i = 0; i < nst; i += 2) {
+                if (!produce(i, xa)) break;
+                if (i + 2 < nst) load_x(i + 2, xa);
+                if (i + 1 >= nst) break;
+                if (!produce(i + 1, xb)) break;
+                if (i + 3 < nst) load_x(i + 3, xb);
+            }
+        } else {  // two n-tiles: one stage of x in registers (the two-stage prefetch would spill)
+            uint4 xa[NT][GPS][4];
+            load_x(0, xa);
+            for (int i = 0; i < nst; ++i) {
+                if (!produce(i, xa)) break;
+                if (i + 1 < nst) load_x(i + 1, xa);
             }
         }
         if (lane == 0 && bar->abort) {
@@ -549,8 +587,8 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const bool in = nl + 16 * i + 8 * h < N;
-                    sv[i][h] = in ? __ldg(reinterpret_cast<const uint32_t *>(srow + (2 * i + h) * sstep + gs)) : 0u;
-                    zv[i][h] = in ? __ldg(zrow + (2 * i + h) * zstep + (g0 >> 3)) : 0u;
+                    sv[i][h] = in ? ldg_nc_u32(srow + (2 * i + h) * sstep + gs) : 0u;
+                    zv[i][h] = in ? ldg_nc_u32(zrow + (2 * i + h) * zstep + (g0 >> 3)) : 0u;
                 }
         };
         fetch(0, sw, zw);
@@ -579,11 +617,16 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
                 // once the last group's operands are in registers
 #pragma unroll
                 for (int q = 0; q < GPS; ++q) {
-                    uint4 xv[4];
+                    uint4 xv[NT][4];
                     uint4 wv[RT][2];
+                    float2 xg[NT];
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) xv[v] = lds128(st + L::OFF_XF + q * L::XF_BYTES + v * 512 + lane * 16);
-                    const float2 xg = lds64f(st + L::OFF_XS + q * 32 + t * 8);  // X_g of batches 2t, 2t+1
+                    for (int n = 0; n < NT; ++n) {
+#pragma unroll
+                        for (int v = 0; v < 4; ++v)
+                            xv[n][v] = lds128(st + L::OFF_XF + q * L::XF_BYTES + (n * 4 + v) * 512 + lane * 16);
+                        xg[n] = lds64f(st + L::OFF_XS + (q * NT + n) * 32 + t * 8);  // -X'_g of batches 2t, 2t+1
+                    }
 #pragma unroll
                     for (int i = 0; i < RT; ++i)
 #pragma unroll
@@ -594,31 +637,47 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
                         __syncwarp();
                         if (lane == 0) mbar_arrive(smem_u32(&bar->empty[s]));
                     }
+                    // RT * NT independent accumulation chains, interleaved k-step by k-step
+                    float d[RT][NT][4];
+#pragma unroll
+                    for (int i = 0; i < RT; ++i)
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) d[i][n][0] = d[i][n][1] = d[i][n][2] = d[i][n][3] = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                        for (int hn = 0; hn < 2; ++hn) {
+#pragma unroll
+                            for (int i = 0; i < RT; ++i) {
+                                const uint32_t wa = j == 0 ? wv[i][0].x : j == 1 ? wv[i][0].y : j == 2 ? wv[i][0].z : wv[i][0].w;
+                                const uint32_t wb = j == 0 ? wv[i][1].x : j == 1 ? wv[i][1].y : j == 2 ? wv[i][1].z : wv[i][1].w;
+                                const uint32_t ua = hn ? wa >> 8 : wa, ub = hn ? wb >> 8 : wb;
+                                const uint32_t af[4] = {ua & 0x000F000Fu, ub & 0x000F000Fu, ua & 0x00F000F0u,
+                                                        ub & 0x00F000F0u};
+#pragma unroll
+                                for (int n = 0; n < NT; ++n) {
+                                    if (hn == 0)
+                                        mma_16816(d[i][n], af, xv[n][j].x, xv[n][j].y);
+                                    else
+                                        mma_16816(d[i][n], af, xv[n][j].z, xv[n][j].w);
+                                }
+                            }
+                        }
+                    }
+                    // acc += s (D - z X'_g)  (rows r and r + 8 of each m-tile)
 #pragma unroll
                     for (int i = 0; i < RT; ++i) {
-                        float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-                        const uint32_t wa[4] = {wv[i][0].x, wv[i][0].y, wv[i][0].z, wv[i][0].w};
-                        const uint32_t wb[4] = {wv[i][1].x, wv[i][1].y, wv[i][1].z, wv[i][1].w};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t a8 = wa[j] >> 8, b8 = wb[j] >> 8;
-                            const uint32_t a0[4] = {wa[j] & 0x000F000Fu, wb[j] & 0x000F000Fu, wa[j] & 0x00F000F0u,
-                                                    wb[j] & 0x00F000F0u};
-                            const uint32_t a1[4] = {a8 & 0x000F000Fu, b8 & 0x000F000Fu, a8 & 0x00F000F0u,
-                                                    b8 & 0x00F000F0u};
-                            mma_16816(d, a0, xv[j].x, xv[j].y);
-                            mma_16816(d, a1, xv[j].z, xv[j].w);
-                        }
                         const float s0 = half_bits_to_float((uint16_t)(scw[i][0] >> (16 * q)));
                         const float s1 = half_bits_to_float((uint16_t)(scw[i][1] >> (16 * q)));
                         const float z0 = (float)((zw[i][0] >> (zsh + 4 * q)) & 0xFu);
                         const float z1 = (float)((zw[i][1] >> (zsh + 4 * q)) & 0xFu);
-                        const float a0s = s0 * 16777216.0f, a1s = s1 * 16777216.0f;  // exact: times 2^24
-                        const float b0s = -s0 * z0, b1s = -s1 * z1;                  // exact: fp16 x 4-bit integer
-                        acc[i][0] = fmaf(a0s, d[0], fmaf(b0s, xg.x, acc[i][0]));
-                        acc[i][1] = fmaf(a0s, d[1], fmaf(b0s, xg.y, acc[i][1]));
-                        acc[i][2] = fmaf(a1s, d[2], fmaf(b1s, xg.x, acc[i][2]));
-                        acc[i][3] = fmaf(a1s, d[3], fmaf(b1s, xg.y, acc[i][3]));
+#pragma unroll
+                        for (int n = 0; n < NT; ++n) {
+                            acc[i][n][0] = fmaf(s0, fmaf(z0, xg[n].x, d[i][n][0]), acc[i][n][0]);
+                            acc[i][n][1] = fmaf(s0, fmaf(z0, xg[n].y, d[i][n][1]), acc[i][n][1]);
+                            acc[i][n][2] = fmaf(s1, fmaf(z1, xg[n].x, d[i][n][2]), acc[i][n][2]);
+                            acc[i][n][3] = fmaf(s1, fmaf(z1, xg[n].y, d[i][n][3]), acc[i][n][3]);
+                        }
                     }
                 }
             }
@@ -632,7 +691,8 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
         }
     }
 
-    // ---------------------------------------------------------------------- results
+    // ---------------------------------------------------------------------- results (times 2^24)
+    constexpr float kUnscale = 16777216.0f;
     const bool cons = warp < CW;
     const int wrow = warp * RT * 16;
     if (splits == 1) {
@@ -640,13 +700,17 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
 #pragma unroll
             for (int i = 0; i < RT; ++i)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int n = n0 + wrow + 16 * i + r + 8 * h;
-                    if (n < N) {
-                        if (2 * t < B) y[(size_t)(2 * t) * N + n] = float_to_half_bits_rn(acc[i][2 * h]);
-                        if (2 * t + 1 < B) y[(size_t)(2 * t + 1) * N + n] = float_to_half_bits_rn(acc[i][2 * h + 1]);
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int row = n0 + wrow + 16 * i + r + 8 * h;
+                        const int b0 = 8 * n + 2 * t;
+                        if (row < N) {
+                            if (b0 < B) y[(size_t)b0 * N + row] = float_to_half_bits_rn(acc[i][n][2 * h] * kUnscale);
+                            if (b0 + 1 < B)
+                                y[(size_t)(b0 + 1) * N + row] = float_to_half_bits_rn(acc[i][n][2 * h + 1] * kUnscale);
+                        }
                     }
-                }
         }
     } else {
         cluster_sync();  // every CTA of the cluster is done with its ring
@@ -655,13 +719,15 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
 #pragma unroll
             for (int i = 0; i < RT; ++i)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int row = wrow + 16 * i + r + 8 * h;
-                    const uint32_t a = red + (uint32_t)(((rank - 1) * L::ROWS + row) * 8 + 2 * t) * 4;
-                    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(acc[i][2 * h]),
-                                 "f"(acc[i][2 * h + 1])
-                                 : "memory");
-                }
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int row = wrow + 16 * i + r + 8 * h;
+                        const uint32_t a = red + (uint32_t)((((rank - 1) * L::ROWS + row) * NT + n) * 8 + 2 * t) * 4;
+                        asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(acc[i][n][2 * h]),
+                                     "f"(acc[i][n][2 * h + 1])
+                                     : "memory");
+                    }
         }
         cluster_sync();  // partials landed in the leading CTA
         if (cons && rank == 0 && !bar->abort) {
@@ -669,36 +735,38 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, GPS>::THREADS, 2)
 #pragma unroll
             for (int i = 0; i < RT; ++i)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int row = wrow + 16 * i + r + 8 * h;
-                    float v0 = acc[i][2 * h], v1 = acc[i][2 * h + 1];
-                    for (int sl = 0; sl < splits - 1; ++sl) {
-                        v0 += red[(sl * L::ROWS + row) * 8 + 2 * t];
-                        v1 += red[(sl * L::ROWS + row) * 8 + 2 * t + 1];
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int row = wrow + 16 * i + r + 8 * h;
+                        float v0 = acc[i][n][2 * h], v1 = acc[i][n][2 * h + 1];
+                        for (int sl = 0; sl < splits - 1; ++sl) {
+                            v0 += red[((sl * L::ROWS + row) * NT + n) * 8 + 2 * t];
+                            v1 += red[((sl * L::ROWS + row) * NT + n) * 8 + 2 * t + 1];
+                        }
+                        const int gr = n0 + row, b0 = 8 * n + 2 * t;
+                        if (gr < N) {
+                            if (b0 < B) y[(size_t)b0 * N + gr] = float_to_half_bits_rn(v0 * kUnscale);
+                            if (b0 + 1 < B) y[(size_t)(b0 + 1) * N + gr] = float_to_half_bits_rn(v1 * kUnscale);
+                        }
                     }
-                    const int n = n0 + row;
-                    if (n < N) {
-                        if (2 * t < B) y[(size_t)(2 * t) * N + n] = float_to_half_bits_rn(v0);
-                        if (2 * t + 1 < B) y[(size_t)(2 * t + 1) * N + n] = float_to_half_bits_rn(v1);
-                    }
-                }
         }
     }
 }
 
-template <int CW, int RT, int GPS>
+template <int CW, int RT, int NT>
 wq_status launch_stream(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
-                        int K, int splits, uint16_t *y, cudaStream_t st) {
-    using L = StreamLayout<CW, RT, GPS>;
+                        int K, int splits, uint16_t *y, cudaStream_t st, const char *who) {
+    using L = StreamLayout<CW, RT, NT>;
     unsigned int *status = device_status_word();
     if (!status) return WQ_ERR_CUDA;
     CUtensorMap tw;
     if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qw, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2, 64,
                         L::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE))
         return WQ_ERR_CUDA;
-    auto kern = gemv_w4a16_stream_kernel<CW, RT, GPS>;
+    auto kern = gemv_w4a16_stream_kernel<CW, RT, NT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L::SMEM);
-    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_gemv_w4a16: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "%s: cudaFuncSetAttribute: %s", who, cudaGetErrorString(e));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(splits, (N + L::ROWS - 1) / L::ROWS, 1);
     cfg.blockDim = dim3(L::THREADS);
@@ -712,16 +780,19 @@ wq_status launch_stream(const uint16_t *x, int B, const uint32_t *qw, const uint
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, tw, x, sc, qz, N, K, B, splits, y, status, wait_limit());
-    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_gemv_w4a16: launch failed: %s", cudaGetErrorString(e));
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "%s: launch failed: %s", who, cudaGetErrorString(e));
     return WQ_OK;
 }
 
 // Tile height and K split of the streaming GEMV.  Two CTAs are resident per
-// SM; the split (cluster size, at most 8, dividing the stage count, partials
-// fitting the leading CTA's ring) is the smallest one that reaches the best
-// fill of those slots over whole waves.  The 256-row tile (4 consumer warps x
-// 4 m-tiles) is the fastest on B200; the 128-row tile serves matrices with too
-// few 256-row tiles.
+// SM; the split (cluster size, at most 8, keeping every CTA's start on a
+// zero-point word, partials fitting the leading CTA's ring) is the smallest one
+// that reaches the best fill of those slots over whole waves.  Measured on
+// B200, for one and for two n-tiles: the 224-row tile (7 consumer warps x 2
+// m-tiles, 8 warps and at most 128 registers per thread, so that 16 warps
+// share an SM) is the fastest; the 128-row tile serves matrices with too few
+// 224-row tiles.  (Unaligned splits that fill every slot, e.g. 8-CTA clusters
+// on the 28672-wide down projection, measured slower.)
 template <typename L>
 int stream_splits(int N, int K, int sms) {
     const int tiles = (N + L::ROWS - 1) / L::ROWS;
@@ -730,7 +801,7 @@ int stream_splits(int N, int K, int sms) {
     double best_fill = 0.0;
     for (int s = 1; s <= 8; ++s) {
         if (s > 1 && (K / 128) % (8 * s)) continue;  // every CTA starts on a zero-point word
-        if ((size_t)(s - 1) * L::ROWS * 8 * 4 > L::OFF_BAR) continue;
+        if ((size_t)(s - 1) * L::ROWS * L::MAX_B * 4 > L::OFF_BAR) continue;
         const long long ctas = (long long)tiles * s;
         const long long waves = (ctas + slots - 1) / slots;
         const double fill = (double)ctas / (double)(waves * slots);
@@ -742,16 +813,28 @@ int stream_splits(int N, int K, int sms) {
     return best;
 }
 
-wq_status gemv_stream(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
-                      int K, uint16_t *y, cudaStream_t st) {
+template <int NT, int BCW, int BRT>
+wq_status gemv_stream_nt(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
+                         int K, uint16_t *y, cudaStream_t st, const char *who) {
     const int sms = num_sms();
-    using Big = StreamLayout<4, 4, 2>;
-    using Small = StreamLayout<4, 2, 2>;
+    using Big = StreamLayout<BCW, BRT, NT>;
+    using Small = StreamLayout<4, 2, NT>;
     const int tiles_big = (N + Big::ROWS - 1) / Big::ROWS;
     if (tiles_big * 8 >= 2 * sms)
-        return launch_stream<4, 4, 2>(x, B, qw, sc, qz, N, K, stream_splits<Big>(N, K, sms), y, st);
-    return launch_stream<4, 2, 2>(x, B, qw, sc, qz, N, K, stream_splits<Small>(N, K, sms), y, st);
+        return launch_stream<BCW, BRT, NT>(x, B, qw, sc, qz, N, K, stream_splits<Big>(N, K, sms), y, st, who);
+    return launch_stream<4, 2, NT>(x, B, qw, sc, qz, N, K, stream_splits<Small>(N, K, sms), y, st, who);
 }
+
+}  // namespace
+
+// Batch 1..16 with K % 256 == 0, group size 128 (also serves wq_gemm_w4a16 at M <= 16).
+wq_status gemv_stream(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
+                      int K, uint16_t *y, cudaStream_t st, const char *who) {
+    if (B <= 8) return gemv_stream_nt<1, 7, 2>(x, B, qw, sc, qz, N, K, y, st, who);
+    return gemv_stream_nt<2, 7, 2>(x, B, qw, sc, qz, N, K, y, st, who);
+}
+
+namespace {
 
 template <int RT>
 cudaError_t launch_mma(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
@@ -798,7 +881,7 @@ extern "C" wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qwe
                "wq_gemv_w4a16: K (%d) must be a multiple of group_size (%d)", K, group_size);
     cudaStream_t st = wq::as_stream(stream);
     cudaError_t e;
-    if (group_size == 128 && K % 256 == 0) return wq::gemv_stream(x, B, qweight, scales, qzeros, N, K, y, st);
+    if (group_size == 128 && K % 256 == 0) return wq::gemv_stream(x, B, qweight, scales, qzeros, N, K, y, st, "wq_gemv_w4a16");
     if (group_size == 128) {
         // Two 16-row MMA tiles per CTA when that still gives every SM several CTAs.
         const long long blocks2 = (N + 31) / 32;

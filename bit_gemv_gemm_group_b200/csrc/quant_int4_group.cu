@@ -17,6 +17,8 @@
 // weight: 2 (fp16 in) + 0.5 + 2.5/G (out).  The codes rne(w / s) are decided
 // from w * RN(1/s) with an exact near-tie fallback (rne_quotient), which gives
 // the same integers as the IEEE division at a third of its instructions.
+#include <type_traits>
+
 #include "wq_device.cuh"
 #include "wq_host.h"
 
@@ -121,6 +123,132 @@ __global__ void __launch_bounds__(256) quant_int4_group_kernel(const TIn *__rest
     if (lane == 0) qzeros[(size_t)n * zwords + zw] = zword;
 }
 
+// ---------------------------------------------------------------------------
+// fp16 input: the same decomposition with packed arithmetic.  The range comes
+// from fp16x2 min/max on the raw bits (exact); a pair of codes is decided with
+// f32x2 operations:  t = w * RN(1/s),  r = t + 1.5*2^23 (rne(t) lands in r's
+// low mantissa bits),  d = t - (r - 1.5*2^23) (exact).  The pair is exact
+// unless |d| comes within 2^-16 of 1/2 (a near-tie of w*RN(1/s), the guard of
+// rne_quotient widened), in which case the lane recomputes its 8 codes with
+// the IEEE quotient.  Adding z, clamping and nibble packing run on 16-bit
+// SIMD lanes.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t hmin2_bits(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// rne(w * rs) of an fp16 pair as int16x2; `bad` collects the sign bit of
+// (1/2 - 2^-16)^2 - d^2 (set when a lane lies in the guard band).
+__device__ __forceinline__ uint32_t pair_rne(uint32_t h2, float rs, uint32_t &bad) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    constexpr float kGuardSq = (0.5f - 0x1p-16f) * (0.5f - 0x1p-16f);
+    const float2 f = half2_bits_to_float2(h2);
+    const float2 t = __fmul2_rn(f, make_float2(rs, rs));
+    const float2 r = __fadd2_rn(t, make_float2(kMagic, kMagic));
+    const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
+    const float2 d = __fadd2_rn(t, make_float2(-n.x, -n.y));
+    const float2 e = __ffma2_rn(d, make_float2(-d.x, -d.y), make_float2(kGuardSq, kGuardSq));
+    bad |= __float_as_uint(e.x) | __float_as_uint(e.y);
+    return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);  // low 16 bits: rne(t)
+}
+
+// codes c_e (int16x2 pairs (c0,c1), (c2,c3), ...) -> one word, code e at bits 4e
+__device__ __forceinline__ uint32_t pack8(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3) {
+    const uint32_t u0 = p0 | (p0 >> 12), u1 = p1 | (p1 >> 12);  // byte 0: c_e | c_{e+1} << 4
+    const uint32_t u2 = p2 | (p2 >> 12), u3 = p3 | (p3 >> 12);
+    return __byte_perm(__byte_perm(u0, u1, 0x3140), __byte_perm(u2, u3, 0x3140), 0x5410);
+}
+
+template <int G>
+__global__ void __launch_bounds__(256) quant_int4_group_f16_kernel(const uint16_t *__restrict__ w, int N, int K,
+                                                                    uint32_t *__restrict__ qweight,
+                                                                    uint16_t *__restrict__ scales,
+                                                                    uint32_t *__restrict__ qzeros) {
+    constexpr int LPG = G / 8;       // lanes per group
+    constexpr int GPI = 32 / LPG;    // groups per warp iteration
+    constexpr int ITERS = 8 / GPI;   // iterations per zero word (8 groups)
+    const int groups = K / G;
+    const int zwords = (groups + 7) / 8;
+    const int lane = threadIdx.x & 31;
+    const long long unit = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (unit >= (long long)N * zwords) return;
+    const int n = (int)(unit / zwords);
+    const int zw = (int)(unit % zwords);
+    const int sub = lane / LPG;  // group slot within an iteration
+    const int li = lane % LPG;   // lane within the group
+
+    // Issue every load of this warp first.
+    uint4 raw[ITERS];
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int j = zw * 8 + it * GPI + sub;
+        raw[it] = j < groups ? ld_stream_u4(w + (size_t)n * K + (size_t)j * G + li * 8) : make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    uint32_t zacc = 0;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int j = zw * 8 + it * GPI + sub;
+        const uint4 c = raw[it];
+        // Range of the group, widened to contain 0.
+        const uint32_t mn = hmin2_bits(hmin2_bits(c.x, c.y), hmin2_bits(c.z, c.w));
+        const uint32_t mx = hmax2_bits(hmax2_bits(c.x, c.y), hmax2_bits(c.z, c.w));
+        const float2 mnf = half2_bits_to_float2(mn), mxf = half2_bits_to_float2(mx);
+        float lo = fminf(0.0f, fminf(mnf.x, mnf.y));
+        float hi = fmaxf(0.0f, fmaxf(mxf.x, mxf.y));
+#pragma unroll
+        for (int off = LPG / 2; off >= 1; off >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+        }
+        // s = fp16((hi - lo) / 15); a zero scale becomes 1.
+        uint16_t s16 = float_to_half_bits_rn(__fdiv_rn(hi - lo, 15.0f));
+        if (s16 == 0) s16 = 0x3c00;
+        const float s = half_bits_to_float(s16);
+        const float rs = __frcp_rn(s);
+        // z = round(-lo / s) in [0, 15]; |-lo / s| and |w / s| stay below 32 (E = 4)
+        const int z = clampi(rne_quotient<4>(-lo, s, rs), 0, 15);
+        if (j < groups) {
+            uint32_t bad = 0;
+            uint32_t p0 = pair_rne(c.x, rs, bad), p1 = pair_rne(c.y, rs, bad);
+            uint32_t p2 = pair_rne(c.z, rs, bad), p3 = pair_rne(c.w, rs, bad);
+            if (bad >> 31) {  // a near-tie: the IEEE quotient decides every code of this lane
+                const uint32_t h[4] = {c.x, c.y, c.z, c.w};
+                uint32_t pp[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = half2_bits_to_float2(h[e]);
+                    const uint32_t a = (uint32_t)__float2int_rn(__fdiv_rn(f.x, s)) & 0xFFFFu;
+                    const uint32_t b = (uint32_t)__float2int_rn(__fdiv_rn(f.y, s)) & 0xFFFFu;
+                    pp[e] = a | (b << 16);
+                }
+                p0 = pp[0]; p1 = pp[1]; p2 = pp[2]; p3 = pp[3];
+            }
+            const uint32_t z2 = (uint32_t)z * 0x00010001u;
+            const uint32_t top = 0x000F000Fu;
+            p0 = __vmins2(__vmaxs2(__vadd2(p0, z2), 0u), top);
+            p1 = __vmins2(__vmaxs2(__vadd2(p1, z2), 0u), top);
+            p2 = __vmins2(__vmaxs2(__vadd2(p2, z2), 0u), top);
+            p3 = __vmins2(__vmaxs2(__vadd2(p3, z2), 0u), top);
+            qweight[(size_t)n * (K / 8) + (size_t)j * (G / 8) + li] = pack8(p0, p1, p2, p3);
+            if (li == 0) {
+                scales[(size_t)n * groups + j] = s16;
+                zacc |= (uint32_t)z << (4 * (j & 7));
+            }
+        }
+    }
+    const uint32_t zword = __reduce_or_sync(0xffffffffu, zacc);
+    if (lane == 0) qzeros[(size_t)n * zwords + zw] = zword;
+}
+
 template <typename TIn, int G>
 cudaError_t launch(const void *w, int N, int K, uint32_t *qweight, uint16_t *scales, uint32_t *qzeros,
                    cudaStream_t stream) {
@@ -128,8 +256,12 @@ cudaError_t launch(const void *w, int N, int K, uint32_t *qweight, uint16_t *sca
     const long long units = (long long)N * zwords;
     const int warps_per_block = 8;
     const long long blocks = (units + warps_per_block - 1) / warps_per_block;
-    quant_int4_group_kernel<TIn, G><<<(unsigned)blocks, warps_per_block * 32, 0, stream>>>(
-        static_cast<const TIn *>(w), N, K, qweight, scales, qzeros);
+    if (std::is_same<TIn, __half>::value)
+        quant_int4_group_f16_kernel<G><<<(unsigned)blocks, warps_per_block * 32, 0, stream>>>(
+            static_cast<const uint16_t *>(w), N, K, qweight, scales, qzeros);
+    else
+        quant_int4_group_kernel<TIn, G><<<(unsigned)blocks, warps_per_block * 32, 0, stream>>>(
+            static_cast<const TIn *>(w), N, K, qweight, scales, qzeros);
     return cudaGetLastError();
 }
 

@@ -39,6 +39,11 @@ int num_sms();
 // Encodes a 2-D tiled TMA descriptor over a row-major [outer][inner] array
 // (element size `elem_bytes`, row pitch `row_bytes`) with box
 // [box_outer][box_inner].  Returns false and records a message on failure.
+// Streaming W4A16 matmul for 1..16 activation rows (K % 256 == 0, group size 128); defined in
+// gemv_w4a16.cu and shared by wq_gemv_w4a16 and wq_gemm_w4a16.  `who` names the entry point in errors.
+wq_status gemv_stream(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
+                      int K, uint16_t *y, cudaStream_t st, const char *who);
+
 bool encode_tmap_2d(CUtensorMap *map, CUtensorMapDataType dtype, int elem_bytes, const void *base, uint64_t inner,
                     uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
                     CUtensorMapSwizzle swizzle);

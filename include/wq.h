@@ -170,12 +170,14 @@ wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qweight, const
                         void *stream);
 
 /*
- * W4A16 GEMM on the tensor cores for M >= 16 rows of activations: tiles of
- * packed weights are dequantized into shared memory and fed to tcgen05 MMAs
- * with fp32 accumulation in tensor memory ([P1] "Inference view").  Same
- * arithmetic and layouts as wq_gemv_w4a16 (each dequantized weight is
- * rounded to fp16 before the MMA); M in [16, 256]; group_size == 128;
- * K % 128 == 0.
+ * W4A16 GEMM for M >= 16 rows of activations ([P1] "Inference view"), same
+ * arithmetic and layouts as wq_gemv_w4a16.  M == 16 with K % 256 == 0 runs
+ * the streaming kernel of wq_gemv_w4a16 (codes dequantized in registers,
+ * exact products, two 8-row batch tiles per weight fragment).  Other M run on
+ * the tensor cores: tiles of packed weights are dequantized into shared
+ * memory (each dequantized weight rounded to fp16) and fed to tcgen05 MMAs
+ * with fp32 accumulation in tensor memory.  M in [16, 256]; group_size ==
+ * 128; K % 128 == 0.
  */
 wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
                         const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y,

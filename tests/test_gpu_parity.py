@@ -118,7 +118,7 @@ def test_gemv_w4a16_small(wq, N, K, g, B):
     assert_within_bound(host(y).astype(np.float64), y_ref, bound, f"gemv N={N} K={K} B={B}")
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3])
+@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
 def test_gemv_w4a16_configs(wq, cfg):
     c = workloads.CONFIGS[cfg]
     for si, (N, K) in enumerate(c.shapes):
