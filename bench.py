@@ -340,7 +340,8 @@ def run_gpu(args):
                      "peak": rdom["peak"], "unit": rdom["unit"], "frac": round(rdom["frac"], 4),
                      "traffic": traffic, "peak_source": peaks["source"]},
         "gemv_roofline": {"bound": "hbm", "achieved": round(value / world, 1), "peak": gemv_roof["peak"],
-                          "unit": "GB/s", "frac": round(value / world / gemv_roof["peak"], 4)},
+                          "unit": "GB/s", "frac": round(value / world / gemv_roof["peak"], 4),
+                          "traffic": load_traffic("gemv_w4a16_b1_up")},
         "kernels": kernels,
         "e2e": e2e,
         "gpu_launches": len(launches) * args.steps,
