@@ -241,7 +241,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                          : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
                          : "r"(sP + p * P_BYTES + row * 32 + half * 16));
-            mbar_arrive(smem_u32(&bar->pk_empty[p]));
             if (!wait_parity(smem_u32(&bar->st_empty[s]), (u & 1) ^ 1, ctl, SITE_DEQUANT)) return false;
             const uint32_t dst = a_row + s * A_BYTES;
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -255,6 +254,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             fence_proxy_async_smem();
             mbar_arrive(smem_u32(&bar->a_full[s]));
+            // The packed slot is released only now: its codes have been consumed and the
+            // proxy fence above orders this thread's read of it before the next TMA write.
+            mbar_arrive(smem_u32(&bar->pk_empty[p]));
             return true;
         };
         if (SB) {

@@ -336,3 +336,24 @@ def test_gemm_w4a16_configs(wq, cfg):
             y_ref, bound = oracle.matmul_w4a16_ref(x, hqw[rows], hsc[rows], hqz[rows], K, 128)
             assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"cfg{cfg} {N}x{K} B={B}")
     assert wq.device_status() == 0
+
+
+# --------------------------------------------------------------------------
+# Determinism at full size: every launch of a kernel on the same inputs gives
+# the same bits.  This holds at any size; a race between a ring slot's release
+# and its refill would show up as a difference somewhere in the output.
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("shape_index", [0, 1])
+def test_w4a16_matmuls_repeat_bit_identically(wq, shape_index):
+    w = workloads.config_weight(4, shape_index)
+    N, K = w.shape
+    qw, sc, qz = wq.quantize_group_int4(dev(w), 128)
+    del w
+    for B in (1, 16, 64):
+        x = dev(workloads.config_activations(4, B, K))
+        first = wq.matmul_w4a16(x, qw, sc, qz, 128)
+        for _ in range(3):
+            again = wq.matmul_w4a16(x, qw, sc, qz, 128)
+            torch.cuda.synchronize()
+            assert torch.equal(first.view(torch.int16), again.view(torch.int16)), f"{N}x{K} B={B}"
+    assert wq.device_status() == 0
