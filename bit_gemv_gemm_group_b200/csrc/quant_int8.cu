@@ -11,7 +11,10 @@
 // One CTA of 256 threads per row.  Each thread owns 16-byte chunks of 8 fp16
 // values; for K <= 16384 the (smoothed) row stays in registers between the
 // absmax pass and the quantize pass, so HBM sees 2 B read + 1 B written per
-// element.  Longer rows are read twice (the second read hits L2).
+// element.  Rows of 8192 < K <= 16384 are split over a cluster of two CTAs
+// (the partial maxima meet in distributed shared memory); longer rows are read
+// twice (the second read hits L2).
+#include "sm100.cuh"
 #include "wq_device.cuh"
 #include "wq_host.h"
 
@@ -125,10 +128,84 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
     }
 }
 
+// 8192 < K <= 16384: a row is split over a cluster of C = 2 CTAs (at most
+// 8192 columns each), each keeping its (smoothed) part in registers
+// with at most 4 chunks per thread (few registers, four CTAs per SM); the
+// partial maxima are exchanged through distributed shared memory, so HBM still
+// sees each element once.
+template <int C, int MODE>
+__global__ void __launch_bounds__(kThreads) quant_int8_rows_cluster_kernel(const uint16_t *__restrict__ x, int K,
+                                                                           const float *__restrict__ smooth,
+                                                                           int8_t *__restrict__ q,
+                                                                           float *__restrict__ scales) {
+    constexpr int NCH = 4;
+    __shared__ float red[kThreads / 32];
+    __shared__ float part_max[C];
+    const size_t row = blockIdx.y;
+    const uint32_t rank = sm100::cluster_ctarank();  // cluster (C, 1, 1) along x
+    const int part = K / C;                          // K % (8 C) == 0: whole chunks per CTA
+    const int kb = (int)rank * part;
+    const uint16_t *xr = x + row * K + kb;
+    int8_t *qr = q + row * K + kb;
+    const int t0 = threadIdx.x * kChunk;
+    float amax = 0.0f;
+    float v[NCH][8];
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        const int k = c * kRowStep + t0;
+        if (k < part) {
+            load8(xr + k, v[c]);
+            smooth8<MODE>(v[c], smooth, kb + k);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[c][e]));
+        }
+    }
+    const float mine = block_max(amax, red);
+    if (threadIdx.x < C) {  // this CTA's maximum into slot `rank` of every CTA of the cluster
+        const uint32_t slot = sm100::smem_u32(&part_max[rank]);
+        asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(sm100::mapa_shared(slot, threadIdx.x)), "f"(mine)
+                     : "memory");
+    }
+    sm100::cluster_sync();
+    float a = part_max[0];
+#pragma unroll
+    for (int c = 1; c < C; ++c) a = fmaxf(a, part_max[c]);
+    a = fmaxf(a, 1e-8f);
+    const float s = __fdiv_rn(a, 127.0f);
+    const float rs = __frcp_rn(s);
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) {
+        const int k = c * kRowStep + t0;
+        if (k < part) *reinterpret_cast<uint2 *>(qr + k) = quant8(v[c], s, rs);
+    }
+    if (threadIdx.x == 0 && rank == 0) scales[row] = s;
+}
+
+template <int C, int MODE>
+cudaError_t launch_cluster(const uint16_t *x, int R, int K, const float *smooth, int8_t *q, float *scales,
+                           cudaStream_t st) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(C, R, 1);
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quant_int8_rows_cluster_kernel<C, MODE>, x, K, smooth, q, scales);
+}
+
 template <int MODE>
 cudaError_t launch_mode(const uint16_t *x, int R, int K, const float *smooth, int8_t *q, float *scales,
                         cudaStream_t st) {
     const int nch = (K + kRowStep - 1) / kRowStep;
+    // Measured on B200: pairs beat the 8-chunk single CTA; for longer rows the
+    // two-pass kernel (second read from L2) beats clusters of 4 or 8.
+    if (nch > 4 && nch <= 8 && R < 65536 && K % 16 == 0)
+        return launch_cluster<2, MODE>(x, R, K, smooth, q, scales, st);
     dim3 grid(R), block(kThreads);
     if (nch <= 1)
         quant_int8_rows_kernel<1, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);

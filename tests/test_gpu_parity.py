@@ -137,7 +137,8 @@ def test_gemv_w4a16_configs(wq, cfg):
 # --------------------------------------------------------------------------
 # INT8 quantizers and smoothing
 # --------------------------------------------------------------------------
-INT8_SMALL = [(1, 16), (7, 48), (33, 2048), (5, 2064), (64, 4096), (3, 16384), (2, 16400), (4, 40960)]
+INT8_SMALL = [(1, 16), (7, 48), (33, 2048), (5, 2064), (64, 4096), (3, 16384), (2, 16400), (4, 40960),
+              (5, 28672), (3, 32768), (2, 24592)]
 
 
 @pytest.mark.parametrize("R,K", INT8_SMALL)
