@@ -171,10 +171,11 @@ wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qweight, const
 
 /*
  * W4A16 GEMM for M >= 16 rows of activations ([P1] "Inference view"), same
- * arithmetic and layouts as wq_gemv_w4a16.  M == 16 with K % 256 == 0 runs
- * the streaming kernel of wq_gemv_w4a16 (codes dequantized in registers,
- * exact products, two 8-row batch tiles per weight fragment).  Other M run on
- * the tensor cores: tiles of packed weights are dequantized into shared
+ * arithmetic and layouts as wq_gemv_w4a16.  M <= 32 with K % 256 == 0 runs
+ * the streaming kernel of wq_gemv_w4a16 in passes of 16 rows (codes
+ * dequantized in registers, exact products, two 8-row batch tiles per weight
+ * fragment).  Other M run on the tensor cores: tiles of packed weights are
+ * dequantized into shared
  * memory (each dequantized weight rounded to fp16) and fed to tcgen05 MMAs
  * with fp32 accumulation in tensor memory.  M in [16, 256]; group_size ==
  * 128; K % 128 == 0.
