@@ -14,7 +14,7 @@
 // dimension is the activation tile (16..128 rows of x), so small batches still
 // use full 128-row MMAs.  Per CTA (480 threads):
 //   warp 0      TMA: packed weight tiles (128 rows x 32 bytes = 64 codes) into
-//               a 12-deep ring
+//               a 6- or 12-deep ring (two or one CTAs per SM, see Layout)
 //   warp 1      TMA: x tiles (MT rows x 64 fp16, 128-byte swizzle)
 //   warp 2      TMEM allocation and tcgen05.mma issue (4 x K=16 per stage)
 //   warps 3-10  dequantize: each thread turns 32 codes of one row into fp16
@@ -39,8 +39,8 @@ using namespace sm100;
 
 constexpr int BMW = 128;                    // weight rows per tile (MMA M)
 constexpr int BK = 64;                      // k per stage: one 128-byte fp16 row
-constexpr int STAGES = 4;                   // dequantized A stages
-constexpr int PSTAGES = 12;                 // packed-tile ring
+constexpr int MAX_STAGES = 4;               // dequantized A stages (barrier arrays)
+constexpr int MAX_PSTAGES = 12;             // packed-tile ring (barrier arrays)
 constexpr uint32_t A_BYTES = BMW * BK * 2;  // 16 KB
 constexpr uint32_t P_BYTES = BMW * BK / 2;  // 4 KB of packed codes
 constexpr int THREADS = 480;
@@ -49,13 +49,21 @@ constexpr uint64_t DRAIN_NS = 2000000000ull;
 constexpr unsigned SITE_PRODUCER = 0x201, SITE_MMA = 0x202, SITE_DEQUANT = 0x204, SITE_EPILOGUE = 0x208,
                    SITE_DRAIN = 0x210;
 
+// Activation tiles of up to 64 rows run two CTAs per SM (smaller rings, at most
+// 64 registers per thread): measured on B200 that halves the time of the
+// 64-row GEMM on the 28672x8192 projection, because a CTA's stage loop is
+// bound by handoff latency rather than by any unit's throughput.  128-row
+// tiles need the deeper activation ring and keep one CTA per SM.
 template <int MT>
 struct Layout {
+    static constexpr int CTAS_PER_SM = MT <= 64 ? 2 : 1;
+    static constexpr int STAGES = MT <= 64 ? 3 : 4;
+    static constexpr int PSTAGES = MT <= 64 ? 6 : 12;
     static constexpr uint32_t B_BYTES = MT * 128;
     // activation tiles get their own ring, deep enough that a tile is requested
     // well before the MMA needs it (x comes from L2; its latency would otherwise
     // stall the MMA warp every few stages)
-    static constexpr int XSTAGES = MT <= 32 ? 12 : MT <= 64 ? 8 : 4;
+    static constexpr int XSTAGES = MT <= 32 ? 6 : 4;
     static constexpr uint32_t OFF_A = 0;
     static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
     static constexpr uint32_t OFF_P = OFF_B + XSTAGES * B_BYTES;
@@ -64,10 +72,10 @@ struct Layout {
 };
 
 struct Bars {
-    uint64_t pk_full[PSTAGES];
-    uint64_t pk_empty[PSTAGES];
-    uint64_t a_full[STAGES];   // dequantized weight tile written (256 arrivals)
-    uint64_t st_empty[STAGES]; // A stage consumed by the MMAs
+    uint64_t pk_full[MAX_PSTAGES];
+    uint64_t pk_empty[MAX_PSTAGES];
+    uint64_t a_full[MAX_STAGES];   // dequantized weight tile written (256 arrivals)
+    uint64_t st_empty[MAX_STAGES]; // A stage consumed by the MMAs
     uint64_t x_full[12];       // activation tile landed (TMA transaction count)
     uint64_t x_empty[12];      // activation tile consumed by the MMAs
     uint64_t tmem_full;
@@ -115,7 +123,7 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t zc, uint32_t 
 }
 
 template <int MT, bool SB>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
                       const uint16_t *__restrict__ scales, const uint32_t *__restrict__ qzeros,
                       uint16_t *__restrict__ y, int M, int N, int K, int splits, unsigned int *status,
@@ -137,11 +145,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr uint32_t TMEM_COLS = MT < 32 ? 32 : MT;
 
     if (threadIdx.x == 0) {
-        for (int p = 0; p < PSTAGES; ++p) {
+        for (int p = 0; p < L::PSTAGES; ++p) {
             mbar_init(smem_u32(&bar->pk_full[p]), 1);
             mbar_init(smem_u32(&bar->pk_empty[p]), DQ_THREADS);
         }
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < L::STAGES; ++s) {
             mbar_init(smem_u32(&bar->a_full[s]), DQ_THREADS);
             mbar_init(smem_u32(&bar->st_empty[s]), 1);
         }
@@ -172,14 +180,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {  // ------------------------------------------------ packed-code producer
             int i = 0;
             for (; i < nkb; ++i) {
-                const int p = i % PSTAGES, up = i / PSTAGES;
+                const int p = i % L::PSTAGES, up = i / L::PSTAGES;
                 if (!wait_parity(smem_u32(&bar->pk_empty[p]), (up & 1) ^ 1, ctl, SITE_PRODUCER)) break;
                 const uint32_t fb = smem_u32(&bar->pk_full[p]);
                 mbar_arrive_expect_tx(fb, P_BYTES);
                 tma_load_2d(sP + p * P_BYTES, &tmap_q, fb, (kb0 + i) * (BK / 2), n0);
             }
-            for (int p = 0; p < PSTAGES; ++p) {
-                const int issued = i > p ? (i - p - 1) / PSTAGES + 1 : 0;
+            for (int p = 0; p < L::PSTAGES; ++p) {
+                const int issued = i > p ? (i - p - 1) / L::PSTAGES + 1 : 0;
                 if (issued) drain_parity(smem_u32(&bar->pk_full[p]), (issued - 1) & 1, DRAIN_NS, status, SITE_DRAIN);
             }
         }
@@ -202,7 +210,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (lane == 0) {  // ------------------------------------------------ MMA issuer
             bool ok = true;
             for (int i = 0; i < nkb; ++i) {
-                const int s = i % STAGES, u = i / STAGES;
+                const int s = i % L::STAGES, u = i / L::STAGES;
                 const int xs = i % L::XSTAGES, xu = i / L::XSTAGES;
                 if (!wait_parity(smem_u32(&bar->x_full[xs]), xu & 1, ctl, SITE_MMA) ||
                     !wait_parity(smem_u32(&bar->a_full[s]), u & 1, ctl, SITE_MMA)) {
@@ -234,8 +242,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t *zrow = qzeros + (size_t)n * zwords;
         bool ok = true;
         auto stage = [&](int i, uint32_t zc, uint32_t s2) -> bool {
-            const int p = i % PSTAGES, up = i / PSTAGES;
-            const int s = i % STAGES, u = i / STAGES;
+            const int p = i % L::PSTAGES, up = i / L::PSTAGES;
+            const int s = i % L::STAGES, u = i / L::STAGES;
             if (!wait_parity(smem_u32(&bar->pk_full[p]), up & 1, ctl, SITE_DEQUANT)) return false;
             uint4 w;
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -425,7 +433,7 @@ wq_status dispatch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t 
                    uint16_t *y, int M, int N, int K, unsigned int *status, cudaStream_t st) {
     const bool fast = (K % 1024) == 0;
     const int tiles = ((N + BMW - 1) / BMW) * ((M + MT - 1) / MT);
-    const int splits = choose_splits(tiles, K, MT, fast, Layout<MT>::PIPE_BYTES, num_sms());
+    const int splits = choose_splits(tiles, K, MT, fast, Layout<MT>::PIPE_BYTES, Layout<MT>::CTAS_PER_SM * num_sms());
     if (fast && (K / BK / splits) % 16 == 0)
         return launch<MT, true>(tq, tx, scales, qzeros, y, M, N, K, splits, status, st);
     return launch<MT, false>(tq, tx, scales, qzeros, y, M, N, K, splits, status, st);
