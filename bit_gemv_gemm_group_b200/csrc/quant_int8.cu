@@ -104,9 +104,23 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
         }
         if (threadIdx.x == 0) scales[row] = s;
     } else {
+        // Two passes over the row: the first pass keeps its lines in L2 (evict-last policy)
+        // so that the second pass, the lines' last use (evict-first), hits L2.  Without the
+        // hint most second-pass reads went back to DRAM (ncu: 1.9x the algorithmic bytes).
+        uint64_t keep, drop;
+        asm("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(keep));
+        asm("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(drop));
         for (int k = t0; k < K; k += kRowStep) {
             float v[8];
-            load8(xr + k, v);
+            uint4 r;
+            asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                         : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(xr + k), "l"(keep));
+            {
+                const float2 a0 = half2_bits_to_float2(r.x), a1 = half2_bits_to_float2(r.y);
+                const float2 a2 = half2_bits_to_float2(r.z), a3 = half2_bits_to_float2(r.w);
+                v[0] = a0.x; v[1] = a0.y; v[2] = a1.x; v[3] = a1.y;
+                v[4] = a2.x; v[5] = a2.y; v[6] = a3.x; v[7] = a3.y;
+            }
             smooth8<MODE>(v, smooth, k);
 #pragma unroll
             for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
@@ -116,7 +130,9 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
         const float rs = __frcp_rn(s);
         for (int k = t0; k < K; k += kRowStep) {
             float v[8];
-            const uint4 r = *reinterpret_cast<const uint4 *>(xr + k);  // L2-resident re-read
+            uint4 r;  // L2-resident re-read, last use
+            asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+                         : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(xr + k), "l"(drop));
             const float2 a0 = half2_bits_to_float2(r.x), a1 = half2_bits_to_float2(r.y);
             const float2 a2 = half2_bits_to_float2(r.z), a3 = half2_bits_to_float2(r.w);
             v[0] = a0.x; v[1] = a0.y; v[2] = a1.x; v[3] = a1.y;
