@@ -6,16 +6,21 @@
 // Mathematics" (s_j = max(|X_j|)^a / max(|W_j|)^(1-a), computed offline).
 //
 // Both operands are [rows][K] row-major, so the column maxima are reductions
-// across rows.  One kernel covers X and W: each CTA owns a tile of 256
-// columns x kTileRows rows, keeps 8 running maxima per thread (one 16-byte
-// load per row), reduces its 8 warps through shared memory and folds the tile
-// into the global maxima with atomicMax on the float bit patterns (exact: for
-// non-negative floats the bit patterns order like the values).  The last CTA
-// to finish (ticket counter) turns the two maxima into s.  HBM traffic is one
+// across rows.  One kernel covers X and W: CTA (ct, g) owns the 256-column
+// tile ct and an equal share g of the rows of both matrices, with as many
+// shares as make the grid fill every CTA slot of the GPU once (no partial
+// second wave).  A thread keeps 8 running maxima (one 16-byte load per row, 8
+// rows in flight), the CTA reduces its 8 warps through shared memory and folds
+// its maxima into the global ones with atomicMax on the float bit patterns
+// (exact: for non-negative floats the bit patterns order like the values).  The last CTA
+// of a column tile's CTAs to finish (a ticket per tile) turns the tile's two
+// maxima into s.  HBM traffic is one
 // read of X and W: 2 B per element.
 //
-// Workspace layout (bytes): ax float[Kp] | aw float[Kp] | ticket uint32,
+// Workspace layout (words): ax float[Kp] | aw float[Kp] | tickets uint32[ceil4(K/256)],
 // Kp = K rounded up to 4.
+#include <algorithm>
+
 #include "wq_device.cuh"
 #include "wq_host.h"
 
@@ -24,47 +29,27 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kTileCols = 256;  // 32 lanes x 8 columns
-constexpr int kTileRows = 256;
 
 __host__ __device__ inline size_t padded(int K) { return ((size_t)K + 3) & ~(size_t)3; }
 
 __device__ __forceinline__ uint32_t umax2(uint32_t a, uint32_t b) { return __vmaxu2(a, b); }
 
-__global__ void __launch_bounds__(kThreads) smooth_kernel(const uint16_t *__restrict__ x, int M,
-                                                          const uint16_t *__restrict__ w, int N, int K,
-                                                          float alpha, float *__restrict__ s,
-                                                          unsigned int *__restrict__ ws, int tiles_x,
-                                                          int col_tiles, unsigned int total_blocks) {
-    __shared__ uint32_t part[kThreads / 32][kTileCols / 2];  // packed fp16 |max| pairs per warp
-    __shared__ bool last;
-    const size_t Kp = padded(K);
-    unsigned int *ax = ws;
-    unsigned int *aw = ws + Kp;
-    unsigned int *ticket = ws + 2 * Kp;
-
-    int tile = blockIdx.x;
-    const bool is_x = tile < tiles_x;
-    if (!is_x) tile -= tiles_x;
-    const uint16_t *src = is_x ? x : w;
-    const int rows = is_x ? M : N;
-    unsigned int *dst = is_x ? ax : aw;
-    const int ct = tile % col_tiles;
-    const int rt = tile / col_tiles;
+// Column maxima of rows [r0, r1) of one 256-column tile, folded into `dst` with
+// atomicMax on the float bit patterns.  All of the CTA's threads call it.
+__device__ __forceinline__ void tile_column_max(const uint16_t *__restrict__ src, int K, int col, int r0, int r1,
+                                                int ct, unsigned int *__restrict__ dst,
+                                                uint32_t (*part)[kTileCols / 2]) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int col = ct * kTileCols + lane * 8;
-    const int r0 = rt * kTileRows;
-    const int r1 = min(rows, r0 + kTileRows);
-
     // |value| as fp16 bits; for non-negative fp16 the bit patterns order like the values.
     uint32_t m0 = 0, m1 = 0, m2 = 0, m3 = 0;
     if (col < K) {
         int r = r0 + warp;
-        for (; r + 3 * 8 < r1; r += 4 * 8) {
-            uint4 v[4];
+        for (; r + 7 * 8 < r1; r += 8 * 8) {  // 8 rows of 16-byte loads in flight per thread
+            uint4 v[8];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) v[u] = ld_stream_u4(src + (size_t)(r + 8 * u) * K + col);
+            for (int u = 0; u < 8; ++u) v[u] = ld_stream_u4(src + (size_t)(r + 8 * u) * K + col);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
+            for (int u = 0; u < 8; ++u) {
                 m0 = umax2(m0, v[u].x & 0x7fff7fffu);
                 m1 = umax2(m1, v[u].y & 0x7fff7fffu);
                 m2 = umax2(m2, v[u].z & 0x7fff7fffu);
@@ -79,12 +64,13 @@ __global__ void __launch_bounds__(kThreads) smooth_kernel(const uint16_t *__rest
             m3 = umax2(m3, v.w & 0x7fff7fffu);
         }
     }
+    __syncthreads();  // `part` is free (a previous call's readers are done)
     part[warp][lane * 4 + 0] = m0;
     part[warp][lane * 4 + 1] = m1;
     part[warp][lane * 4 + 2] = m2;
     part[warp][lane * 4 + 3] = m3;
     __syncthreads();
-    if (threadIdx.x < kTileCols / 2) {
+    if (threadIdx.x < kTileCols / 2 && r0 < r1) {
         uint32_t m = 0;
 #pragma unroll
         for (int i = 0; i < kThreads / 32; ++i) m = umax2(m, part[i][threadIdx.x]);
@@ -92,15 +78,36 @@ __global__ void __launch_bounds__(kThreads) smooth_kernel(const uint16_t *__rest
         if (c < K) atomicMax(dst + c, __float_as_uint(half_bits_to_float((uint16_t)(m & 0xffffu))));
         if (c + 1 < K) atomicMax(dst + c + 1, __float_as_uint(half_bits_to_float((uint16_t)(m >> 16))));
     }
+}
 
-    // The last CTA to arrive turns the maxima into smoothing factors.
+// CTA (ct, g): column tile ct of both matrices, row share g of `groups` (X and W
+// rows split evenly), so that the grid fills the SMs' CTA slots exactly once.
+__global__ void __launch_bounds__(kThreads) smooth_kernel(const uint16_t *__restrict__ x, int M,
+                                                          const uint16_t *__restrict__ w, int N, int K,
+                                                          float alpha, float *__restrict__ s,
+                                                          unsigned int *__restrict__ ws, int col_tiles, int groups) {
+    __shared__ uint32_t part[kThreads / 32][kTileCols / 2];  // packed fp16 |max| pairs per warp
+    __shared__ bool last;
+    const size_t Kp = padded(K);
+    unsigned int *ax = ws;
+    unsigned int *aw = ws + Kp;
+    unsigned int *ticket = ws + 2 * Kp;  // one per column tile
+
+    const int ct = blockIdx.x % col_tiles;
+    const int g = blockIdx.x / col_tiles;
+    const int lane = threadIdx.x & 31;
+    const int col = ct * kTileCols + lane * 8;
+    tile_column_max(x, K, col, (int)((long long)M * g / groups), (int)((long long)M * (g + 1) / groups), ct, ax, part);
+    tile_column_max(w, K, col, (int)((long long)N * g / groups), (int)((long long)N * (g + 1) / groups), ct, aw, part);
+
+    // The last of the column tile's CTAs to arrive turns its 256 maxima into smoothing factors.
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) last = atomicAdd(ticket, 1u) == total_blocks - 1;
+    if (threadIdx.x == 0) last = atomicAdd(ticket + ct, 1u) == (unsigned int)groups - 1;
     __syncthreads();
     if (!last) return;
     __threadfence();
-    for (int j = threadIdx.x; j < K; j += kThreads) {
+    for (int j = ct * kTileCols + threadIdx.x; j < min(K, (ct + 1) * kTileCols); j += kThreads) {
         const float a_x = fmaxf(__uint_as_float(__ldcg(ax + j)), 1e-5f);
         const float a_w = fmaxf(__uint_as_float(__ldcg(aw + j)), 1e-5f);
         float num, den;
@@ -115,12 +122,27 @@ __global__ void __launch_bounds__(kThreads) smooth_kernel(const uint16_t *__rest
     }
 }
 
+// Resident CTAs of smooth_kernel on the current device (SMs x CTAs per SM), cached.
+int smooth_slots() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148 * 8;
+    if (!cached[dev]) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, smooth_kernel, kThreads, 0) != cudaSuccess ||
+            per_sm <= 0)
+            per_sm = 8;
+        cached[dev] = per_sm * num_sms();
+    }
+    return cached[dev];
+}
+
 }  // namespace
 }  // namespace wq
 
 extern "C" size_t wq_smooth_workspace_bytes(int K) {
     if (K <= 0) return 0;
-    return (2 * wq::padded(K) + 4) * sizeof(unsigned int);
+    return (2 * wq::padded(K) + wq::padded((K + wq::kTileCols - 1) / wq::kTileCols)) * sizeof(unsigned int);
 }
 
 extern "C" wq_status wq_smooth(const uint16_t *x, int M, const uint16_t *w, int N, int K, float alpha, float *s,
@@ -134,17 +156,17 @@ extern "C" wq_status wq_smooth(const uint16_t *x, int M, const uint16_t *w, int 
     WQ_REQUIRE(K % 8 == 0, WQ_ERR_UNSUPPORTED, "wq_smooth: K (%d) must be a multiple of 8", K);
     WQ_REQUIRE(alpha >= 0.0f && alpha <= 1.0f, WQ_ERR_INVALID_ARG, "wq_smooth: alpha must lie in [0, 1]");
     const int col_tiles = (K + wq::kTileCols - 1) / wq::kTileCols;
-    const long long tx = (long long)col_tiles * ((M + wq::kTileRows - 1) / wq::kTileRows);
-    const long long tw = (long long)col_tiles * ((N + wq::kTileRows - 1) / wq::kTileRows);
-    WQ_REQUIRE(tx + tw < (1ll << 31), WQ_ERR_UNSUPPORTED, "wq_smooth: problem too large");
+    // row shares per column tile: fill every CTA slot of the GPU exactly once
+    const int slots = wq::smooth_slots();
+    const int groups = std::max(1, std::min(std::max(M, N), slots / col_tiles));
+    WQ_REQUIRE((long long)col_tiles * groups < (1ll << 31), WQ_ERR_UNSUPPORTED, "wq_smooth: problem too large");
     cudaStream_t st = wq::as_stream(stream);
     cudaError_t e = cudaMemsetAsync(workspace, 0, wq_smooth_workspace_bytes(K), st);
     if (e != cudaSuccess) return wq::fail(WQ_ERR_CUDA, "wq_smooth: clearing the workspace failed: %s",
                                           cudaGetErrorString(e));
-    const unsigned int total = (unsigned int)(tx + tw);
+    const unsigned int total = (unsigned int)(col_tiles * groups);
     wq::smooth_kernel<<<total, wq::kThreads, 0, st>>>(x, M, w, N, K, alpha, s,
-                                                      static_cast<unsigned int *>(workspace), (int)tx, col_tiles,
-                                                      total);
+                                                      static_cast<unsigned int *>(workspace), col_tiles, groups);
     return wq::check_launch("wq_smooth");
 }
 
@@ -166,7 +188,8 @@ extern "C" wq_status wq_smooth(const uint16_t *x, int M, const uint16_t *w, int 
 namespace wq {
 namespace {
 
-constexpr size_t kNoAllocWords = 2 * (size_t)WQ_SMOOTH_NOALLOC_MAX_K + 4;  // ax | aw | ticket, K padded to 4
+// ax | aw | one ticket per 256-column tile, each padded to 4 words
+constexpr size_t kNoAllocWords = 2 * (size_t)WQ_SMOOTH_NOALLOC_MAX_K + WQ_SMOOTH_NOALLOC_MAX_K / 256;
 static __device__ __align__(256) unsigned int g_smooth_scratch[kNoAllocWords];
 
 constexpr int kScratchDevices = 64;

@@ -139,8 +139,8 @@ wq_status wq_smooth(const uint16_t *x, int M, const uint16_t *w, int N, int K, f
  * Same arguments, result and restrictions as wq_smooth, plus K <=
  * WQ_SMOOTH_NOALLOC_MAX_K (larger K returns WQ_ERR_UNSUPPORTED and launches
  * nothing).
- * The workspace is a fixed array of 2 * WQ_SMOOTH_NOALLOC_MAX_K + 4 words
- * (512 KiB) held in the device memory of every GPU that loads the library,
+ * The workspace is a fixed array of 2 * WQ_SMOOTH_NOALLOC_MAX_K + 256 words
+ * (513 KiB) held in the device memory of every GPU that loads the library,
  * until the process exits.  The call allocates nothing: no cudaMalloc, no
  * cudaFree, no allocating library routine.  The first call on a device (made
  * while that device is current) looks up the array's device address with

@@ -74,8 +74,10 @@ def test_sizes_rejected(wq):
 
 
 def test_workspace_size(wq):
-    assert wq.smooth_workspace_bytes(8192) == (2 * 8192 + 4) * 4
+    # column maxima of X and W (K padded to 4 words each) + one ticket per 256 columns (padded to 4)
+    assert wq.smooth_workspace_bytes(8192) == (2 * 8192 + 32) * 4
     assert wq.smooth_workspace_bytes(10) == (2 * 12 + 4) * 4
+    assert wq.smooth_workspace_bytes(1300) == (2 * 1300 + 8) * 4
     assert wq.smooth_workspace_bytes(0) == 0
 
 
