@@ -249,6 +249,93 @@ __global__ void __launch_bounds__(256) quant_int4_group_f16_kernel(const uint16_
     if (lane == 0) qzeros[(size_t)n * zwords + zw] = zword;
 }
 
+// G >= 64: 16 elements (two 16-byte loads) per lane, so the per-group work
+// (range butterfly, scale, zero point), which a warp pays once for all its
+// lanes, is spread over twice the elements; the range travels as one fp16x2
+// value (-lo, hi) (negation and max are exact in fp16), one shuffle and one
+// max per butterfly step.
+template <int G>
+__global__ void __launch_bounds__(256) quant_int4_group_f16x16_kernel(const uint16_t *__restrict__ w, int N, int K,
+                                                                      uint32_t *__restrict__ qweight,
+                                                                      uint16_t *__restrict__ scales,
+                                                                      uint32_t *__restrict__ qzeros) {
+    constexpr int LPG = G / 16;      // lanes per group
+    constexpr int GPI = 32 / LPG;    // groups per warp iteration
+    constexpr int ITERS = 8 / GPI;   // iterations per zero word (8 groups)
+    static_assert(ITERS >= 1, "G >= 64");
+    const int groups = K / G;
+    const int zwords = (groups + 7) / 8;
+    const int lane = threadIdx.x & 31;
+    const long long unit = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (unit >= (long long)N * zwords) return;
+    const int n = (int)(unit / zwords);
+    const int zw = (int)(unit % zwords);
+    const int sub = lane / LPG;  // group slot within an iteration
+    const int li = lane % LPG;   // lane within the group
+
+    // Issue every load of this warp first.
+    uint4 raw[ITERS][2];
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int j = zw * 8 + it * GPI + sub;
+        const uint16_t *p = w + (size_t)n * K + (size_t)j * G + li * 16;
+        raw[it][0] = j < groups ? ld_stream_u4(p) : make_uint4(0u, 0u, 0u, 0u);
+        raw[it][1] = j < groups ? ld_stream_u4(p + 8) : make_uint4(0u, 0u, 0u, 0u);
+    }
+
+    uint32_t zacc = 0;
+#pragma unroll
+    for (int it = 0; it < ITERS; ++it) {
+        const int j = zw * 8 + it * GPI + sub;
+        const uint4 c0 = raw[it][0], c1 = raw[it][1];
+        // (-lo, hi) with lo = min(0, min w), hi = max(0, max w), as fp16x2
+        const uint32_t mn = hmin2_bits(hmin2_bits(hmin2_bits(c0.x, c0.y), hmin2_bits(c0.z, c0.w)),
+                                       hmin2_bits(hmin2_bits(c1.x, c1.y), hmin2_bits(c1.z, c1.w)));
+        const uint32_t mx = hmax2_bits(hmax2_bits(hmax2_bits(c0.x, c0.y), hmax2_bits(c0.z, c0.w)),
+                                       hmax2_bits(hmax2_bits(c1.x, c1.y), hmax2_bits(c1.z, c1.w)));
+        uint32_t r = hmax2_bits(__byte_perm(mn, mx, 0x5410) ^ 0x00008000u, __byte_perm(mn, mx, 0x7632) ^ 0x00008000u);
+        r = hmax2_bits(r, 0u);
+#pragma unroll
+        for (int off = LPG / 2; off >= 1; off >>= 1) r = hmax2_bits(r, __shfl_xor_sync(0xffffffffu, r, off));
+        const float2 rf = half2_bits_to_float2(r);
+        const float lo = -rf.x, hi = rf.y;
+        // s = fp16((hi - lo) / 15); a zero scale becomes 1.
+        uint16_t s16 = float_to_half_bits_rn(__fdiv_rn(hi - lo, 15.0f));
+        if (s16 == 0) s16 = 0x3c00;
+        const float s = half_bits_to_float(s16);
+        const float rs = __frcp_rn(s);
+        // z = round(-lo / s) in [0, 15]; |-lo / s| and |w / s| stay below 32 (E = 4)
+        const int z = clampi(rne_quotient<4>(-lo, s, rs), 0, 15);
+        if (j < groups) {
+            const uint32_t h[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+            uint32_t p[8];
+            uint32_t bad = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) p[e] = pair_rne(h[e], rs, bad);
+            if (bad >> 31) {  // a near-tie: the IEEE quotient decides every code of this lane
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float2 f = half2_bits_to_float2(h[e]);
+                    const uint32_t a = (uint32_t)__float2int_rn(__fdiv_rn(f.x, s)) & 0xFFFFu;
+                    const uint32_t b = (uint32_t)__float2int_rn(__fdiv_rn(f.y, s)) & 0xFFFFu;
+                    p[e] = a | (b << 16);
+                }
+            }
+            const uint32_t z2 = (uint32_t)z * 0x00010001u;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) p[e] = __vmins2(__vmaxs2(__vadd2(p[e], z2), 0u), 0x000F000Fu);
+            *reinterpret_cast<uint2 *>(qweight + (size_t)n * (K / 8) + (size_t)j * (G / 8) + li * 2) =
+                make_uint2(pack8(p[0], p[1], p[2], p[3]), pack8(p[4], p[5], p[6], p[7]));
+            if (li == 0) {
+                scales[(size_t)n * groups + j] = s16;
+                zacc |= (uint32_t)z << (4 * (j & 7));
+            }
+        }
+    }
+    const uint32_t zword = __reduce_or_sync(0xffffffffu, zacc);
+    if (lane == 0) qzeros[(size_t)n * zwords + zw] = zword;
+}
+
 template <typename TIn, int G>
 cudaError_t launch(const void *w, int N, int K, uint32_t *qweight, uint16_t *scales, uint32_t *qzeros,
                    cudaStream_t stream) {
@@ -256,7 +343,10 @@ cudaError_t launch(const void *w, int N, int K, uint32_t *qweight, uint16_t *sca
     const long long units = (long long)N * zwords;
     const int warps_per_block = 8;
     const long long blocks = (units + warps_per_block - 1) / warps_per_block;
-    if (std::is_same<TIn, __half>::value)
+    if (std::is_same<TIn, __half>::value && G >= 64)
+        quant_int4_group_f16x16_kernel<G < 64 ? 64 : G><<<(unsigned)blocks, warps_per_block * 32, 0, stream>>>(
+            static_cast<const uint16_t *>(w), N, K, qweight, scales, qzeros);
+    else if (std::is_same<TIn, __half>::value)
         quant_int4_group_f16_kernel<G><<<(unsigned)blocks, warps_per_block * 32, 0, stream>>>(
             static_cast<const uint16_t *>(w), N, K, qweight, scales, qzeros);
     else
