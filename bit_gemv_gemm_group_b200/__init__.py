@@ -274,5 +274,6 @@ def device_status(stream=None) -> int:
     return int(lib.wq_device_status(_P(_stream(stream))))
 
 
-def set_wait_limit(polls: int) -> None:
-    lib.wq_set_wait_limit(int(polls))
+def set_wait_limit(nanoseconds: int) -> None:
+    """Wall-clock limit of each bounded wait in the pipelined kernels (0 restores the 2 s default)."""
+    lib.wq_set_wait_limit(int(nanoseconds))
