@@ -18,7 +18,7 @@ import torch
 
 __all__ = ["WQError", "lib", "quantize_group_int4", "quantize_int8_per_channel", "quantize_int8_per_token",
            "smooth", "smooth_workspace_bytes", "smooth_noalloc", "gemv_w4a16", "gemm_w4a16", "gemm_w8a8", "gemv_w8a16",
-           "matmul_w4a16", "device_status", "set_wait_limit", "LIB_PATH"]
+           "matmul_w4a16", "device_status", "set_wait_limit", "selftest_wait_timeout", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwq.so")
 
@@ -51,6 +51,7 @@ _SIGS = {
     "wq_gemm_w8a8": [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P],
     "wq_gemv_w8a16": [_P, _I, _P, _P, _I, _I, _P, _P],
     "wq_device_status": [_P],
+    "wq_selftest_wait_timeout": [_P],
 }
 for _name, _args in _SIGS.items():
     _fn = getattr(lib, _name)
@@ -272,6 +273,11 @@ def gemv_w8a16(x, wq, sw, out=None, stream=None):
 def device_status(stream=None) -> int:
     """Synchronizes the stream and returns (and clears) the device status word (0 = WQ_OK)."""
     return int(lib.wq_device_status(_P(_stream(stream))))
+
+
+def selftest_wait_timeout(stream=None) -> None:
+    """Launches the bounded-wait self-test (a wait that must time out; see wq.h)."""
+    _check(lib.wq_selftest_wait_timeout(_P(_stream(stream))), "wq_selftest_wait_timeout")
 
 
 def set_wait_limit(nanoseconds: int) -> None:

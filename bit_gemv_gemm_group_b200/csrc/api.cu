@@ -127,3 +127,44 @@ extern "C" wq_status wq_device_status(void *stream) {
     }
     return WQ_OK;
 }
+
+// ---------------------------------------------------------------------------
+// Self-test of the bounded waits: one thread waits, through the same code the
+// pipelined kernels use, on an mbarrier that nothing ever arrives on.  The wait
+// must give up after the current limit and record its site code in the status
+// word, which the next wq_device_status() reports as WQ_ERR_TIMEOUT.
+// ---------------------------------------------------------------------------
+#include "sm100.cuh"
+
+namespace wq {
+namespace {
+
+constexpr unsigned kSelftestSite = 0x800;
+
+__global__ void selftest_wait_kernel(unsigned int *status, uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        sm100::mbar_init(sm100::smem_u32(&bar), 1);
+        abort_flag = 0;
+        sm100::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const sm100::WaitCtl ctl{&abort_flag, status, limit_ns};
+        sm100::wait_parity(sm100::smem_u32(&bar), 0, ctl, kSelftestSite);  // phase 0 never completes
+    }
+}
+
+}  // namespace
+}  // namespace wq
+
+extern "C" wq_status wq_selftest_wait_timeout(void *stream) {
+    unsigned int *status = wq::device_status_word();
+    if (!status) return WQ_ERR_CUDA;
+    wq::selftest_wait_kernel<<<1, 32, 0, wq::as_stream(stream)>>>(status, wq::wait_limit());
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return wq::fail(WQ_ERR_CUDA, "wq_selftest_wait_timeout: launch failed: %s", cudaGetErrorString(e));
+    return WQ_OK;
+}

@@ -228,6 +228,16 @@ wq_status wq_device_status(void *stream);
  */
 void wq_set_wait_limit(uint64_t nanoseconds);
 
+/*
+ * Self-test of the bounded waits (failure detection; the pages have no
+ * counterpart): launches one thread that waits, through the same bounded-wait
+ * code as the pipelined kernels, on a barrier that nothing completes.  After
+ * the current wait limit (wq_set_wait_limit) it gives up, so the next
+ * wq_device_status() returns WQ_ERR_TIMEOUT.  Set a short limit first: with
+ * the default the wait lasts two seconds.
+ */
+wq_status wq_selftest_wait_timeout(void *stream);
+
 #ifdef __cplusplus
 }
 #endif
