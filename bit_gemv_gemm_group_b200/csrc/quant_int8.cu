@@ -45,17 +45,40 @@ __device__ __forceinline__ void load8(const uint16_t *p, float (&v)[8]) {
     v[4] = c.x; v[5] = c.y; v[6] = d.x; v[7] = d.y;
 }
 
-// |v / s| <= 127 (1 + 2^-23) < 2^8 (E = 7): codes via rne_quotient, identical to rne(fl(v / s)).
+// |v / s| <= 127 (1 + 2^-23) < 2^8 (E = 7): the codes equal rne(fl(v / s)).  Pairs are
+// decided with f32x2 arithmetic: t = v * RN(1/s), r = t + 1.5*2^23 (rne(t) lands in r's low
+// mantissa bits), d = t - (r - 1.5*2^23) (exact).  rne(t) is rne(v / s) unless |d| comes
+// within the guard band of 1/2 (t is within 2^(E-22) of v / s, so a band of 2^-13 > 2^(E-21)
+// suffices); a chunk with such a near-tie is redone with rne_quotient (IEEE quotient).
+__device__ __forceinline__ uint32_t pair_rne8(float a, float b, float rs, uint32_t &bad) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+    constexpr float kGuardSq = (0.5f - 0x1p-13f) * (0.5f - 0x1p-13f);
+    const float2 t = __fmul2_rn(make_float2(a, b), make_float2(rs, rs));
+    const float2 r = __fadd2_rn(t, make_float2(kMagic, kMagic));
+    const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
+    const float2 d = __fadd2_rn(t, make_float2(-n.x, -n.y));
+    const float2 e = __ffma2_rn(d, make_float2(-d.x, -d.y), make_float2(kGuardSq, kGuardSq));
+    bad |= __float_as_uint(e.x) | __float_as_uint(e.y);
+    return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);  // int16x2 rne(t)
+}
+
 __device__ __forceinline__ uint2 quant8(const float (&v)[8], float s, float rs) {
-    uint32_t lo = 0, hi = 0;
+    uint32_t bad = 0;
+    uint32_t p0 = pair_rne8(v[0], v[1], rs, bad), p1 = pair_rne8(v[2], v[3], rs, bad);
+    uint32_t p2 = pair_rne8(v[4], v[5], rs, bad), p3 = pair_rne8(v[6], v[7], rs, bad);
+    if (bad >> 31) {  // a near-tie: the IEEE quotient decides every code of this chunk
+        uint32_t c[8];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int q0 = clampi(rne_quotient<7>(v[e], s, rs), -128, 127);
-        const int q1 = clampi(rne_quotient<7>(v[e + 4], s, rs), -128, 127);
-        lo |= (uint32_t)(q0 & 0xff) << (8 * e);
-        hi |= (uint32_t)(q1 & 0xff) << (8 * e);
+        for (int e = 0; e < 8; ++e) c[e] = (uint32_t)rne_quotient<7>(v[e], s, rs) & 0xFFFFu;
+        p0 = c[0] | (c[1] << 16); p1 = c[2] | (c[3] << 16); p2 = c[4] | (c[5] << 16); p3 = c[6] | (c[7] << 16);
     }
-    return make_uint2(lo, hi);
+    const uint32_t lo = 0xFF80FF80u, hi = 0x007F007Fu;  // [-128, 127] per 16-bit lane
+    p0 = __vmins2(__vmaxs2(p0, lo), hi);
+    p1 = __vmins2(__vmaxs2(p1, lo), hi);
+    p2 = __vmins2(__vmaxs2(p2, lo), hi);
+    p3 = __vmins2(__vmaxs2(p3, lo), hi);
+    // low byte of every 16-bit lane, in element order
+    return make_uint2(__byte_perm(p0, p1, 0x6420), __byte_perm(p2, p3, 0x6420));
 }
 
 __device__ __forceinline__ float block_max(float a, float *red) {
