@@ -126,12 +126,11 @@ __global__ void __launch_bounds__(256) quant_int4_group_kernel(const TIn *__rest
 // ---------------------------------------------------------------------------
 // fp16 input: the same decomposition with packed arithmetic.  The range comes
 // from fp16x2 min/max on the raw bits (exact); a pair of codes is decided with
-// f32x2 operations:  t = w * RN(1/s),  r = t + 1.5*2^23 (rne(t) lands in r's
-// low mantissa bits),  d = t - (r - 1.5*2^23) (exact).  The pair is exact
+// f32x2 operations:  t = w * RN(1/s),  r = t + (1.5*2^23 + z) (rne(t) + z lands
+// in r's low mantissa bits),  d = t - (r - (1.5*2^23 + z)) (exact).  The pair is exact
 // unless |d| comes within 2^-16 of 1/2 (a near-tie of w*RN(1/s), the guard of
 // rne_quotient widened), in which case the lane recomputes its 8 codes with
-// the IEEE quotient.  Adding z, clamping and nibble packing run on 16-bit
-// SIMD lanes.
+// the IEEE quotient.  Clamping and nibble packing run on 16-bit SIMD lanes.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t hmin2_bits(uint32_t a, uint32_t b) {
     uint32_t d;
@@ -145,19 +144,19 @@ __device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
     return d;
 }
 
-// rne(w * rs) of an fp16 pair as int16x2; `bad` collects the sign bit of
-// (1/2 - 2^-16)^2 - d^2 (set when a lane lies in the guard band).
-__device__ __forceinline__ uint32_t pair_rne(uint32_t h2, float rs, uint32_t &bad) {
-    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+// rne(w * rs) + z of an fp16 pair as int16x2, with magic = 1.5 * 2^23 + z (adding the
+// integer z before rounding is exact, so it folds into the rounding add); `bad` collects
+// the sign bit of (1/2 - 2^-16)^2 - d^2 (set when a lane lies in the guard band).
+__device__ __forceinline__ uint32_t pair_rne(uint32_t h2, float rs, float magic, uint32_t &bad) {
     constexpr float kGuardSq = (0.5f - 0x1p-16f) * (0.5f - 0x1p-16f);
     const float2 f = half2_bits_to_float2(h2);
     const float2 t = __fmul2_rn(f, make_float2(rs, rs));
-    const float2 r = __fadd2_rn(t, make_float2(kMagic, kMagic));
-    const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
+    const float2 r = __fadd2_rn(t, make_float2(magic, magic));
+    const float2 n = __fadd2_rn(r, make_float2(-magic, -magic));
     const float2 d = __fadd2_rn(t, make_float2(-n.x, -n.y));
     const float2 e = __ffma2_rn(d, make_float2(-d.x, -d.y), make_float2(kGuardSq, kGuardSq));
     bad |= __float_as_uint(e.x) | __float_as_uint(e.y);
-    return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);  // low 16 bits: rne(t)
+    return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);  // low 16 bits: rne(t) + z
 }
 
 // codes c_e (int16x2 pairs (c0,c1), (c2,c3), ...) -> one word, code e at bits 4e
@@ -218,26 +217,26 @@ __global__ void __launch_bounds__(256) quant_int4_group_f16_kernel(const uint16_
         const int z = clampi(rne_quotient<4>(-lo, s, rs), 0, 15);
         if (j < groups) {
             uint32_t bad = 0;
-            uint32_t p0 = pair_rne(c.x, rs, bad), p1 = pair_rne(c.y, rs, bad);
-            uint32_t p2 = pair_rne(c.z, rs, bad), p3 = pair_rne(c.w, rs, bad);
+            const float magic = 12582912.0f + (float)z;  // 1.5 * 2^23 + z
+            uint32_t p0 = pair_rne(c.x, rs, magic, bad), p1 = pair_rne(c.y, rs, magic, bad);
+            uint32_t p2 = pair_rne(c.z, rs, magic, bad), p3 = pair_rne(c.w, rs, magic, bad);
             if (bad >> 31) {  // a near-tie: the IEEE quotient decides every code of this lane
                 const uint32_t h[4] = {c.x, c.y, c.z, c.w};
                 uint32_t pp[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 f = half2_bits_to_float2(h[e]);
-                    const uint32_t a = (uint32_t)__float2int_rn(__fdiv_rn(f.x, s)) & 0xFFFFu;
-                    const uint32_t b = (uint32_t)__float2int_rn(__fdiv_rn(f.y, s)) & 0xFFFFu;
+                    const uint32_t a = (uint32_t)(__float2int_rn(__fdiv_rn(f.x, s)) + z) & 0xFFFFu;
+                    const uint32_t b = (uint32_t)(__float2int_rn(__fdiv_rn(f.y, s)) + z) & 0xFFFFu;
                     pp[e] = a | (b << 16);
                 }
                 p0 = pp[0]; p1 = pp[1]; p2 = pp[2]; p3 = pp[3];
             }
-            const uint32_t z2 = (uint32_t)z * 0x00010001u;
             const uint32_t top = 0x000F000Fu;
-            p0 = __vmins2(__vmaxs2(__vadd2(p0, z2), 0u), top);
-            p1 = __vmins2(__vmaxs2(__vadd2(p1, z2), 0u), top);
-            p2 = __vmins2(__vmaxs2(__vadd2(p2, z2), 0u), top);
-            p3 = __vmins2(__vmaxs2(__vadd2(p3, z2), 0u), top);
+            p0 = __vmins2(__vmaxs2(p0, 0u), top);
+            p1 = __vmins2(__vmaxs2(p1, 0u), top);
+            p2 = __vmins2(__vmaxs2(p2, 0u), top);
+            p3 = __vmins2(__vmaxs2(p3, 0u), top);
             qweight[(size_t)n * (K / 8) + (size_t)j * (G / 8) + li] = pack8(p0, p1, p2, p3);
             if (li == 0) {
                 scales[(size_t)n * groups + j] = s16;
@@ -310,20 +309,20 @@ __global__ void __launch_bounds__(256) quant_int4_group_f16x16_kernel(const uint
             const uint32_t h[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
             uint32_t p[8];
             uint32_t bad = 0;
+            const float magic = 12582912.0f + (float)z;  // 1.5 * 2^23 + z
 #pragma unroll
-            for (int e = 0; e < 8; ++e) p[e] = pair_rne(h[e], rs, bad);
+            for (int e = 0; e < 8; ++e) p[e] = pair_rne(h[e], rs, magic, bad);
             if (bad >> 31) {  // a near-tie: the IEEE quotient decides every code of this lane
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const float2 f = half2_bits_to_float2(h[e]);
-                    const uint32_t a = (uint32_t)__float2int_rn(__fdiv_rn(f.x, s)) & 0xFFFFu;
-                    const uint32_t b = (uint32_t)__float2int_rn(__fdiv_rn(f.y, s)) & 0xFFFFu;
+                    const uint32_t a = (uint32_t)(__float2int_rn(__fdiv_rn(f.x, s)) + z) & 0xFFFFu;
+                    const uint32_t b = (uint32_t)(__float2int_rn(__fdiv_rn(f.y, s)) + z) & 0xFFFFu;
                     p[e] = a | (b << 16);
                 }
             }
-            const uint32_t z2 = (uint32_t)z * 0x00010001u;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) p[e] = __vmins2(__vmaxs2(__vadd2(p[e], z2), 0u), 0x000F000Fu);
+            for (int e = 0; e < 8; ++e) p[e] = __vmins2(__vmaxs2(p[e], 0u), 0x000F000Fu);
             *reinterpret_cast<uint2 *>(qweight + (size_t)n * (K / 8) + (size_t)j * (G / 8) + li * 2) =
                 make_uint2(pack8(p[0], p[1], p[2], p[3]), pack8(p[4], p[5], p[6], p[7]));
             if (li == 0) {

@@ -33,8 +33,17 @@ __device__ __forceinline__ void smooth8(float (&v)[8], const float *__restrict__
     const float4 a = __ldg(reinterpret_cast<const float4 *>(smooth + k));
     const float4 b = __ldg(reinterpret_cast<const float4 *>(smooth + k + 4));
     const float s[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    if (MODE == kMul) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) v[e] = (MODE == kMul) ? __fmul_rn(v[e], s[e]) : __fdiv_rn(v[e], s[e]);
+        for (int e = 0; e < 8; e += 2) {
+            const float2 p = __fmul2_rn(make_float2(v[e], v[e + 1]), make_float2(s[e], s[e + 1]));
+            v[e] = p.x;
+            v[e + 1] = p.y;
+        }
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = __fdiv_rn(v[e], s[e]);
+    }
 }
 
 __device__ __forceinline__ void load8(const uint16_t *p, float (&v)[8]) {
