@@ -8,7 +8,15 @@
 //
 //   y[b][n] = fp16_rn( sum_j s[n][j] * sum_{k in group j} (q[n][k] - z[n][j]) * x[b][k] )
 //
-// Work decomposition: a warp owns R weight rows and walks K in steps of 1024
+// Three kernels, chosen by wq_gemv_w4a16:
+//   - group size 128, K % 256 == 0 (every decode shape): the streaming
+//     tensor-core kernel further below (TMA ring, producer-built B fragments,
+//     codes fed to mma.sync as fp16 subnormals); it also serves wq_gemm_w4a16
+//     for up to 32 rows in passes of 16;
+//   - group size 128, other K: a register-prefetch mma.sync kernel;
+//   - other group sizes: the CUDA-core kernel that follows.
+//
+// CUDA-core kernel.  Work decomposition: a warp owns R weight rows and walks K in steps of 1024
 // weights: lane l of step t reads the 16-byte chunk c = 32 t + l of each of
 // its rows (32 consecutive codes, all in one group since g >= 32), so a warp
 // load instruction covers 512 contiguous bytes of a row.  Loads bypass L1
@@ -827,7 +835,8 @@ wq_status gemv_stream_nt(const uint16_t *x, int B, const uint32_t *qw, const uin
 
 }  // namespace
 
-// Batch 1..16 with K % 256 == 0, group size 128 (also serves wq_gemm_w4a16 at M <= 16).
+// Batch 1..16 with K % 256 == 0, group size 128 (also serves wq_gemm_w4a16 for up to 32 rows,
+// in passes of 16).
 wq_status gemv_stream(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
                       int K, uint16_t *y, cudaStream_t st, const char *who) {
     if (B <= 8) return gemv_stream_nt<1, 7, 2>(x, B, qw, sc, qz, N, K, y, st, who);
