@@ -12,16 +12,21 @@
 //
 // Swap-AB: the MMA's M dimension is 128 weight rows (TMEM lanes) and its N
 // dimension is the activation tile (16..128 rows of x), so small batches still
-// use full 128-row MMAs.  Per CTA (480 threads):
+// use full 128-row MMAs.  Per CTA (512 threads):
 //   warp 0      TMA: packed weight tiles (128 rows x 32 bytes = 64 codes) into
 //               a 6- or 12-deep ring (two or one CTAs per SM, see Layout)
 //   warp 1      TMA: x tiles (MT rows x 64 fp16, 128-byte swizzle)
-//   warp 2      TMEM allocation and tcgen05.mma issue (4 x K=16 per stage)
+//   warps 2, 15 tcgen05.mma issue (4 x K=16 per stage), warp 2 for the even
+//               stages and warp 15 for the odd ones, each into its own fp32
+//               accumulator in TMEM (warp 2 also allocates it); one thread
+//               issues a tcgen05.mma only every ~50 cycles, so a second issuer
+//               measured 6% (64 rows) to 16% (100-128 rows) faster on B200
 //   warps 3-10  dequantize: each thread turns 32 codes of one row into fp16
 //               with PRMT/LOP3 (code -> 1024 + q), one exact fp16x2 fma
 //               (-> q - z) and one fp16x2 multiply by the scale, and stores
 //               them into the 128-byte-swizzled K-major A tile
-//   warps 11-14 epilogue: tcgen05.ld of the 128 x MT fp32 accumulator
+//   warps 11-14 epilogue: tcgen05.ld of the two 128 x MT fp32 accumulators,
+//               summed
 // K is split over the S CTAs of a thread-block cluster when the weight tiles
 // alone would leave SMs idle; their fp32 partial tiles are summed in the
 // leading CTA's shared memory through distributed shared memory, so the
@@ -43,7 +48,7 @@ constexpr int MAX_STAGES = 4;               // dequantized A stages (barrier arr
 constexpr int MAX_PSTAGES = 12;             // packed-tile ring (barrier arrays)
 constexpr uint32_t A_BYTES = BMW * BK * 2;  // 16 KB
 constexpr uint32_t P_BYTES = BMW * BK / 2;  // 4 KB of packed codes
-constexpr int THREADS = 480;
+constexpr int THREADS = 512;
 constexpr int DQ_THREADS = 256;
 constexpr uint64_t DRAIN_NS = 2000000000ull;
 constexpr unsigned SITE_PRODUCER = 0x201, SITE_MMA = 0x202, SITE_DEQUANT = 0x204, SITE_EPILOGUE = 0x208,
@@ -79,7 +84,8 @@ struct Bars {
     uint64_t x_full[12];       // activation tile landed (TMA transaction count)
     uint64_t x_empty[12];      // activation tile consumed by the MMAs
     uint64_t tmem_full;
-    uint64_t drain;
+    uint64_t drain;            // issuer 0's outstanding MMAs (exit drain)
+    uint64_t drain2;           // issuer 1's
     uint32_t tmem_base;
     int abort;
 };
@@ -122,6 +128,25 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t zc, uint32_t 
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// Columns [c, c + 16) of the tile's accumulator for this warp's 32 TMEM lanes:
+// the even-stage accumulator, plus the odd-stage one (MT columns further) when
+// the second issuer ran.
+__device__ __forceinline__ void load_acc16(uint32_t t_row, int c, int mt, bool two, uint32_t (&r)[16]) {
+    tmem_ld_32x32b_x16(t_row + c, r);
+    tmem_ld_wait();
+    if (two) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t r2[8];
+            tmem_ld_32x32b_x8(t_row + mt + c + 8 * h, r2);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                r[8 * h + k] = __float_as_uint(__uint_as_float(r[8 * h + k]) + __uint_as_float(r2[k]));
+        }
+    }
+}
+
 template <int MT, bool SB>
 __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
@@ -142,7 +167,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     const int kb0 = rank * nkb;
     const int groups = K / 128, zwords = (groups + 7) / 8;
     constexpr uint32_t IDESC = make_idesc(/*f32*/ 1, /*f16*/ 0, /*f16*/ 0, BMW, MT);
-    constexpr uint32_t TMEM_COLS = MT < 32 ? 32 : MT;
+    constexpr uint32_t TMEM_COLS = 2 * MT;  // two MT-column accumulators; MT >= 16
 
     if (threadIdx.x == 0) {
         for (int p = 0; p < L::PSTAGES; ++p) {
@@ -157,8 +182,9 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
             mbar_init(smem_u32(&bar->x_full[s]), 1);
             mbar_init(smem_u32(&bar->x_empty[s]), 1);
         }
-        mbar_init(smem_u32(&bar->tmem_full), 1);
+        mbar_init(smem_u32(&bar->tmem_full), 2);  // one commit per issuer
         mbar_init(smem_u32(&bar->drain), 1);
+        mbar_init(smem_u32(&bar->drain2), 1);
         bar->abort = 0;
         fence_mbar_init();
     }
@@ -206,10 +232,16 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
                 if (issued) drain_parity(smem_u32(&bar->x_full[s]), (issued - 1) & 1, DRAIN_NS, status, SITE_DRAIN);
             }
         }
-    } else if (warp == 2) {
-        if (lane == 0) {  // ------------------------------------------------ MMA issuer
+    } else if (warp == 2 || warp == 15) {
+        if (lane == 0) {  // ------------------------------------------------ MMA issuers
+            // Issuer j takes stages j, j + 2, ...  A-stage and x slots pass between the two
+            // issuers in stage order: slot reuse waits for the dequantizers / producer, which
+            // wait for the previous user's commit, so each barrier's phases stay in order.
+            const int j = warp == 2 ? 0 : 1;
+            const uint32_t acc = tmem_base + (uint32_t)(j * MT);
+            const uint32_t drb = smem_u32(j ? &bar->drain2 : &bar->drain);
             bool ok = true;
-            for (int i = 0; i < nkb; ++i) {
+            for (int i = j; i < nkb; i += 2) {
                 const int s = i % L::STAGES, u = i / L::STAGES;
                 const int xs = i % L::XSTAGES, xu = i / L::XSTAGES;
                 if (!wait_parity(smem_u32(&bar->x_full[xs]), xu & 1, ctl, SITE_MMA) ||
@@ -221,14 +253,14 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
                 const uint32_t a_addr = sA + s * A_BYTES, b_addr = sB + xs * L::B_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
-                    mma_f16(tmem_base, umma_desc_sw128_kmajor(a_addr + kk * 32), umma_desc_sw128_kmajor(b_addr + kk * 32),
-                            IDESC, (i | kk) != 0);
+                    mma_f16(acc, umma_desc_sw128_kmajor(a_addr + kk * 32), umma_desc_sw128_kmajor(b_addr + kk * 32),
+                            IDESC, i != j || kk != 0);
                 tc_commit(smem_u32(&bar->st_empty[s]));
                 tc_commit(smem_u32(&bar->x_empty[xs]));
             }
             if (ok) tc_commit(smem_u32(&bar->tmem_full));
-            tc_commit(smem_u32(&bar->drain));
-            drain_parity(smem_u32(&bar->drain), 0, DRAIN_NS, status, SITE_DRAIN);
+            tc_commit(drb);
+            drain_parity(drb, 0, DRAIN_NS, status, SITE_DRAIN);
         }
         __syncwarp();
     } else if (warp < 11) {
@@ -305,7 +337,8 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     }
 
     // ------------------------------------------------------------------------ epilogue
-    const bool epi = warp >= 11;
+    const bool epi = warp >= 11 && warp < 15;
+    const bool two = nkb > 1;  // issuer 1 ran at least one stage
     const int q = warp & 3;
     const int erow = q * 32 + lane;
     const int n = n0 + erow;
@@ -321,8 +354,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
 #pragma unroll 1
             for (int c = 0; c < MT; c += 16) {
                 uint32_t r[16];
-                tmem_ld_32x32b_x16(t_row + c, r);
-                tmem_ld_wait();
+                load_acc16(t_row, c, MT, two, r);
                 if (n < N) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
@@ -341,8 +373,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
 #pragma unroll 1
             for (int c = 0; c < MT; c += 16) {
                 uint32_t r[16];
-                tmem_ld_32x32b_x16(t_row + c, r);
-                tmem_ld_wait();
+                load_acc16(t_row, c, MT, two, r);
 #pragma unroll
                 for (int j = 0; j < 16; j += 4)
                     st_cluster_v4(slot + (c + j) * 4, __uint_as_float(r[j]), __uint_as_float(r[j + 1]),
@@ -355,8 +386,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
 #pragma unroll 1
             for (int c = 0; c < MT; c += 16) {
                 uint32_t r[16];
-                tmem_ld_32x32b_x16(t_row + c, r);
-                tmem_ld_wait();
+                load_acc16(t_row, c, MT, two, r);
                 float acc[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) acc[j] = __uint_as_float(r[j]);
