@@ -126,11 +126,13 @@ __global__ void __launch_bounds__(256) quant_int4_group_kernel(const TIn *__rest
 // ---------------------------------------------------------------------------
 // fp16 input: the same decomposition with packed arithmetic.  The range comes
 // from fp16x2 min/max on the raw bits (exact); a pair of codes is decided with
-// f32x2 operations:  t = w * RN(1/s),  r = t + (1.5*2^23 + z) (rne(t) + z lands
-// in r's low mantissa bits),  d = t - (r - (1.5*2^23 + z)) (exact).  The pair is exact
-// unless |d| comes within 2^-16 of 1/2 (a near-tie of w*RN(1/s), the guard of
-// rne_quotient widened), in which case the lane recomputes its 8 codes with
-// the IEEE quotient.  Clamping and nibble packing run on 16-bit SIMD lanes.
+// f32x2 fused operations on the exact product w * RN(1/s):
+//   r = RN(w * RN(1/s) + (1.5*2^23 + z))   (rne + z lands in r's low mantissa bits),
+//   d = RN(w * RN(1/s) - (r - (1.5*2^23 + z)))   (within 2^-25 of the true remainder).
+// w * RN(1/s) is within 2^-19 of w/s (|w/s| < 32), so the pair is exact unless
+// |d| comes within 2^-16 of 1/2, in which case the lane recomputes its codes
+// with the IEEE quotient.  Clamping (one min.relu.s16x2 per pair) and nibble
+// packing run on 16-bit SIMD lanes.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t hmin2_bits(uint32_t a, uint32_t b) {
     uint32_t d;
@@ -144,26 +146,32 @@ __device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
     return d;
 }
 
-// rne(w * rs) + z of an fp16 pair as int16x2, with magic = 1.5 * 2^23 + z (adding the
-// integer z before rounding is exact, so it folds into the rounding add); `bad` collects
-// the sign bit of (1/2 - 2^-16)^2 - d^2 (set when a lane lies in the guard band).
+// rne(w * rs) + z of an fp16 pair as int16x2, with magic = 1.5 * 2^23 + z: one fused
+// multiply-add rounds w * rs + magic to an integer, which is magic + rne(w * rs) away from a
+// tie (at a tie the parity of z decides, and the guard band below catches it); `bad`
+// collects the sign bit of (1/2 - 2^-16)^2 - d^2 (set when a lane lies in the guard band).
 __device__ __forceinline__ uint32_t pair_rne(uint32_t h2, float rs, float magic, uint32_t &bad) {
     constexpr float kGuardSq = (0.5f - 0x1p-16f) * (0.5f - 0x1p-16f);
     const float2 f = half2_bits_to_float2(h2);
-    const float2 t = __fmul2_rn(f, make_float2(rs, rs));
-    const float2 r = __fadd2_rn(t, make_float2(magic, magic));
+    const float2 r = __ffma2_rn(f, make_float2(rs, rs), make_float2(magic, magic));
     const float2 n = __fadd2_rn(r, make_float2(-magic, -magic));
-    const float2 d = __fadd2_rn(t, make_float2(-n.x, -n.y));
+    const float2 d = __ffma2_rn(f, make_float2(rs, rs), make_float2(-n.x, -n.y));
     const float2 e = __ffma2_rn(d, make_float2(-d.x, -d.y), make_float2(kGuardSq, kGuardSq));
     bad |= __float_as_uint(e.x) | __float_as_uint(e.y);
     return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);  // low 16 bits: rne(t) + z
 }
 
-// codes c_e (int16x2 pairs (c0,c1), (c2,c3), ...) -> one word, code e at bits 4e
+// int16x2 -> each half clamped to [0, 15] in one instruction
+__device__ __forceinline__ uint32_t clamp15x2(uint32_t p) {
+    uint32_t d;
+    asm("min.relu.s16x2 %0, %1, %2;" : "=r"(d) : "r"(p), "r"(0x000F000Fu));
+    return d;
+}
+
+// codes c_e in [0, 15] (int16x2 pairs (c0,c1), (c2,c3), ...) -> one word, code e at bits 4e
 __device__ __forceinline__ uint32_t pack8(uint32_t p0, uint32_t p1, uint32_t p2, uint32_t p3) {
-    const uint32_t u0 = p0 | (p0 >> 12), u1 = p1 | (p1 >> 12);  // byte 0: c_e | c_{e+1} << 4
-    const uint32_t u2 = p2 | (p2 >> 12), u3 = p3 | (p3 >> 12);
-    return __byte_perm(__byte_perm(u0, u1, 0x3140), __byte_perm(u2, u3, 0x3140), 0x5410);
+    const uint32_t x0 = p0 + (p1 << 8), x1 = p2 + (p3 << 8);  // c0 | c2 << 8 | c1 << 16 | c3 << 24
+    return __byte_perm(x0 | (x0 >> 12), x1 | (x1 >> 12), 0x5410);
 }
 
 template <int G>
@@ -232,11 +240,10 @@ __global__ void __launch_bounds__(256) quant_int4_group_f16_kernel(const uint16_
                 }
                 p0 = pp[0]; p1 = pp[1]; p2 = pp[2]; p3 = pp[3];
             }
-            const uint32_t top = 0x000F000Fu;
-            p0 = __vmins2(__vmaxs2(p0, 0u), top);
-            p1 = __vmins2(__vmaxs2(p1, 0u), top);
-            p2 = __vmins2(__vmaxs2(p2, 0u), top);
-            p3 = __vmins2(__vmaxs2(p3, 0u), top);
+            p0 = clamp15x2(p0);
+            p1 = clamp15x2(p1);
+            p2 = clamp15x2(p2);
+            p3 = clamp15x2(p3);
             qweight[(size_t)n * (K / 8) + (size_t)j * (G / 8) + li] = pack8(p0, p1, p2, p3);
             if (li == 0) {
                 scales[(size_t)n * groups + j] = s16;
@@ -322,7 +329,7 @@ __global__ void __launch_bounds__(256) quant_int4_group_f16x16_kernel(const uint
                 }
             }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) p[e] = __vmins2(__vmaxs2(p[e], 0u), 0x000F000Fu);
+            for (int e = 0; e < 8; ++e) p[e] = clamp15x2(p[e]);
             *reinterpret_cast<uint2 *>(qweight + (size_t)n * (K / 8) + (size_t)j * (G / 8) + li * 2) =
                 make_uint2(pack8(p[0], p[1], p[2], p[3]), pack8(p[4], p[5], p[6], p[7]));
             if (li == 0) {
