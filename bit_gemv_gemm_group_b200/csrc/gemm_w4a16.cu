@@ -266,7 +266,9 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     } else if (warp < 11) {
         // -------------------------------------------------------------------- dequantizers
         const int d = threadIdx.x - 96;
-        const int row = d & (BMW - 1), half = d >> 7;
+        // Thread pairs take the two 16-byte halves of one row, so a warp's code load reads 512
+        // contiguous bytes (16 rows) without bank conflicts; the swizzled stores stay conflict-free.
+        const int row = d >> 1, half = d & 1;
         const int n = min(n0 + row, N - 1);
         const uint32_t a_row = sA + row * 128;
         const int sw = row & 7;
