@@ -55,17 +55,19 @@ __device__ __forceinline__ void load8(const uint16_t *p, float (&v)[8]) {
 }
 
 // |v / s| <= 127 (1 + 2^-23) < 2^8 (E = 7): the codes equal rne(fl(v / s)).  Pairs are
-// decided with f32x2 arithmetic: t = v * RN(1/s), r = t + 1.5*2^23 (rne(t) lands in r's low
-// mantissa bits), d = t - (r - 1.5*2^23) (exact).  rne(t) is rne(v / s) unless |d| comes
-// within the guard band of 1/2 (t is within 2^(E-22) of v / s, so a band of 2^-13 > 2^(E-21)
-// suffices); a chunk with such a near-tie is redone with rne_quotient (IEEE quotient).
+// decided with f32x2 fused arithmetic on the exact product t = v * RN(1/s):
+// r = RN(t + 1.5*2^23) (rne(t) lands in r's low mantissa bits), d = RN(t - (r - 1.5*2^23)).
+// rne(t) is rne(v / s) unless |d| comes within the guard band of 1/2 (t is within 2^(E-23)
+// of v / s, so a band of 2^-13 suffices); a chunk with such a near-tie is redone with
+// rne_quotient (IEEE quotient).  No clamp is needed: s = RN(a / 127) with a = max |v| over
+// the same values, so |v| * RN(1/s) <= 127 (1 + 2^-22) and every code lies in [-127, 127].
 __device__ __forceinline__ uint32_t pair_rne8(float a, float b, float rs, uint32_t &bad) {
     constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
     constexpr float kGuardSq = (0.5f - 0x1p-13f) * (0.5f - 0x1p-13f);
-    const float2 t = __fmul2_rn(make_float2(a, b), make_float2(rs, rs));
-    const float2 r = __fadd2_rn(t, make_float2(kMagic, kMagic));
+    const float2 v = make_float2(a, b), r2 = make_float2(rs, rs);
+    const float2 r = __ffma2_rn(v, r2, make_float2(kMagic, kMagic));
     const float2 n = __fadd2_rn(r, make_float2(-kMagic, -kMagic));
-    const float2 d = __fadd2_rn(t, make_float2(-n.x, -n.y));
+    const float2 d = __ffma2_rn(v, r2, make_float2(-n.x, -n.y));
     const float2 e = __ffma2_rn(d, make_float2(-d.x, -d.y), make_float2(kGuardSq, kGuardSq));
     bad |= __float_as_uint(e.x) | __float_as_uint(e.y);
     return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);  // int16x2 rne(t)
@@ -81,11 +83,6 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float s, float rs) 
         for (int e = 0; e < 8; ++e) c[e] = (uint32_t)rne_quotient<7>(v[e], s, rs) & 0xFFFFu;
         p0 = c[0] | (c[1] << 16); p1 = c[2] | (c[3] << 16); p2 = c[4] | (c[5] << 16); p3 = c[6] | (c[7] << 16);
     }
-    const uint32_t lo = 0xFF80FF80u, hi = 0x007F007Fu;  // [-128, 127] per 16-bit lane
-    p0 = __vmins2(__vmaxs2(p0, lo), hi);
-    p1 = __vmins2(__vmaxs2(p1, lo), hi);
-    p2 = __vmins2(__vmaxs2(p2, lo), hi);
-    p3 = __vmins2(__vmaxs2(p3, lo), hi);
     // low byte of every 16-bit lane, in element order
     return make_uint2(__byte_perm(p0, p1, 0x6420), __byte_perm(p2, p3, 0x6420));
 }
