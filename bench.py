@@ -514,7 +514,7 @@ def run_profile_case(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["wq", "reference"], default="wq")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="size of the CPU oracle sample")
