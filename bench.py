@@ -312,16 +312,7 @@ def run_gpu(args):
         r = roofline_for(n, mean_us[n], work[n], peaks)
         kernels.append({"name": n, "us": round(mean_us[n], 2), "achieved": round(r["achieved"], 1),
                         "unit": r["unit"], "bound": r["bound"], "frac": round(r["frac"], 4)})
-    # dominant kernel of the step: the one whose launches (on both projections) take the most
-    # time; the roofline is that of its first launch, and traffic comes from a committed ncu
-    # capture of that launch
-    def family(n):
-        return n.rsplit("_", 1)[0] if n.endswith(("_up", "_down")) else n
-    share = {}
-    for n in names:
-        share[family(n)] = share.get(family(n), 0.0) + mean_us[n]
-    top = max(share, key=share.get)
-    dom = next(n for n in names if family(n) == top)
+    dom = dominant_kernel(names, mean_us)
     rdom = roofline_for(dom, mean_us[dom], work[dom], peaks)
     traffic = load_traffic(dom)
     gemv_roof = roofline_for("gemv_w4a16_b1_up", 1.0, {"bytes": 1, "ops": 0}, peaks)
@@ -425,6 +416,19 @@ def run_e2e(torch, wq, step, steps, stream):
             "launch": how,
             "what": "batch-1 W4A16 GEMV on both weights via the Python/C API, x copied from pinned host memory "
                     "and y read back each step (one copy each way)"}
+
+
+def dominant_kernel(names, mean_us):
+    """The kernel whose launches (on both projections: `_up` and `_down`) take the largest share
+    of the step; returns its first launch, whose roofline the bench line reports and whose DRAM
+    traffic comes from a committed ncu capture."""
+    def family(n):
+        return n.rsplit("_", 1)[0] if n.endswith(("_up", "_down")) else n
+    share = {}
+    for n in names:
+        share[family(n)] = share.get(family(n), 0.0) + mean_us[n]
+    top = max(share, key=share.get)
+    return next(n for n in names if family(n) == top)
 
 
 def load_traffic(kernel):
