@@ -177,8 +177,9 @@ wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qweight, const
  * fragment).  Other M run on the tensor cores: tiles of packed weights are
  * dequantized into shared
  * memory (each dequantized weight rounded to fp16) and fed to tcgen05 MMAs
- * with fp32 accumulation in tensor memory.  M in [16, 256]; group_size ==
- * 128; K % 128 == 0.
+ * with fp32 accumulation in tensor memory (activation tiles of up to 128
+ * rows; larger M is several tiles).  M >= 16; group_size == 128;
+ * K % 128 == 0.
  */
 wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
                         const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y,
