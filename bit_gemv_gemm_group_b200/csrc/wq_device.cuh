@@ -25,12 +25,6 @@ __device__ __forceinline__ uint4 ld_shared_ro_u4(const void *p) {
     return r;
 }
 
-__device__ __forceinline__ void st_stream_u4(void *p, uint4 v) {
-    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
-                 "r"(v.w)
-                 : "memory");
-}
-
 __device__ __forceinline__ float half_bits_to_float(uint16_t b) {
     return __half2float(__ushort_as_half(b));
 }
