@@ -217,7 +217,7 @@ def gemv_w4a16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stre
 
 
 def gemm_w4a16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stream=None):
-    """y [M, N] fp16 = x [M, K] @ dequant(W)^T for M >= 16 on the tensor cores."""
+    """y [M, N] fp16 = x [M, K] @ dequant(W)^T for M >= 16 (or 9..15 with K % 256 == 0)."""
     M, N, K = _w4_args(x, qweight, scales, qzeros, group_size)
     y = out if out is not None else _empty((M, N), torch.float16, x)
     _cuda(y, "out", (torch.float16,), 2)
@@ -227,7 +227,7 @@ def gemm_w4a16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stre
 
 
 def matmul_w4a16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stream=None):
-    """GEMV for up to 8 activation rows, tensor-core GEMM above (the caller's choice made for it)."""
+    """GEMV for up to 8 activation rows, GEMM above (the caller's choice made for it)."""
     if x.shape[0] <= 8:
         return gemv_w4a16(x, qweight, scales, qzeros, group_size, out, stream)
     return gemm_w4a16(x, qweight, scales, qzeros, group_size, out, stream)

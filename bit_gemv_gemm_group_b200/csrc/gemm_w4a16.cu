@@ -527,9 +527,11 @@ extern "C" wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qwe
                M, N, K);
     WQ_REQUIRE(group_size == 128, WQ_ERR_UNSUPPORTED, "wq_gemm_w4a16: group_size must be 128 (got %d)", group_size);
     WQ_REQUIRE(K % 128 == 0, WQ_ERR_INVALID_ARG, "wq_gemm_w4a16: K (%d) must be a multiple of 128", K);
-    WQ_REQUIRE(M >= 16, WQ_ERR_UNSUPPORTED, "wq_gemm_w4a16: M (%d) below 16: use wq_gemv_w4a16", M);
+    WQ_REQUIRE(M >= 16 || (M >= 9 && K % 256 == 0), WQ_ERR_UNSUPPORTED,
+               "wq_gemm_w4a16: M (%d) below 16 needs K %% 256 == 0 (K = %d); use wq_gemv_w4a16 for M <= 8", M, K);
     // Up to 32 activation rows the byte stream dominates: the streaming mma.sync kernel (codes
-    // dequantized in registers, no shared-memory fp16 tile) takes 16 rows per pass and, measured
+    // dequantized in registers, no shared-memory fp16 tile) takes up to 16 rows per pass (it also
+    // serves 9 <= M < 16, which the tensor-core kernel below does not take) and, measured
     // on B200, beats the tensor-core kernel below at M <= 32 (2 passes at M = 32 take 0.36x its
     // time on the 28672x8192 projection; at three passes the two are even).
     if (M <= 32 && K % 256 == 0) {

@@ -170,7 +170,7 @@ wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qweight, const
                         void *stream);
 
 /*
- * W4A16 GEMM for M >= 16 rows of activations ([P1] "Inference view"), same
+ * W4A16 GEMM for M >= 9 rows of activations ([P1] "Inference view"), same
  * arithmetic and layouts as wq_gemv_w4a16.  M <= 32 with K % 256 == 0 runs
  * the streaming kernel of wq_gemv_w4a16 in passes of 16 rows (codes
  * dequantized in registers, exact products, two 8-row batch tiles per weight
@@ -178,7 +178,8 @@ wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qweight, const
  * dequantized into shared
  * memory (each dequantized weight rounded to fp16) and fed to tcgen05 MMAs
  * with fp32 accumulation in tensor memory (activation tiles of up to 128
- * rows; larger M is several tiles).  M >= 16; group_size == 128;
+ * rows; larger M is several tiles).  M >= 16, or 9 <= M < 16 with
+ * K % 256 == 0 (the streaming kernel, one pass); group_size == 128;
  * K % 128 == 0.
  */
 wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,

@@ -64,6 +64,10 @@ def test_sizes_rejected(wq):
     assert L.wq_gemv_w4a16(FAKE, 9, FAKE, FAKE, FAKE, 16, 128, 128, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
     assert L.wq_gemv_w4a16(FAKE, 0, FAKE, FAKE, FAKE, 16, 128, 128, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
     assert L.wq_gemv_w8a16(FAKE, 9, FAKE, FAKE, 16, 128, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    # W4A16 GEMM below 16 rows: only 9..15 rows with K % 256 == 0 (one streaming pass)
+    assert L.wq_gemm_w4a16(FAKE, 12, FAKE, FAKE, FAKE, 16, 640, 128, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_gemm_w4a16(FAKE, 8, FAKE, FAKE, FAKE, 16, 512, 128, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    assert "K % 256" in L.wq_last_error().decode()
     # K granularity of the INT8 paths
     assert L.wq_quantize_int8_per_token(FAKE, 4, 24, None, FAKE, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
     assert L.wq_gemv_w8a16(FAKE, 1, FAKE, FAKE, 16, 24, FAKE, None) == wq.WQ_ERR_UNSUPPORTED

@@ -306,6 +306,7 @@ GEMM_W4_SMALL = [  # (M, N, K): ragged M/N, K on and off the 1024-code fast path
     (16, 128, 128), (16, 300, 1024), (20, 256, 2048), (64, 1000, 4096), (33, 129, 1152),
     (128, 512, 8192), (100, 384, 3072), (16, 4096, 14336), (48, 640, 16384), (17, 130, 640),
     (200, 384, 2048), (300, 260, 1024),  # two and three 128-row activation tiles, ragged
+    (12, 300, 1280), (25, 520, 2304),  # 9..15 rows in one streaming pass; 16 + 9 rows
 ]
 
 
