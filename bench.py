@@ -176,14 +176,14 @@ def make_inputs(torch, dev):
     import workloads
     ins = {}
     for tag, (N, K), si in (("up", UP, 0), ("down", DOWN, 1)):
-        w = workloads.config_weight(4, si)
+        w = workloads.config_weight("llama70b_class", si)
         ins[f"w_{tag}"] = torch.from_numpy(w).to(dev)
         del w
         for B in (1, 16, 64):
-            ins[f"x{B}_{tag}"] = torch.from_numpy(workloads.config_activations(4, B, K)).to(dev)
+            ins[f"x{B}_{tag}"] = torch.from_numpy(workloads.config_activations("llama70b_class", B, K)).to(dev)
     M, N, K = W8A8_SHAPE
-    ins["X5"] = torch.from_numpy(workloads.config_activations(5, M, K)).to(dev)
-    ins["W5"] = torch.from_numpy(workloads.config_weight(5)).to(dev)
+    ins["x_w8a8"] = torch.from_numpy(workloads.config_activations("w8a8_smoothquant", M, K)).to(dev)
+    ins["w_w8a8"] = torch.from_numpy(workloads.config_weight("w8a8_smoothquant")).to(dev)
     return ins
 
 
@@ -197,7 +197,7 @@ class Step:
         self.qB = {t: wq.quantize_group_int4(ins[f"w_{t}"], 128) for t in ("up", "down")}
         self.q8B = {t: wq.quantize_int8_per_channel(ins[f"w_{t}"]) for t in ("up", "down")}
         torch.cuda.synchronize()
-        self.ws = torch.empty(wq.smooth_workspace_bytes(W8A8_SHAPE[2]), dtype=torch.uint8, device=ins["X5"].device)
+        self.ws = torch.empty(wq.smooth_workspace_bytes(W8A8_SHAPE[2]), dtype=torch.uint8, device=ins["x_w8a8"].device)
         self.out = {}
 
     def launches(self):
@@ -210,17 +210,17 @@ class Step:
             L.append((f"quant_int4_{t}", lambda t=t: wq.quantize_group_int4(ins[f"w_{t}"], 128)))
 
         def smooth():
-            self.out["s"] = wq.smooth(ins["X5"], ins["W5"], 0.5, workspace=self.ws)
+            self.out["s"] = wq.smooth(ins["x_w8a8"], ins["w_w8a8"], 0.5, workspace=self.ws)
 
         def q_w():
-            self.out["wq5"] = wq.quantize_int8_per_channel(ins["W5"], self.out["s"])
+            self.out["wq_w8a8"] = wq.quantize_int8_per_channel(ins["w_w8a8"], self.out["s"])
 
         def q_x():
-            self.out["xq5"] = wq.quantize_int8_per_token(ins["X5"], self.out["s"])
+            self.out["xq_w8a8"] = wq.quantize_int8_per_token(ins["x_w8a8"], self.out["s"])
 
         def w8a8():
-            xq, sx = self.out["xq5"]
-            w8, sw = self.out["wq5"]
+            xq, sx = self.out["xq_w8a8"]
+            w8, sw = self.out["wq_w8a8"]
             self.out["y5"] = wq.gemm_w8a8(xq, sx, w8, sw)
 
         L += [("smooth", smooth), ("quant_int8_pc_smooth", q_w), ("quant_int8_pt_smooth", q_x), ("gemm_w8a8", w8a8)]
@@ -373,8 +373,8 @@ def run_e2e(torch, wq, step, steps, stream):
     ny = {"up": UP[0], "down": DOWN[0]}
     hx = torch.cat([ins["x1_up"].reshape(-1), ins["x1_down"].reshape(-1)]).cpu().pin_memory()
     hy = torch.empty(ny["up"] + ny["down"], dtype=torch.float16).pin_memory()
-    dx = torch.empty_like(hx, device=ins["X5"].device)
-    dy = torch.empty(hy.numel(), dtype=torch.float16, device=ins["X5"].device)
+    dx = torch.empty_like(hx, device=ins["x_w8a8"].device)
+    dy = torch.empty(hy.numel(), dtype=torch.float16, device=ins["x_w8a8"].device)
     xv = {"up": dx[:kx["up"]].view(1, -1), "down": dx[kx["up"]:].view(1, -1)}
     yv = {"up": dy[:ny["up"]].view(1, -1), "down": dy[ny["up"]:].view(1, -1)}
 
@@ -451,8 +451,8 @@ def _oracle_inputs(rows=4096):
     if rows not in _ORACLE_INPUTS:
         import oracle
         import workloads
-        w = workloads.config_weight(4, 0, shape=(rows, UP[1]))
-        _ORACLE_INPUTS[rows] = (oracle.quantize_group_int4(w, 128), workloads.config_activations(4, 1, UP[1]))
+        w = workloads.config_weight("llama70b_class", 0, shape=(rows, UP[1]))
+        _ORACLE_INPUTS[rows] = (oracle.quantize_group_int4(w, 128), workloads.config_activations("llama70b_class", 1, UP[1]))
     return _ORACLE_INPUTS[rows]
 
 

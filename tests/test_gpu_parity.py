@@ -83,12 +83,12 @@ def test_int4_quantizer_bit_exact_small(wq, N, K, g, dtype):
     assert np.array_equal(host(qz, np.uint32), rqz)
 
 
-@pytest.mark.parametrize("cfg,shape_index", [(1, 0), (2, 0), (3, 0), (3, 1)])
+@pytest.mark.parametrize("cfg,shape_index", [("tiny_w4a16", 0), ("decode_4096", 0), ("mlp_8b", 0), ("mlp_8b", 1)])
 def test_int4_quantizer_bit_exact_configs(wq, cfg, shape_index):
     w = workloads.config_weight(cfg, shape_index)
     qw, sc, qz = wq.quantize_group_int4(dev(w), 128)
     torch.cuda.synchronize()
-    rows = sample_rows(w.shape[0], 512, seed=cfg)
+    rows = sample_rows(w.shape[0], 512, seed=workloads.CONFIGS[cfg].seed)
     rqw, rsc, rqz = oracle.quantize_group_int4(w[rows], 128)
     assert np.array_equal(host(qw, np.uint32)[rows], rqw)
     assert np.array_equal(host(sc).view(np.uint16)[rows], rsc.view(np.uint16))
@@ -118,7 +118,7 @@ def test_gemv_w4a16_small(wq, N, K, g, B):
     assert_within_bound(host(y).astype(np.float64), y_ref, bound, f"gemv N={N} K={K} B={B}")
 
 
-@pytest.mark.parametrize("cfg", [1, 2, 3, 4])
+@pytest.mark.parametrize("cfg", ["tiny_w4a16", "decode_4096", "mlp_8b", "llama70b_class"])
 def test_gemv_w4a16_configs(wq, cfg):
     c = workloads.CONFIGS[cfg]
     for si, (N, K) in enumerate(c.shapes):
@@ -131,7 +131,7 @@ def test_gemv_w4a16_configs(wq, cfg):
             y = wq.gemv_w4a16(dev(x), qw, sc, qz, 128)
             torch.cuda.synchronize()
             y_ref, bound = oracle.matmul_w4a16_ref(x, hqw, hsc, hqz, K, 128, rows=rows)
-            assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"cfg{cfg} {N}x{K} B={B}")
+            assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"{cfg} {N}x{K} B={B}")
 
 
 # --------------------------------------------------------------------------
@@ -209,20 +209,20 @@ def test_gemv_w8a16_small(wq, N, K, B):
     assert_within_bound(y.astype(np.float64), y_ref, bound, f"w8a16 N={N} K={K} B={B}")
 
 
-def test_w8a16_config3(wq):
-    c = workloads.CONFIGS[3]
+def test_w8a16_mlp_8b(wq):
+    c = workloads.CONFIGS["mlp_8b"]
     for si, (N, K) in enumerate(c.shapes):
-        w = workloads.config_weight(3, si)
+        w = workloads.config_weight("mlp_8b", si)
         q, s = wq.quantize_int8_per_channel(dev(w))
         rows = sample_rows(N, 256, seed=si)
         rq, rs = oracle.quantize_int8_per_channel(w[rows])
         hq, hs = host(q), host(s)
         assert np.array_equal(hq[rows], rq) and np.array_equal(hs[rows].view(np.uint32), rs.view(np.uint32))
         for B in (1, 8):
-            x = workloads.config_activations(3, B, K)
+            x = workloads.config_activations("mlp_8b", B, K)
             y = host(wq.gemv_w8a16(dev(x), q, s))
             y_ref, bound = oracle.matmul_w8a16_ref(x, hq, hs, rows=rows)
-            assert_within_bound(y.astype(np.float64)[:, rows], y_ref, bound, f"w8a16 cfg3 {N}x{K} B={B}")
+            assert_within_bound(y.astype(np.float64)[:, rows], y_ref, bound, f"w8a16 mlp_8b {N}x{K} B={B}")
 
 
 # --------------------------------------------------------------------------
@@ -274,11 +274,11 @@ def test_gemm_w8a8_extreme_accumulators(wq):
 
 
 def test_w8a8_smoothquant_pipeline_full_size(wq):
-    # Config 5: smoothing -> per-channel(W * s) -> per-token(X / s) -> INT8 GEMM, in the
+    # The W8A8 SmoothQuant layer: smoothing -> per-channel(W * s) -> per-token(X / s) -> INT8 GEMM, in the
     # launch configuration the benchmark times; sampled rows checked one by one.
     M, N, K = 2048, 8192, 8192
-    X = workloads.config_activations(5, M, K)
-    W = workloads.config_weight(5)
+    X = workloads.config_activations("w8a8_smoothquant", M, K)
+    W = workloads.config_weight("w8a8_smoothquant")
     Xd, Wd = dev(X), dev(W)
     s = wq.smooth(Xd, Wd, 0.5)
     wq8, sw = wq.quantize_int8_per_channel(Wd, s)
@@ -295,7 +295,7 @@ def test_w8a8_smoothquant_pipeline_full_size(wq):
     assert np.array_equal(host(wq8)[ns], rwq) and np.array_equal(host(sw)[ns], rsw)
     racc, ry, rb = oracle.gemm_w8a8_ref(rxq, rsx, rwq, rsw)
     assert np.array_equal(host(acc)[np.ix_(ms, ns)].astype(np.int64), racc)
-    assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, "w8a8 config 5")
+    assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, "w8a8_smoothquant")
     assert wq.device_status() == 0
 
 
@@ -323,7 +323,7 @@ def test_gemm_w4a16_small(wq, M, N, K):
     assert wq.device_status() == 0
 
 
-@pytest.mark.parametrize("cfg", [3, 4])
+@pytest.mark.parametrize("cfg", ["mlp_8b", "llama70b_class"])
 def test_gemm_w4a16_configs(wq, cfg):
     c = workloads.CONFIGS[cfg]
     for si, (N, K) in enumerate(c.shapes):
@@ -337,7 +337,7 @@ def test_gemm_w4a16_configs(wq, cfg):
             y = wq.matmul_w4a16(dev(x), qw, sc, qz, 128)
             torch.cuda.synchronize()
             y_ref, bound = oracle.matmul_w4a16_ref(x, hqw[rows], hsc[rows], hqz[rows], K, 128)
-            assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"cfg{cfg} {N}x{K} B={B}")
+            assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"{cfg} {N}x{K} B={B}")
     assert wq.device_status() == 0
 
 
@@ -348,12 +348,12 @@ def test_gemm_w4a16_configs(wq, cfg):
 # --------------------------------------------------------------------------
 @pytest.mark.parametrize("shape_index", [0, 1])
 def test_w4a16_matmuls_repeat_bit_identically(wq, shape_index):
-    w = workloads.config_weight(4, shape_index)
+    w = workloads.config_weight("llama70b_class", shape_index)
     N, K = w.shape
     qw, sc, qz = wq.quantize_group_int4(dev(w), 128)
     del w
     for B in (1, 16, 64):
-        x = dev(workloads.config_activations(4, B, K))
+        x = dev(workloads.config_activations("llama70b_class", B, K))
         first = wq.matmul_w4a16(x, qw, sc, qz, 128)
         for _ in range(3):
             again = wq.matmul_w4a16(x, qw, sc, qz, 128)

@@ -94,49 +94,51 @@ class Config:
 
 
 CONFIGS = {
-    1: Config("tiny_w4a16", 0, ((256, 512),), (1,),
+    "tiny_w4a16": Config("tiny_w4a16", 0, ((256, 512),), (1,),
               "fp32 W 256x512 N(0,0.02), every 97th element x20; x fp16 [1,512] N(0,1)"),
-    2: Config("decode_4096", 2, ((4096, 4096),), (1, 4),
+    "decode_4096": Config("decode_4096", 2, ((4096, 4096),), (1, 4),
               "fp16 W 4096x4096, row sigma lognormal(ln 0.02, 0.5), 0.1% entries x30; "
               "x N(0,1) with 1% of channels x50"),
-    3: Config("mlp_8b", 3, ((14336, 4096), (4096, 14336)), (1, 8, 16),
+    "mlp_8b": Config("mlp_8b", 3, ((14336, 4096), (4096, 14336)), (1, 8, 16),
               "fp16 W N(0,0.02) gate/up 14336x4096 and down 4096x14336; x with 1% channels x50; "
               "also INT8 per-channel (W8A16) on the same weights"),
-    4: Config("llama70b_class", 4, ((28672, 8192), (8192, 28672)), (1, 16, 64),
+    "llama70b_class": Config("llama70b_class", 4, ((28672, 8192), (8192, 28672)), (1, 16, 64),
               "fp16 W N(0,0.015) 28672x8192 and 8192x28672; x with 0.5% channels x100"),
-    5: Config("w8a8_smoothquant", 5, ((8192, 8192),), (2048,),
+    "w8a8_smoothquant": Config("w8a8_smoothquant", 5, ((8192, 8192),), (2048,),
               "X fp16 [2048, 8192] N(0,1) with 64 fixed channels x60; W fp16 8192x8192 N(0,0.02); "
               "alpha 0.5"),
 }
 
-_X_OUTLIERS = {1: (0.0, 1.0), 2: (0.01, 50.0), 3: (0.01, 50.0), 4: (0.005, 100.0)}
-_W_SIGMA = {3: 0.02, 4: 0.015}
+_X_OUTLIERS = {"tiny_w4a16": (0.0, 1.0), "decode_4096": (0.01, 50.0), "mlp_8b": (0.01, 50.0),
+               "llama70b_class": (0.005, 100.0)}
+_W_SIGMA = {"mlp_8b": 0.02, "llama70b_class": 0.015}
 
 
-def config_weight(cfg: int, shape_index: int = 0, shape=None) -> np.ndarray:
-    """The weight matrix of a W4A16 config (optionally at a different [N, K])."""
+def config_weight(cfg: str, shape_index: int = 0, shape=None) -> np.ndarray:
+    """The weight matrix of workload `cfg` (a key of CONFIGS), optionally at another [N, K]."""
     c = CONFIGS[cfg]
     N, K = shape if shape is not None else c.shapes[shape_index]
-    if cfg == 1:
+    if cfg == "tiny_w4a16":
         return weight_every_nth_outlier(N, K, 0.02, 97, 20.0, c.seed, shape_index, np.float32)
-    if cfg == 2:
+    if cfg == "decode_4096":
         return weight_lognormal_rows(N, K, c.seed, shape_index)
-    if cfg in (3, 4):
+    if cfg in ("mlp_8b", "llama70b_class"):
         return weight_normal(N, K, _W_SIGMA[cfg], c.seed, shape_index)
-    if cfg == 5:
+    if cfg == "w8a8_smoothquant":
         return weight_normal(N, K, 0.02, c.seed, 1)
     raise KeyError(cfg)
 
 
-def config_activations(cfg: int, B: int, K: int, tensor_id: int = 100) -> np.ndarray:
+def config_activations(cfg: str, B: int, K: int, tensor_id: int = 100) -> np.ndarray:
+    """Activation rows [B, K] of workload `cfg` (a key of CONFIGS)."""
     c = CONFIGS[cfg]
-    if cfg == 5:
+    if cfg == "w8a8_smoothquant":
         return w8a8_activations(B, K, seed=c.seed)
     frac, mult = _X_OUTLIERS[cfg]
     return activations(B, K, frac, mult, c.seed, tensor_id + B)
 
 
-def config_inputs(cfg: int):
+def config_inputs(cfg: str):
     """All tensors of a config: {"weights": [W...], "x": {B: [x per weight]}}."""
     c = CONFIGS[cfg]
     ws = [config_weight(cfg, i) for i in range(len(c.shapes))]
