@@ -12,7 +12,7 @@
 //   - group size 128, K % 256 == 0 (every decode shape): the streaming
 //     tensor-core kernel further below (TMA ring, producer-built B fragments,
 //     codes fed to mma.sync as fp16 subnormals); it also serves wq_gemm_w4a16
-//     for up to 32 rows in passes of 16;
+//     for up to 32 rows in passes of up to 16;
 //   - group size 128, other K: a register-prefetch mma.sync kernel;
 //   - other group sizes: the CUDA-core kernel that follows.
 //
@@ -836,7 +836,7 @@ wq_status gemv_stream_nt(const uint16_t *x, int B, const uint32_t *qw, const uin
 }  // namespace
 
 // Batch 1..16 with K % 256 == 0, group size 128 (also serves wq_gemm_w4a16 for up to 32 rows,
-// in passes of 16).
+// in passes of up to 16).
 wq_status gemv_stream(const uint16_t *x, int B, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
                       int K, uint16_t *y, cudaStream_t st, const char *who) {
     if (B <= 8) return gemv_stream_nt<1, 7, 2>(x, B, qw, sc, qz, N, K, y, st, who);
