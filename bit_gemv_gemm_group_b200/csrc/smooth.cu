@@ -20,6 +20,8 @@
 // Workspace layout (words): ax float[Kp] | aw float[Kp] | tickets uint32[ceil4(K/256)],
 // Kp = K rounded up to 4.
 #include <algorithm>
+#include <atomic>
+#include <mutex>
 
 #include "wq_device.cuh"
 #include "wq_host.h"
@@ -122,19 +124,22 @@ __global__ void __launch_bounds__(kThreads) smooth_kernel(const uint16_t *__rest
     }
 }
 
-// Resident CTAs of smooth_kernel on the current device (SMs x CTAs per SM), cached.
+// Resident CTAs of smooth_kernel on the current device (SMs x CTAs per SM), cached per
+// device; host threads may race to fill an entry, and they all store the same value.
 int smooth_slots() {
-    static int cached[64] = {0};
+    static std::atomic<int> cached[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148 * 8;
-    if (!cached[dev]) {
+    int v = cached[dev].load(std::memory_order_relaxed);
+    if (!v) {
         int per_sm = 0;
         if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, smooth_kernel, kThreads, 0) != cudaSuccess ||
             per_sm <= 0)
             per_sm = 8;
-        cached[dev] = per_sm * num_sms();
+        v = per_sm * num_sms();
+        cached[dev].store(v, std::memory_order_relaxed);
     }
-    return cached[dev];
+    return v;
 }
 
 }  // namespace
@@ -183,7 +188,6 @@ extern "C" wq_status wq_smooth(const uint16_t *x, int M, const uint16_t *w, int 
 // so the device address is looked up once per device with cudaGetSymbolAddress
 // (on the first call made while that device is current) and cached.
 // ---------------------------------------------------------------------------
-#include <mutex>
 
 namespace wq {
 namespace {
