@@ -242,7 +242,8 @@ extern "C" wq_status wq_gemm_w8a8(const int8_t *xq, const float *sx, const int8_
     WQ_REQUIRE(M > 0 && N > 0 && K > 0, WQ_ERR_INVALID_ARG, "wq_gemm_w8a8: sizes must be positive (M=%d N=%d K=%d)", M,
                N, K);
     WQ_REQUIRE(K % 16 == 0, WQ_ERR_UNSUPPORTED, "wq_gemm_w8a8: K (%d) must be a multiple of 16", K);
-    WQ_REQUIRE(K <= 131072, WQ_ERR_UNSUPPORTED, "wq_gemm_w8a8: K (%d) above 131072 could overflow int32", K);
+    // |acc| <= 128 * 128 * K must stay below 2^31 for any int8 codes: K <= 131071, and K % 16 == 0
+    WQ_REQUIRE(K <= 131056, WQ_ERR_UNSUPPORTED, "wq_gemm_w8a8: K (%d) above 131056 could overflow int32", K);
     unsigned int *status = device_status_word();
     if (!status) return WQ_ERR_CUDA;
     CUtensorMap tx, tw;

@@ -195,7 +195,8 @@ wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const
  *   y[m][n]   = fp16_rn( (float)acc * sx[m] * sw[n] )     (fp32 products)
  * xq: int8 [M][K], sx: fp32 [M], wq: int8 [N][K], sw: fp32 [N];
  * y: out fp16 [M][N];  acc_out: nullable, out int32 [M][N] (raw accumulators).
- * K % 16 == 0, K <= 131072 (so |acc| < 2^31).
+ * K % 16 == 0, K <= 131056 (so |acc| <= 128 * 128 * K < 2^31 for any
+ * int8 codes).
  */
 wq_status wq_gemm_w8a8(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
                        int M, int N, int K, uint16_t *y, int32_t *acc_out, void *stream);

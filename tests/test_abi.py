@@ -72,6 +72,14 @@ def test_sizes_rejected(wq):
     assert L.wq_quantize_int8_per_token(FAKE, 4, 24, None, FAKE, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
     assert L.wq_gemv_w8a16(FAKE, 1, FAKE, FAKE, 16, 24, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
     assert L.wq_gemm_w8a8(FAKE, FAKE, FAKE, FAKE, 16, 16, 24, FAKE, None, None) == wq.WQ_ERR_UNSUPPORTED
+    # W8A8: |acc| <= 128 * 128 * K must stay below 2^31; at K = 131072 (-128) * (-128) products
+    # reach 2^31 exactly, so the largest K (a multiple of 16) is 131056
+    assert L.wq_gemm_w8a8(FAKE, FAKE, FAKE, FAKE, 16, 16, 131072, FAKE, None, None) == wq.WQ_ERR_UNSUPPORTED
+    assert "131056" in L.wq_last_error().decode()
+    assert 128 * 128 * 131056 < 2 ** 31 <= 128 * 128 * 131072
+    # the W4A16 GEMM takes group size 128 only; the GEMV takes 32/64/128/256
+    assert L.wq_gemm_w4a16(FAKE, 16, FAKE, FAKE, FAKE, 16, 512, 64, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    assert L.wq_gemv_w4a16(FAKE, 1, FAKE, FAKE, FAKE, 16, 512, 96, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
     # smoothing: alpha range, K granularity
     assert L.wq_smooth(FAKE, 4, FAKE, 4, 64, ctypes.c_float(1.5), FAKE, FAKE, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_smooth(FAKE, 4, FAKE, 4, 60, ctypes.c_float(0.5), FAKE, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
