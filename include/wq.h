@@ -160,7 +160,10 @@ wq_status wq_smooth_noalloc(const uint16_t *x, int M, const uint16_t *w, int N, 
  * scales), [P3] "Scale and zero-point" (w^ = (q - z) s), [P5] "Why It Is
  * Faster" (decode streams the weights).
  *   y[b][n] = fp16_rn( sum_k s[n][k/g] * (q[n][k] - z[n][k/g]) * x[b][k] )
- * accumulated in fp32 (order unspecified).
+ * accumulated in fp32 (order unspecified).  With group size 128 and
+ * K % 256 == 0, half of the products take x pre-scaled by 2^-4 in fp16,
+ * which is exact for |x| >= 2^-10.  A row made only of much smaller
+ * activations (|x| ~ 1e-6) can have relative errors of a few percent.
  * x: fp16 [B][K];  qweight/scales/qzeros: the packed layout above;
  * y: out fp16 [B][N].  group_size in {32, 64, 128, 256}; K % group_size == 0;
  * K % 32 == 0.
