@@ -162,8 +162,11 @@ wq_status wq_smooth_noalloc(const uint16_t *x, int M, const uint16_t *w, int N, 
  *   y[b][n] = fp16_rn( sum_k s[n][k/g] * (q[n][k] - z[n][k/g]) * x[b][k] )
  * accumulated in fp32 (order unspecified).  With group size 128 and
  * K % 256 == 0, half of the products take x pre-scaled by 2^-4 in fp16,
- * which is exact for |x| >= 2^-10.  A row made only of much smaller
- * activations (|x| ~ 1e-6) can have relative errors of a few percent.
+ * which is exact for |x| >= 2^-10.  Rows of ordinary activations are
+ * unaffected (the roundings of small elements cancel), but a row made only
+ * of tiny values loses precision: its error can exceed the 2e-3 relative
+ * tolerance from |x| ~ 1e-5 down, and below ~2^-21 the pre-scaled values
+ * round to zero, so half of the products are lost.
  * x: fp16 [B][K];  qweight/scales/qzeros: the packed layout above;
  * y: out fp16 [B][N].  group_size in {32, 64, 128, 256}; K % group_size == 0;
  * K % 32 == 0.
