@@ -164,8 +164,8 @@ wq_status wq_smooth_noalloc(const uint16_t *x, int M, const uint16_t *w, int N, 
  * K % 256 == 0, half of the products take x pre-scaled by 2^-4 in fp16,
  * which is exact for |x| >= 2^-10.  Rows of ordinary activations are
  * unaffected (the roundings of small elements cancel), but a row made only
- * of tiny values loses precision: its error can exceed the 2e-3 relative
- * tolerance from |x| ~ 1e-5 down, and below ~2^-21 the pre-scaled values
+ * of one tiny value loses precision: its error can exceed the 2e-3 relative
+ * tolerance for values below ~2e-4, and below ~2^-21 the pre-scaled values
  * round to zero, so half of the products are lost.
  * x: fp16 [B][K];  qweight/scales/qzeros: the packed layout above;
  * y: out fp16 [B][N].  group_size in {32, 64, 128, 256}; K % group_size == 0;
