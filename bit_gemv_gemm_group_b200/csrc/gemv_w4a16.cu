@@ -394,7 +394,8 @@ struct StreamLayout {
     static constexpr uint32_t XF_BYTES = NT * 32 * 64; // B fragments of one group: [NT][4][32 lanes][16 B]
     static constexpr uint32_t OFF_XF = W_BYTES;
     static constexpr uint32_t OFF_XS = OFF_XF + XF_BYTES * kGPS;  // X'_g: [kGPS][8 * NT] fp32
-    static constexpr uint32_t STAGE = (OFF_XS + 32 * NT * kGPS + 127) / 128 * 128;  // 128-byte aligned TMA
+    static constexpr uint32_t OFF_FL = OFF_XS + 32 * NT * kGPS;   // per group: fp32 factor of its scales (1 or 1/16)
+    static constexpr uint32_t STAGE = (OFF_FL + 4 * kGPS + 127) / 128 * 128;  // 128-byte aligned TMA
     static constexpr int RING = (kStreamRingBudget / STAGE) < 3 ? 3
                                 : (kStreamRingBudget / STAGE) > 8 ? 8 : (kStreamRingBudget / STAGE);
     static constexpr uint32_t OFF_BAR = RING * STAGE;
@@ -441,6 +442,12 @@ __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint3
 
 __device__ __forceinline__ void sts32f(uint32_t a, float v) {
     asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ float lds32f(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
 }
 
 __device__ __forceinline__ uint32_t hmul2_u(uint32_t a, uint32_t b) {
@@ -522,17 +529,50 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, NT>::THREADS, 2)
             }
             ++issued;
 #pragma unroll
-            for (int n = 0; n < NT; ++n)
+            for (int q = 0; q < GPS; ++q) {
+                // Fragment k-step 2j: (x0,x4) and 2^-4 (x1,x5) of chunk j; 2j+1: (x2,x6) and 2^-4 (x3,x7).
+                // The 2^-4 pre-scaling of the high-nibble lanes is exact unless some |x| < 2^-10
+                // loses bits in fp16 (the round trip x * 2^-4 * 16 then differs from x).  If that
+                // happens anywhere in the group (any lane, any batch row) and no |x| in the
+                // low-nibble lanes reaches 4096, the group's fragments carry 16 x in the low-nibble
+                // lanes and x in the high-nibble lanes instead (both exact), and its flag word
+                // tells the consumers that D and X'_g come out 16 times larger.
+                uint32_t inexact = 0u;
 #pragma unroll
-                for (int q = 0; q < GPS; ++q) {
-                    // fragment k-step 2j: (x0,x4) and 2^-4 (x1,x5) of chunk j; 2j+1: (x2,x6) and 2^-4 (x3,x7)
+                for (int n = 0; n < NT; ++n)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 c = xr[n][q][j];
+                        const uint32_t h0 = prmt_u(c.x, c.z, 0x7632u), h1 = prmt_u(c.y, c.w, 0x7632u);
+                        inexact |= (hmul2_u(hmul2_u(h0, 0x2C002C00u), 0x4C004C00u) ^ h0) |
+                                   (hmul2_u(hmul2_u(h1, 0x2C002C00u), 0x4C004C00u) ^ h1);
+                    }
+                bool x16 = __any_sync(0xffffffffu, inexact != 0u);
+                if (x16) {  // rare: is 16 x finite for every low-nibble lane of the group?
+                    uint32_t big = 0u;
+#pragma unroll
+                    for (int n = 0; n < NT; ++n)
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const uint4 c = xr[n][q][j];
+                            // |x| >= 4096 (0x6C00) sets bit 15 of (|x| + 0x1400) in each half
+                            big |= ((prmt_u(c.x, c.z, 0x5410u) & 0x7FFF7FFFu) + 0x14001400u) |
+                                   ((prmt_u(c.y, c.w, 0x5410u) & 0x7FFF7FFFu) + 0x14001400u);
+                        }
+                    x16 = !__any_sync(0xffffffffu, (big & 0x80008000u) != 0u);
+                }
+                const uint32_t lo_scale = x16 ? 0x4C004C00u : 0x3C003C00u;   // 16 or 1
+                const uint32_t hi_scale = x16 ? 0x3C003C00u : 0x2C002C00u;   // 1 or 2^-4
+                const float xs_scale = x16 ? -9.5367431640625e-7f : -5.9604644775390625e-8f;  // -2^-20 / -2^-24
+#pragma unroll
+                for (int n = 0; n < NT; ++n) {
                     float sum0 = 0.0f, sum1 = 0.0f;
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const uint4 c = xr[n][q][j];
                         sts128(st + L::OFF_XF + q * L::XF_BYTES + (n * 4 + j) * 512 + lane * 16,
-                               prmt_u(c.x, c.z, 0x5410u), hmul2_u(prmt_u(c.x, c.z, 0x7632u), 0x2C002C00u),
-                               prmt_u(c.y, c.w, 0x5410u), hmul2_u(prmt_u(c.y, c.w, 0x7632u), 0x2C002C00u));
+                               hmul2_u(prmt_u(c.x, c.z, 0x5410u), lo_scale), hmul2_u(prmt_u(c.x, c.z, 0x7632u), hi_scale),
+                               hmul2_u(prmt_u(c.y, c.w, 0x5410u), lo_scale), hmul2_u(prmt_u(c.y, c.w, 0x7632u), hi_scale));
                         const float2 f0 = half2_bits_to_float2(c.x), f1 = half2_bits_to_float2(c.y);
                         const float2 f2 = half2_bits_to_float2(c.z), f3 = half2_bits_to_float2(c.w);
                         sum0 += (f0.x + f1.x) + (f2.x + f3.x);
@@ -541,9 +581,11 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, NT>::THREADS, 2)
                     float xg = sum0 + sum1;
                     xg += __shfl_xor_sync(0xffffffffu, xg, 1);
                     xg += __shfl_xor_sync(0xffffffffu, xg, 2);
-                    // -2^-24 X_g of batch row r + 8n (exact scaling)
-                    if (t == 0) sts32f(st + L::OFF_XS + (q * NT + n) * 32 + r * 4, xg * -5.9604644775390625e-8f);
+                    // -2^-24 X_g (or -2^-20 X_g) of batch row r + 8n (exact scaling)
+                    if (t == 0) sts32f(st + L::OFF_XS + (q * NT + n) * 32 + r * 4, xg * xs_scale);
                 }
+                if (lane == 0) sts32f(st + L::OFF_FL + q * 4, x16 ? 0.0625f : 1.0f);
+            }
             mbar_arrive(fb);  // release: the fragments are visible to the consumers' acquire
             return true;
         };
@@ -672,11 +714,13 @@ __global__ void __launch_bounds__(StreamLayout<CW, RT, NT>::THREADS, 2)
                             }
                         }
                     }
-                    // acc += s (D - z X'_g)  (rows r and r + 8 of each m-tile)
+                    // acc += s (D - z X'_g)  (rows r and r + 8 of each m-tile); a group whose fragments
+                    // carry 16 x in the low-nibble lanes has D and X'_g 16 times larger
+                    const float gf = lds32f(st + L::OFF_FL + q * 4);  // 1 or 1/16
 #pragma unroll
                     for (int i = 0; i < RT; ++i) {
-                        const float s0 = half_bits_to_float((uint16_t)(scw[i][0] >> (16 * q)));
-                        const float s1 = half_bits_to_float((uint16_t)(scw[i][1] >> (16 * q)));
+                        const float s0 = half_bits_to_float((uint16_t)(scw[i][0] >> (16 * q))) * gf;
+                        const float s1 = half_bits_to_float((uint16_t)(scw[i][1] >> (16 * q))) * gf;
                         const float z0 = (float)((zw[i][0] >> (zsh + 4 * q)) & 0xFu);
                         const float z1 = (float)((zw[i][1] >> (zsh + 4 * q)) & 0xFu);
 #pragma unroll

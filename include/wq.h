@@ -145,7 +145,13 @@ wq_status wq_smooth(const uint16_t *x, int M, const uint16_t *w, int N, int K, f
  * cudaFree, no allocating library routine.  The first call on a device (made
  * while that device is current) looks up the array's device address with
  * cudaGetSymbolAddress and caches it; make that first call before any stream
- * capture.  All calls on a device share the one array, which keeps the last
+ * capture.  Under CUDA's lazy module loading (the default) the first use of
+ * the library on a device -- this look-up or the first launch of any entry
+ * point -- loads the library's device code on that device, which allocates
+ * device memory for the code and the array and may synchronize: make one
+ * ordinary call during set-up, or load modules eagerly
+ * (CUDA_MODULE_LOADING=EAGER), if later calls must not do either.  All
+ * calls on a device share the one array, which keeps the last
  * call's contents (each call clears what must start at zero), so calls that
  * overlap on the GPU (concurrent streams, several host threads) race and
  * give wrong results: order them on one stream or with events.
@@ -160,13 +166,14 @@ wq_status wq_smooth_noalloc(const uint16_t *x, int M, const uint16_t *w, int N, 
  * scales), [P3] "Scale and zero-point" (w^ = (q - z) s), [P5] "Why It Is
  * Faster" (decode streams the weights).
  *   y[b][n] = fp16_rn( sum_k s[n][k/g] * (q[n][k] - z[n][k/g]) * x[b][k] )
- * accumulated in fp32 (order unspecified).  With group size 128 and
- * K % 256 == 0, half of the products take x pre-scaled by 2^-4 in fp16,
- * which is exact for |x| >= 2^-10.  Rows of ordinary activations are
- * unaffected (the roundings of small elements cancel), but a row made only
- * of one tiny value loses precision: its error can exceed the 2e-3 relative
- * tolerance for values below ~2e-4, and below ~2^-21 the pre-scaled values
- * round to zero, so half of the products are lost.
+ * accumulated in fp32 (order unspecified).  Every product s * (q - z) * x
+ * enters the accumulation exactly, for any finite fp16 x, with one
+ * exception: with group size 128 and K % 256 == 0 the kernel pre-scales half
+ * of a group's x by 2^-4 (or, when that would drop bits of some |x| < 2^-10,
+ * the other half by 16); if one activation row's group holds both a value
+ * of magnitude >= 4096 in the second half and such a small value in the
+ * first, the small values keep the 2^-4 pre-scaling and each product with
+ * them is off by at most 2^-21 * s * q.
  * x: fp16 [B][K];  qweight/scales/qzeros: the packed layout above;
  * y: out fp16 [B][N].  group_size in {32, 64, 128, 256}; K % group_size == 0;
  * K % 32 == 0.
