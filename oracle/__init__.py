@@ -71,6 +71,18 @@ def _declare(L):
     L.orc_matmul_w8a16_ref.restype = None
     L.orc_gemm_w8a8_ref.argtypes = [_P, _P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _P]
     L.orc_gemm_w8a8_ref.restype = _I
+    L.orc_e4m3_to_float.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_to_float.restype = ctypes.c_float
+    L.orc_float_to_e4m3.argtypes = [ctypes.c_float]
+    L.orc_float_to_e4m3.restype = ctypes.c_uint8
+    L.orc_quantize_fp8_e4m3.argtypes = [_P, _I, _I, _I, _P, _P]
+    L.orc_quantize_fp8_e4m3.restype = _I
+    L.orc_gemm_fp8_ref.argtypes = [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _I, _P, _I, _P, _P]
+    L.orc_gemm_fp8_ref.restype = None
+    L.orc_outlier_columns.argtypes = [_P, _I, _I, ctypes.c_float, _I, _P]
+    L.orc_outlier_columns.restype = _I
+    L.orc_llm_int8_ref.argtypes = [_P, _I, _I, _P, _P, _I, _P, _I, _P, _I, _P, _I, _P, _P, _P, _P]
+    L.orc_llm_int8_ref.restype = _I
 
 
 def _ptr(a: np.ndarray | None):
@@ -255,3 +267,81 @@ def gemm_w8a8_ref(xq, sx, wq, sw, ms=None, ns=None):
     if rc == -2:
         raise OverflowError("an int8 accumulator left the int32 range")
     return acc, y, bd
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 ("Quantization from Scratch", Formats; "Quantization: Smaller
+# Weights, Same Answers (Mostly)", FP8 section; "How quantization works",
+# quant.py fake_quant_fp8: scale = max|w| / 448)
+# --------------------------------------------------------------------------
+def e4m3_to_float(code: int) -> float:
+    return float(lib().orc_e4m3_to_float(int(code) & 0xFF))
+
+
+def float_to_e4m3(x: float) -> int:
+    return int(lib().orc_float_to_e4m3(float(np.float32(x))))
+
+
+def quantize_fp8_e4m3(a, per_row: bool = True):
+    """fp16 [R, K] -> (E4M3 codes uint8 [R, K], fp32 scales [R] per row or [1] per tensor)."""
+    bits16 = _f16_bits(a)
+    R, K = bits16.shape
+    q = np.zeros((R, K), np.uint8)
+    s = np.zeros(R if per_row else 1, np.float32)
+    rc = lib().orc_quantize_fp8_e4m3(_ptr(bits16), R, K, 1 if per_row else 0, _ptr(q), _ptr(s))
+    if rc != 0:
+        raise ValueError("orc_quantize_fp8_e4m3: bad arguments")
+    return q, s
+
+
+def gemm_fp8_ref(xq, sx, wq, sw, ms=None, ns=None):
+    """(y fp64 [nm, nn], bound fp64): y = sx * sw * sum_k e4m3(xq) e4m3(wq); a scale vector of
+    length 1 applies to every row of its operand (per-tensor scale)."""
+    a = _c(xq, np.uint8)
+    b = _c(wq, np.uint8)
+    M, K = a.shape
+    N = b.shape[0]
+    sxa = _c(np.atleast_1d(sx), np.float32)
+    swa = _c(np.atleast_1d(sw), np.float32)
+    m_arr, nm = _rows_arg(ms, M)
+    n_arr, nn = _rows_arg(ns, N)
+    y = np.zeros((nm, nn), np.float64)
+    bd = np.zeros((nm, nn), np.float64)
+    lib().orc_gemm_fp8_ref(_ptr(a), _ptr(sxa), int(sxa.size == M), _ptr(b), _ptr(swa), int(swa.size == N),
+                           M, N, K, _ptr(m_arr), nm, _ptr(n_arr), nn, _ptr(y), _ptr(bd))
+    return y, bd
+
+
+# --------------------------------------------------------------------------
+# LLM.int8() decomposition ("Quantization" (engine-room ch. 15), The
+# Mathematics: C ~= S_out (.) (X_q W_q) + X_16 W_16)
+# --------------------------------------------------------------------------
+def outlier_columns(x, threshold: float, cap: int):
+    """(idx int32 [min(total, cap)], total): columns with max |x| >= threshold, lowest first."""
+    xb = _f16_bits(x)
+    M, K = xb.shape
+    idx = np.zeros(max(1, cap), np.int32)
+    total = lib().orc_outlier_columns(_ptr(xb), M, K, float(np.float32(threshold)), int(cap), _ptr(idx))
+    return idx[: min(total, cap)].copy(), int(total)
+
+
+def llm_int8_ref(x, wq, sw, idx, ms=None, ns=None):
+    """(y fp64 [nm, nn], bound, xq int8 [M, K], sx fp32 [M]) of the decomposed product with the
+    columns `idx` carved out of the INT8 path (weights: per-channel INT8 codes wq and scales sw)."""
+    xb = _f16_bits(x)
+    M, K = xb.shape
+    q = _c(wq, np.int8)
+    s = _c(sw, np.float32)
+    N = q.shape[0]
+    ix = _c(idx, np.int32)
+    m_arr, nm = _rows_arg(ms, M)
+    n_arr, nn = _rows_arg(ns, N)
+    xq = np.zeros((M, K), np.int8)
+    sx = np.zeros(M, np.float32)
+    y = np.zeros((nm, nn), np.float64)
+    bd = np.zeros((nm, nn), np.float64)
+    rc = lib().orc_llm_int8_ref(_ptr(xb), M, K, _ptr(q), _ptr(s), N, _ptr(ix), int(ix.size), _ptr(m_arr), nm,
+                                _ptr(n_arr), nn, _ptr(xq), _ptr(sx), _ptr(y), _ptr(bd))
+    if rc != 0:
+        raise ValueError("orc_llm_int8_ref: bad arguments")
+    return y, bd, xq, sx

@@ -46,6 +46,7 @@
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 
 /* ------------------------------------------------------------------------ */
@@ -351,5 +352,223 @@ int orc_gemm_w8a8_ref(const int8_t *xq, const float *sx, const int8_t *wq, const
             bound[(size_t)a * nn + c] = (double)sa * (double)sx[m] * (double)sw[n];
         }
     }
+    return rc;
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8 E4M3 ([P3] "Formats": 4 exponent bits, 3 mantissa bits, up to 448;   */
+/* [P4] "What about FP8, MXFP4, NVFP4 and GGUF?": E4M3 reaches +-448), the  */
+/* variant without infinities:                                               */
+/*   exponent field e in 1..15: (-1)^s * 2^(e-7) * (1 + m/8)                 */
+/*   e == 0 (subnormal):        (-1)^s * 2^(-6)  * (m/8)                     */
+/*   e == 15 and m == 7:        NaN  (so the largest finite value is 448)    */
+/* ------------------------------------------------------------------------ */
+float orc_e4m3_to_float(uint8_t c)
+{
+    int sign = (c >> 7) & 1;
+    int e = (c >> 3) & 0xf;
+    int m = c & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);                  /* 2^-6 * m/8 */
+    else
+        v = ldexp((double)(8 + m), e - 10);        /* 2^(e-7) * (8+m)/8 */
+    return (float)(sign ? -v : v);
+}
+
+/* Nearest E4M3 value, ties to even mantissa; magnitudes beyond 448 saturate
+   to 448 (reading: the format has no infinity, and every quantizer below
+   chooses its scale so that |x/s| <= 448 up to one rounding).  The sign of a
+   value that rounds to zero is kept. */
+uint8_t orc_float_to_e4m3(float f)
+{
+    uint8_t sign = signbit(f) ? 0x80 : 0;
+    double a = fabs((double)f);
+    if (isnan(f))
+        return 0x7f;
+    if (a >= 448.0)
+        return sign | 0x7e;
+    if (a < ldexp(1.0, -6)) {
+        /* subnormal grid: multiples of 2^-9; m == 8 is the smallest normal */
+        double m = nearbyint(a / ldexp(1.0, -9));
+        return sign | (uint8_t)m;
+    }
+    int E;
+    frexp(a, &E);                                  /* a in [2^(E-1), 2^E) */
+    int e = E - 1;
+    double m = nearbyint(a / ldexp(1.0, e - 3));   /* in [8, 16] */
+    if (m == 16.0) {
+        m = 8.0;
+        e += 1;
+    }
+    int field = e + 7;
+    if (field > 15 || (field == 15 && (int)m - 8 == 7))
+        return sign | 0x7e;                        /* rounds past 448: saturate */
+    return sign | (uint8_t)((field << 3) | ((int)m - 8));
+}
+
+/* ------------------------------------------------------------------------ */
+/* FP8 E4M3 quantizer ([P1] quant.py fake_quant_fp8: scale = max|w| / 448,  */
+/* codes = (w / scale) cast to E4M3).  x: fp16 bits [R][K].  per_row != 0:  */
+/* one scale per row (per output channel for weights, per token for          */
+/* activations; scales [R]); per_row == 0: one scale for the whole tensor   */
+/* (scales [1]), as in the listing.  The absmax is clamped at 1e-8 (the     */
+/* same guard as the listing's integer quantizer) so that an all-zero input */
+/* gets a finite scale.  w / scale is one IEEE fp32 division, then rounded  */
+/* to E4M3.                                                                  */
+/* ------------------------------------------------------------------------ */
+int orc_quantize_fp8_e4m3(const uint16_t *x, int R, int K, int per_row, uint8_t *q, float *scales)
+{
+    if (R <= 0 || K <= 0)
+        return -1;
+    float tensor_a = 0.0f;
+    if (!per_row) {
+        for (size_t i = 0; i < (size_t)R * K; ++i) {
+            float v = fabsf(orc_half_to_float(x[i]));
+            if (v > tensor_a) tensor_a = v;
+        }
+        if (tensor_a < 1e-8f) tensor_a = 1e-8f;
+        scales[0] = tensor_a / 448.0f;
+    }
+    for (int r = 0; r < R; ++r) {
+        const uint16_t *row = x + (size_t)r * K;
+        float s;
+        if (per_row) {
+            float a = 0.0f;
+            for (int k = 0; k < K; ++k) {
+                float v = fabsf(orc_half_to_float(row[k]));
+                if (v > a) a = v;
+            }
+            if (a < 1e-8f) a = 1e-8f;
+            s = a / 448.0f;
+            scales[r] = s;
+        } else {
+            s = scales[0];
+        }
+        for (int k = 0; k < K; ++k)
+            q[(size_t)r * K + k] = orc_float_to_e4m3(orc_half_to_float(row[k]) / s);
+    }
+    return 0;
+}
+
+/* FP8 W8A8 reference: y[m][n] = sx * sw * sum_k e4m3(xq[m][k]) e4m3(wq[n][k])
+   in fp64 (every product and partial sum is exact in fp64 for K <= 2^20),
+   bound = sx * sw * sum_k |products|.  sx_per_row / sw_per_row == 0 means one
+   scale for the whole operand (element 0).  ms/ns select rows of X and W. */
+void orc_gemm_fp8_ref(const uint8_t *xq, const float *sx, int sx_per_row, const uint8_t *wq,
+                      const float *sw, int sw_per_row, int M, int N, int K, const int *ms, int nm,
+                      const int *ns, int nn, double *y, double *bound)
+{
+    if (!ms) nm = M;
+    if (!ns) nn = N;
+    for (int a = 0; a < nm; ++a) {
+        int m = ms ? ms[a] : a;
+        double sxm = (double)sx[sx_per_row ? m : 0];
+        for (int c = 0; c < nn; ++c) {
+            int n = ns ? ns[c] : c;
+            double swn = (double)sw[sw_per_row ? n : 0];
+            double acc = 0.0, abs_acc = 0.0;
+            for (int k = 0; k < K; ++k) {
+                double p = (double)orc_e4m3_to_float(xq[(size_t)m * K + k]) *
+                           (double)orc_e4m3_to_float(wq[(size_t)n * K + k]);
+                acc += p;
+                abs_acc += fabs(p);
+            }
+            y[(size_t)a * nn + c] = acc * sxm * swn;
+            bound[(size_t)a * nn + c] = abs_acc * sxm * swn;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* LLM.int8() mixed-precision decomposition ([P2] "The Mathematics":        */
+/* C ~= S_out (.) (X_q W_q) + X_16 W_16, the outlier feature dimensions     */
+/* removed from the integer path and multiplied in 16-bit; [P2] "The         */
+/* Breakthrough": vector-wise scales per row and per column; [P4] outlier  */
+/* schemes: LLM.int8()-style mixed precision keeps the outlier dimensions  */
+/* in FP16 and quantizes the rest).                                          */
+/* Readings: an outlier dimension is an input column j with                  */
+/* max_m |X[m][j]| >= threshold (the threshold is a parameter; the pages do */
+/* not give its value); at most `cap` of them, the lowest column indices,   */
+/* are carved out; the weights are stored once, as per-output-channel INT8 */
+/* (the method halves weight memory, so no 16-bit copy exists) and W_16 is  */
+/* their dequantized outlier columns s_w[n] * W_q[n][j].                     */
+/* ------------------------------------------------------------------------ */
+
+/* Outlier columns of X [M][K] (fp16 bits): writes the first min(total, cap)
+   qualifying column indices in increasing order to idx and returns the
+   total number that qualify. */
+int orc_outlier_columns(const uint16_t *X, int M, int K, float threshold, int cap, int *idx)
+{
+    int total = 0;
+    for (int j = 0; j < K; ++j) {
+        float a = 0.0f;
+        for (int m = 0; m < M; ++m) {
+            float v = fabsf(orc_half_to_float(X[(size_t)m * K + j]));
+            if (v > a) a = v;
+        }
+        if (a >= threshold) {
+            if (total < cap)
+                idx[total] = j;
+            ++total;
+        }
+    }
+    return total;
+}
+
+/* The decomposed product for the carved-out columns idx[0..n_out):
+     keep[j] = 0 for carved columns, 1 otherwise
+     X_q, s_x = per-row symmetric INT8 of X * keep   (orc_quantize_sym_rows)
+     y[m][n]  = s_w[n] * ( s_x[m] * sum_{j not carved} X_q[m][j] W_q[n][j]
+                           + sum_{j carved} X[m][j] W_q[n][j] )       (fp64)
+   bound = s_w (s_x sum |X_q W_q| + sum |X W_q|).  xq/sx receive X_q and s_x
+   (both [M][K] / [M], required).  ms/ns select rows of X and of W. */
+int orc_llm_int8_ref(const uint16_t *X, int M, int K, const int8_t *wq, const float *sw, int N,
+                     const int *idx, int n_out, const int *ms, int nm, const int *ns, int nn,
+                     int8_t *xq, float *sx, double *y, double *bound)
+{
+    if (M <= 0 || N <= 0 || K <= 0 || n_out < 0 || n_out > K)
+        return -1;
+    float *keep = (float *)malloc(sizeof(float) * (size_t)K);
+    char *carved = (char *)calloc((size_t)K, 1);
+    if (!keep || !carved) {
+        free(keep);
+        free(carved);
+        return -1;
+    }
+    for (int j = 0; j < K; ++j)
+        keep[j] = 1.0f;
+    for (int i = 0; i < n_out; ++i) {
+        keep[idx[i]] = 0.0f;
+        carved[idx[i]] = 1;
+    }
+    int rc = orc_quantize_sym_rows(X, M, K, keep, 1, 8, xq, sx);
+    if (!ms) nm = M;
+    if (!ns) nn = N;
+    for (int a = 0; rc == 0 && a < nm; ++a) {
+        int m = ms ? ms[a] : a;
+        for (int c = 0; c < nn; ++c) {
+            int n = ns ? ns[c] : c;
+            double acc8 = 0.0, abs8 = 0.0, acc16 = 0.0, abs16 = 0.0;
+            for (int k = 0; k < K; ++k) {
+                double w = (double)wq[(size_t)n * K + k];
+                if (carved[k]) {
+                    double p = (double)orc_half_to_float(X[(size_t)m * K + k]) * w;
+                    acc16 += p;
+                    abs16 += fabs(p);
+                } else {
+                    double p = (double)xq[(size_t)m * K + k] * w;
+                    acc8 += p;
+                    abs8 += fabs(p);
+                }
+            }
+            y[(size_t)a * nn + c] = (double)sw[n] * ((double)sx[m] * acc8 + acc16);
+            bound[(size_t)a * nn + c] = (double)sw[n] * ((double)sx[m] * abs8 + abs16);
+        }
+    }
+    free(keep);
+    free(carved);
     return rc;
 }

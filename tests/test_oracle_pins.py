@@ -317,6 +317,15 @@ def test_w8a8_ref_is_exact_integer_matmul():
     big = np.full((1, 8192), -128, np.int8)
     acc2, _, _ = oracle.gemm_w8a8_ref(big, np.ones(1, np.float32), big, np.ones(1, np.float32))
     assert acc2[0, 0] == 128 * 128 * 8192
+    # selected rows of X (ms) and of W (ns), in any order and with repeats, agree with the
+    # full result indexed the same way (a swapped or misapplied selection fails here)
+    ms, ns = [6, 0, 3, 3], [8, 1, 4]
+    accs, ys, bs = oracle.gemm_w8a8_ref(xq, sx, wq, sw, ms=ms, ns=ns)
+    assert np.array_equal(accs, acc[np.ix_(ms, ns)])
+    assert np.array_equal(ys, y[np.ix_(ms, ns)]) and np.array_equal(bs, bound[np.ix_(ms, ns)])
+    acc_m, _, _ = oracle.gemm_w8a8_ref(xq, sx, wq, sw, ms=[2])
+    acc_n, _, _ = oracle.gemm_w8a8_ref(xq, sx, wq, sw, ns=[7, 5])
+    assert np.array_equal(acc_m, acc[[2]]) and np.array_equal(acc_n, acc[:, [7, 5]])
 
 
 def test_w8a16_ref_reduces_to_numpy():
@@ -327,6 +336,10 @@ def test_w8a16_ref_reduces_to_numpy():
     y, b = oracle.matmul_w8a16_ref(x, wq, sw)
     what = wq.astype(np.float64) * sw[:, None].astype(np.float64)
     assert np.allclose(y, x.astype(np.float64) @ what.T, rtol=1e-12, atol=1e-15)
+    assert np.allclose(b, np.abs(x.astype(np.float64)) @ np.abs(what).T, rtol=1e-12)
+    # selected rows (any order) agree with the full result's columns
+    ys, bs = oracle.matmul_w8a16_ref(x, wq, sw, rows=[11, 0, 4])
+    assert np.array_equal(ys, y[:, [11, 0, 4]]) and np.array_equal(bs, b[:, [11, 0, 4]])
 
 
 # --------------------------------------------------------------------------
@@ -386,3 +399,184 @@ def test_bad_arguments_rejected():
         oracle.quantize_group_int4(np.zeros((2, 100), np.float16), 128)
     with pytest.raises(ValueError):
         oracle.quantize_sym_rows(np.zeros((2, 8), np.float16), bits=9)
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3: the format pinned to torch's float8_e4m3fn conversions (an
+# independent library implementation), the pages' 448 maximum and scale
+# rule, and closed-form error bounds
+# --------------------------------------------------------------------------
+def _torch_e4m3_decode(codes):
+    import torch
+    return torch.tensor(np.asarray(codes, np.uint8)).view(torch.float8_e4m3fn).float().numpy()
+
+
+def test_e4m3_decode_all_codes_matches_torch_and_pages():
+    codes = np.arange(256)
+    ours = np.array([oracle.e4m3_to_float(c) for c in codes], np.float32)
+    ref = _torch_e4m3_decode(codes)
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan) and list(codes[nan]) == [0x7F, 0xFF]
+    assert np.array_equal(ours[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+    # "E4M3 ... reaches +-448" (the largest finite code); no infinities
+    assert np.nanmax(ours) == 448.0 and np.nanmin(ours) == -448.0 and not np.isinf(ours).any()
+    assert oracle.e4m3_to_float(0x01) == 2.0 ** -9       # smallest subnormal
+    assert oracle.e4m3_to_float(0x08) == 2.0 ** -6       # smallest normal
+
+
+def test_e4m3_encode_matches_torch_rne():
+    import torch
+    g = np.random.default_rng(21)
+    # every finite code, every midpoint between neighbours (ties to even), and random values
+    fin = np.array([oracle.e4m3_to_float(c) for c in range(0x7F)], np.float64)   # 0 .. 448
+    mids = (fin[:-1] + fin[1:]) / 2
+    rnd = np.exp(g.uniform(np.log(2.0 ** -12), np.log(448.0), 20000))
+    vals = np.concatenate([fin, mids, rnd, mids * (1 + 2 ** -20), mids * (1 - 2 ** -20)])
+    vals = np.concatenate([vals, -vals]).astype(np.float32)
+    ours = np.array([oracle.float_to_e4m3(v) for v in vals], np.uint8)
+    ref = torch.from_numpy(vals).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, ref)
+    # ties to even: 17 lies halfway between 16 (mantissa 0) and 18 (mantissa 1) -> 16
+    assert oracle.e4m3_to_float(oracle.float_to_e4m3(17.0)) == 16.0
+    assert oracle.e4m3_to_float(oracle.float_to_e4m3(19.0)) == 20.0
+    # beyond the largest finite value the reading saturates to 448 (the format has no infinity)
+    for v in (448.0, 460.0, 470.0, 1e6):
+        assert oracle.float_to_e4m3(v) == 0x7E and oracle.float_to_e4m3(-v) == 0xFE
+
+
+def test_fp8_quantizer_scale_rule_and_error_bound():
+    # "scale = max|w| / 448": the largest magnitude maps to the largest code, exactly
+    g = np.random.default_rng(22)
+    w = (g.standard_normal((6, 256)) * 0.02).astype(np.float32)
+    w.reshape(-1)[96::97] *= 20
+    w = w.astype(np.float16)
+    for per_row in (True, False):
+        q, s = oracle.quantize_fp8_e4m3(w, per_row=per_row)
+        wf = w.astype(np.float32)
+        amax = np.abs(wf).max(axis=1) if per_row else np.full(6, np.abs(wf).max())
+        assert np.array_equal(s, (amax / np.float32(448.0)).astype(np.float32)[: s.size])
+        dec = _torch_e4m3_decode(q).astype(np.float64)
+        srow = (s if per_row else np.repeat(s, 6)).astype(np.float64)[:, None]
+        what = dec * srow
+        # relative error at most half a step of a 3-bit mantissa (2^-4) on the normal range,
+        # absolute error at most half the subnormal step (2^-10 * s) below it
+        v = wf.astype(np.float64) / srow
+        err = np.abs(what - wf)
+        lim = np.where(np.abs(v) >= 2.0 ** -6, 2.0 ** -4 * np.abs(wf), 2.0 ** -10 * srow) * (1 + 1e-6)
+        assert np.all(err <= lim)
+        for r in range(6):
+            k = np.argmax(np.abs(wf[r])) if per_row else None
+            if per_row:
+                assert q[r, k] & 0x7F == 0x7E
+        if not per_row:
+            assert (q & 0x7F == 0x7E).sum() >= 1
+    # an all-zero tensor: finite scale (absmax clamped at 1e-8), all codes zero
+    q0, s0 = oracle.quantize_fp8_e4m3(np.zeros((2, 32), np.float16))
+    assert np.all(s0 == np.float32(1e-8) / np.float32(448.0)) and not q0.any()
+
+
+def test_fp8_per_tensor_beats_int8_per_tensor():
+    # "FP8, even per tensor, has less error than INT8 per tensor" on weights with outliers
+    g = np.random.default_rng(23)
+    w = (g.standard_normal((128, 1024)) * 0.02).astype(np.float32)
+    w.reshape(-1)[96::97] *= 20
+    w = w.astype(np.float16)
+    wf = w.astype(np.float64)
+    q8, s8 = oracle.quantize_fp8_e4m3(w, per_row=False)
+    fp8 = _torch_e4m3_decode(q8).astype(np.float64) * float(s8[0])
+    qi, si = oracle.quantize_sym_rows(w.reshape(1, -1), None, 0, 8)
+    int8 = (qi.astype(np.float64) * float(si[0])).reshape(w.shape)
+    assert _rel(fp8, wf) < _rel(int8, wf)
+
+
+def test_fp8_gemm_ref_reduces_to_numpy():
+    g = np.random.default_rng(24)
+    xq = g.integers(0, 256, (5, 64), dtype=np.uint8)
+    wq = g.integers(0, 256, (7, 64), dtype=np.uint8)
+    xq[(xq & 0x7F) == 0x7F] = 0x10      # no NaN codes
+    wq[(wq & 0x7F) == 0x7F] = 0x22
+    sx = g.random(5, dtype=np.float32) + 0.5
+    sw = g.random(7, dtype=np.float32) + 0.5
+    y, b = oracle.gemm_fp8_ref(xq, sx, wq, sw)
+    dx, dw = _torch_e4m3_decode(xq).astype(np.float64), _torch_e4m3_decode(wq).astype(np.float64)
+    ref = (dx @ dw.T) * sx[:, None].astype(np.float64) * sw[None, :].astype(np.float64)
+    assert np.allclose(y, ref, rtol=1e-15, atol=0)
+    assert np.allclose(b, (np.abs(dx) @ np.abs(dw).T) * sx[:, None] * sw[None, :], rtol=1e-12)
+    # a per-tensor scale (one element) applies to every row
+    y1, _ = oracle.gemm_fp8_ref(xq, sx[:1], wq, sw[:1])
+    assert np.allclose(y1, (dx @ dw.T) * float(sx[0]) * float(sw[0]), rtol=1e-15)
+    ys, _ = oracle.gemm_fp8_ref(xq, sx, wq, sw, ms=[4, 1], ns=[6, 0, 3])
+    assert np.array_equal(ys, y[np.ix_([4, 1], [6, 0, 3])])
+
+
+# --------------------------------------------------------------------------
+# LLM.int8() decomposition: reduces to the plain W8A8 and W8A16 references at
+# its two extremes, finds planted outlier columns, and beats plain W8A8 on
+# activations with outlier features
+# --------------------------------------------------------------------------
+def _llm_case(seed=31, M=24, N=20, K=256, planted=(3, 70, 71, 200)):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((M, K)).astype(np.float32)
+    x[:, list(planted)] *= 40.0
+    x = x.astype(np.float16)
+    w = (g.standard_normal((N, K)) * 0.02).astype(np.float16)
+    wq, sw = oracle.quantize_int8_per_channel(w)
+    return x, w, wq, sw
+
+
+def test_outlier_columns_found_and_capped():
+    x, _, _, _ = _llm_case()
+    idx, total = oracle.outlier_columns(x, 6.0, 16)
+    assert total == 4 and list(idx) == [3, 70, 71, 200]
+    idx2, total2 = oracle.outlier_columns(x, 6.0, 2)           # cap keeps the lowest columns
+    assert total2 == 4 and list(idx2) == [3, 70]
+    # the threshold compares max |x| >= t: a column whose max equals t qualifies
+    e = np.zeros((2, 16), np.float16)
+    e[1, 5], e[0, 9] = 6.0, -5.996
+    assert oracle.outlier_columns(e, 6.0, 4) == (np.array([5], np.int32), 1)
+
+
+def test_llm_int8_reduces_to_w8a8_without_outliers():
+    x, _, wq, sw = _llm_case()
+    y, b, xq, sx = oracle.llm_int8_ref(x, wq, sw, np.zeros(0, np.int32))
+    rxq, rsx = oracle.quantize_int8_per_token(x)
+    assert np.array_equal(xq, rxq) and np.array_equal(sx, rsx)
+    _, ry, rb = oracle.gemm_w8a8_ref(rxq, rsx, wq, sw)
+    assert np.allclose(y, ry, rtol=1e-14, atol=0) and np.allclose(b, rb, rtol=1e-14)
+
+
+def test_llm_int8_reduces_to_w8a16_with_every_column_carved():
+    x, _, wq, sw = _llm_case()
+    y, b, xq, _ = oracle.llm_int8_ref(x, wq, sw, np.arange(x.shape[1], dtype=np.int32))
+    assert not xq.any()
+    ry, rb = oracle.matmul_w8a16_ref(x, wq, sw)
+    assert np.allclose(y, ry.T.T, rtol=1e-13, atol=1e-18) and np.allclose(b, rb, rtol=1e-13)
+
+
+def test_llm_int8_carves_exactly_the_listed_columns():
+    x, _, wq, sw = _llm_case()
+    idx = np.array([3, 70, 71, 200], np.int32)
+    y, _, xq, sx = oracle.llm_int8_ref(x, wq, sw, idx)
+    assert not xq[:, idx].any()
+    keep = np.ones(x.shape[1], np.float32)
+    keep[idx] = 0
+    rxq, rsx = oracle.quantize_sym_rows(x, keep, 1, 8)
+    assert np.array_equal(xq, rxq) and np.array_equal(sx, rsx)
+    # S_out (.) (X_q W_q) + X_16 W_16 written out with numpy in fp64
+    xf = x.astype(np.float64)
+    w16 = wq[:, idx].astype(np.float64) * sw[:, None]
+    ref = (xq.astype(np.float64) @ wq.astype(np.float64).T) * sx[:, None].astype(np.float64) * sw[None, :] \
+        + xf[:, idx] @ w16.T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-15)
+    ys, _, _, _ = oracle.llm_int8_ref(x, wq, sw, idx, ms=[5, 0], ns=[19, 2, 7])
+    assert np.array_equal(ys, y[np.ix_([5, 0], [19, 2, 7])])
+
+
+def test_llm_int8_beats_plain_w8a8_on_outlier_features():
+    # carving the outlier dimensions out keeps the other values' precision
+    x, w, wq, sw = _llm_case(seed=32, M=64, N=48, K=512, planted=(11, 40, 300))
+    exact = x.astype(np.float64) @ (wq.astype(np.float64) * sw[:, None]).T
+    idx, _ = oracle.outlier_columns(x, 6.0, 64)
+    y_llm, _, _, _ = oracle.llm_int8_ref(x, wq, sw, idx)
+    y_w8a8, _, _, _ = oracle.llm_int8_ref(x, wq, sw, np.zeros(0, np.int32))
+    assert _rel(y_llm, exact) < 0.5 * _rel(y_w8a8, exact)
