@@ -83,6 +83,19 @@ def _declare(L):
     L.orc_outlier_columns.restype = _I
     L.orc_llm_int8_ref.argtypes = [_P, _I, _I, _P, _P, _I, _P, _I, _P, _I, _P, _I, _P, _P, _P, _P]
     L.orc_llm_int8_ref.restype = _I
+    L.orc_e2m1_to_float.argtypes = [ctypes.c_uint8]
+    L.orc_e2m1_to_float.restype = ctypes.c_float
+    L.orc_float_to_e2m1.argtypes = [ctypes.c_float]
+    L.orc_float_to_e2m1.restype = ctypes.c_uint8
+    L.orc_e8m0_to_float.argtypes = [ctypes.c_uint8]
+    L.orc_e8m0_to_float.restype = ctypes.c_float
+    L.orc_quantize_mxfp4.argtypes = [_P, _I, _I, _P, _P]
+    L.orc_quantize_mxfp4.restype = _I
+    L.orc_quantize_nvfp4.argtypes = [_P, _I, _I, _P, _P, _P]
+    L.orc_quantize_nvfp4.restype = _I
+    L.orc_gemm_fp4_ref.argtypes = [_I, _P, _P, ctypes.c_float, _P, _P, ctypes.c_float, _I, _I, _I, _P, _I, _P, _I,
+                                   _P, _P]
+    L.orc_gemm_fp4_ref.restype = None
 
 
 def _ptr(a: np.ndarray | None):
@@ -345,3 +358,66 @@ def llm_int8_ref(x, wq, sw, idx, ms=None, ns=None):
     if rc != 0:
         raise ValueError("orc_llm_int8_ref: bad arguments")
     return y, bd, xq, sx
+
+
+# --------------------------------------------------------------------------
+# Block-scaled FP4: MXFP4 (E2M1, blocks of 32, E8M0 power-of-two scales) and
+# NVFP4 (E2M1, blocks of 16, E4M3 scales, one fp32 tensor scale)
+# ("Quantization: Smaller Weights, Same Answers (Mostly)", FP8/MXFP4/NVFP4
+# section; "Quantization from Scratch", Formats)
+# --------------------------------------------------------------------------
+def e2m1_to_float(code: int) -> float:
+    return float(lib().orc_e2m1_to_float(int(code) & 0xF))
+
+
+def float_to_e2m1(x: float) -> int:
+    return int(lib().orc_float_to_e2m1(float(np.float32(x))))
+
+
+def e8m0_to_float(code: int) -> float:
+    return float(lib().orc_e8m0_to_float(int(code) & 0xFF))
+
+
+def quantize_mxfp4(a):
+    """fp16 [R, K] -> (packed E2M1 uint8 [R, K/2], E8M0 scales uint8 [R, K/32])."""
+    xb = _f16_bits(a)
+    R, K = xb.shape
+    q = np.zeros((R, K // 2), np.uint8)
+    s = np.zeros((R, K // 32), np.uint8)
+    if lib().orc_quantize_mxfp4(_ptr(xb), R, K, _ptr(q), _ptr(s)) != 0:
+        raise ValueError("orc_quantize_mxfp4: bad arguments")
+    return q, s
+
+
+def quantize_nvfp4(a):
+    """fp16 [R, K] -> (packed E2M1 uint8 [R, K/2], E4M3 scales uint8 [R, K/16], fp32 tensor scale [1])."""
+    xb = _f16_bits(a)
+    R, K = xb.shape
+    q = np.zeros((R, K // 2), np.uint8)
+    s = np.zeros((R, K // 16), np.uint8)
+    t = np.zeros(1, np.float32)
+    if lib().orc_quantize_nvfp4(_ptr(xb), R, K, _ptr(q), _ptr(s), _ptr(t)) != 0:
+        raise ValueError("orc_quantize_nvfp4: bad arguments")
+    return q, s, t
+
+
+def unpack_fp4(q, K: int) -> np.ndarray:
+    """E2M1 codes [R, K] from the packed layout (element 2i in the low nibble of byte i)."""
+    q = _c(q, np.uint8)
+    out = np.empty((q.shape[0], K), np.uint8)
+    out[:, 0::2] = q & 0xF
+    out[:, 1::2] = q >> 4
+    return out
+
+
+def gemm_fp4_ref(nvfp4: bool, a, sa, ta, b, sb, tb, K: int, ms=None, ns=None):
+    """(y fp64, bound) of the block-scaled FP4 product (tensor scales ta/tb: 1.0 for MXFP4)."""
+    A, SA, B, SB = _c(a, np.uint8), _c(sa, np.uint8), _c(b, np.uint8), _c(sb, np.uint8)
+    M, N = A.shape[0], B.shape[0]
+    m_arr, nm = _rows_arg(ms, M)
+    n_arr, nn = _rows_arg(ns, N)
+    y = np.zeros((nm, nn), np.float64)
+    bd = np.zeros((nm, nn), np.float64)
+    lib().orc_gemm_fp4_ref(1 if nvfp4 else 0, _ptr(A), _ptr(SA), float(ta), _ptr(B), _ptr(SB), float(tb), M, N, K,
+                           _ptr(m_arr), nm, _ptr(n_arr), nn, _ptr(y), _ptr(bd))
+    return y, bd

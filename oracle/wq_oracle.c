@@ -572,3 +572,175 @@ int orc_llm_int8_ref(const uint16_t *X, int M, int K, const int8_t *wq, const fl
     free(carved);
     return rc;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Block-scaled FP4 ([P4] "What about FP8, MXFP4, NVFP4 and GGUF?": MXFP4   */
+/* stores blocks of 32 four-bit floats (E2M1) sharing one 8-bit power-of-two */
+/* scale; NVFP4 uses blocks of 16 with an FP8 scale per block plus one FP32 */
+/* scale per tensor; [P3] "Formats": blocks of 32 share one 8-bit           */
+/* power-of-two scale; [P1] "Mainstream schemes": FP4 (NVFP4 / MXFP4) on    */
+/* Blackwell).                                                               */
+/* E2M1: 1 sign, 2 exponent bits (bias 1), 1 mantissa bit, no inf/NaN:       */
+/*   e in 1..3: (-1)^s * 2^(e-1) * (1 + m/2);  e == 0: (-1)^s * m/2          */
+/*   i.e. 0, 0.5, 1, 1.5, 2, 3, 4, 6.                                        */
+/* Readings (the pages name the formats, not their rounding rules):          */
+/*  - MXFP4 follows the microscaling specification the pages cite: shared    */
+/*    exponent floor(log2(max|v|)) - 2 (2 = the exponent of E2M1's largest   */
+/*    value 6), stored as E8M0 = exponent + 127 (an all-zero block gets 0,   */
+/*    i.e. 2^-127); elements v / 2^e rounded to nearest even, saturating at  */
+/*    +-6.                                                                   */
+/*  - NVFP4: tensor scale S = max(max|v|, 1e-8) / (6 * 448); block scale     */
+/*    E4M3 code of (max_block|v| / 6) / S (positive); elements               */
+/*    e2m1_rn(v / (e4m3(block) * S)), all zero when the block code is 0.     */
+/*  - two elements per byte, element 2i in the low nibble.                   */
+/* ------------------------------------------------------------------------ */
+float orc_e2m1_to_float(uint8_t c)
+{
+    int sign = (c >> 3) & 1;
+    int e = (c >> 1) & 3;
+    int m = c & 1;
+    double v = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return (float)(sign ? -v : v);
+}
+
+/* Nearest E2M1 value, ties to even mantissa, magnitudes beyond 6 saturate. */
+uint8_t orc_float_to_e2m1(float f)
+{
+    uint8_t sign = signbit(f) ? 8 : 0;
+    double a = fabs((double)f);
+    if (a >= 6.0)
+        return sign | 7;
+    if (a < 1.0) {                                 /* subnormal grid: multiples of 0.5 */
+        double m = nearbyint(a / 0.5);             /* 0, 1 or 2 (2 = the value 1.0) */
+        return sign | (uint8_t)m;
+    }
+    int E;
+    frexp(a, &E);                                  /* a in [2^(E-1), 2^E) */
+    int e = E - 1;                                 /* 0..2 */
+    double m = nearbyint(a / ldexp(1.0, e - 1));   /* in [2, 4] */
+    if (m == 4.0) {
+        m = 2.0;
+        e += 1;
+    }
+    if (e + 1 > 3)
+        return sign | 7;
+    return sign | (uint8_t)(((e + 1) << 1) | ((int)m - 2));
+}
+
+float orc_e8m0_to_float(uint8_t c)
+{
+    return (float)ldexp(1.0, (int)c - 127);        /* 255 would be NaN; never produced */
+}
+
+static void put_nibble(uint8_t *q, size_t k, uint8_t v)
+{
+    if (k % 2 == 0)
+        q[k / 2] = (uint8_t)((q[k / 2] & 0xf0) | (v & 0xf));
+    else
+        q[k / 2] = (uint8_t)((q[k / 2] & 0x0f) | ((v & 0xf) << 4));
+}
+
+uint8_t orc_fp4_code(const uint8_t *q, size_t k)
+{
+    return (k % 2 == 0) ? (q[k / 2] & 0xf) : (q[k / 2] >> 4);
+}
+
+/* MXFP4: x fp16 [R][K], K % 32 == 0 -> q [R][K/2], scales E8M0 [R][K/32]. */
+int orc_quantize_mxfp4(const uint16_t *x, int R, int K, uint8_t *q, uint8_t *scales)
+{
+    if (R <= 0 || K <= 0 || K % 32 != 0)
+        return -1;
+    for (int r = 0; r < R; ++r) {
+        for (int b = 0; b < K / 32; ++b) {
+            const uint16_t *blk = x + (size_t)r * K + (size_t)b * 32;
+            float a = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float v = fabsf(orc_half_to_float(blk[i]));
+                if (v > a) a = v;
+            }
+            int e;
+            if (a == 0.0f) {
+                e = -127;
+            } else {
+                int E;
+                frexp((double)a, &E);              /* floor(log2 a) = E - 1 */
+                e = (E - 1) - 2;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            scales[(size_t)r * (K / 32) + b] = (uint8_t)(e + 127);
+            for (int i = 0; i < 32; ++i) {
+                float v = orc_half_to_float(blk[i]);
+                float t = (float)ldexp((double)v, -e); /* exact: a power-of-two scaling */
+                put_nibble(q + (size_t)r * (K / 2), (size_t)b * 32 + i, a == 0.0f ? 0 : orc_float_to_e2m1(t));
+            }
+        }
+    }
+    return 0;
+}
+
+/* NVFP4: x fp16 [R][K], K % 16 == 0 -> q [R][K/2], scales E4M3 [R][K/16], tensor scale [1]. */
+int orc_quantize_nvfp4(const uint16_t *x, int R, int K, uint8_t *q, uint8_t *scales, float *tensor_scale)
+{
+    if (R <= 0 || K <= 0 || K % 16 != 0)
+        return -1;
+    float at = 0.0f;
+    for (size_t i = 0; i < (size_t)R * K; ++i) {
+        float v = fabsf(orc_half_to_float(x[i]));
+        if (v > at) at = v;
+    }
+    if (at < 1e-8f) at = 1e-8f;
+    const float S = at / 2688.0f;                  /* 6 * 448 */
+    tensor_scale[0] = S;
+    for (int r = 0; r < R; ++r) {
+        for (int b = 0; b < K / 16; ++b) {
+            const uint16_t *blk = x + (size_t)r * K + (size_t)b * 16;
+            float a = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float v = fabsf(orc_half_to_float(blk[i]));
+                if (v > a) a = v;
+            }
+            const float e = (a / 6.0f) / S;
+            const uint8_t sb = orc_float_to_e4m3(e);
+            scales[(size_t)r * (K / 16) + b] = sb;
+            const float d = orc_e4m3_to_float(sb) * S;
+            for (int i = 0; i < 16; ++i) {
+                float v = orc_half_to_float(blk[i]);
+                put_nibble(q + (size_t)r * (K / 2), (size_t)b * 16 + i, sb == 0 ? 0 : orc_float_to_e2m1(v / d));
+            }
+        }
+    }
+    return 0;
+}
+
+/* Block-scaled FP4 GEMM reference: y[m][n] = ta * tb * sum_k dec(a[m][k]) sa(m, k/bs)
+   dec(b[n][k]) sb(n, k/bs) in fp64 (bs = 32 with E8M0 scales for MXFP4, 16 with E4M3
+   scales for NVFP4; ta/tb are the tensor scales, 1 for MXFP4), bound = the same with
+   absolute values.  ms/ns select rows of A and B. */
+void orc_gemm_fp4_ref(int nvfp4, const uint8_t *a, const uint8_t *sa, float ta, const uint8_t *b,
+                      const uint8_t *sb, float tb, int M, int N, int K, const int *ms, int nm,
+                      const int *ns, int nn, double *y, double *bound)
+{
+    const int bs = nvfp4 ? 16 : 32;
+    const int nb = K / bs;
+    if (!ms) nm = M;
+    if (!ns) nn = N;
+    for (int i = 0; i < nm; ++i) {
+        int m = ms ? ms[i] : i;
+        for (int j = 0; j < nn; ++j) {
+            int n = ns ? ns[j] : j;
+            double acc = 0.0, abs_acc = 0.0;
+            for (int k = 0; k < K; ++k) {
+                uint8_t ca = sa[(size_t)m * nb + k / bs], cb = sb[(size_t)n * nb + k / bs];
+                double fa = nvfp4 ? (double)orc_e4m3_to_float(ca) : (double)orc_e8m0_to_float(ca);
+                double fb = nvfp4 ? (double)orc_e4m3_to_float(cb) : (double)orc_e8m0_to_float(cb);
+                double p = (double)orc_e2m1_to_float(orc_fp4_code(a + (size_t)m * (K / 2), k)) * fa *
+                           (double)orc_e2m1_to_float(orc_fp4_code(b + (size_t)n * (K / 2), k)) * fb;
+                acc += p;
+                abs_acc += fabs(p);
+            }
+            y[(size_t)i * nn + j] = acc * (double)ta * (double)tb;
+            bound[(size_t)i * nn + j] = abs_acc * (double)ta * (double)tb;
+        }
+    }
+}

@@ -580,3 +580,109 @@ def test_llm_int8_beats_plain_w8a8_on_outlier_features():
     y_llm, _, _, _ = oracle.llm_int8_ref(x, wq, sw, idx)
     y_w8a8, _, _, _ = oracle.llm_int8_ref(x, wq, sw, np.zeros(0, np.int32))
     assert _rel(y_llm, exact) < 0.5 * _rel(y_w8a8, exact)
+
+
+# --------------------------------------------------------------------------
+# Block-scaled FP4 (MXFP4, NVFP4): E2M1 by brute force over its 16 codes,
+# the pages' storage figures, block-scale properties, the GEMM reference
+# against numpy on dequantized values
+# --------------------------------------------------------------------------
+def _e2m1_table():
+    return np.array([oracle.e2m1_to_float(c) for c in range(16)], np.float64)
+
+
+def test_e2m1_codes_and_brute_force_rounding():
+    tab = _e2m1_table()
+    # "four-bit floats (E2M1)": 8 magnitudes, the largest 6, a sign bit
+    assert sorted(set(np.abs(tab))) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert np.array_equal(tab[8:], -tab[:8])
+    g = np.random.default_rng(41)
+    vals = np.concatenate([g.uniform(-7, 7, 4000), (np.arange(-28, 29) / 4.0)]).astype(np.float32)
+    for v in vals:
+        code = oracle.float_to_e2m1(v)
+        # brute force: the nearest code (within the sign of v); a tie goes to the even mantissa
+        cands = range(8, 16) if np.signbit(v) else range(0, 8)
+        dist = {c: abs(tab[c] - min(max(v, -6.0), 6.0)) for c in cands}
+        best = min(dist.values())
+        near = [c for c in cands if dist[c] == best]
+        want = near[0] if len(near) == 1 else [c for c in near if c % 2 == 0][0]
+        assert code == want, (v, code, want)
+
+
+def test_fp4_storage_figures_from_the_pages():
+    # MXFP4: 32 four-bit values + one 8-bit scale = "about 4.25 bits per weight"
+    assert (32 * 4 + 8) / 32 == 4.25
+    # NVFP4: 16 values + an FP8 scale: 4.5 bits, "about 3.5 times" smaller than FP16
+    assert abs(16 / ((16 * 4 + 8) / 16) - 3.5) < 0.1
+    q, s = oracle.quantize_mxfp4(np.zeros((3, 64), np.float16))
+    assert q.shape == (3, 32) and s.shape == (3, 2)
+    q2, s2, t2 = oracle.quantize_nvfp4(np.zeros((3, 64), np.float16))
+    assert q2.shape == (3, 32) and s2.shape == (3, 4) and t2.shape == (1,)
+
+
+def test_mxfp4_block_scale_rule():
+    g = np.random.default_rng(42)
+    x = (g.standard_normal((8, 256)) * np.exp(g.uniform(-6, 6, (8, 1)))).astype(np.float16)
+    x[0, :32] = 0.0                                                # an all-zero block
+    q, s = oracle.quantize_mxfp4(x)
+    codes = oracle.unpack_fp4(q, 256)
+    tab = _e2m1_table()
+    xf = x.astype(np.float64).reshape(8, 8, 32)
+    deq = tab[codes].reshape(8, 8, 32) * np.ldexp(1.0, s.astype(np.int64) - 127)[:, :, None]
+    amax = np.abs(xf).max(axis=2)
+    nz = amax > 0
+    # the block maximum lands in [4, 8) units of the shared power of two (so it may saturate to 6)
+    ratio = amax[nz] / np.ldexp(1.0, s[nz].astype(np.int64) - 127)
+    assert np.all((ratio >= 4) & (ratio < 8))
+    assert s[0, 0] == 0 and not codes[0, :32].any()
+    # every element is the nearest grid value of the scaled block (saturating at 6)
+    scale = np.ldexp(1.0, s.astype(np.int64) - 127)[:, :, None]
+    err = np.abs(deq - np.clip(xf, -6 * scale, 6 * scale))
+    assert np.all(err <= 1.0 * scale + 1e-300)        # half of the widest step (2 between 4 and 6)
+
+
+def test_nvfp4_scale_rule_and_error():
+    g = np.random.default_rng(43)
+    x = (g.standard_normal((6, 128)) * 0.05).astype(np.float32)
+    x[:, 5] *= 30
+    x = x.astype(np.float16)
+    q, s, t = oracle.quantize_nvfp4(x)
+    xf = x.astype(np.float64)
+    assert t[0] == np.float32(np.float32(np.abs(xf).max()) / np.float32(2688.0))
+    sb = np.array([oracle.e4m3_to_float(c) for c in s.reshape(-1)]).reshape(s.shape)
+    # the block maximum divided by its decoded scale x tensor scale stays near 6 (E4M3 rounding of the
+    # block scale is within 2^-4 relative)
+    amax = np.abs(xf).reshape(6, 8, 16).max(axis=2)
+    r = amax / (sb * float(t[0]))
+    assert np.all((r > 6 / (1 + 2 ** -4) - 1e-9) & (r < 6 / (1 - 2 ** -4) + 1e-9))
+    deq = _e2m1_table()[oracle.unpack_fp4(q, 128)].reshape(6, 8, 16) * (sb * float(t[0]))[:, :, None]
+    # relative error of the block maximum's quantization: a step of E2M1 near 6 is 2 (1/3 of 6)
+    assert np.all(np.abs(deq - xf.reshape(6, 8, 16)) <= (sb * float(t[0]))[:, :, None] * 1.0 + 1e-12)
+
+
+def test_fp4_gemm_ref_reduces_to_numpy():
+    g = np.random.default_rng(44)
+    a = (g.standard_normal((5, 128))).astype(np.float16)
+    b = (g.standard_normal((7, 128)) * 0.1).astype(np.float16)
+    tab = _e2m1_table()
+    for nv in (False, True):
+        if nv:
+            qa, sa, ta = oracle.quantize_nvfp4(a)
+            qb, sb, tb = oracle.quantize_nvfp4(b)
+            da = np.array([oracle.e4m3_to_float(c) for c in sa.reshape(-1)]).reshape(sa.shape) * float(ta[0])
+            db = np.array([oracle.e4m3_to_float(c) for c in sb.reshape(-1)]).reshape(sb.shape) * float(tb[0])
+            bs, tav, tbv = 16, float(ta[0]), float(tb[0])
+        else:
+            qa, sa = oracle.quantize_mxfp4(a)
+            qb, sb = oracle.quantize_mxfp4(b)
+            da, db = np.ldexp(1.0, sa.astype(np.int64) - 127), np.ldexp(1.0, sb.astype(np.int64) - 127)
+            bs, tav, tbv = 32, 1.0, 1.0
+        wa = tab[oracle.unpack_fp4(qa, 128)] * np.repeat(da, bs, axis=1)
+        wb = tab[oracle.unpack_fp4(qb, 128)] * np.repeat(db, bs, axis=1)
+        y, bd = oracle.gemm_fp4_ref(nv, qa, sa, tav, qb, sb, tbv, 128)
+        assert np.allclose(y, wa @ wb.T, rtol=1e-12, atol=1e-300)
+        assert np.allclose(bd, np.abs(wa) @ np.abs(wb).T, rtol=1e-12)
+        # dequantized values approximate the inputs (the format works): relative Frobenius error < 20%
+        assert _rel(wa, a.astype(np.float64)) < 0.2
+        ys, _ = oracle.gemm_fp4_ref(nv, qa, sa, tav, qb, sb, tbv, 128, ms=[4, 0], ns=[6, 1])
+        assert np.array_equal(ys, y[np.ix_([4, 0], [6, 1])])
