@@ -18,7 +18,9 @@ import torch
 
 __all__ = ["WQError", "lib", "quantize_group_int4", "quantize_int8_per_channel", "quantize_int8_per_token",
            "smooth", "smooth_workspace_bytes", "smooth_noalloc", "gemv_w4a16", "gemm_w4a16", "gemm_w8a8", "gemv_w8a16",
-           "matmul_w4a16", "device_status", "set_wait_limit", "selftest_wait_timeout", "LIB_PATH"]
+           "matmul_w4a16", "quantize_fp8_e4m3", "gemm_fp8", "outlier_columns", "gather_outliers",
+           "gemm_w8a8_outliers", "llm_int8_matmul", "device_status", "set_wait_limit",
+           "selftest_wait_timeout", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwq.so")
 
@@ -50,6 +52,11 @@ _SIGS = {
     "wq_gemm_w4a16": [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P],
     "wq_gemm_w8a8": [_P, _P, _P, _P, _I, _I, _I, _P, _P, _P],
     "wq_gemv_w8a16": [_P, _I, _P, _P, _I, _I, _P, _P],
+    "wq_quantize_fp8_e4m3": [_P, _I, _I, _I, _P, _P, _P],
+    "wq_gemm_fp8": [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P],
+    "wq_outlier_columns": [_P, _I, _I, _F, _I, _P, _P, _P, _P],
+    "wq_gather_outliers": [_P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _P],
+    "wq_gemm_w8a8_outliers": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P],
     "wq_device_status": [_P],
     "wq_selftest_wait_timeout": [_P],
 }
@@ -268,6 +275,93 @@ def gemv_w8a16(x, wq, sw, out=None, stream=None):
     _cuda(y, "out", (torch.float16,), 2)
     _check(lib.wq_gemv_w8a16(_ptr(x), B, _ptr(wq), _ptr(sw), N, K, _ptr(y), _P(_stream(stream))), "wq_gemv_w8a16")
     return y
+
+
+def quantize_fp8_e4m3(a: torch.Tensor, per_row: bool = True, stream=None):
+    """FP8 E4M3 codes (torch.uint8 [R, K]) and fp32 scales ([R] per row, [1] per tensor) of fp16 `a`."""
+    _cuda(a, "input", (torch.float16,), 2)
+    R, K = a.shape
+    q = _empty((R, K), torch.uint8, a)
+    s = _empty((R if per_row else 1,), torch.float32, a)
+    _check(lib.wq_quantize_fp8_e4m3(_ptr(a), R, K, 1 if per_row else 0, _ptr(q), _ptr(s), _P(_stream(stream))),
+           "wq_quantize_fp8_e4m3")
+    return q, s
+
+
+def gemm_fp8(xq, sx, wq, sw, out=None, return_acc: bool = False, stream=None):
+    """y [M, N] fp16 = fp16((e4m3(xq) @ e4m3(wq)^T) * sx * sw); a scale tensor of one element is per tensor."""
+    _cuda(xq, "xq", (torch.uint8,), 2)
+    _cuda(wq, "wq", (torch.uint8,), 2)
+    _cuda(sx, "sx", (torch.float32,), 1)
+    _cuda(sw, "sw", (torch.float32,), 1)
+    M, K = xq.shape
+    N, K2 = wq.shape
+    if K != K2 or sx.numel() not in (1, M) or sw.numel() not in (1, N):
+        raise ValueError("shape mismatch: xq [M,K], wq [N,K], sx [M] or [1], sw [N] or [1]")
+    y = out if out is not None else _empty((M, N), torch.float16, xq)
+    _cuda(y, "out", (torch.float16,), 2)
+    acc = _empty((M, N), torch.float32, xq) if return_acc else None
+    _check(lib.wq_gemm_fp8(_ptr(xq), _ptr(sx), int(sx.numel() == M), _ptr(wq), _ptr(sw), int(sw.numel() == N),
+                           M, N, K, _ptr(y), _ptr(acc), _P(_stream(stream))), "wq_gemm_fp8")
+    return (y, acc) if return_acc else y
+
+
+def outlier_columns(x: torch.Tensor, threshold: float = 6.0, cap: int = 64, stream=None):
+    """LLM.int8() outlier columns of fp16 x [M, K]: (idx int32 [cap], count int32 [1], keep fp32 [K]).
+
+    idx[:min(count, cap)] are the carved columns (lowest first); keep is 0 there and 1 elsewhere."""
+    _cuda(x, "x", (torch.float16,), 2)
+    M, K = x.shape
+    idx = torch.zeros((cap,), dtype=torch.int32, device=x.device)
+    count = _empty((1,), torch.int32, x)
+    keep = _empty((K,), torch.float32, x)
+    _check(lib.wq_outlier_columns(_ptr(x), M, K, float(threshold), int(cap), _ptr(idx), _ptr(count), _ptr(keep),
+                                  _P(_stream(stream))), "wq_outlier_columns")
+    return idx, count, keep
+
+
+def gather_outliers(x, wq, idx, count, cap: int, stream=None):
+    """(X_16 fp16 [M, cap], W_16 fp16 [N, cap]): the carved columns of x and of the INT8 weight codes."""
+    _cuda(x, "x", (torch.float16,), 2)
+    _cuda(wq, "wq", (torch.int8,), 2)
+    _cuda(idx, "idx", (torch.int32,), 1)
+    _cuda(count, "count", (torch.int32,), 1)
+    M, K = x.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K or idx.numel() < cap:
+        raise ValueError("shape mismatch: x [M,K], wq [N,K], idx [>= cap]")
+    x16 = _empty((M, cap), torch.float16, x)
+    w16 = _empty((N, cap), torch.float16, x)
+    _check(lib.wq_gather_outliers(_ptr(x), M, K, _ptr(wq), N, _ptr(idx), _ptr(count), int(cap), _ptr(x16), _ptr(w16),
+                                  _P(_stream(stream))), "wq_gather_outliers")
+    return x16, w16
+
+
+def gemm_w8a8_outliers(xq, sx, wq, sw, x16, w16, out=None, stream=None):
+    """y [M, N] fp16 = fp16((xq @ wq^T * sx[m] + x16 @ w16^T) * sw[n]) (LLM.int8() product)."""
+    for t, n, d in ((xq, "xq", torch.int8), (wq, "wq", torch.int8), (sx, "sx", torch.float32),
+                    (sw, "sw", torch.float32), (x16, "x16", torch.float16), (w16, "w16", torch.float16)):
+        _cuda(t, n, (d,))
+    M, K = xq.shape
+    N = wq.shape[0]
+    cap = x16.shape[1]
+    if wq.shape[1] != K or sx.numel() != M or sw.numel() != N or tuple(x16.shape) != (M, cap) or \
+            tuple(w16.shape) != (N, cap):
+        raise ValueError("shape mismatch: xq [M,K], wq [N,K], sx [M], sw [N], x16 [M,cap], w16 [N,cap]")
+    y = out if out is not None else _empty((M, N), torch.float16, xq)
+    _cuda(y, "out", (torch.float16,), 2)
+    _check(lib.wq_gemm_w8a8_outliers(_ptr(xq), _ptr(sx), _ptr(wq), _ptr(sw), _ptr(x16), _ptr(w16), int(cap), M, N, K,
+                                     _ptr(y), _P(_stream(stream))), "wq_gemm_w8a8_outliers")
+    return y
+
+
+def llm_int8_matmul(x, wq, sw, threshold: float = 6.0, cap: int = 64, stream=None):
+    """The LLM.int8() sequence on fp16 x [M, K] and per-channel INT8 weights (wq [N, K], sw [N]):
+    outlier columns -> per-token INT8 of the rest -> gather -> GEMM.  Returns (y, count)."""
+    idx, count, keep = outlier_columns(x, threshold, cap, stream)
+    xq, sx = quantize_int8_per_channel(x, keep, stream)
+    x16, w16 = gather_outliers(x, wq, idx, count, cap, stream)
+    return gemm_w8a8_outliers(xq, sx, wq, sw, x16, w16, stream=stream), count
 
 
 def device_status(stream=None) -> int:

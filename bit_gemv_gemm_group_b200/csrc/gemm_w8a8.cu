@@ -1,5 +1,6 @@
-// W8A8 INT8 GEMM on the 5th-generation tensor cores (tcgen05, kind::i8) with
-// a fused per-token x per-channel dequantization epilogue.
+// W8A8 GEMMs on the 5th-generation tensor cores with a fused per-token x
+// per-channel dequantization epilogue: INT8 (tcgen05 kind::i8, int32
+// accumulators) and FP8 E4M3 (kind::f8f6f4, fp32 accumulators).
 //
 // Source: "Quantization: Smaller Weights, Same Answers (Mostly)", section
 // "How does quantized matrix multiplication actually run on the GPU?" (int8
@@ -10,6 +11,12 @@
 //
 //   acc[m][n] = sum_k xq[m][k] * wq[n][k]          (int32, exact)
 //   y[m][n]   = fp16_rn( (float)acc * sx[m] * sw[n] )
+//
+// FP8: "How quantization works", "Mainstream schemes at a glance" (FP8 W8A8:
+// FP8 weights and activations on FP8 tensor cores); "Quantization:
+// Smaller Weights, Same Answers (Mostly)", "What about FP8, MXFP4, NVFP4 and
+// GGUF?".  Same data flow with E4M3 codes; acc is the tensor cores' fp32 sum
+// and a scale vector may hold one per-tensor value (stride 0).
 //
 // Persistent, warp-specialized CTA (one per SM, 192 threads):
 //   warp 0      TMA producer: 128x128-byte tiles of xq and 256x128-byte
@@ -23,6 +30,16 @@
 //               MMAs of tile i+1.
 // Tiles are 128 (M) x 256 (N), visited M-fastest so CTAs running together
 // share the same weight tile.  No multicast of any kind.
+//
+// LLM.int8() variant ("Quantization" (engine-room ch. 15), "The Mathematics":
+// C ~= S_out (.) (X_q W_q) + X_16 W_16): the INT8 GEMM above, whose epilogue
+// warps also multiply the carved-out outlier columns in 16-bit.  Per 32 x 32
+// chunk of its accumulator a warp runs mma.sync m16n8k16 (fp16 x fp16 -> fp32)
+// over X_16 [M][cap] and W_16 [N][cap] (the INT8 weight codes of those columns
+// as fp16, exact), transposes the fragments to one row per lane through 4 KB
+// of shared memory, and stores y = fp16((acc * s_x + X_16 W_16^T) * s_w).  The
+// epilogue of tile i runs while the MMAs of tile i + 1 proceed, so for a few
+// dozen outlier columns the 16-bit product costs no extra time.
 #include "sm100.cuh"
 #include "wq_device.cuh"
 #include "wq_host.h"
@@ -41,8 +58,19 @@ constexpr uint32_t B_BYTES = BN * BK;        // 32 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr uint32_t TMEM_COLS = 512;          // two 256-column fp32/int32 accumulators
 constexpr int THREADS = 192;
-constexpr uint32_t IDESC = make_idesc(/*s32*/ 2, /*s8*/ 1, /*s8*/ 1, BM, BN);
+constexpr uint32_t IDESC_I8 = make_idesc(/*s32*/ 2, /*s8*/ 1, /*s8*/ 1, BM, BN);
+constexpr uint32_t IDESC_E4M3 = make_idesc(/*f32*/ 1, /*e4m3*/ 0, /*e4m3*/ 0, BM, BN);
 constexpr size_t SMEM_BYTES = 1024 /*alignment slack*/ + STAGES * STAGE_BYTES + 256 /*barriers etc.*/;
+constexpr int TR_PITCH = 33;                                     // fp32 words per row of a transpose buffer
+constexpr size_t TR_BYTES = 4 * 32 * TR_PITCH * sizeof(float);    // one 32 x 32 buffer per epilogue warp
+constexpr size_t SMEM_BYTES_OUTL = SMEM_BYTES + TR_BYTES;
+
+// The carved-out outlier columns of the LLM.int8() variant (cap == 0: none).
+struct Outliers {
+    const uint16_t *x16;  // fp16 [M][cap]
+    const uint16_t *w16;  // fp16 [N][cap]
+    int cap;              // multiple of 16
+};
 constexpr uint64_t DRAIN_NS = 2000000000ull;
 
 // Site codes recorded in the device status word when a wait runs out.
@@ -58,21 +86,34 @@ struct Smem {
     int abort;
 };
 
+// Accumulator bits to float: int32 (INT8) or fp32 (FP8).
+template <bool FP8>
+__device__ __forceinline__ float acc_value(uint32_t r) {
+    return FP8 ? __uint_as_float(r) : (float)(int32_t)r;
+}
+
+template <bool FP8>
 __device__ __forceinline__ void store_chunk(uint16_t *__restrict__ y, int32_t *__restrict__ acc_out, int m, int n0,
-                                            int N, float sxm, const float *__restrict__ sw, const uint32_t (&r)[32],
-                                            bool vec_ok) {
+                                            int N, float sxm, const float *__restrict__ sw, int sw_stride,
+                                            const uint32_t (&r)[32], bool vec_ok) {
     float swv[32];
     if (vec_ok && n0 + 32 <= N) {
+        if (sw_stride) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float4 v = __ldg(reinterpret_cast<const float4 *>(sw + n0) + j);
-            swv[4 * j] = v.x; swv[4 * j + 1] = v.y; swv[4 * j + 2] = v.z; swv[4 * j + 3] = v.w;
+            for (int j = 0; j < 8; ++j) {
+                const float4 v = __ldg(reinterpret_cast<const float4 *>(sw + n0) + j);
+                swv[4 * j] = v.x; swv[4 * j + 1] = v.y; swv[4 * j + 2] = v.z; swv[4 * j + 3] = v.w;
+            }
+        } else {
+            const float v = __ldg(sw);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) swv[j] = v;
         }
         uint32_t h[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-            const float a = __fmul_rn(__fmul_rn((float)(int32_t)r[2 * j], sxm), swv[2 * j]);
-            const float b = __fmul_rn(__fmul_rn((float)(int32_t)r[2 * j + 1], sxm), swv[2 * j + 1]);
+            const float a = __fmul_rn(__fmul_rn(acc_value<FP8>(r[2 * j]), sxm), swv[2 * j]);
+            const float b = __fmul_rn(__fmul_rn(acc_value<FP8>(r[2 * j + 1]), sxm), swv[2 * j + 1]);
             h[j] = (uint32_t)float_to_half_bits_rn(a) | ((uint32_t)float_to_half_bits_rn(b) << 16);
         }
         uint4 *yp = reinterpret_cast<uint4 *>(y + (size_t)m * N + n0);
@@ -88,7 +129,7 @@ __device__ __forceinline__ void store_chunk(uint16_t *__restrict__ y, int32_t *_
         for (int j = 0; j < 32; ++j) {
             const int n = n0 + j;
             if (n < N) {
-                const float v = __fmul_rn(__fmul_rn((float)(int32_t)r[j], sxm), __ldg(sw + n));
+                const float v = __fmul_rn(__fmul_rn(acc_value<FP8>(r[j]), sxm), __ldg(sw + n * sw_stride));
                 y[(size_t)m * N + n] = float_to_half_bits_rn(v);
                 if (acc_out) acc_out[(size_t)m * N + n] = (int32_t)r[j];
             }
@@ -96,10 +137,118 @@ __device__ __forceinline__ void store_chunk(uint16_t *__restrict__ y, int32_t *_
     }
 }
 
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t ldg_u32(const uint16_t *p) { return __ldg(reinterpret_cast<const uint32_t *>(p)); }
+
+// o[j] = sum_i X_16[r0 + lane][i] * W_16[n0 + j][i] for j < 32 (one row per lane), by the whole
+// warp: 2 x 4 tiles of m16n8k16 over cap / 16 k-steps, then a transpose through `tr`.  Rows and
+// columns past M and N read the last valid ones (their results are never stored).
+__device__ __forceinline__ void outlier_chunk(const Outliers &ol, int M, int N, int r0, int n0, int lane,
+                                              float *__restrict__ tr, float (&o)[32]) {
+    const int g = lane >> 2, t = lane & 3;
+    const uint16_t *xa[2][2], *wb[4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) xa[mt][h] = ol.x16 + (size_t)min(r0 + 16 * mt + 8 * h + g, M - 1) * ol.cap + 2 * t;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) wb[nt] = ol.w16 + (size_t)min(n0 + 8 * nt + g, N - 1) * ol.cap + 2 * t;
+    float cf[2][4][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) cf[mt][nt][0] = cf[mt][nt][1] = cf[mt][nt][2] = cf[mt][nt][3] = 0.0f;
+    for (int kk = 0; kk < ol.cap; kk += 16) {
+        uint32_t a[2][4], b[4][2];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            a[mt][0] = ldg_u32(xa[mt][0] + kk);
+            a[mt][1] = ldg_u32(xa[mt][1] + kk);
+            a[mt][2] = ldg_u32(xa[mt][0] + kk + 8);
+            a[mt][3] = ldg_u32(xa[mt][1] + kk + 8);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            b[nt][0] = ldg_u32(wb[nt] + kk);
+            b[nt][1] = ldg_u32(wb[nt] + kk + 8);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) mma_16816_f16(cf[mt][nt], a[mt], b[nt][0], b[nt][1]);
+    }
+    __syncwarp();  // the previous chunk's readers are done with tr
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            float *p = tr + (16 * mt + g) * TR_PITCH + 8 * nt + 2 * t;
+            p[0] = cf[mt][nt][0];
+            p[1] = cf[mt][nt][1];
+            p[8 * TR_PITCH] = cf[mt][nt][2];
+            p[8 * TR_PITCH + 1] = cf[mt][nt][3];
+        }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) o[j] = tr[lane * TR_PITCH + j];
+}
+
+// y = fp16((acc * s_x + o) * s_w) for one row's 32-column chunk (INT8 accumulators).
+__device__ __forceinline__ void store_chunk_outliers(uint16_t *__restrict__ y, int m, int n0, int N, float sxm,
+                                                     const float *__restrict__ sw, const uint32_t (&r)[32],
+                                                     const float (&o)[32], bool vec_ok) {
+    if (vec_ok && n0 + 32 <= N) {
+        uint32_t h[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 v = __ldg(reinterpret_cast<const float4 *>(sw + n0) + j);
+            const float sv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; e += 2) {
+                const int c = 4 * j + e;
+                const float a = __fmul_rn(__fmaf_rn((float)(int32_t)r[c], sxm, o[c]), sv[e]);
+                const float b = __fmul_rn(__fmaf_rn((float)(int32_t)r[c + 1], sxm, o[c + 1]), sv[e + 1]);
+                h[c / 2] = (uint32_t)float_to_half_bits_rn(a) | ((uint32_t)float_to_half_bits_rn(b) << 16);
+            }
+        }
+        uint4 *yp = reinterpret_cast<uint4 *>(y + (size_t)m * N + n0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) yp[j] = make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int n = n0 + j;
+            if (n < N)
+                y[(size_t)m * N + n] =
+                    float_to_half_bits_rn(__fmul_rn(__fmaf_rn((float)(int32_t)r[j], sxm, o[j]), __ldg(sw + n)));
+        }
+    }
+}
+
+// D (+)= A * B^T for one 128 x 256 x 32 step: kind::i8 (int32) or kind::f8f6f4 E4M3 (fp32).
+template <bool FP8>
+__device__ __forceinline__ void mma_step(uint32_t d, uint64_t a, uint64_t b, uint32_t acc) {
+    if (FP8)
+        mma_f8f6f4(d, a, b, IDESC_E4M3, acc);
+    else
+        mma_i8(d, a, b, IDESC_I8, acc);
+}
+
+// sx_stride / sw_stride: 1 for one scale per row, 0 for one scale for the whole operand.
+// OUTL (INT8 only): the epilogue adds the 16-bit product of the outlier columns `ol`.
+template <bool FP8, bool OUTL = false>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                     const float *__restrict__ sx, const float *__restrict__ sw, uint16_t *__restrict__ y,
-                     int32_t *__restrict__ acc_out, int M, int N, int K, unsigned int *status, uint64_t limit_ns) {
+                     const float *__restrict__ sx, int sx_stride, const float *__restrict__ sw, int sw_stride,
+                     uint16_t *__restrict__ y, int32_t *__restrict__ acc_out, int M, int N, int K, Outliers ol,
+                     unsigned int *status, uint64_t limit_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
@@ -183,8 +332,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     const uint32_t a_addr = smem_u32(sA + s * A_BYTES), b_addr = smem_u32(sB + s * B_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk)
-                        mma_i8(d, umma_desc_sw128_kmajor(a_addr + kk * 32), umma_desc_sw128_kmajor(b_addr + kk * 32),
-                               IDESC, (kb | kk) != 0);
+                        mma_step<FP8>(d, umma_desc_sw128_kmajor(a_addr + kk * 32),
+                                      umma_desc_sw128_kmajor(b_addr + kk * 32), (kb | kk) != 0);
                     tc_commit(smem_u32(&sm->empty[s]));
                 }
                 if (ok) tc_commit(smem_u32(&sm->tmem_full[a]));
@@ -208,13 +357,23 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const int m = (tile % mt) * BM + row;
             const int nb = (tile / mt) * BN;
-            const float sxm = m < M ? __ldg(sx + m) : 0.0f;
+            const float sxm = m < M ? __ldg(sx + m * sx_stride) : 0.0f;
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + a * BN + c * 32, r);
                 tmem_ld_wait();
-                if (m < M && nb + c * 32 < N) store_chunk(y, acc_out, m, nb + c * 32, N, sxm, sw, r, vec_ok);
+                if (OUTL) {
+                    if (nb + c * 32 < N) {  // warp-uniform: the whole warp runs the outlier MMAs
+                        float o[32];
+                        float *tr = reinterpret_cast<float *>(base + STAGES * STAGE_BYTES + 256) +
+                                    (warp - 2) * 32 * TR_PITCH;
+                        outlier_chunk(ol, M, N, m - row + q * 32, nb + c * 32, lane, tr, o);
+                        if (m < M) store_chunk_outliers(y, m, nb + c * 32, N, sxm, sw, r, o, vec_ok);
+                    }
+                } else if (m < M && nb + c * 32 < N) {
+                    store_chunk<FP8>(y, acc_out, m, nb + c * 32, N, sxm, sw, sw_stride, r, vec_ok);
+                }
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&sm->tmem_empty[a]));
@@ -225,6 +384,39 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         tmem_dealloc(tmem_base, TMEM_COLS);
     }
+}
+
+}  // namespace
+}  // namespace wq
+
+namespace wq {
+namespace {
+
+// Shared launch path of the INT8, FP8 and LLM.int8() GEMMs (arguments already validated).
+template <bool FP8, bool OUTL = false>
+wq_status launch_gemm(const void *xq, const float *sx, int sx_stride, const void *wq_, const float *sw, int sw_stride,
+                      int M, int N, int K, uint16_t *y, void *acc_out, void *stream, const char *who,
+                      Outliers ol = Outliers{nullptr, nullptr, 0}) {
+    unsigned int *status = device_status_word();
+    if (!status) return WQ_ERR_CUDA;
+    CUtensorMap tx, tw;
+    if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return WQ_ERR_CUDA;
+    if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq_, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BN,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return WQ_ERR_CUDA;
+    constexpr size_t smem = OUTL ? SMEM_BYTES_OUTL : SMEM_BYTES;
+    cudaError_t e = cudaFuncSetAttribute(gemm_w8a8_kernel<FP8, OUTL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "%s: cudaFuncSetAttribute failed: %s", who, cudaGetErrorString(e));
+    const long long tiles = (long long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    WQ_REQUIRE(tiles < (1ll << 31), WQ_ERR_UNSUPPORTED, "%s: problem too large", who);
+    const int grid = (int)std::min<long long>(tiles, num_sms());
+    gemm_w8a8_kernel<FP8, OUTL><<<grid, THREADS, smem, as_stream(stream)>>>(
+        tx, tw, sx, sx_stride, sw, sw_stride, y, reinterpret_cast<int32_t *>(acc_out), M, N, K, ol, status,
+        wait_limit());
+    return check_launch(who);
 }
 
 }  // namespace
@@ -244,23 +436,43 @@ extern "C" wq_status wq_gemm_w8a8(const int8_t *xq, const float *sx, const int8_
     WQ_REQUIRE(K % 16 == 0, WQ_ERR_UNSUPPORTED, "wq_gemm_w8a8: K (%d) must be a multiple of 16", K);
     // |acc| <= 128 * 128 * K must stay below 2^31 for any int8 codes: K <= 131071, and K % 16 == 0
     WQ_REQUIRE(K <= 131056, WQ_ERR_UNSUPPORTED, "wq_gemm_w8a8: K (%d) above 131056 could overflow int32", K);
-    unsigned int *status = device_status_word();
-    if (!status) return WQ_ERR_CUDA;
-    CUtensorMap tx, tw;
-    if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, xq, (uint64_t)K, (uint64_t)M, (uint64_t)K, BK, BM,
-                        CU_TENSOR_MAP_SWIZZLE_128B))
-        return WQ_ERR_CUDA;
-    if (!encode_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, wq_, (uint64_t)K, (uint64_t)N, (uint64_t)K, BK, BN,
-                        CU_TENSOR_MAP_SWIZZLE_128B))
-        return WQ_ERR_CUDA;
-    cudaError_t e = cudaFuncSetAttribute(gemm_w8a8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
-    if (e != cudaSuccess)
-        return fail(WQ_ERR_CUDA, "wq_gemm_w8a8: cudaFuncSetAttribute failed: %s", cudaGetErrorString(e));
-    const long long tiles = (long long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    WQ_REQUIRE(tiles < (1ll << 31), WQ_ERR_UNSUPPORTED, "wq_gemm_w8a8: problem too large");
-    const int grid = (int)std::min<long long>(tiles, num_sms());
-    gemm_w8a8_kernel<<<grid, THREADS, SMEM_BYTES, as_stream(stream)>>>(tx, tw, sx, sw, y, acc_out, M, N, K, status,
-                                                                        wait_limit());
-    return check_launch("wq_gemm_w8a8");
+    return launch_gemm<false>(xq, sx, 1, wq_, sw, 1, M, N, K, y, acc_out, stream, "wq_gemm_w8a8");
+}
+
+extern "C" wq_status wq_gemm_fp8(const uint8_t *xq, const float *sx, int sx_per_row, const uint8_t *wq_,
+                                 const float *sw, int sw_per_row, int M, int N, int K, uint16_t *y, float *acc_out,
+                                 void *stream) {
+    using namespace wq;
+    WQ_REQUIRE_PTR(xq, "xq");
+    WQ_REQUIRE_PTR(sx, "sx");
+    WQ_REQUIRE_PTR(wq_, "wq");
+    WQ_REQUIRE_PTR(sw, "sw");
+    WQ_REQUIRE_PTR(y, "y");
+    if (acc_out) WQ_REQUIRE(aligned16(acc_out), WQ_ERR_ALIGNMENT, "acc_out is not 16-byte aligned");
+    WQ_REQUIRE(M > 0 && N > 0 && K > 0, WQ_ERR_INVALID_ARG, "wq_gemm_fp8: sizes must be positive (M=%d N=%d K=%d)", M,
+               N, K);
+    WQ_REQUIRE(K % 16 == 0, WQ_ERR_UNSUPPORTED, "wq_gemm_fp8: K (%d) must be a multiple of 16", K);
+    return launch_gemm<true>(xq, sx, sx_per_row ? 1 : 0, wq_, sw, sw_per_row ? 1 : 0, M, N, K, y, acc_out, stream,
+                             "wq_gemm_fp8");
+}
+
+extern "C" wq_status wq_gemm_w8a8_outliers(const int8_t *xq, const float *sx, const int8_t *wq_, const float *sw,
+                                           const uint16_t *x16, const uint16_t *w16, int cap, int M, int N, int K,
+                                           uint16_t *y, void *stream) {
+    using namespace wq;
+    WQ_REQUIRE_PTR(xq, "xq");
+    WQ_REQUIRE_PTR(sx, "sx");
+    WQ_REQUIRE_PTR(wq_, "wq");
+    WQ_REQUIRE_PTR(sw, "sw");
+    WQ_REQUIRE_PTR(x16, "x16");
+    WQ_REQUIRE_PTR(w16, "w16");
+    WQ_REQUIRE_PTR(y, "y");
+    WQ_REQUIRE(M > 0 && N > 0 && K > 0, WQ_ERR_INVALID_ARG,
+               "wq_gemm_w8a8_outliers: sizes must be positive (M=%d N=%d K=%d)", M, N, K);
+    WQ_REQUIRE(K % 16 == 0, WQ_ERR_UNSUPPORTED, "wq_gemm_w8a8_outliers: K (%d) must be a multiple of 16", K);
+    WQ_REQUIRE(K <= 131056, WQ_ERR_UNSUPPORTED, "wq_gemm_w8a8_outliers: K (%d) above 131056 could overflow int32", K);
+    WQ_REQUIRE(cap >= 16 && cap <= 256 && cap % 16 == 0, WQ_ERR_UNSUPPORTED,
+               "wq_gemm_w8a8_outliers: cap (%d) must be a multiple of 16 in [16, 256]", cap);
+    return launch_gemm<false, true>(xq, sx, 1, wq_, sw, 1, M, N, K, y, nullptr, stream, "wq_gemm_w8a8_outliers",
+                                    Outliers{x16, w16, cap});
 }

@@ -1,12 +1,17 @@
 // Symmetric INT8 row quantizers: per output channel (weights, optional
-// SmoothQuant W * s) and per token (activations, optional X / s).
+// SmoothQuant W * s) and per token (activations, optional X / s); and the FP8
+// E4M3 quantizer per row or per tensor, which shares their row machinery.
 //
 // Source: "How quantization works", sections "The math of quantization"
 // (s = max|x| / (2^(b-1) - 1), q = clamp(round(x/s), -2^(b-1), 2^(b-1)-1)),
 // the quant.py listing (absmax clamped at 1e-8), q8_per_row and SmoothQuant's
 // "Xs, Ws = X / s, W * s" in "Activation quantization and outliers";
 // "Quantization: Smaller Weights, Same Answers (Mostly)", Quick Reference
-// (per-token dynamic activation scales).
+// (per-token dynamic activation scales).  FP8: "How quantization works",
+// quant.py fake_quant_fp8 (scale = max|w| / 448, then the cast to E4M3);
+// "Quantization from Scratch", Formats, and "Quantization: Smaller Weights,
+// Same Answers (Mostly)", "What about FP8, MXFP4, NVFP4 and GGUF?" (E4M3
+// reaches +-448).
 //
 // One CTA of 256 threads per row.  Each thread owns 16-byte chunks of 8 fp16
 // values; for K <= 16384 the (smoothed) row stays in registers between the
@@ -17,6 +22,8 @@
 #include "sm100.cuh"
 #include "wq_device.cuh"
 #include "wq_host.h"
+
+#include <algorithm>
 
 namespace wq {
 namespace {
@@ -87,6 +94,52 @@ __device__ __forceinline__ uint2 quant8(const float (&v)[8], float s, float rs) 
     return make_uint2(__byte_perm(p0, p1, 0x6420), __byte_perm(p2, p3, 0x6420));
 }
 
+enum Format { kInt8 = 0, kE4M3 = 1 };
+
+// Two fp32 values to E4M3 (round to nearest even, saturating at +-448); `lo` lands in the low byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// E4M3 codes of v / s for one chunk: e4m3_rn(fl(v / s)).  t = RN(v * RN(1/s)) is within
+// 1.5 * 2^-23 |t| of v / s and fl(v / s) within 2^-24 of v / s, so fl(v / s) lies in
+// [t (1 - 2^-21), t (1 + 2^-21)], which the two products t (1 -+ 2^-20) enclose even after
+// their own rounding.  Rounding to E4M3 is monotone: when both ends give the same code, so
+// does fl(v / s).  Otherwise (v / s next to an E4M3 midpoint, rare) the chunk is redone from
+// the IEEE quotient.  Saturation never applies: |v / s| <= 448 (1 + 2^-22) rounds to 448.
+__device__ __forceinline__ uint2 quant8_e4m3(const float (&v)[8], float s, float rs) {
+    constexpr float kDown = 1.0f - 0x1p-20f, kUp = 1.0f + 0x1p-20f;
+    uint32_t c[4], bad = 0;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const float2 t = __fmul2_rn(make_float2(v[2 * p], v[2 * p + 1]), make_float2(rs, rs));
+        const float2 a = __fmul2_rn(t, make_float2(kDown, kDown));
+        const float2 b = __fmul2_rn(t, make_float2(kUp, kUp));
+        c[p] = cvt_e4m3x2(a.x, a.y);
+        bad |= c[p] ^ cvt_e4m3x2(b.x, b.y);
+    }
+    if (bad) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) c[p] = cvt_e4m3x2(__fdiv_rn(v[2 * p], s), __fdiv_rn(v[2 * p + 1], s));
+    }
+    return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+template <int FMT>
+struct FormatTraits;
+template <>
+struct FormatTraits<kInt8> {
+    static constexpr float kMax = 127.0f;  // 2^(b-1) - 1
+    __device__ static uint2 chunk(const float (&v)[8], float s, float rs) { return quant8(v, s, rs); }
+};
+template <>
+struct FormatTraits<kE4M3> {
+    static constexpr float kMax = 448.0f;  // largest finite E4M3 value
+    __device__ static uint2 chunk(const float (&v)[8], float s, float rs) { return quant8_e4m3(v, s, rs); }
+};
+
 __device__ __forceinline__ float block_max(float a, float *red) {
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
@@ -100,11 +153,15 @@ __device__ __forceinline__ float block_max(float a, float *red) {
 }
 
 // NCH > 0: the row is kept in registers (K <= NCH * 2048).  NCH == 0: two passes.
-template <int NCH, int MODE>
+// tensor_amax (FP8 per tensor): the tensor's max |x| (float bits), used instead of the
+// row's; the scale is then written by finish_tensor_scale_kernel, not here.
+template <int NCH, int MODE, int FMT = kInt8>
 __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_t *__restrict__ x, int K,
                                                                    const float *__restrict__ smooth,
                                                                    int8_t *__restrict__ q,
-                                                                   float *__restrict__ scales) {
+                                                                   float *__restrict__ scales,
+                                                                   const unsigned int *__restrict__ tensor_amax = nullptr) {
+    using F = FormatTraits<FMT>;
     __shared__ float red[kThreads / 32];
     const size_t row = blockIdx.x;
     const uint16_t *xr = x + row * K;
@@ -123,15 +180,15 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
                 for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[c][e]));
             }
         }
-        const float a = fmaxf(block_max(amax, red), 1e-8f);
-        const float s = __fdiv_rn(a, 127.0f);
+        const float a = fmaxf(tensor_amax ? __uint_as_float(*tensor_amax) : block_max(amax, red), 1e-8f);
+        const float s = __fdiv_rn(a, F::kMax);
         const float rs = __frcp_rn(s);
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
             const int k = c * kRowStep + t0;
-            if (k < K) *reinterpret_cast<uint2 *>(qr + k) = quant8(v[c], s, rs);
+            if (k < K) *reinterpret_cast<uint2 *>(qr + k) = F::chunk(v[c], s, rs);
         }
-        if (threadIdx.x == 0) scales[row] = s;
+        if (threadIdx.x == 0 && !tensor_amax) scales[row] = s;
     } else {
         // Two passes over the row: the first pass keeps its lines in L2 (evict-last policy)
         // so that the second pass, the lines' last use (evict-first), hits L2.  Without the
@@ -154,8 +211,8 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
 #pragma unroll
             for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
         }
-        const float a = fmaxf(block_max(amax, red), 1e-8f);
-        const float s = __fdiv_rn(a, 127.0f);
+        const float a = fmaxf(tensor_amax ? __uint_as_float(*tensor_amax) : block_max(amax, red), 1e-8f);
+        const float s = __fdiv_rn(a, F::kMax);
         const float rs = __frcp_rn(s);
         for (int k = t0; k < K; k += kRowStep) {
             float v[8];
@@ -167,9 +224,9 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
             v[0] = a0.x; v[1] = a0.y; v[2] = a1.x; v[3] = a1.y;
             v[4] = a2.x; v[5] = a2.y; v[6] = a3.x; v[7] = a3.y;
             smooth8<MODE>(v, smooth, k);
-            *reinterpret_cast<uint2 *>(qr + k) = quant8(v, s, rs);
+            *reinterpret_cast<uint2 *>(qr + k) = F::chunk(v, s, rs);
         }
-        if (threadIdx.x == 0) scales[row] = s;
+        if (threadIdx.x == 0 && !tensor_amax) scales[row] = s;
     }
 }
 
@@ -178,7 +235,7 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
 // with at most 4 chunks per thread (few registers, four CTAs per SM); the
 // partial maxima are exchanged through distributed shared memory, so HBM still
 // sees each element once.
-template <int C, int MODE>
+template <int C, int MODE, int FMT = kInt8>
 __global__ void __launch_bounds__(kThreads) quant_int8_rows_cluster_kernel(const uint16_t *__restrict__ x, int K,
                                                                            const float *__restrict__ smooth,
                                                                            int8_t *__restrict__ q,
@@ -216,17 +273,17 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_cluster_kernel(const
 #pragma unroll
     for (int c = 1; c < C; ++c) a = fmaxf(a, part_max[c]);
     a = fmaxf(a, 1e-8f);
-    const float s = __fdiv_rn(a, 127.0f);
+    const float s = __fdiv_rn(a, FormatTraits<FMT>::kMax);
     const float rs = __frcp_rn(s);
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
         const int k = c * kRowStep + t0;
-        if (k < part) *reinterpret_cast<uint2 *>(qr + k) = quant8(v[c], s, rs);
+        if (k < part) *reinterpret_cast<uint2 *>(qr + k) = FormatTraits<FMT>::chunk(v[c], s, rs);
     }
     if (threadIdx.x == 0 && rank == 0) scales[row] = s;
 }
 
-template <int C, int MODE>
+template <int C, int MODE, int FMT = kInt8>
 cudaError_t launch_cluster(const uint16_t *x, int R, int K, const float *smooth, int8_t *q, float *scales,
                            cudaStream_t st) {
     cudaLaunchConfig_t cfg = {};
@@ -240,29 +297,50 @@ cudaError_t launch_cluster(const uint16_t *x, int R, int K, const float *smooth,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, quant_int8_rows_cluster_kernel<C, MODE>, x, K, smooth, q, scales);
+    return cudaLaunchKernelEx(&cfg, quant_int8_rows_cluster_kernel<C, MODE, FMT>, x, K, smooth, q, scales);
 }
 
-template <int MODE>
+template <int MODE, int FMT = kInt8>
 cudaError_t launch_mode(const uint16_t *x, int R, int K, const float *smooth, int8_t *q, float *scales,
-                        cudaStream_t st) {
+                        cudaStream_t st, const unsigned int *tensor_amax = nullptr) {
     const int nch = (K + kRowStep - 1) / kRowStep;
     // Measured on B200: pairs beat the 8-chunk single CTA; for longer rows the
     // two-pass kernel (second read from L2) beats clusters of 4 or 8.
-    if (nch > 4 && nch <= 8 && R < 65536 && K % 16 == 0)
-        return launch_cluster<2, MODE>(x, R, K, smooth, q, scales, st);
+    if (!tensor_amax && nch > 4 && nch <= 8 && R < 65536 && K % 16 == 0)
+        return launch_cluster<2, MODE, FMT>(x, R, K, smooth, q, scales, st);
     dim3 grid(R), block(kThreads);
     if (nch <= 1)
-        quant_int8_rows_kernel<1, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+        quant_int8_rows_kernel<1, MODE, FMT><<<grid, block, 0, st>>>(x, K, smooth, q, scales, tensor_amax);
     else if (nch <= 2)
-        quant_int8_rows_kernel<2, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+        quant_int8_rows_kernel<2, MODE, FMT><<<grid, block, 0, st>>>(x, K, smooth, q, scales, tensor_amax);
     else if (nch <= 4)
-        quant_int8_rows_kernel<4, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+        quant_int8_rows_kernel<4, MODE, FMT><<<grid, block, 0, st>>>(x, K, smooth, q, scales, tensor_amax);
     else if (nch <= 8)
-        quant_int8_rows_kernel<8, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+        quant_int8_rows_kernel<8, MODE, FMT><<<grid, block, 0, st>>>(x, K, smooth, q, scales, tensor_amax);
     else
-        quant_int8_rows_kernel<0, MODE><<<grid, block, 0, st>>>(x, K, smooth, q, scales);
+        quant_int8_rows_kernel<0, MODE, FMT><<<grid, block, 0, st>>>(x, K, smooth, q, scales, tensor_amax);
     return cudaGetLastError();
+}
+
+// Per-tensor FP8: the tensor's max |x| by atomicMax on the float bits (non-negative floats
+// order like their bit patterns) into the scale slot, which the call clears first.
+__global__ void __launch_bounds__(kThreads) tensor_absmax_kernel(const uint16_t *__restrict__ x, size_t n8,
+                                                                 unsigned int *__restrict__ amax) {
+    __shared__ float red[kThreads / 32];
+    float m = 0.0f;
+    for (size_t i = (size_t)blockIdx.x * kThreads + threadIdx.x; i < n8; i += (size_t)gridDim.x * kThreads) {
+        float v[8];
+        load8(x + 8 * i, v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(v[e]));
+    }
+    m = block_max(m, red);
+    if (threadIdx.x == 0) atomicMax(amax, __float_as_uint(m));
+}
+
+// Turns the tensor's max |x| into its scale once every row has been quantized with it.
+__global__ void finish_tensor_scale_kernel(float *scale) {
+    *scale = __fdiv_rn(fmaxf(*scale, 1e-8f), 448.0f);
 }
 
 wq_status quantize_rows(const char *name, const uint16_t *x, int R, int K, const float *smooth, int mode,
@@ -297,4 +375,39 @@ extern "C" wq_status wq_quantize_int8_per_channel(const uint16_t *w, int N, int 
 extern "C" wq_status wq_quantize_int8_per_token(const uint16_t *x, int M, int K, const float *smooth,
                                                 int8_t *q, float *scales, void *stream) {
     return wq::quantize_rows("wq_quantize_int8_per_token", x, M, K, smooth, wq::kDiv, q, scales, stream);
+}
+
+extern "C" wq_status wq_quantize_fp8_e4m3(const uint16_t *x, int R, int K, int per_row, uint8_t *q, float *scales,
+                                          void *stream) {
+    using namespace wq;
+    WQ_REQUIRE_PTR(x, "input");
+    WQ_REQUIRE_PTR(q, "q");
+    WQ_REQUIRE_PTR(scales, "scales");
+    WQ_REQUIRE(R > 0 && K > 0, WQ_ERR_INVALID_ARG, "wq_quantize_fp8_e4m3: sizes must be positive (rows=%d K=%d)",
+               R, K);
+    WQ_REQUIRE(K % 16 == 0, WQ_ERR_UNSUPPORTED, "wq_quantize_fp8_e4m3: K (%d) must be a multiple of 16", K);
+    WQ_REQUIRE(R < (1 << 30), WQ_ERR_UNSUPPORTED, "wq_quantize_fp8_e4m3: too many rows");
+    cudaStream_t st = as_stream(stream);
+    int8_t *q8 = reinterpret_cast<int8_t *>(q);
+    cudaError_t e;
+    if (per_row) {
+        e = launch_mode<kPlain, kE4M3>(x, R, K, nullptr, q8, scales, st);
+    } else {
+        unsigned int *amax = reinterpret_cast<unsigned int *>(scales);
+        e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), st);
+        if (e == cudaSuccess) {
+            const size_t n8 = (size_t)R * K / 8;
+            const size_t want = (n8 + kThreads - 1) / kThreads;
+            const int grid = (int)std::min<size_t>(want, (size_t)num_sms() * 8);
+            tensor_absmax_kernel<<<grid, kThreads, 0, st>>>(x, n8, amax);
+            e = cudaGetLastError();
+        }
+        if (e == cudaSuccess) e = launch_mode<kPlain, kE4M3>(x, R, K, nullptr, q8, scales, st, amax);
+        if (e == cudaSuccess) {
+            finish_tensor_scale_kernel<<<1, 1, 0, st>>>(scales);
+            e = cudaGetLastError();
+        }
+    }
+    if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_quantize_fp8_e4m3: launch failed: %s", cudaGetErrorString(e));
+    return WQ_OK;
 }

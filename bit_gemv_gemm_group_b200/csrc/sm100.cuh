@@ -145,6 +145,68 @@ __device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_
         : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (FP8/FP6/FP4 -> fp32; the formats are in idesc).
+__device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Block-scaled FP4 MMAs: D[tmem] (+)= (A . SFA) * (B . SFB)^T with E2M1 operands in shared memory
+// (two per byte) and per-block scale factors in tensor memory (sfa/sfb are TMEM addresses; the
+// byte of the 32-bit column that holds this MMA's factors is selected in idesc).
+// MXFP4: blocks of 32, E8M0 scales.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+}
+
+// NVFP4: blocks of 16, E4M3 scales.
+__device__ __forceinline__ void mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t sfa, uint32_t sfb, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa), "r"(sfb), "r"(accumulate)
+        : "memory");
+}
+
+// Copies 32 rows x 16 bytes of shared memory (described by sdesc) into tensor memory: row r lands in
+// lane r of each of the four 32-lane subpartitions, as 4 consecutive 32-bit columns from taddr.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of a 32-row x 16-byte source for tmem_cp_32x128b_warpx4: no swizzle,
+// K-major core matrices of 8 rows x 16 bytes stored 128 bytes apart (SBO), 512 bytes in all.
+__device__ __forceinline__ uint64_t utccp_desc_32x16(uint32_t smem_addr) {
+    const uint64_t start = (smem_addr >> 4) & 0x3FFFu;
+    const uint64_t lbo = 128 >> 4;
+    const uint64_t sbo = 128 >> 4;
+    return start | (lbo << 16) | (sbo << 32) | (1ull << 46) /* descriptor version */ | (0ull << 61) /* no swizzle */;
+}
+
+// Instruction descriptor of the block-scaled kinds (K-major E2M1 A and B, fp32 D):
+//   bits 7-9 / 10-12 A / B format (E2M1 = 1), 17-22 N >> 3, 23 scale format (0 = E4M3, 1 = E8M0),
+//   24-28 M >> 4; the scale-factor byte of B goes in bits 4-5 and that of A in bits 29-30.
+__host__ __device__ constexpr uint32_t make_idesc_fp4(uint32_t scale_e8m0, int M, int N) {
+    return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | (scale_e8m0 << 23) | ((uint32_t)(M >> 4) << 24);
+}
+
+__host__ __device__ constexpr uint32_t idesc_sf_bytes(uint32_t idesc, uint32_t a_byte, uint32_t b_byte) {
+    return idesc | (b_byte << 4) | (a_byte << 29);
+}
+
 // D[tmem] (+)= A[smem] * B[smem]^T, kind::f16 (fp16/bf16 -> fp32).
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                         uint32_t accumulate) {
@@ -233,7 +295,8 @@ __device__ __forceinline__ uint64_t umma_desc_sw128_kmajor(uint32_t smem_addr) {
 }
 
 // Instruction descriptor (dense, K-major A and B).
-//   c_format: 1 = f32, 2 = s32;  ab_format: kind::i8 1 = s8;  kind::f16 0 = f16.
+//   c_format: 1 = f32, 2 = s32;  ab_format: kind::i8 1 = s8;  kind::f16 0 = f16, 1 = bf16;
+//   kind::f8f6f4 0 = E4M3, 1 = E5M2.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t c_format, uint32_t a_format, uint32_t b_format, int M,
                                                   int N) {
     return (c_format << 4) | (a_format << 7) | (b_format << 10) | ((uint32_t)(N >> 3) << 17) |

@@ -224,6 +224,86 @@ wq_status wq_gemm_w8a8(const int8_t *xq, const float *sx, const int8_t *wq, cons
 wq_status wq_gemv_w8a16(const uint16_t *x, int B, const int8_t *wq, const float *sw, int N, int K,
                         uint16_t *y, void *stream);
 
+/*
+ * FP8 E4M3 quantization, per row or per tensor.  Source: [P1] quant.py
+ * fake_quant_fp8 (scale = max|w| / 448, then the cast to E4M3) and
+ * "Mainstream schemes at a glance" (FP8 W8A8, dynamic or static scales);
+ * [P3] "Formats" and [P4] "What about FP8, MXFP4, NVFP4 and GGUF?" (E4M3:
+ * 4 exponent bits, 3 mantissa bits, up to +-448).  E4M3 here is the variant
+ * without infinities (exponent bias 7; 0x7F/0xFF are NaN).
+ *   a = max(max |x| over the row (per_row) or the tensor, 1e-8)
+ *   s = a / 448                                    (fp32 IEEE division)
+ *   q = e4m3_rn(x / s)       (fp32 IEEE division, then round to nearest even)
+ * x: fp16 [R][K];  q: out E4M3 codes [R][K];  scales: out fp32, [R] when
+ * per_row != 0 (per output channel for weights, per token for activations),
+ * else [1] (one scale for the whole tensor; the call uses it as its
+ * reduction word first).  K % 16 == 0.  Inputs must be finite.
+ */
+wq_status wq_quantize_fp8_e4m3(const uint16_t *x, int R, int K, int per_row, uint8_t *q, float *scales,
+                               void *stream);
+
+/*
+ * FP8 E4M3 W8A8 GEMM on the tensor cores (tcgen05 kind::f8f6f4, fp32
+ * accumulation) with the fused dequantization epilogue.  Source: [P1]
+ * "Mainstream schemes at a glance" (FP8 weights and activations on FP8
+ * tensor cores), [P4] FP8 section.
+ *   acc[m][n] = sum_k e4m3(xq[m][k]) * e4m3(wq[n][k])    (fp32, order unspecified)
+ *   y[m][n]   = fp16_rn( acc * sx[m or 0] * sw[n or 0] )   (fp32 products)
+ * xq: E4M3 [M][K], wq: E4M3 [N][K];  sx: fp32 [M] if sx_per_row else [1];
+ * sw: fp32 [N] if sw_per_row else [1];  y: out fp16 [M][N];  acc_out:
+ * nullable, out fp32 [M][N] (raw accumulators).  K % 16 == 0.
+ */
+wq_status wq_gemm_fp8(const uint8_t *xq, const float *sx, int sx_per_row, const uint8_t *wq, const float *sw,
+                      int sw_per_row, int M, int N, int K, uint16_t *y, float *acc_out, void *stream);
+
+/*
+ * LLM.int8() mixed-precision decomposition.  Source: [P2] "The Breakthrough"
+ * and "The Mathematics" (C ~= S_out (.) (X_q W_q) + X_16 W_16: INT8 with a
+ * scale per row of X and per column of the product, the outlier feature
+ * dimensions removed from the integer path and multiplied in 16-bit); [P4]
+ * "How do LLM-specific quantization schemes protect against outliers?".
+ * The weights are stored once, as per-output-channel INT8 (codes wq, scales
+ * sw from wq_quantize_int8_per_channel without smoothing), and the 16-bit
+ * outlier slice of W is their dequantized columns.  The sequence is:
+ *   wq_outlier_columns  -> idx, count, keep
+ *   wq_quantize_int8_per_channel(x, keep)  -> X_q, s_x  (the carved columns
+ *       of x multiplied by 0: per-token INT8 over the other columns)
+ *   wq_gather_outliers  -> X_16, W_16
+ *   wq_gemm_w8a8_outliers -> y
+ *
+ * wq_outlier_columns: an outlier column is a column j of x [M][K] (fp16) with
+ * max_m |x[m][j]| >= threshold.  idx (int32 [cap]) receives the first
+ * min(total, cap) of them in increasing order (the ones carved out), *count
+ * (int32, device) the total that qualify, keep (fp32 [K]) 0 for the carved
+ * columns and 1 elsewhere (keep also serves as the call's reduction buffer).
+ * K % 8 == 0; 1 <= cap <= K; threshold > 0.
+ */
+wq_status wq_outlier_columns(const uint16_t *x, int M, int K, float threshold, int cap, int32_t *idx,
+                             int32_t *count, float *keep, void *stream);
+
+/*
+ * wq_gather_outliers: X_16 (fp16 [M][cap]) = x[:, idx[i]] and W_16 (fp16
+ * [N][cap]) = (fp16) wq[:, idx[i]] (exact: |code| <= 128) for i <
+ * min(*count, cap); zero for the other i.  idx/count as written by
+ * wq_outlier_columns.  cap % 16 == 0, 16 <= cap <= 256.
+ */
+wq_status wq_gather_outliers(const uint16_t *x, int M, int K, const int8_t *wq, int N, const int32_t *idx,
+                             const int32_t *count, int cap, uint16_t *x16, uint16_t *w16, void *stream);
+
+/*
+ * wq_gemm_w8a8_outliers: the INT8 tensor-core GEMM of wq_gemm_w8a8 whose
+ * epilogue adds the 16-bit product of the carved columns:
+ *   y[m][n] = fp16_rn( (acc[m][n] * sx[m] + sum_i x16[m][i] w16[n][i]) * sw[n] )
+ * acc as in wq_gemm_w8a8 (int32, exact), the 16-bit sum in fp32 (order
+ * unspecified).  xq: int8 [M][K] (carved columns zero), sx: fp32 [M],
+ * wq: int8 [N][K], sw: fp32 [N], x16: fp16 [M][cap], w16: fp16 [N][cap],
+ * y: out fp16 [M][N].  K % 16 == 0, K <= 131056; cap % 16 == 0,
+ * 16 <= cap <= 256.
+ */
+wq_status wq_gemm_w8a8_outliers(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
+                                const uint16_t *x16, const uint16_t *w16, int cap, int M, int N, int K, uint16_t *y,
+                                void *stream);
+
 /* Message describing the last error status returned on this host thread. */
 const char *wq_last_error(void);
 

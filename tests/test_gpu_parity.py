@@ -427,3 +427,179 @@ def test_w4a16_matmuls_repeat_bit_identically(wq, shape_index):
             torch.cuda.synchronize()
             assert torch.equal(first.view(torch.int16), again.view(torch.int16)), f"{N}x{K} B={B}"
     assert wq.device_status() == 0
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 W8A8: quantizer bit-exact, tensor-core GEMM within the tolerance
+# --------------------------------------------------------------------------
+FP8_Q_SMALL = [(1, 16), (7, 48), (33, 2048), (5, 2064), (64, 4096), (3, 16384), (2, 16400), (4, 40960), (300, 1024)]
+
+
+@pytest.mark.parametrize("R,K", FP8_Q_SMALL)
+@pytest.mark.parametrize("per_row", [True, False])
+def test_fp8_quantizer_bit_exact_small(wq, R, K, per_row):
+    g = np.random.default_rng(R * K + per_row)
+    a = (g.standard_normal((R, K)) * 2).astype(np.float32)
+    a[:, g.choice(K, size=max(1, K // 100), replace=False)] *= 40
+    if R > 2:
+        a[1] = 0.0                                        # an all-zero row: the 1e-8 clamp (per row)
+        a[2, : K // 2] *= 1e-6                            # E4M3 subnormals and values that round to 0
+    a = a.astype(np.float16)
+    q, s = wq.quantize_fp8_e4m3(dev(a), per_row=per_row)
+    torch.cuda.synchronize()
+    rq, rs = oracle.quantize_fp8_e4m3(a, per_row=per_row)
+    assert np.array_equal(host(s).view(np.uint32), rs.view(np.uint32))
+    assert np.array_equal(host(q), rq)
+
+
+def test_fp8_quantizer_every_e4m3_midpoint(wq):
+    # x / s placed next to every E4M3 rounding boundary (both sides and on it): the decisions
+    # that the fast path hands to the IEEE quotient
+    fin = np.array([oracle.e4m3_to_float(c) for c in range(0x7F)], np.float64)
+    mids = (fin[:-1] + fin[1:]) / 2
+    vals = np.concatenate([mids, mids * (1 + 2 ** -10), mids * (1 - 2 ** -10), fin])
+    K = 16 * ((vals.size + 15) // 16)
+    row = np.zeros(K, np.float64)
+    row[: vals.size] = vals
+    a = np.stack([row, -row]).astype(np.float16)          # scale 448 / 448: x / s is x
+    a[:, -1] = 448.0
+    q, s = wq.quantize_fp8_e4m3(dev(a), per_row=True)
+    torch.cuda.synchronize()
+    rq, rs = oracle.quantize_fp8_e4m3(a, per_row=True)
+    assert np.array_equal(host(s), rs) and np.array_equal(host(q), rq)
+
+
+def _fp8_gemm_check(wq, xq, sx, wq8, sw, ms=None, ns=None):
+    y = wq.gemm_fp8(dev(xq), dev(sx), dev(wq8), dev(sw))
+    torch.cuda.synchronize()
+    ry, rb = oracle.gemm_fp8_ref(xq, sx, wq8, sw, ms, ns)
+    hy = host(y).astype(np.float64)
+    if ms is not None:
+        hy = hy[np.ix_(ms, ns)]
+    assert_within_bound(hy, ry, rb, "fp8 gemm")
+
+
+def _random_e4m3(g, shape):
+    c = g.integers(0, 256, shape, dtype=np.uint8)
+    c[(c & 0x7F) == 0x7F] = 0x3A                          # no NaN codes
+    return c
+
+
+FP8_GEMM_SMALL = [(1, 1, 16), (128, 256, 128), (130, 300, 144), (64, 40, 1040), (257, 513, 256),
+                  (300, 1000, 2000), (512, 1024, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", FP8_GEMM_SMALL)
+def test_gemm_fp8_small(wq, M, N, K):
+    g = np.random.default_rng(M * N + K + 1)
+    xq, wq8 = _random_e4m3(g, (M, K)), _random_e4m3(g, (N, K))
+    sx = (g.random(M, dtype=np.float32) + 0.01) * 0.05
+    sw = (g.random(N, dtype=np.float32) + 0.01) * 0.01
+    _fp8_gemm_check(wq, xq, sx, wq8, sw)
+    _fp8_gemm_check(wq, xq, sx[:1], wq8, sw[:1])           # per-tensor scales
+
+
+def test_gemm_fp8_every_code_pair(wq):
+    # acc[m][n] = e4m3(m) * e4m3(n): every product of two finite E4M3 codes
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    xq = np.zeros((codes.size, 16), np.uint8)
+    xq[:, 0] = codes
+    wq8 = np.zeros((codes.size, 16), np.uint8)
+    wq8[:, 0] = codes
+    y, acc = wq.gemm_fp8(dev(xq), dev(np.ones(1, np.float32)), dev(wq8), dev(np.ones(1, np.float32)),
+                         return_acc=True)
+    torch.cuda.synchronize()
+    dec = np.array([oracle.e4m3_to_float(c) for c in codes], np.float64)
+    assert np.array_equal(host(acc).astype(np.float64), np.outer(dec, dec))
+
+
+def test_fp8_w8a8_pipeline_full_size(wq):
+    # The W8A8 layer in FP8: per-token activations, per-channel weights (and the per-tensor
+    # variant of the listing), tensor-core GEMM; sampled rows checked one by one.
+    M, N, K = 2048, 8192, 8192
+    X = workloads.config_activations("w8a8_smoothquant", M, K)
+    W = workloads.config_weight("w8a8_smoothquant")
+    ms = sample_rows(M, 64, seed=3)
+    ns = sample_rows(N, 96, seed=4)
+    for per_row in (True, False):
+        xq, sx = wq.quantize_fp8_e4m3(dev(X), per_row=per_row)
+        w8, sw = wq.quantize_fp8_e4m3(dev(W), per_row=per_row)
+        y = wq.gemm_fp8(xq, sx, w8, sw)
+        torch.cuda.synchronize()
+        hxq, hsx, hw8, hsw = host(xq), host(sx), host(w8), host(sw)
+        if per_row:
+            rxq, rsx = oracle.quantize_fp8_e4m3(X[ms], per_row=True)
+            rwq, rsw = oracle.quantize_fp8_e4m3(W[ns], per_row=True)
+            assert np.array_equal(hxq[ms], rxq) and np.array_equal(hsx[ms], rsx)
+            assert np.array_equal(hw8[ns], rwq) and np.array_equal(hsw[ns], rsw)
+        else:  # one scale over the whole tensor: the oracle quantizes all of it
+            rxq, rsx = oracle.quantize_fp8_e4m3(X, per_row=False)
+            rwq, rsw = oracle.quantize_fp8_e4m3(W, per_row=False)
+            assert np.array_equal(hsx, rsx) and np.array_equal(hsw, rsw)
+            assert np.array_equal(hxq, rxq) and np.array_equal(hw8, rwq)
+            del rxq, rwq
+        ry, rb = oracle.gemm_fp8_ref(hxq, hsx, hw8, hsw, ms, ns)
+        assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, f"fp8 per_row={per_row}")
+    assert wq.device_status() == 0
+
+
+# --------------------------------------------------------------------------
+# LLM.int8() decomposition: outlier columns and codes bit-exact, the fused
+# GEMM (INT8 tensor cores + 16-bit outlier product in the epilogue) within
+# the tolerance
+# --------------------------------------------------------------------------
+def _llm_inputs(M, N, K, planted, seed, scale=40.0):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((M, K)).astype(np.float32)
+    x[:, list(planted)] *= scale
+    x = x.astype(np.float16)
+    w = (g.standard_normal((N, K)) * 0.02).astype(np.float16)
+    wq8, sw = oracle.quantize_int8_per_channel(w)
+    return x, wq8, sw
+
+
+LLM_SMALL = [  # (M, N, K, planted columns, cap)
+    (1, 1, 16, (3,), 16), (128, 256, 128, (0, 127), 16), (130, 300, 144, (5, 6, 7, 100), 16),
+    (64, 40, 1040, tuple(range(0, 1040, 41)), 32), (257, 513, 256, (), 16), (300, 1000, 2000, (7, 1999), 64),
+    (200, 260, 512, tuple(range(3, 512, 9)), 48),  # 57 outlier columns, 48 carved: the rest stay INT8
+]
+
+
+@pytest.mark.parametrize("M,N,K,planted,cap", LLM_SMALL)
+def test_llm_int8_small(wq, M, N, K, planted, cap):
+    x, wq8, sw = _llm_inputs(M, N, K, planted, seed=M + N + K)
+    xd, wd, sd = dev(x), dev(wq8), dev(sw)
+    idx, count, keep = wq.outlier_columns(xd, 6.0, cap)
+    xq, sx = wq.quantize_int8_per_channel(xd, keep)
+    x16, w16 = wq.gather_outliers(xd, wd, idx, count, cap)
+    y = wq.gemm_w8a8_outliers(xq, sx, wd, sd, x16, w16)
+    torch.cuda.synchronize()
+    ridx, total = oracle.outlier_columns(x, 6.0, cap)
+    assert int(host(count)[0]) == total
+    assert np.array_equal(host(idx)[: ridx.size], ridx)
+    assert np.array_equal(host(keep) == 0, np.isin(np.arange(K), ridx))
+    ry, rb, rxq, rsx = oracle.llm_int8_ref(x, wq8, sw, ridx)
+    assert np.array_equal(host(xq), rxq) and np.array_equal(host(sx), rsx)
+    hx16, hw16 = host(x16), host(w16)
+    assert np.array_equal(hx16[:, : ridx.size], x[:, ridx]) and not hx16[:, ridx.size:].any()
+    assert np.array_equal(hw16[:, : ridx.size], wq8[:, ridx].astype(np.float16)) and not hw16[:, ridx.size:].any()
+    assert_within_bound(host(y).astype(np.float64), ry, rb, f"llm.int8 M={M} N={N} K={K}")
+    assert wq.device_status() == 0
+
+
+def test_llm_int8_full_size(wq):
+    # The W8A8 layer's activations (64 outlier channels x60) through the whole sequence at
+    # threshold 6: the 64 planted columns are carved out; sampled rows checked one by one.
+    M, N, K = 2048, 8192, 8192
+    X = workloads.config_activations("w8a8_smoothquant", M, K)
+    W = workloads.config_weight("w8a8_smoothquant")
+    wq8, sw = wq.quantize_int8_per_channel(dev(W))
+    y, count = wq.llm_int8_matmul(dev(X), wq8, sw, 6.0, 64)
+    torch.cuda.synchronize()
+    ridx, total = oracle.outlier_columns(X, 6.0, 64)
+    assert int(host(count)[0]) == total == 64
+    ms = sample_rows(M, 64, seed=5)
+    ns = sample_rows(N, 96, seed=6)
+    ry, rb, _, _ = oracle.llm_int8_ref(X, host(wq8), host(sw), ridx, ms=ms, ns=ns)
+    assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, "llm.int8 full size")
+    assert wq.device_status() == 0
