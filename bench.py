@@ -46,6 +46,9 @@ WORKLOAD = "llama70b_class_w4a16_layer+w8a8_smoothquant_2048x8192x8192"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 UP, DOWN = (28672, 8192), (8192, 28672)
 W8A8_SHAPE = (2048, 8192, 8192)
+LLM_THRESHOLD, LLM_CAP = 6.0, 64      # LLM.int8(): outlier threshold and carved-column capacity
+# nominal dense tensor throughput relative to bf16 (FP8/INT8 2x, FP4 4x)
+TENSOR_RATIO = {"gemm_w8a8": 2.0, "gemm_fp8": 2.0, "gemm_llm_int8": 2.0, "gemm_mxfp4": 4.0, "gemm_nvfp4": 4.0}
 
 
 # ----------------------------------------------------------------------------- peaks
@@ -76,6 +79,19 @@ def work_table():
         t[f"quant_int8_pc_{tag}"] = {"bytes": 3 * N * K + 4 * N, "ops": 0}
         t[f"gemv_w8a16_b1_{tag}"] = {"bytes": N * K + 4 * N + 2 * K + 2 * N, "ops": 2 * N * K}
     M, N, K = W8A8_SHAPE
+    # FP8 E4M3 W8A8 (per-token X, per-channel W), LLM.int8() and block-scaled FP4 on the same layer
+    t["quant_fp8_w"] = {"bytes": 3 * N * K + 4 * N, "ops": 0}
+    t["quant_fp8_x"] = {"bytes": 3 * M * K + 4 * M, "ops": 0}
+    t["gemm_fp8"] = {"bytes": M * K + N * K + 4 * (M + N) + 2 * M * N, "ops": 2 * M * N * K}
+    t["llm_outlier_columns"] = {"bytes": 2 * M * K + 4 * K, "ops": 0}
+    t["llm_quant_x"] = {"bytes": 3 * M * K + 4 * M + 4 * K, "ops": 0}
+    t["llm_gather"] = {"bytes": 4 * (M + N) * LLM_CAP + 4 * LLM_CAP, "ops": 0}
+    t["gemm_llm_int8"] = {"bytes": M * K + N * K + 4 * (M + N) + 2 * (M + N) * LLM_CAP + 2 * M * N,
+                          "ops": 2 * M * N * (K + LLM_CAP)}
+    for fmt, bs in (("mxfp4", 32), ("nvfp4", 16)):
+        t[f"quant_{fmt}_w"] = {"bytes": 2 * N * K + N * K // 2 + N * K // bs, "ops": 0}
+        t[f"quant_{fmt}_x"] = {"bytes": 2 * M * K + M * K // 2 + M * K // bs, "ops": 0}
+        t[f"gemm_{fmt}"] = {"bytes": (M + N) * (K // 2 + K // bs) + 2 * M * N, "ops": 2 * M * N * K}
     t["smooth"] = {"bytes": 2 * (M + N) * K + 4 * K, "ops": 0}
     t["quant_int8_pc_smooth"] = {"bytes": 3 * N * K + 4 * N + 4 * K, "ops": 0}
     t["quant_int8_pt_smooth"] = {"bytes": 3 * M * K + 4 * M + 4 * K, "ops": 0}
@@ -86,12 +102,12 @@ def work_table():
 def roofline_for(name, us, work, peaks):
     """Achieved rate against the kernel's binding roofline (measured peaks)."""
     hbm = peaks["hbm_gbs"]
-    int8 = 2.0 * peaks["bf16_tflops"]          # INT8 dense = 2 x bf16 (nominal ratio)
     f16 = peaks["bf16_tflops"]                 # fp16 dense = bf16
     b, ops = work["bytes"], work["ops"]
-    if name == "gemm_w8a8":
+    if name in TENSOR_RATIO:
+        peak = TENSOR_RATIO[name] * peaks["bf16_tflops"]
         ach = ops / (us * 1e-6) / 1e12
-        return {"bound": "tensor", "achieved": ach, "peak": int8, "unit": "TOPS", "frac": ach / int8}
+        return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TOPS", "frac": ach / peak}
     if name.startswith("gemm_w4a16"):
         t_mem, t_tc = b / (hbm * 1e9), ops / (f16 * 1e12)
         if t_tc > t_mem:
@@ -196,6 +212,7 @@ class Step:
         # read-side packed weights (previous "model state"), never written inside a step
         self.qB = {t: wq.quantize_group_int4(ins[f"w_{t}"], 128) for t in ("up", "down")}
         self.q8B = {t: wq.quantize_int8_per_channel(ins[f"w_{t}"]) for t in ("up", "down")}
+        self.w8_plain = wq.quantize_int8_per_channel(ins["w_w8a8"])  # LLM.int8() weights (no smoothing)
         torch.cuda.synchronize()
         self.ws = torch.empty(wq.smooth_workspace_bytes(W8A8_SHAPE[2]), dtype=torch.uint8, device=ins["x_w8a8"].device)
         self.out = {}
@@ -224,6 +241,50 @@ class Step:
             self.out["y5"] = wq.gemm_w8a8(xq, sx, w8, sw)
 
         L += [("smooth", smooth), ("quant_int8_pc_smooth", q_w), ("quant_int8_pt_smooth", q_x), ("gemm_w8a8", w8a8)]
+        X, W = ins["x_w8a8"], ins["w_w8a8"]
+        o = self.out
+
+        # FP8 E4M3 W8A8: W first, so that its 200 MB stream evicts X from L2 before X is read
+        def fp8_w():
+            o["fp8_w"] = wq.quantize_fp8_e4m3(W, per_row=True)
+
+        def fp8_x():
+            o["fp8_x"] = wq.quantize_fp8_e4m3(X, per_row=True)
+
+        def fp8_gemm():
+            o["y_fp8"] = wq.gemm_fp8(o["fp8_x"][0], o["fp8_x"][1], o["fp8_w"][0], o["fp8_w"][1])
+
+        # LLM.int8(): weights are the plain per-channel INT8 codes of W (model state, made once)
+        def llm_cols():
+            o["llm_cols"] = wq.outlier_columns(X, LLM_THRESHOLD, LLM_CAP)
+
+        def llm_qx():
+            o["llm_x"] = wq.quantize_int8_per_channel(X, o["llm_cols"][2])
+
+        def llm_gather():
+            idx, count, _ = o["llm_cols"]
+            o["llm_16"] = wq.gather_outliers(X, self.w8_plain[0], idx, count, LLM_CAP)
+
+        def llm_gemm():
+            xq, sx = o["llm_x"]
+            o["y_llm"] = wq.gemm_w8a8_outliers(xq, sx, self.w8_plain[0], self.w8_plain[1], *o["llm_16"])
+
+        L += [("quant_fp8_w", fp8_w), ("quant_fp8_x", fp8_x), ("gemm_fp8", fp8_gemm), ("llm_outlier_columns", llm_cols),
+              ("llm_quant_x", llm_qx), ("llm_gather", llm_gather), ("gemm_llm_int8", llm_gemm)]
+        for fmt in ("mxfp4", "nvfp4"):
+            qf = wq.quantize_mxfp4 if fmt == "mxfp4" else wq.quantize_nvfp4
+
+            def q_w(qf=qf, fmt=fmt):
+                o[f"{fmt}_w"] = qf(W)
+
+            def q_x(qf=qf, fmt=fmt):
+                o[f"{fmt}_x"] = qf(X)
+
+            def mm(fmt=fmt):
+                a, b = o[f"{fmt}_x"], o[f"{fmt}_w"]
+                o[f"y_{fmt}"] = wq.gemm_fp4(a[0], a[1], b[0], b[1], *((a[2], b[2]) if fmt == "nvfp4" else ()))
+
+            L += [(f"quant_{fmt}_w", q_w), (f"quant_{fmt}_x", q_x), (f"gemm_{fmt}", mm)]
         for t in ("up", "down"):
             L.append((f"quant_int8_pc_{t}", lambda t=t: wq.quantize_int8_per_channel(ins[f"w_{t}"])))
         for M in (16, 64):
@@ -277,6 +338,9 @@ def run_gpu(args):
     barrier()
     t_wall0 = time.time()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # A 50 ms spin (before the timed region) lets the host queue the step's launches ahead of the
+    # GPU, so the per-kernel events bracket device work rather than host launch gaps.
+    torch.cuda._sleep(int(0.05 * 1.9e9))
     start.record(stream)
     for k in range(args.steps):
         for (name, fn), (e0, e1) in zip(launches, evs[k]):
@@ -294,7 +358,7 @@ def run_gpu(args):
     for k in range(args.steps):
         for n, (e0, e1) in zip(names, evs[k]):
             per_kernel_us[n].append(e0.elapsed_time(e1) * 1e3)
-    mean_us = {n: sum(v) / len(v) for n, v in per_kernel_us.items()}
+    mean_us = {n: statistics.median(v) for n, v in per_kernel_us.items()}  # median device time per launch
 
     # max over ranks of the timed region and of each kernel's summed time
     red = reduce_max([total_ms] + [sum(per_kernel_us[n]) for n in names], world, dev)
@@ -399,21 +463,19 @@ def run_e2e(torch, wq, step, steps, stream):
     w = work_table()
     byts = w["gemv_w4a16_b1_up"]["bytes"] + w["gemv_w4a16_b1_down"]["bytes"]
     t_eager = timed(one, stream)
-    value, how = byts * steps / t_eager / 1e9, "eager"
-    graph = None
+    graph, graph_value = None, None
     try:
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
             one()
-        t_graph = timed(graph.replay, stream)
-        value, how = byts * steps / t_graph / 1e9, "cuda graph of the same calls"
-    except Exception as exc:  # capture unsupported: report the eager number
-        how = f"eager (graph capture failed: {type(exc).__name__})"
+        graph_value = round(byts * steps / timed(graph.replay, stream) / 1e9, 1)
+    except Exception:  # capture unsupported: only the call-by-call number
+        graph_value = None
     finally:
         del graph
-    return {"value": round(value, 1), "unit": "GB/s", "h2d_bytes_per_step": hx.numel() * 2,
-            "d2h_bytes_per_step": hy.numel() * 2, "eager_value": round(byts * steps / t_eager / 1e9, 1),
-            "launch": how,
+    return {"value": round(byts * steps / t_eager / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": hx.numel() * 2,
+            "d2h_bytes_per_step": hy.numel() * 2, "graph_value": graph_value,
+            "launch": "call by call from Python (value); the same calls replayed as one CUDA graph (graph_value)",
             "what": "batch-1 W4A16 GEMV on both weights via the Python/C API, x copied from pinned host memory "
                     "and y read back each step (one copy each way)"}
 
@@ -512,8 +574,16 @@ def run_profile_case(args):
     launches = dict(step.launches())
     if args.profile_case not in launches:
         raise SystemExit(f"unknown kernel {args.profile_case!r}; one of {sorted(launches)}")
-    for name in ("smooth", "quant_int8_pc_smooth", "quant_int8_pt_smooth"):  # producers of the W8A8 operands
-        if args.profile_case in ("quant_int8_pc_smooth", "quant_int8_pt_smooth", "gemm_w8a8") and name != args.profile_case:
+    # producers of a profiled kernel's operands run first (in step order), then the kernel itself
+    names = [n for n, _ in step.launches()]
+    producers = {"quant_int8_pc_smooth": ["smooth"], "quant_int8_pt_smooth": ["smooth"],
+                 "gemm_w8a8": ["smooth", "quant_int8_pc_smooth", "quant_int8_pt_smooth"],
+                 "gemm_fp8": ["quant_fp8_w", "quant_fp8_x"], "llm_quant_x": ["llm_outlier_columns"],
+                 "llm_gather": ["llm_outlier_columns"],
+                 "gemm_llm_int8": ["llm_outlier_columns", "llm_quant_x", "llm_gather"],
+                 "gemm_mxfp4": ["quant_mxfp4_w", "quant_mxfp4_x"], "gemm_nvfp4": ["quant_nvfp4_w", "quant_nvfp4_x"]}
+    for name in names:
+        if name in producers.get(args.profile_case, []):
             launches[name]()
     torch.cuda.synchronize()
     for _ in range(args.profile_launches):

@@ -19,7 +19,8 @@ import torch
 __all__ = ["WQError", "lib", "quantize_group_int4", "quantize_int8_per_channel", "quantize_int8_per_token",
            "smooth", "smooth_workspace_bytes", "smooth_noalloc", "gemv_w4a16", "gemm_w4a16", "gemm_w8a8", "gemv_w8a16",
            "matmul_w4a16", "quantize_fp8_e4m3", "gemm_fp8", "outlier_columns", "gather_outliers",
-           "gemm_w8a8_outliers", "llm_int8_matmul", "device_status", "set_wait_limit",
+           "gemm_w8a8_outliers", "llm_int8_matmul", "quantize_mxfp4", "quantize_nvfp4", "gemm_fp4",
+           "device_status", "set_wait_limit",
            "selftest_wait_timeout", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwq.so")
@@ -57,6 +58,9 @@ _SIGS = {
     "wq_outlier_columns": [_P, _I, _I, _F, _I, _P, _P, _P, _P],
     "wq_gather_outliers": [_P, _I, _I, _P, _I, _P, _P, _I, _P, _P, _P],
     "wq_gemm_w8a8_outliers": [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _P],
+    "wq_quantize_mxfp4": [_P, _I, _I, _P, _P, _P],
+    "wq_quantize_nvfp4": [_P, _I, _I, _P, _P, _P, _P],
+    "wq_gemm_fp4": [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P],
     "wq_device_status": [_P],
     "wq_selftest_wait_timeout": [_P],
 }
@@ -362,6 +366,50 @@ def llm_int8_matmul(x, wq, sw, threshold: float = 6.0, cap: int = 64, stream=Non
     xq, sx = quantize_int8_per_channel(x, keep, stream)
     x16, w16 = gather_outliers(x, wq, idx, count, cap, stream)
     return gemm_w8a8_outliers(xq, sx, wq, sw, x16, w16, stream=stream), count
+
+
+def quantize_mxfp4(x: torch.Tensor, stream=None):
+    """MXFP4 of fp16 x [R, K]: (packed E2M1 codes uint8 [R, K/2], E8M0 scales uint8 [R, K/32])."""
+    _cuda(x, "x", (torch.float16,), 2)
+    R, K = x.shape
+    q = _empty((R, K // 2), torch.uint8, x)
+    s = _empty((R, K // 32), torch.uint8, x)
+    _check(lib.wq_quantize_mxfp4(_ptr(x), R, K, _ptr(q), _ptr(s), _P(_stream(stream))), "wq_quantize_mxfp4")
+    return q, s
+
+
+def quantize_nvfp4(x: torch.Tensor, stream=None):
+    """NVFP4 of fp16 x [R, K]: (packed E2M1 uint8 [R, K/2], E4M3 scales uint8 [R, K/16], fp32 tensor scale [1])."""
+    _cuda(x, "x", (torch.float16,), 2)
+    R, K = x.shape
+    q = _empty((R, K // 2), torch.uint8, x)
+    s = _empty((R, K // 16), torch.uint8, x)
+    t = _empty((1,), torch.float32, x)
+    _check(lib.wq_quantize_nvfp4(_ptr(x), R, K, _ptr(q), _ptr(s), _ptr(t), _P(_stream(stream))),
+           "wq_quantize_nvfp4")
+    return q, s, t
+
+
+def gemm_fp4(a, sfa, b, sfb, ta=None, tb=None, out=None, return_acc: bool = False, stream=None):
+    """Block-scaled FP4 GEMM: NVFP4 when the tensor scales ta/tb are given, MXFP4 otherwise.
+    a [M, K/2], sfa [M, K/bs], b [N, K/2], sfb [N, K/bs] -> y fp16 [M, N]."""
+    nv = ta is not None
+    for t, n in ((a, "a"), (sfa, "sfa"), (b, "b"), (sfb, "sfb")):
+        _cuda(t, n, (torch.uint8,), 2)
+    if nv:
+        _cuda(ta, "ta", (torch.float32,), 1)
+        _cuda(tb, "tb", (torch.float32,), 1)
+    M, K = a.shape[0], a.shape[1] * 2
+    N = b.shape[0]
+    bs = 16 if nv else 32
+    if b.shape[1] * 2 != K or tuple(sfa.shape) != (M, K // bs) or tuple(sfb.shape) != (N, K // bs):
+        raise ValueError("shape mismatch: a [M,K/2], b [N,K/2], sfa [M,K/bs], sfb [N,K/bs]")
+    y = out if out is not None else _empty((M, N), torch.float16, a)
+    _cuda(y, "out", (torch.float16,), 2)
+    acc = _empty((M, N), torch.float32, a) if return_acc else None
+    _check(lib.wq_gemm_fp4(1 if nv else 0, _ptr(a), _ptr(sfa), _ptr(ta), _ptr(b), _ptr(sfb), _ptr(tb), M, N, K,
+                           _ptr(y), _ptr(acc), _P(_stream(stream))), "wq_gemm_fp4")
+    return (y, acc) if return_acc else y
 
 
 def device_status(stream=None) -> int:

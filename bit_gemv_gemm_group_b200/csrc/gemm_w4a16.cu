@@ -8,7 +8,12 @@
 // zero-point" (w^ = (q - z) s) and "What it buys at decode" (a batch of B
 // sequences reads every weight once and does 2 FLOPs per weight per sequence).
 //
-//   y[m][n] = fp16_rn( sum_k fp16_rn(s[n][k/128] * (q[n][k] - z[n][k/128])) * x[m][k] )
+//   y[m][n] = fp16_rn( sum_k fp16_rn(s[n][k/g] * (q[n][k] - z[n][k/g])) * x[m][k] )
+//
+// Group size g = 128 runs the paths tuned for it (scales of 8 groups fetched
+// ahead, split-K in 16-stage parts); g = 32, 64 and 256 fetch each stage's
+// scale and zero point one stage ahead (a thread's 32 codes of a stage always
+// lie in one group).
 //
 // Swap-AB: the MMA's M dimension is 128 weight rows (TMEM lanes) and its N
 // dimension is the activation tile (16..128 rows of x), so small batches still
@@ -151,7 +156,7 @@ template <int MT, bool SB>
 __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
                       const uint16_t *__restrict__ scales, const uint32_t *__restrict__ qzeros,
-                      uint16_t *__restrict__ y, int M, int N, int K, int splits, unsigned int *status,
+                      uint16_t *__restrict__ y, int M, int N, int K, int gs, int splits, unsigned int *status,
                       uint64_t limit_ns) {
     using L = Layout<MT>;
     extern __shared__ uint8_t smem_raw[];
@@ -165,7 +170,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     const int kb_total = K / BK;
     const int nkb = kb_total / splits;
     const int kb0 = rank * nkb;
-    const int groups = K / 128, zwords = (groups + 7) / 8;
+    const int groups = K / gs, zwords = (groups + 7) / 8;
     constexpr uint32_t IDESC = make_idesc(/*f32*/ 1, /*f16*/ 0, /*f16*/ 0, BMW, MT);
     constexpr uint32_t TMEM_COLS = 2 * MT;  // two MT-column accumulators; MT >= 16
 
@@ -368,13 +373,31 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
                 cs = ns;
                 cz = nz;
             }
-        } else {
+        } else if (gs == 128) {
             for (int i = 0; i < nkb && ok; i += 2) {
                 const int g = (kb0 + i) >> 1;
                 const uint32_t sh = __ldg(srow + g);
                 const uint32_t s2 = sh | (sh << 16);
                 const uint32_t zc = zero_consts((__ldg(zrow + (g >> 3)) >> (4 * (g & 7))) & 0xFu);
                 ok = two_stages(i, zc, s2);
+            }
+        } else {
+            // Group sizes 32, 64 and 256: a thread's 32 codes of a stage lie in one group (groups
+            // start on multiples of 32), whose scale and zero point it fetches one stage ahead.
+            auto fetch = [&](int i, uint32_t &zc, uint32_t &s2) {
+                const int g = ((kb0 + i) * BK + half * 32) / gs;
+                const uint32_t sh = __ldg(srow + g);
+                s2 = sh | (sh << 16);
+                zc = zero_consts((__ldg(zrow + (g >> 3)) >> (4 * (g & 7))) & 0xFu);
+            };
+            uint32_t zc, s2;
+            fetch(0, zc, s2);
+            for (int i = 0; i < nkb && ok; ++i) {
+                uint32_t zn = zc, sn = s2;
+                if (i + 1 < nkb) fetch(i + 1, zn, sn);
+                ok = stage(i, zc, s2);
+                zc = zn;
+                s2 = sn;
             }
         }
     }
@@ -456,7 +479,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
 
 template <int MT, bool SB>
 wq_status launch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t *scales, const uint32_t *qzeros,
-                 uint16_t *y, int M, int N, int K, int splits, unsigned int *status, cudaStream_t st) {
+                 uint16_t *y, int M, int N, int K, int gs, int splits, unsigned int *status, cudaStream_t st) {
     auto kern = gemm_w4a16_kernel<MT, SB>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Layout<MT>::SMEM);
@@ -473,7 +496,7 @@ wq_status launch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t *s
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, kern, tq, tx, scales, qzeros, y, M, N, K, splits, status, wait_limit());
+    e = cudaLaunchKernelEx(&cfg, kern, tq, tx, scales, qzeros, y, M, N, K, gs, splits, status, wait_limit());
     if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: launch failed: %s", cudaGetErrorString(e));
     return WQ_OK;
 }
@@ -481,15 +504,16 @@ wq_status launch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t *s
 // Number of CTAs sharing one weight tile's K range: a divisor of the stage
 // count (a multiple of 16 stages each on the fast path), at most 8, whose
 // partial tiles fit the leading CTA's pipeline buffers, chosen to fill the
-// SMs in as few, as full waves as possible.
-int choose_splits(int tiles, int K, int MT, bool fast, size_t pipe_bytes, int sms) {
+// SMs in as few, as full waves as possible.  The group-size-128 path without
+// the fast path takes no split; the other group sizes take any divisor.
+int choose_splits(int tiles, int K, int MT, bool fast, bool generic, size_t pipe_bytes, int sms) {
     const int kb = K / BK;
     int best = 1;
     double best_eff = -1.0;
     for (int s = 1; s <= 8; ++s) {
         if (kb % s) continue;
         if (fast && (kb / s) % 16) continue;
-        if (!fast && s > 1) continue;
+        if (!fast && !generic && s > 1) continue;
         if ((size_t)(s - 1) * BMW * MT * 4 > pipe_bytes) continue;
         const double waves = (double)tiles * s / sms;
         const double eff = waves / std::ceil(waves);
@@ -503,13 +527,14 @@ int choose_splits(int tiles, int K, int MT, bool fast, size_t pipe_bytes, int sm
 
 template <int MT>
 wq_status dispatch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t *scales, const uint32_t *qzeros,
-                   uint16_t *y, int M, int N, int K, unsigned int *status, cudaStream_t st) {
-    const bool fast = (K % 1024) == 0;
+                   uint16_t *y, int M, int N, int K, int gs, unsigned int *status, cudaStream_t st) {
+    const bool fast = gs == 128 && (K % 1024) == 0;
     const int tiles = ((N + BMW - 1) / BMW) * ((M + MT - 1) / MT);
-    const int splits = choose_splits(tiles, K, MT, fast, Layout<MT>::PIPE_BYTES, Layout<MT>::CTAS_PER_SM * num_sms());
+    const int splits = choose_splits(tiles, K, MT, fast, gs != 128, Layout<MT>::PIPE_BYTES,
+                                     Layout<MT>::CTAS_PER_SM * num_sms());
     if (fast && (K / BK / splits) % 16 == 0)
-        return launch<MT, true>(tq, tx, scales, qzeros, y, M, N, K, splits, status, st);
-    return launch<MT, false>(tq, tx, scales, qzeros, y, M, N, K, splits, status, st);
+        return launch<MT, true>(tq, tx, scales, qzeros, y, M, N, K, gs, splits, status, st);
+    return launch<MT, false>(tq, tx, scales, qzeros, y, M, N, K, gs, splits, status, st);
 }
 
 }  // namespace
@@ -525,16 +550,28 @@ extern "C" wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qwe
     WQ_REQUIRE_PTR(y, "y");
     WQ_REQUIRE(M > 0 && N > 0 && K > 0, WQ_ERR_INVALID_ARG, "wq_gemm_w4a16: sizes must be positive (M=%d N=%d K=%d)",
                M, N, K);
-    WQ_REQUIRE(group_size == 128, WQ_ERR_UNSUPPORTED, "wq_gemm_w4a16: group_size must be 128 (got %d)", group_size);
+    WQ_REQUIRE(group_size == 32 || group_size == 64 || group_size == 128 || group_size == 256, WQ_ERR_UNSUPPORTED,
+               "wq_gemm_w4a16: group_size must be 32, 64, 128 or 256 (got %d)", group_size);
+    WQ_REQUIRE(K % group_size == 0, WQ_ERR_INVALID_ARG, "wq_gemm_w4a16: K (%d) must be a multiple of group_size (%d)",
+               K, group_size);
     WQ_REQUIRE(K % 128 == 0, WQ_ERR_INVALID_ARG, "wq_gemm_w4a16: K (%d) must be a multiple of 128", K);
-    WQ_REQUIRE(M >= 16 || (M >= 9 && K % 256 == 0), WQ_ERR_UNSUPPORTED,
+    WQ_REQUIRE(M >= 16 || (M >= 9 && (K % 256 == 0 || group_size != 128)), WQ_ERR_UNSUPPORTED,
                "wq_gemm_w4a16: M (%d) below 16 needs K %% 256 == 0 (K = %d); use wq_gemv_w4a16 for M <= 8", M, K);
+    // Other group sizes below 16 rows: the CUDA-core GEMV kernel in passes of up to 8 rows.
+    if (group_size != 128 && M < 16) {
+        for (int r0 = 0; r0 < M; r0 += 8) {
+            const wq_status e = wq_gemv_w4a16(x + (size_t)r0 * K, std::min(8, M - r0), qweight, scales, qzeros, N, K,
+                                              group_size, y + (size_t)r0 * N, stream);
+            if (e != WQ_OK) return e;
+        }
+        return WQ_OK;
+    }
     // Up to 32 activation rows the byte stream dominates: the streaming mma.sync kernel (codes
     // dequantized in registers, no shared-memory fp16 tile) takes up to 16 rows per pass (it also
     // serves 9 <= M < 16, which the tensor-core kernel below does not take) and, measured
     // on B200, beats the tensor-core kernel below at M <= 32 (2 passes at M = 32 take 0.36x its
     // time on the 28672x8192 projection; at three passes the two are even).
-    if (M <= 32 && K % 256 == 0) {
+    if (group_size == 128 && M <= 32 && K % 256 == 0) {
         for (int r0 = 0; r0 < M; r0 += 16) {
             const wq_status e = gemv_stream(x + (size_t)r0 * K, std::min(16, M - r0), qweight, scales, qzeros, N, K,
                                             y + (size_t)r0 * N, as_stream(stream), "wq_gemm_w4a16");
@@ -554,9 +591,9 @@ extern "C" wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qwe
         return WQ_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     switch (MT) {
-        case 16: return dispatch<16>(tq, tx, scales, qzeros, y, M, N, K, status, st);
-        case 32: return dispatch<32>(tq, tx, scales, qzeros, y, M, N, K, status, st);
-        case 64: return dispatch<64>(tq, tx, scales, qzeros, y, M, N, K, status, st);
-        default: return dispatch<128>(tq, tx, scales, qzeros, y, M, N, K, status, st);
+        case 16: return dispatch<16>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
+        case 32: return dispatch<32>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
+        case 64: return dispatch<64>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
+        default: return dispatch<128>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
     }
 }

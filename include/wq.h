@@ -184,16 +184,17 @@ wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qweight, const
 
 /*
  * W4A16 GEMM for M >= 9 rows of activations ([P1] "Inference view"), same
- * arithmetic and layouts as wq_gemv_w4a16.  M <= 32 with K % 256 == 0 runs
- * the streaming kernel of wq_gemv_w4a16 in passes of 16 rows (codes
- * dequantized in registers, exact products, two 8-row batch tiles per weight
- * fragment).  Other M run on the tensor cores: tiles of packed weights are
- * dequantized into shared
- * memory (each dequantized weight rounded to fp16) and fed to tcgen05 MMAs
- * with fp32 accumulation in tensor memory (activation tiles of up to 128
- * rows; larger M is several tiles).  M >= 16, or 9 <= M < 16 with
- * K % 256 == 0 (the streaming kernel, one pass); group_size == 128;
- * K % 128 == 0.
+ * arithmetic and layouts as wq_gemv_w4a16, for every group size the
+ * quantizer writes.  Group size 128: M <= 32 with K % 256 == 0 runs the
+ * streaming kernel of wq_gemv_w4a16 in passes of 16 rows (codes dequantized
+ * in registers, exact products, two 8-row batch tiles per weight fragment).
+ * Other group sizes below 16 rows run wq_gemv_w4a16 in passes of 8 rows.
+ * Everything else runs on the tensor cores: tiles of packed weights are
+ * dequantized into shared memory (each dequantized weight rounded to fp16)
+ * and fed to tcgen05 MMAs with fp32 accumulation in tensor memory
+ * (activation tiles of up to 128 rows; larger M is several tiles).
+ * M >= 16, or 9 <= M < 16 with K % 256 == 0 or group_size != 128;
+ * group_size in {32, 64, 128, 256}, K % group_size == 0; K % 128 == 0.
  */
 wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
                         const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y,
@@ -303,6 +304,45 @@ wq_status wq_gather_outliers(const uint16_t *x, int M, int K, const int8_t *wq, 
 wq_status wq_gemm_w8a8_outliers(const int8_t *xq, const float *sx, const int8_t *wq, const float *sw,
                                 const uint16_t *x16, const uint16_t *w16, int cap, int M, int N, int K, uint16_t *y,
                                 void *stream);
+
+/*
+ * Block-scaled FP4 quantization.  Source: [P4] "What about FP8, MXFP4, NVFP4
+ * and GGUF?" (MXFP4: blocks of 32 four-bit floats (E2M1) sharing one 8-bit
+ * power-of-two scale; NVFP4: blocks of 16 with an FP8 scale per block plus
+ * one FP32 scale per tensor); [P3] "Formats"; [P1] "Mainstream schemes" (FP4
+ * on Blackwell).  E2M1 values: 0, 0.5, 1, 1.5, 2, 3, 4, 6 and negatives;
+ * codes are packed two per byte along K, element 2i in the low nibble.
+ * MXFP4 (the microscaling rule): per block of 32 consecutive values of a row,
+ *   e = floor(log2 max|v|) - 2,  scale byte = e + 127 (E8M0; 0 for an all-zero
+ *   block),  q = e2m1_rn(v * 2^-e)  (exact scaling, round to nearest even,
+ *   saturating at +-6).
+ * NVFP4: S = max(max|v| over the tensor, 1e-8) / 2688  (6 * 448, fp32 division;
+ *   written to *tensor_scale); per block of 16, scale byte
+ *   b = e4m3_rn((max|v| / 6) / S) (two fp32 divisions), d = e4m3(b) * S,
+ *   q = e2m1_rn(v / d) (fp32 IEEE division; all zero when b == 0).
+ * x: fp16 [R][K];  q: out [R][K/2];  scales: out [R][K/32] (MX) or [R][K/16]
+ * (NV);  tensor_scale: out fp32 [1] (also the call's reduction word).
+ * K % 32 == 0 (MX) or K % 16 == 0 (NV).  Inputs must be finite.
+ */
+wq_status wq_quantize_mxfp4(const uint16_t *x, int R, int K, uint8_t *q, uint8_t *scales, void *stream);
+wq_status wq_quantize_nvfp4(const uint16_t *x, int R, int K, uint8_t *q, uint8_t *scales, float *tensor_scale,
+                            void *stream);
+
+/*
+ * Block-scaled FP4 GEMM on the tensor cores (tcgen05 kind::mxf4 for MXFP4,
+ * kind::mxf4nvf4 for NVFP4; fp32 accumulation).  Source: as above; the
+ * hardware block scale is what group-wise quantization does in software
+ * ([P3] "Formats").
+ *   y[m][n] = fp16_rn( ta * tb * sum_k e2m1(a[m][k]) sa(m, k/bs) e2m1(b[n][k]) sb(n, k/bs) )
+ * nvfp4 = 0: MXFP4 (bs = 32, E8M0 scales, ta = tb = 1, both may be NULL);
+ * nvfp4 = 1: NVFP4 (bs = 16, E4M3 scales, ta/tb: device fp32 [1] tensor
+ * scales).  a: [M][K/2], sfa: [M][K/bs], b: [N][K/2], sfb: [N][K/bs] in the
+ * layouts the quantizers write;  y: out fp16 [M][N];  acc_out: nullable,
+ * out fp32 [M][N] (the block-scaled sums before ta * tb).  K % 256 == 0.
+ */
+wq_status wq_gemm_fp4(int nvfp4, const uint8_t *a, const uint8_t *sfa, const float *ta, const uint8_t *b,
+                      const uint8_t *sfb, const float *tb, int M, int N, int K, uint16_t *y, float *acc_out,
+                      void *stream);
 
 /* Message describing the last error status returned on this host thread. */
 const char *wq_last_error(void);

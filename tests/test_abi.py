@@ -77,9 +77,10 @@ def test_sizes_rejected(wq):
     assert L.wq_gemm_w8a8(FAKE, FAKE, FAKE, FAKE, 16, 16, 131072, FAKE, None, None) == wq.WQ_ERR_UNSUPPORTED
     assert "131056" in L.wq_last_error().decode()
     assert 128 * 128 * 131056 < 2 ** 31 <= 128 * 128 * 131072
-    # the W4A16 GEMM takes group size 128 only; the GEMV takes 32/64/128/256
-    assert L.wq_gemm_w4a16(FAKE, 16, FAKE, FAKE, FAKE, 16, 512, 64, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    # both W4A16 matmuls take the group sizes the quantizer writes (32/64/128/256) and no other
+    assert L.wq_gemm_w4a16(FAKE, 16, FAKE, FAKE, FAKE, 16, 512, 96, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
     assert L.wq_gemv_w4a16(FAKE, 1, FAKE, FAKE, FAKE, 16, 512, 96, FAKE, None) == wq.WQ_ERR_UNSUPPORTED
+    assert "32, 64, 128 or 256" in L.wq_last_error().decode()
     # smoothing: alpha range, K granularity
     assert L.wq_smooth(FAKE, 4, FAKE, 4, 64, ctypes.c_float(1.5), FAKE, FAKE, None) == wq.WQ_ERR_INVALID_ARG
     assert L.wq_smooth(FAKE, 4, FAKE, 4, 60, ctypes.c_float(0.5), FAKE, FAKE, None) == wq.WQ_ERR_UNSUPPORTED

@@ -390,6 +390,28 @@ def test_gemm_w4a16_small(wq, M, N, K):
     assert wq.device_status() == 0
 
 
+GEMM_W4_GROUPS = [  # (M, N, K, g): the group sizes the quantizer writes, ragged M/N, split-K, M < 16
+    (16, 300, 1024, 32), (64, 1000, 4096, 64), (100, 384, 3072, 256), (130, 260, 2048, 32),
+    (48, 640, 16384, 64), (12, 300, 1280, 256), (9, 130, 640, 32), (33, 129, 1152, 64),
+]
+
+
+@pytest.mark.parametrize("M,N,K,g", GEMM_W4_GROUPS)
+def test_gemm_w4a16_group_sizes(wq, M, N, K, g):
+    # A layout wq_quantize_group_int4 writes is one wq_gemm_w4a16 consumes, for every group size.
+    w = _special_weights(N, K, seed=M + N + K + g)
+    qw, sc, qz = wq.quantize_group_int4(dev(w), g)
+    x = workloads.activations(M, K, 0.01, 50.0, seed=M + g, tensor_id=N)
+    y = wq.gemm_w4a16(dev(x), qw, sc, qz, g)
+    torch.cuda.synchronize()
+    rqw, rsc, rqz = oracle.quantize_group_int4(w, g)
+    assert np.array_equal(host(qw, np.uint32), rqw) and np.array_equal(host(qz, np.uint32), rqz)
+    rows = sample_rows(N, 300, seed=K)
+    y_ref, bound = oracle.matmul_w4a16_ref(x, rqw, rsc, rqz, K, g, rows=rows)
+    assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"gemm_w4a16 g={g} M={M} N={N} K={K}")
+    assert wq.device_status() == 0
+
+
 @pytest.mark.parametrize("cfg", ["mlp_8b", "llama70b_class"])
 def test_gemm_w4a16_configs(wq, cfg):
     c = workloads.CONFIGS[cfg]
@@ -602,4 +624,134 @@ def test_llm_int8_full_size(wq):
     ns = sample_rows(N, 96, seed=6)
     ry, rb, _, _ = oracle.llm_int8_ref(X, host(wq8), host(sw), ridx, ms=ms, ns=ns)
     assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, "llm.int8 full size")
+    assert wq.device_status() == 0
+
+
+# --------------------------------------------------------------------------
+# Block-scaled FP4 (MXFP4, NVFP4): quantizers bit-exact, tcgen05 block-scaled
+# GEMM within the tolerance
+# --------------------------------------------------------------------------
+FP4_Q_SMALL = [(1, 32), (7, 64), (33, 2048), (5, 2080), (64, 4096), (3, 16384), (300, 1024)]
+
+
+def _fp4_inputs(R, K, seed):
+    g = np.random.default_rng(seed)
+    a = (g.standard_normal((R, K)) * np.exp(g.uniform(-3, 3, (R, 1)))).astype(np.float32)
+    a[:, g.choice(K, size=max(1, K // 100), replace=False)] *= 40
+    if R > 2:
+        a[1, :64] = 0.0                                   # all-zero blocks
+        a[2, : K // 2] *= 1e-5                            # tiny blocks (E4M3 block scales near 0)
+    return a.astype(np.float16)
+
+
+@pytest.mark.parametrize("R,K", FP4_Q_SMALL)
+def test_mxfp4_quantizer_bit_exact(wq, R, K):
+    a = _fp4_inputs(R, K, seed=R * K + 5)
+    q, s = wq.quantize_mxfp4(dev(a))
+    torch.cuda.synchronize()
+    rq, rs = oracle.quantize_mxfp4(a)
+    assert np.array_equal(host(s), rs) and np.array_equal(host(q), rq)
+
+
+@pytest.mark.parametrize("R,K", [rk for rk in FP4_Q_SMALL if rk[1] % 16 == 0])
+def test_nvfp4_quantizer_bit_exact(wq, R, K):
+    a = _fp4_inputs(R, K, seed=R * K + 6)
+    q, s, t = wq.quantize_nvfp4(dev(a))
+    torch.cuda.synchronize()
+    rq, rs, rt = oracle.quantize_nvfp4(a)
+    assert np.array_equal(host(t), rt)
+    assert np.array_equal(host(s), rs) and np.array_equal(host(q), rq)
+
+
+def test_fp4_quantizers_every_e2m1_midpoint(wq):
+    # v / scale next to every E2M1 rounding boundary, both signs: the row maximum 6 fixes the
+    # MX exponent at 0 (2^floor(log2 6) / 4 = 1) and the NV block scale at 1 x S
+    vals = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float64)
+    row = np.concatenate([vals, vals * (1 + 2 ** -9), vals * (1 - 2 ** -9), [6.0] * 11])
+    a = np.stack([row[:32], -row[:32]]).astype(np.float16)
+    q, s = wq.quantize_mxfp4(dev(a))
+    rq, rs = oracle.quantize_mxfp4(a)
+    assert np.array_equal(host(s), rs) and np.array_equal(host(q), rq)
+    q, s, t = wq.quantize_nvfp4(dev(a))
+    rq, rs, rt = oracle.quantize_nvfp4(a)
+    assert np.array_equal(host(t), rt) and np.array_equal(host(s), rs) and np.array_equal(host(q), rq)
+
+
+FP4_GEMM_SMALL = [(1, 1, 256), (128, 128, 256), (130, 300, 512), (64, 40, 1024), (257, 513, 256),
+                  (300, 1000, 2048), (512, 1024, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", FP4_GEMM_SMALL)
+@pytest.mark.parametrize("nv", [False, True])
+def test_gemm_fp4_small(wq, M, N, K, nv):
+    a = _fp4_inputs(M, K, seed=M + K)
+    b = (_fp4_inputs(N, K, seed=N + 2 * K).astype(np.float32) * 0.05).astype(np.float16)
+    if nv:
+        qa, sa, ta = oracle.quantize_nvfp4(a)
+        qb, sb, tb = oracle.quantize_nvfp4(b)
+        y = wq.gemm_fp4(dev(qa), dev(sa), dev(qb), dev(sb), dev(ta), dev(tb))
+        tav, tbv = float(ta[0]), float(tb[0])
+    else:
+        qa, sa = oracle.quantize_mxfp4(a)
+        qb, sb = oracle.quantize_mxfp4(b)
+        y = wq.gemm_fp4(dev(qa), dev(sa), dev(qb), dev(sb))
+        tav = tbv = 1.0
+    torch.cuda.synchronize()
+    ms, ns = sample_rows(M, 64, seed=1), sample_rows(N, 96, seed=2)
+    ry, rb = oracle.gemm_fp4_ref(nv, qa, sa, tav, qb, sb, tbv, K, ms, ns)
+    assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, f"fp4 nv={nv} M={M} N={N} K={K}")
+    assert wq.device_status() == 0
+
+
+@pytest.mark.parametrize("nv", [False, True])
+def test_gemm_fp4_scale_factor_placement(wq, nv):
+    # Every A row and every K block gets its own power-of-two scale (B all ones with scale 1): each
+    # output is the sum of A's decoded row, so a misplaced factor (row, block or byte) shows up.
+    # Scales 2^-3 .. 2^3 keep every partial sum a multiple of 2^-4 below 2^15: exact in fp32.
+    M, N, K = 256, 128, 512
+    bs = 16 if nv else 32
+    g = np.random.default_rng(7)
+    qa = g.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    qb = np.full((N, K // 2), 0x22, np.uint8)                       # E2M1 1.0 in both nibbles
+    if nv:   # E4M3 codes of 2^e: exponent field e + 7, mantissa 0
+        sa = ((g.integers(-3, 4, (M, K // bs)) + 7) << 3).astype(np.uint8)
+        sb = np.full((N, K // bs), 7 << 3, np.uint8)                # 1.0
+        one = np.ones(1, np.float32)
+        y, acc = wq.gemm_fp4(dev(qa), dev(sa), dev(qb), dev(sb), dev(one), dev(one), return_acc=True)
+    else:
+        sa = (g.integers(-3, 4, (M, K // bs)) + 127).astype(np.uint8)
+        sb = np.full((N, K // bs), 127, np.uint8)
+        y, acc = wq.gemm_fp4(dev(qa), dev(sa), dev(qb), dev(sb), return_acc=True)
+    torch.cuda.synchronize()
+    ry, _ = oracle.gemm_fp4_ref(nv, qa, sa, 1.0, qb, sb, 1.0, K)
+    assert np.array_equal(host(acc).astype(np.float64), ry)
+
+
+def test_fp4_w4a4_full_size(wq):
+    # The W8A8 layer's shapes (X [2048, 8192], W [8192, 8192]) in MXFP4 and NVFP4, quantized on the
+    # GPU and multiplied on the tensor cores; codes and scales checked on sampled rows.
+    M, N, K = 2048, 8192, 8192
+    X = workloads.config_activations("w8a8_smoothquant", M, K)
+    W = workloads.config_weight("w8a8_smoothquant")
+    ms, ns = sample_rows(M, 48, seed=8), sample_rows(N, 64, seed=9)
+    xa, wa = dev(X), dev(W)
+    for nv in (False, True):
+        if nv:
+            qx, sx, tx = wq.quantize_nvfp4(xa)
+            qw, sw, tw = wq.quantize_nvfp4(wa)
+            y = wq.gemm_fp4(qx, sx, qw, sw, tx, tw)
+            rqx, rsx, rtx = oracle.quantize_nvfp4(X)
+            assert np.array_equal(host(tx), rtx)
+            tv = (float(host(tx)[0]), float(host(tw)[0]))
+        else:
+            qx, sx = wq.quantize_mxfp4(xa)
+            qw, sw = wq.quantize_mxfp4(wa)
+            y = wq.gemm_fp4(qx, sx, qw, sw)
+            rqx, rsx = oracle.quantize_mxfp4(X[ms])
+            tv = (1.0, 1.0)
+        torch.cuda.synchronize()
+        hqx, hsx, hqw, hsw = host(qx), host(sx), host(qw), host(sw)
+        assert np.array_equal(hqx[ms], rqx[ms] if nv else rqx) and np.array_equal(hsx[ms], rsx[ms] if nv else rsx)
+        ry, rb = oracle.gemm_fp4_ref(nv, hqx, hsx, tv[0], hqw, hsw, tv[1], K, ms, ns)
+        assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, f"fp4 full nv={nv}")
     assert wq.device_status() == 0
