@@ -96,6 +96,14 @@ def _declare(L):
     L.orc_gemm_fp4_ref.argtypes = [_I, _P, _P, ctypes.c_float, _P, _P, ctypes.c_float, _I, _I, _I, _P, _I, _P, _I,
                                    _P, _P]
     L.orc_gemm_fp4_ref.restype = None
+    L.orc_hessian.argtypes = [_P, _I, _I, _P]
+    L.orc_hessian.restype = None
+    L.orc_gptq_hinv_chol.argtypes = [_P, _I, ctypes.c_double, _P]
+    L.orc_gptq_hinv_chol.restype = _I
+    L.orc_gptq.argtypes = [_P, _I, _I, _I, _P, _P, _P, _P]
+    L.orc_gptq.restype = _I
+    L.orc_awq.argtypes = [_P, _I, _I, _I, _P, _I, _P, _P, _I, _P, _P, _P, _P, _P]
+    L.orc_awq.restype = _I
 
 
 def _ptr(a: np.ndarray | None):
@@ -421,3 +429,63 @@ def gemm_fp4_ref(nvfp4: bool, a, sa, ta, b, sb, tb, K: int, ms=None, ns=None):
     lib().orc_gemm_fp4_ref(1 if nvfp4 else 0, _ptr(A), _ptr(SA), float(ta), _ptr(B), _ptr(SB), float(tb), M, N, K,
                            _ptr(m_arr), nm, _ptr(n_arr), nn, _ptr(y), _ptr(bd))
     return y, bd
+
+
+# --------------------------------------------------------------------------
+# Calibration-driven INT4 ("Quantization from Scratch": GPTQ, AWQ, gptq()/awq()
+# in "Measured on two real layers"; "Quantization" (engine-room ch. 15): H = 2 X^T X)
+# --------------------------------------------------------------------------
+def hessian(x) -> np.ndarray:
+    """H = 2 X^T X in fp64 from fp16 calibration activations X [T, K]."""
+    xb = _f16_bits(x)
+    T, K = xb.shape
+    H = np.zeros((K, K), np.float64)
+    lib().orc_hessian(_ptr(xb), T, K, _ptr(H))
+    return H
+
+
+def gptq_hinv_chol(H, damp: float = 0.01) -> np.ndarray:
+    """U, upper triangular with U^T U = (H + damp * mean(diag H) I)^-1."""
+    Hc = _c(H, np.float64)
+    K = Hc.shape[0]
+    U = np.zeros((K, K), np.float64)
+    if lib().orc_gptq_hinv_chol(_ptr(Hc), K, float(damp), _ptr(U)) != 0:
+        raise ValueError("H + damping is not positive definite")
+    return U
+
+
+def gptq(w, U, group_size: int = 128):
+    """GPTQ in the stored INT4 format: (qweight u32 [N, K/8], scales fp16 [N, K/g], qzeros u32)."""
+    wb = _f16_bits(w)
+    N, K = wb.shape
+    Uc = _c(U, np.float64)
+    G = K // group_size
+    qw = np.zeros((N, K // 8), np.uint32)
+    sc = np.zeros((N, G), np.uint16)
+    qz = np.zeros((N, (G + 7) // 8), np.uint32)
+    if lib().orc_gptq(_ptr(wb), N, K, group_size, _ptr(Uc), _ptr(qw), _ptr(sc), _ptr(qz)) != 0:
+        raise ValueError("orc_gptq: bad arguments")
+    return qw, sc.view(np.float16), qz
+
+
+AWQ_GRID = np.linspace(0.0, 1.0, 11)
+
+
+def awq(w, x, H, group_size: int = 128, grid=AWQ_GRID):
+    """AWQ's scaling search: (qweight, scales, qzeros of W diag(s), s fp32 [K], alpha index, errors)."""
+    wb, xb = _f16_bits(w), _f16_bits(x)
+    N, K = wb.shape
+    T = xb.shape[0]
+    Hc = _c(H, np.float64)
+    gr = _c(grid, np.float64)
+    G = K // group_size
+    qw = np.zeros((N, K // 8), np.uint32)
+    sc = np.zeros((N, G), np.uint16)
+    qz = np.zeros((N, (G + 7) // 8), np.uint32)
+    s = np.zeros(K, np.float32)
+    err = np.zeros(gr.size, np.float64)
+    best = lib().orc_awq(_ptr(wb), N, K, group_size, _ptr(xb), T, _ptr(Hc), _ptr(gr), int(gr.size), _ptr(qw),
+                         _ptr(sc), _ptr(qz), _ptr(s), _ptr(err))
+    if best < 0:
+        raise ValueError("orc_awq: bad arguments")
+    return qw, sc.view(np.float16), qz, s, int(best), err

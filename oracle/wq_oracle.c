@@ -744,3 +744,229 @@ void orc_gemm_fp4_ref(int nvfp4, const uint8_t *a, const uint8_t *sa, float ta, 
         }
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* Calibration-driven INT4: GPTQ and AWQ's scaling search ([P3] "GPTQ:      */
+/* rounding with error compensation", "AWQ: protect the channels that      */
+/* matter" and the gptq()/awq() routines of "Measured on two real layers"; */
+/* [P2] "The Mathematics": H = 2 X^T X; [P5] GPTQ and AWQ sections).        */
+/* Both produce the stored INT4 format of orc_quantize_group_int4; readings:*/
+/*  - a group's grid is the stored-format rule of orc_quantize_group_int4   */
+/*    (range widened to contain 0, fp16 scale, zero clamped to [0,15]),     */
+/*    applied to the fp32 values of the weights it quantizes;               */
+/*  - GPTQ's blocks are the groups (block = group size), its per-element    */
+/*    rounding is that rule's fp32 decision on the compensated weight       */
+/*    rounded to fp32; compensation runs in fp64;                           */
+/*  - H's damping adds damp * mean(diag H) to the diagonal.                 */
+/* ------------------------------------------------------------------------ */
+
+/* One group's stored-format grid from n fp32 values: *s16 (fp16 bits), *z. */
+static void group_grid(const float *v, int n, uint16_t *s16_out, int *z_out)
+{
+    float lo = 0.0f, hi = 0.0f;
+    for (int t = 0; t < n; ++t) {
+        if (v[t] < lo) lo = v[t];
+        if (v[t] > hi) hi = v[t];
+    }
+    uint16_t s16 = orc_float_to_half((hi - lo) / 15.0f);
+    if (s16 == 0) s16 = 0x3c00;
+    float s = orc_half_to_float(s16);
+    *s16_out = s16;
+    *z_out = clampi(rne_to_int(-lo / s), 0, 15);
+}
+
+static int group_code(float w, float s, int z)
+{
+    return clampi(rne_to_int(w / s) + z, 0, 15);
+}
+
+/* H = 2 X^T X in fp64, X fp16 bits [T][K]; H [K][K]. */
+void orc_hessian(const uint16_t *X, int T, int K, double *H)
+{
+    memset(H, 0, sizeof(double) * (size_t)K * K);
+    for (int t = 0; t < T; ++t)
+        for (int i = 0; i < K; ++i) {
+            double xi = (double)orc_half_to_float(X[(size_t)t * K + i]);
+            if (xi == 0.0) continue;
+            for (int j = 0; j < K; ++j)
+                H[(size_t)i * K + j] += 2.0 * xi * (double)orc_half_to_float(X[(size_t)t * K + j]);
+        }
+}
+
+/* In-place lower Cholesky factor of the SPD matrix A [n][n] (upper part untouched). */
+static int cholesky_lower(double *A, int n)
+{
+    for (int j = 0; j < n; ++j) {
+        double d = A[(size_t)j * n + j];
+        for (int k = 0; k < j; ++k) d -= A[(size_t)j * n + k] * A[(size_t)j * n + k];
+        if (!(d > 0.0)) return -1;
+        d = sqrt(d);
+        A[(size_t)j * n + j] = d;
+        for (int i = j + 1; i < n; ++i) {
+            double v = A[(size_t)i * n + j];
+            for (int k = 0; k < j; ++k) v -= A[(size_t)i * n + k] * A[(size_t)j * n + k];
+            A[(size_t)i * n + j] = v / d;
+        }
+    }
+    return 0;
+}
+
+/* U = upper Cholesky factor of (H + damp * mean(diag H) * I)^{-1}: U^T U = H'^{-1}.
+   Written as the inverse of H' via its Cholesky factor, then the Cholesky factor of
+   that inverse.  H, U: [K][K] fp64.  Returns 0, or -1 if H' is not positive definite. */
+int orc_gptq_hinv_chol(const double *H, int K, double damp, double *U)
+{
+    double *A = (double *)malloc(sizeof(double) * (size_t)K * K);
+    double *Li = (double *)calloc((size_t)K * K, sizeof(double));
+    if (!A || !Li) { free(A); free(Li); return -1; }
+    double mean = 0.0;
+    for (int i = 0; i < K; ++i) mean += H[(size_t)i * K + i];
+    mean /= K;
+    memcpy(A, H, sizeof(double) * (size_t)K * K);
+    for (int i = 0; i < K; ++i) A[(size_t)i * K + i] += damp * mean;
+    int rc = cholesky_lower(A, K);                 /* H' = L L^T */
+    if (rc == 0) {
+        /* Li = L^{-1} (lower), column by column by forward substitution */
+        for (int c = 0; c < K; ++c) {
+            for (int i = c; i < K; ++i) {
+                double v = (i == c) ? 1.0 : 0.0;
+                for (int k = c; k < i; ++k) v -= A[(size_t)i * K + k] * Li[(size_t)k * K + c];
+                Li[(size_t)i * K + c] = v / A[(size_t)i * K + i];
+            }
+        }
+        /* H'^{-1} = Li^T Li into A (full) */
+        for (int i = 0; i < K; ++i)
+            for (int j = 0; j < K; ++j) {
+                double v = 0.0;
+                for (int k = (i > j ? i : j); k < K; ++k) v += Li[(size_t)k * K + i] * Li[(size_t)k * K + j];
+                A[(size_t)i * K + j] = v;
+            }
+        rc = cholesky_lower(A, K);                 /* H'^{-1} = C C^T, U = C^T */
+        if (rc == 0)
+            for (int i = 0; i < K; ++i)
+                for (int j = 0; j < K; ++j)
+                    U[(size_t)i * K + j] = j >= i ? A[(size_t)j * K + i] : 0.0;
+    }
+    free(A);
+    free(Li);
+    return rc;
+}
+
+/* GPTQ: W fp16 bits [N][K] -> the stored INT4 format, quantizing one column at a time within
+   blocks of g columns (one group) and pushing each column's error onto the later columns through
+   U (from orc_gptq_hinv_chol):
+     for each block [i1, i2): grid of every row from its current (compensated) block values;
+       for i in block: q = code of fl32(W[n][i]); e = (W[n][i] - (q - z) s) / U[i][i];
+                       W[n][j] -= e U[i][j] for i < j < i2;  E[n][i] = e
+     then W[n][j] -= sum_i E[n][i] U[i][j] for j >= i2.
+   Returns 0, or -1 on bad arguments. */
+int orc_gptq(const uint16_t *W, int N, int K, int g, const double *U, uint32_t *qweight,
+             uint16_t *scales, uint32_t *qzeros)
+{
+    if (N <= 0 || K <= 0 || g <= 0 || K % g != 0 || K % 8 != 0)
+        return -1;
+    const int G = K / g, ZW = (G + 7) / 8;
+    double *Wd = (double *)malloc(sizeof(double) * (size_t)N * K);
+    double *E = (double *)malloc(sizeof(double) * (size_t)N * g);
+    float *blk = (float *)malloc(sizeof(float) * (size_t)g);
+    if (!Wd || !E || !blk) { free(Wd); free(E); free(blk); return -1; }
+    for (size_t i = 0; i < (size_t)N * K; ++i) Wd[i] = (double)orc_half_to_float(W[i]);
+    memset(qweight, 0, sizeof(uint32_t) * (size_t)N * (K / 8));
+    memset(qzeros, 0, sizeof(uint32_t) * (size_t)N * ZW);
+    for (int b = 0; b < G; ++b) {
+        const int i1 = b * g, i2 = i1 + g;
+        for (int n = 0; n < N; ++n) {
+            double *row = Wd + (size_t)n * K;
+            for (int t = 0; t < g; ++t) blk[t] = (float)row[i1 + t];
+            uint16_t s16;
+            int z;
+            group_grid(blk, g, &s16, &z);
+            const float s = orc_half_to_float(s16);
+            scales[(size_t)n * G + b] = s16;
+            qzeros[(size_t)n * ZW + b / 8] |= (uint32_t)z << (4 * (b % 8));
+            for (int i = i1; i < i2; ++i) {
+                const int q = group_code((float)row[i], s, z);
+                qweight[(size_t)n * (K / 8) + i / 8] |= (uint32_t)q << (4 * (i % 8));
+                const double e = (row[i] - (double)(q - z) * (double)s) / U[(size_t)i * K + i];
+                for (int j = i + 1; j < i2; ++j) row[j] -= e * U[(size_t)i * K + j];
+                E[(size_t)n * g + (i - i1)] = e;
+            }
+            for (int j = i2; j < K; ++j) {
+                double v = 0.0;
+                for (int i = i1; i < i2; ++i) v += E[(size_t)n * g + (i - i1)] * U[(size_t)i * K + j];
+                row[j] -= v;
+            }
+        }
+    }
+    free(Wd);
+    free(E);
+    free(blk);
+    return 0;
+}
+
+/* AWQ's scaling search.  mag[j] = mean_t |X[t][j]|; for each alpha of the grid:
+     s_j = mag_j^alpha, s /= sqrt(max s * min s)            (fp64, then rounded to fp32)
+     codes = stored-format RTN of the fp32 products W[n][j] * s_j
+     D = W - dequant(codes) / s;  err(alpha) = sum_n D[n] H D[n]^T  (fp64)
+   and keeps the first alpha with the smallest error.  Writes that alpha's codes,
+   s [K] (fp32) and err[grid] (all errors); returns the index of the chosen alpha,
+   or -1 on bad arguments. */
+int orc_awq(const uint16_t *W, int N, int K, int g, const uint16_t *X, int T, const double *H,
+            const double *grid, int ngrid, uint32_t *qweight, uint16_t *scales, uint32_t *qzeros,
+            float *s_out, double *err)
+{
+    if (N <= 0 || K <= 0 || T <= 0 || ngrid <= 0 || K % g != 0 || K % 8 != 0)
+        return -1;
+    const int G = K / g, ZW = (G + 7) / 8;
+    double *mag = (double *)calloc((size_t)K, sizeof(double));
+    float *s = (float *)malloc(sizeof(float) * (size_t)K);
+    float *ws = (float *)malloc(sizeof(float) * (size_t)N * K);
+    uint32_t *qw = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)N * (K / 8));
+    uint16_t *sc = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)N * G);
+    uint32_t *qz = (uint32_t *)malloc(sizeof(uint32_t) * (size_t)N * ZW);
+    double *D = (double *)malloc(sizeof(double) * (size_t)K);
+    double *what = (double *)malloc(sizeof(double) * (size_t)N * K);
+    int best = -1;
+    if (!mag || !s || !ws || !qw || !sc || !qz || !D || !what) goto done;
+    for (int t = 0; t < T; ++t)
+        for (int j = 0; j < K; ++j) mag[j] += fabs((double)orc_half_to_float(X[(size_t)t * K + j]));
+    for (int j = 0; j < K; ++j) mag[j] /= T;
+    for (int a = 0; a < ngrid; ++a) {
+        double smax = 0.0, smin = INFINITY;
+        double *sd = D;                             /* reuse D as the fp64 scales */
+        for (int j = 0; j < K; ++j) {
+            sd[j] = pow(mag[j], grid[a]);
+            if (sd[j] > smax) smax = sd[j];
+            if (sd[j] < smin) smin = sd[j];
+        }
+        const double norm = sqrt(smax * smin);
+        for (int j = 0; j < K; ++j) s[j] = (float)(sd[j] / norm);
+        for (int n = 0; n < N; ++n)
+            for (int j = 0; j < K; ++j)
+                ws[(size_t)n * K + j] = orc_half_to_float(W[(size_t)n * K + j]) * s[j];
+        orc_quantize_group_int4(ws, 0, N, K, g, qw, sc, qz);
+        orc_dequant_int4(qw, sc, qz, N, K, g, what);
+        double e = 0.0;
+        for (int n = 0; n < N; ++n) {
+            for (int j = 0; j < K; ++j)
+                D[j] = (double)orc_half_to_float(W[(size_t)n * K + j]) - what[(size_t)n * K + j] / (double)s[j];
+            for (int i = 0; i < K; ++i) {
+                if (D[i] == 0.0) continue;
+                double hd = 0.0;
+                for (int j = 0; j < K; ++j) hd += H[(size_t)i * K + j] * D[j];
+                e += D[i] * hd;
+            }
+        }
+        err[a] = e;
+        if (best < 0 || e < err[best]) {
+            best = a;
+            memcpy(qweight, qw, sizeof(uint32_t) * (size_t)N * (K / 8));
+            memcpy(scales, sc, sizeof(uint16_t) * (size_t)N * G);
+            memcpy(qzeros, qz, sizeof(uint32_t) * (size_t)N * ZW);
+            memcpy(s_out, s, sizeof(float) * (size_t)K);
+        }
+    }
+done:
+    free(mag); free(s); free(ws); free(qw); free(sc); free(qz); free(D); free(what);
+    return best;
+}

@@ -686,3 +686,86 @@ def test_fp4_gemm_ref_reduces_to_numpy():
         assert _rel(wa, a.astype(np.float64)) < 0.2
         ys, _ = oracle.gemm_fp4_ref(nv, qa, sa, tav, qb, sb, tbv, 128, ms=[4, 0], ns=[6, 1])
         assert np.array_equal(ys, y[np.ix_([4, 0], [6, 1])])
+
+
+# --------------------------------------------------------------------------
+# GPTQ and AWQ: the Hessian and its factor against numpy, the degenerate cases
+# that reduce to round-to-nearest, the objective each method lowers, and the
+# pages' direction (GPTQ beats RTN on its calibration data; AWQ's scaling
+# helps where input channels carry outliers)
+# --------------------------------------------------------------------------
+def _calib_case(seed, N=48, K=256, T=384, outlier_channels=(), scale=30.0):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((T, K)).astype(np.float32)
+    # correlated inputs (a few shared directions) so that compensation has something to use
+    x += 0.8 * (g.standard_normal((T, 4)) @ g.standard_normal((4, K))).astype(np.float32)
+    for c in outlier_channels:
+        x[:, c] *= scale
+    w = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    return x.astype(np.float16), w.astype(np.float16)
+
+
+def _objective(x, w, qw, sc, qz, K, g, s=None):
+    what = oracle.dequant_int4(qw, sc, qz, K, g)
+    if s is not None:
+        what = what / s.astype(np.float64)[None, :]
+    d = w.astype(np.float64) - what
+    return float(np.sum((x.astype(np.float64) @ d.T) ** 2))
+
+
+def test_hessian_and_factor_against_numpy():
+    x, _ = _calib_case(51, K=64, T=80)
+    H = oracle.hessian(x)
+    xf = x.astype(np.float64)
+    assert np.allclose(H, 2 * xf.T @ xf, rtol=1e-13, atol=1e-10)
+    U = oracle.gptq_hinv_chol(H, 0.01)
+    Hd = H + 0.01 * np.mean(np.diag(H)) * np.eye(64)
+    assert np.allclose(np.triu(U), U)
+    assert np.allclose(U.T @ U, np.linalg.inv(Hd), rtol=1e-9, atol=1e-12)
+    assert np.allclose(U, np.linalg.cholesky(np.linalg.inv(Hd)).T, rtol=1e-8, atol=1e-12)
+
+
+def test_gptq_with_identity_hessian_is_round_to_nearest():
+    # U = I: no compensation, every block's grid and codes are plain RTN of the weights
+    _, w = _calib_case(52)
+    K = w.shape[1]
+    for g in (64, 128):
+        qw, sc, qz = oracle.gptq(w, np.eye(K), g)
+        rqw, rsc, rqz = oracle.quantize_group_int4(w, g)
+        assert np.array_equal(qw, rqw) and np.array_equal(sc.view(np.uint16), rsc.view(np.uint16))
+        assert np.array_equal(qz, rqz)
+
+
+def test_gptq_lowers_the_calibration_objective():
+    x, w = _calib_case(53)
+    K = w.shape[1]
+    H = oracle.hessian(x)
+    U = oracle.gptq_hinv_chol(H, 0.01)
+    qw, sc, qz = oracle.gptq(w, U, 128)
+    rqw, rsc, rqz = oracle.quantize_group_int4(w, 128)
+    e_gptq = _objective(x, w, qw, sc, qz, K, 128)
+    e_rtn = _objective(x, w, rqw, rsc, rqz, K, 128)
+    # "on its own calibration tokens" GPTQ is well below round-to-nearest
+    assert e_gptq < 0.8 * e_rtn
+
+
+def test_awq_grid_zero_is_round_to_nearest_and_search_picks_the_minimum():
+    x, w = _calib_case(54, outlier_channels=(3, 70, 200))
+    K = w.shape[1]
+    H = oracle.hessian(x)
+    qw, sc, qz, s, best, err = oracle.awq(w, x, H, 128, grid=np.array([0.0]))
+    rqw, rsc, rqz = oracle.quantize_group_int4(w, 128)
+    assert np.all(s == 1.0) and np.array_equal(qw, rqw) and np.array_equal(qz, rqz)
+    # the error the search computes is the calibration objective sum_n D H D^T (H = 2 X^T X)
+    assert abs(err[0] - 2 * _objective(x, w, rqw, rsc, rqz, K, 128)) <= 1e-9 * err[0]
+    qw, sc, qz, s, best, err = oracle.awq(w, x, H, 128)
+    assert best == int(np.argmin(err)) and err[best] <= err[0]
+    assert abs(2 * _objective(x, w, qw, sc, qz, K, 128, s) - err[best]) <= 1e-9 * err[best]
+
+
+def test_awq_helps_with_outlier_channels():
+    # "AWQ's scaling helps where there are outliers": planted channels 30x the others
+    x, w = _calib_case(55, outlier_channels=(3, 70, 200), scale=30.0)
+    H = oracle.hessian(x)
+    _, _, _, _, best, err = oracle.awq(w, x, H, 128)
+    assert best > 0 and err[best] < 0.9 * err[0]
