@@ -165,24 +165,37 @@ __device__ __forceinline__ void outlier_chunk(const Outliers &ol, int M, int N, 
     for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) cf[mt][nt][0] = cf[mt][nt][1] = cf[mt][nt][2] = cf[mt][nt][3] = 0.0f;
-    for (int kk = 0; kk < ol.cap; kk += 16) {
-        uint32_t a[2][4], b[4][2];
+    // Four k-steps (64 carved columns) per round: all of the round's fragments are requested
+    // before its MMAs, so a chunk waits for one L2 round trip per 64 columns, not one per 16.
+    for (int k0 = 0; k0 < ol.cap; k0 += 64) {
+        uint32_t a[4][2][4], b[4][4][2];
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt) {
-            a[mt][0] = ldg_u32(xa[mt][0] + kk);
-            a[mt][1] = ldg_u32(xa[mt][1] + kk);
-            a[mt][2] = ldg_u32(xa[mt][0] + kk + 8);
-            a[mt][3] = ldg_u32(xa[mt][1] + kk + 8);
+        for (int ks = 0; ks < 4; ++ks) {
+            const int kk = k0 + 16 * ks;
+            if (kk < ol.cap) {
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt) {
+                    a[ks][mt][0] = ldg_u32(xa[mt][0] + kk);
+                    a[ks][mt][1] = ldg_u32(xa[mt][1] + kk);
+                    a[ks][mt][2] = ldg_u32(xa[mt][0] + kk + 8);
+                    a[ks][mt][3] = ldg_u32(xa[mt][1] + kk + 8);
+                }
+#pragma unroll
+                for (int nt = 0; nt < 4; ++nt) {
+                    b[ks][nt][0] = ldg_u32(wb[nt] + kk);
+                    b[ks][nt][1] = ldg_u32(wb[nt] + kk + 8);
+                }
+            }
         }
 #pragma unroll
-        for (int nt = 0; nt < 4; ++nt) {
-            b[nt][0] = ldg_u32(wb[nt] + kk);
-            b[nt][1] = ldg_u32(wb[nt] + kk + 8);
+        for (int ks = 0; ks < 4; ++ks) {
+            if (k0 + 16 * ks < ol.cap) {
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int nt = 0; nt < 4; ++nt) mma_16816_f16(cf[mt][nt], a[ks][mt], b[ks][nt][0], b[ks][nt][1]);
+            }
         }
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) mma_16816_f16(cf[mt][nt], a[mt], b[nt][0], b[nt][1]);
     }
     __syncwarp();  // the previous chunk's readers are done with tr
 #pragma unroll
@@ -232,6 +245,36 @@ __device__ __forceinline__ void store_chunk_outliers(uint16_t *__restrict__ y, i
     }
 }
 
+// Work schedule of the persistent CTAs.  Plain: tile blockIdx.x + u * gridDim.x for u = 0, 1, ...
+// Split (the grid is made of CTA pairs, thread-block clusters of 2): `full_rounds` rounds of whole
+// tiles, then the `split_tiles` tiles left over are shared by the pairs, one per pair, each CTA
+// taking one half of K; the pair sums its two partial accumulators through distributed shared
+// memory at the end.  This turns a last round that would keep only part of the SMs busy for a
+// whole tile into a half-length round.
+struct Sched {
+    int tiles, full_rounds, split_tiles;  // split_tiles == 0: plain schedule
+
+    __device__ __forceinline__ bool unit(int u, int kblocks, int &tile, int &kb0, int &kb1, bool &half) const {
+        half = false;
+        kb0 = 0;
+        kb1 = kblocks;
+        if (split_tiles == 0 || u < full_rounds) {
+            tile = (int)blockIdx.x + u * (int)gridDim.x;
+            return split_tiles == 0 ? tile < tiles : true;
+        }
+        const int pair = (int)blockIdx.x >> 1;
+        if (u != full_rounds || pair >= split_tiles) return false;
+        tile = full_rounds * (int)gridDim.x + pair;
+        half = true;
+        const int h = kblocks / 2;
+        if (blockIdx.x & 1) kb0 = h;
+        else kb1 = h;
+        return true;
+    }
+};
+
+constexpr int PART_PITCH = BN + 4;  // 32-bit words per row of the pair's partial tile in shared memory
+
 // D (+)= A * B^T for one 128 x 256 x 32 step: kind::i8 (int32) or kind::f8f6f4 E4M3 (fp32).
 template <bool FP8>
 __device__ __forceinline__ void mma_step(uint32_t d, uint64_t a, uint64_t b, uint32_t acc) {
@@ -243,12 +286,13 @@ __device__ __forceinline__ void mma_step(uint32_t d, uint64_t a, uint64_t b, uin
 
 // sx_stride / sw_stride: 1 for one scale per row, 0 for one scale for the whole operand.
 // OUTL (INT8 only): the epilogue adds the 16-bit product of the outlier columns `ol`.
-template <bool FP8, bool OUTL = false>
+// SPLIT: launched as clusters of 2 with the split schedule (see Sched).
+template <bool FP8, bool OUTL = false, bool SPLIT = false>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                      const float *__restrict__ sx, int sx_stride, const float *__restrict__ sw, int sw_stride,
                      uint16_t *__restrict__ y, int32_t *__restrict__ acc_out, int M, int N, int K, Outliers ol,
-                     unsigned int *status, uint64_t limit_ns) {
+                     Sched sched, unsigned int *status, uint64_t limit_ns) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sA = base;
@@ -286,15 +330,18 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     const uint32_t tmem_base = sm->tmem_base;
     const WaitCtl ctl{&sm->abort, status, limit_ns};
+    int split_acc = -1, split_tile = 0;  // epilogue: accumulator and tile of the pair's shared tile
 
     if (warp == 0) {
         if (lane == 0) {
             // ---------------------------------------------------------------- producer
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+            int tile, kbb, kbe;
+            bool half;
+            for (int u = 0; ok && sched.unit(u, kblocks, tile, kbb, kbe, half); ++u) {
                 const int m0 = (tile % mt) * BM, n0 = (tile / mt) * BN;
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                for (int kb = kbb; kb < kbe; ++kb, ++it) {
                     const uint32_t s = it % STAGES, u = it / STAGES;
                     if (!wait_parity(smem_u32(&sm->empty[s]), (u & 1) ^ 1, ctl, SITE_PRODUCER)) {
                         ok = false;
@@ -317,12 +364,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             // ---------------------------------------------------------------- MMA issuer
             uint32_t it = 0, tcount = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x, ++tcount) {
+            int tile, kbb, kbe;
+            bool half;
+            for (int u = 0; ok && sched.unit(u, kblocks, tile, kbb, kbe, half); ++u, ++tcount) {
                 const uint32_t a = tcount & 1, ua = tcount >> 1;
                 if (!wait_parity(smem_u32(&sm->tmem_empty[a]), (ua & 1) ^ 1, ctl, SITE_MMA)) break;
                 tc_fence_after();
                 const uint32_t d = tmem_base + a * BN;
-                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                for (int kb = kbb; kb < kbe; ++kb, ++it) {
                     const uint32_t s = it % STAGES, u = it / STAGES;
                     if (!wait_parity(smem_u32(&sm->full[s]), u & 1, ctl, SITE_MMA)) {
                         ok = false;
@@ -333,7 +382,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
                     for (int kk = 0; kk < BK / 32; ++kk)
                         mma_step<FP8>(d, umma_desc_sw128_kmajor(a_addr + kk * 32),
-                                      umma_desc_sw128_kmajor(b_addr + kk * 32), (kb | kk) != 0);
+                                      umma_desc_sw128_kmajor(b_addr + kk * 32), (kb != kbb) || kk != 0);
                     tc_commit(smem_u32(&sm->empty[s]));
                 }
                 if (ok) tc_commit(smem_u32(&sm->tmem_full[a]));
@@ -349,12 +398,19 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int row = q * 32 + lane;
         const bool vec_ok = (N % 8) == 0;
         uint32_t tcount = 0;
-        for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tcount) {
+        int tile, kbb, kbe;
+        bool half;
+        for (int u = 0; sched.unit(u, kblocks, tile, kbb, kbe, half); ++u, ++tcount) {
             const uint32_t a = tcount & 1, ua = tcount >> 1;
             bool ok = wait_parity(smem_u32(&sm->tmem_full[a]), ua & 1, ctl, SITE_EPILOGUE);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) break;
             tc_fence_after();
+            if (SPLIT && half) {  // the pair's shared tile: summed and stored after the loop
+                split_acc = (int)a;
+                split_tile = tile;
+                break;
+            }
             const int m = (tile % mt) * BM + row;
             const int nb = (tile / mt) * BN;
             const float sxm = m < M ? __ldg(sx + m * sx_stride) : 0.0f;
@@ -379,6 +435,57 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_arrive(smem_u32(&sm->tmem_empty[a]));
         }
     }
+    if (SPLIT) {
+        // Every CTA of the pair is past its last wait: the MMAs of the shared tile are complete
+        // (the epilogue warps waited for them) and every TMA load has landed, so the leading CTA's
+        // pipeline buffers are free to receive the second CTA's partial accumulator.
+        cluster_sync();
+        const bool epi = warp >= 2;
+        const int q = warp & 3, row = q * 32 + lane;
+        uint32_t *part = reinterpret_cast<uint32_t *>(base);  // [BM][PART_PITCH] in the leading CTA
+        if (epi && split_acc >= 0 && (blockIdx.x & 1)) {
+            const uint32_t dst = mapa_shared(smem_u32(part + row * PART_PITCH), 0);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + split_acc * BN + c * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    asm volatile("st.shared::cluster.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst + (c * 32 + j) * 4),
+                                 "r"(r[j]), "r"(r[j + 1]), "r"(r[j + 2]), "r"(r[j + 3])
+                                 : "memory");
+            }
+        }
+        cluster_sync();
+        if (epi && split_acc >= 0 && !(blockIdx.x & 1) && !sm->abort) {
+            const int m = (split_tile % mt) * BM + row;
+            const int nb = (split_tile / mt) * BN;
+            const float sxm = m < M ? __ldg(sx + m * sx_stride) : 0.0f;
+            const bool vec_ok = (N % 8) == 0;
+            const uint32_t src = smem_u32(part + row * PART_PITCH);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t r[32];
+                tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + split_acc * BN + c * 32, r);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 32; j += 4) {
+                    uint4 v;
+                    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                 : "r"(src + (c * 32 + j) * 4));
+                    const uint32_t o[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)  // int32 sums are exact; fp32 sums of two terms commute
+                        r[j + e] = FP8 ? __float_as_uint(__uint_as_float(r[j + e]) + __uint_as_float(o[e]))
+                                       : r[j + e] + o[e];
+                }
+                if (m < M && nb + c * 32 < N)
+                    store_chunk<FP8>(y, acc_out, m, nb + c * 32, N, sxm, sw, sw_stride, r, vec_ok);
+            }
+        }
+    }
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
@@ -391,6 +498,34 @@ __global__ void __launch_bounds__(THREADS, 1)
 
 namespace wq {
 namespace {
+
+// CTA pairs (clusters of 2, one CTA per SM) that can be resident at once, at most half the SMs;
+// 0 if the query fails.  Cached per device.
+int split_pairs(const void *kern, size_t smem, int sms) {
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+    if (cached[dev]) return cached[dev] > 0 ? cached[dev] : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sms / 2));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        clusters = -1;
+    }
+    const int pairs = clusters > 0 ? std::min(clusters, sms / 2) : -1;
+    cached[dev] = pairs;
+    return pairs > 0 ? pairs : 0;
+}
 
 // Shared launch path of the INT8, FP8 and LLM.int8() GEMMs (arguments already validated).
 template <bool FP8, bool OUTL = false>
@@ -412,10 +547,44 @@ wq_status launch_gemm(const void *xq, const float *sx, int sx_stride, const void
     if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "%s: cudaFuncSetAttribute failed: %s", who, cudaGetErrorString(e));
     const long long tiles = (long long)((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     WQ_REQUIRE(tiles < (1ll << 31), WQ_ERR_UNSUPPORTED, "%s: problem too large", who);
-    const int grid = (int)std::min<long long>(tiles, num_sms());
+    const int sms = num_sms();
+    const int kblocks = (K + BK - 1) / BK;
+    // Split schedule when the tiles left after whole rounds fit one per CTA pair: the last
+    // round then takes half a tile's time instead of a whole one.
+    if (!OUTL && kblocks >= 2 && tiles > sms) {
+        auto kern = gemm_w8a8_kernel<FP8, false, true>;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess)
+            return fail(WQ_ERR_CUDA, "%s: cudaFuncSetAttribute failed: %s", who, cudaGetErrorString(e));
+        const int pairs = split_pairs(reinterpret_cast<const void *>(kern), smem, sms);
+        const int grid = 2 * pairs;
+        const int full_rounds = grid > 0 ? (int)(tiles / grid) : 0;
+        const int left = (int)(tiles - (long long)full_rounds * grid);
+        // estimated time in tiles: full_rounds + 1/2 against ceil(tiles / sms) for the plain grid
+        if (pairs > 0 && left > 0 && left <= pairs && full_rounds + 0.5 < (double)((tiles + sms - 1) / sms)) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(grid);
+            cfg.blockDim = dim3(THREADS);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = as_stream(stream);
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            e = cudaLaunchKernelEx(&cfg, kern, tx, tw, sx, sx_stride, sw, sw_stride, y,
+                                   reinterpret_cast<int32_t *>(acc_out), M, N, K, ol,
+                                   Sched{(int)tiles, full_rounds, left}, status, wait_limit());
+            if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "%s: launch failed: %s", who, cudaGetErrorString(e));
+            return WQ_OK;
+        }
+    }
+    const int grid = (int)std::min<long long>(tiles, sms);
     gemm_w8a8_kernel<FP8, OUTL><<<grid, THREADS, smem, as_stream(stream)>>>(
-        tx, tw, sx, sx_stride, sw, sw_stride, y, reinterpret_cast<int32_t *>(acc_out), M, N, K, ol, status,
-        wait_limit());
+        tx, tw, sx, sx_stride, sw, sw_stride, y, reinterpret_cast<int32_t *>(acc_out), M, N, K, ol,
+        Sched{(int)tiles, 0, 0}, status, wait_limit());
     return check_launch(who);
 }
 

@@ -755,3 +755,38 @@ def test_fp4_w4a4_full_size(wq):
         ry, rb = oracle.gemm_fp4_ref(nv, hqx, hsx, tv[0], hqw, hsw, tv[1], K, ms, ns)
         assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, f"fp4 full nv={nv}")
     assert wq.device_status() == 0
+
+
+# --------------------------------------------------------------------------
+# Split last round of the persistent W8A8 / FP8 GEMMs: 160 tiles of 128 x 256 on 148 SMs leave 12
+# tiles after one whole round; CTA pairs share them (half of K each, summed through distributed
+# shared memory).  Every output of those tiles (n-tiles 14 and 15) is checked, plus a sample.
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("fp8", [False, True])
+def test_w8a8_split_last_round(wq, fp8):
+    M, N, K = 1280, 4096, 512
+    g = np.random.default_rng(17 + fp8)
+    sx = (g.random(M, dtype=np.float32) + 0.01) * 0.05
+    sw = (g.random(N, dtype=np.float32) + 0.01) * 0.01
+    ns = np.arange(14 * 256, 16 * 256, dtype=np.int32)
+    ms = np.arange(M, dtype=np.int32)
+    if fp8:
+        xq, wq8 = _random_e4m3(g, (M, K)), _random_e4m3(g, (N, K))
+        y, acc = wq.gemm_fp8(dev(xq), dev(sx), dev(wq8), dev(sw), return_acc=True)
+        torch.cuda.synchronize()
+        ry, rb = oracle.gemm_fp8_ref(xq, sx, wq8, sw, ms, ns)
+    else:
+        xq = g.integers(-128, 128, (M, K), dtype=np.int8)
+        wq8 = g.integers(-128, 128, (N, K), dtype=np.int8)
+        y, acc = wq.gemm_w8a8(dev(xq), dev(sx), dev(wq8), dev(sw), return_acc=True)
+        torch.cuda.synchronize()
+        racc, ry, rb = oracle.gemm_w8a8_ref(xq, sx, wq8, sw, ms, ns)
+        assert np.array_equal(host(acc)[:, ns].astype(np.int64), racc)
+    assert_within_bound(host(y)[:, ns].astype(np.float64), ry, rb, f"split round fp8={fp8}")
+    ms2, ns2 = sample_rows(M, 64, seed=3), sample_rows(N, 64, seed=4)
+    if fp8:
+        ry2, rb2 = oracle.gemm_fp8_ref(xq, sx, wq8, sw, ms2, ns2)
+    else:
+        _, ry2, rb2 = oracle.gemm_w8a8_ref(xq, sx, wq8, sw, ms2, ns2)
+    assert_within_bound(host(y)[np.ix_(ms2, ns2)].astype(np.float64), ry2, rb2, f"split round sample fp8={fp8}")
+    assert wq.device_status() == 0
