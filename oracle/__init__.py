@@ -67,6 +67,10 @@ def _declare(L):
     L.orc_smooth.restype = _I
     L.orc_matmul_w4a16_ref.argtypes = [_P, _I, _P, _P, _P, _I, _I, _I, _P, _I, _P, _P]
     L.orc_matmul_w4a16_ref.restype = None
+    L.orc_matmul_w4a16_ref_bf16.argtypes = [_P, _I, _P, _P, _P, _I, _I, _I, _P, _I, _P, _P]
+    L.orc_matmul_w4a16_ref_bf16.restype = None
+    L.orc_bf16_to_float.argtypes = [ctypes.c_uint16]
+    L.orc_bf16_to_float.restype = ctypes.c_float
     L.orc_matmul_w8a16_ref.argtypes = [_P, _I, _P, _P, _I, _I, _P, _I, _P, _P]
     L.orc_matmul_w8a16_ref.restype = None
     L.orc_gemm_w8a8_ref.argtypes = [_P, _P, _P, _P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _P]
@@ -239,6 +243,26 @@ def _rows_arg(rows, N):
     if r.size and (r.min() < 0 or r.max() >= N):
         raise ValueError("row index out of range")
     return r, int(r.size)
+
+
+def matmul_w4a16_ref_bf16(x_bits, qweight, scales, qzeros, K: int, group_size: int = 128, rows=None):
+    """matmul_w4a16_ref with bf16 activations given as uint16 bit patterns [B, K]."""
+    xb = np.ascontiguousarray(np.atleast_2d(x_bits), dtype=np.uint16)
+    B = xb.shape[0]
+    qw = _c(qweight, np.uint32)
+    sc = _f16_bits(scales)
+    qz = _c(qzeros, np.uint32)
+    N = qw.shape[0]
+    r, nr = _rows_arg(rows, N)
+    y = np.zeros((B, nr), np.float64)
+    bd = np.zeros((B, nr), np.float64)
+    lib().orc_matmul_w4a16_ref_bf16(_ptr(xb), B, _ptr(qw), _ptr(sc), _ptr(qz), N, K, group_size,
+                                    _ptr(r), nr, _ptr(y), _ptr(bd))
+    return y, bd
+
+
+def bf16_to_float(bits: int) -> float:
+    return float(lib().orc_bf16_to_float(int(bits)))
 
 
 def matmul_w4a16_ref(x, qweight, scales, qzeros, K: int, group_size: int = 128, rows=None):

@@ -275,9 +275,37 @@ int orc_smooth(const uint16_t *X, int M, const uint16_t *W, int N, int K,
 /* x[b][k], plus bound[b][n] = sum_k |w^[n][k] x[b][k]|.  rows (nullable)    */
 /* selects output rows; results are [B][nrows].                              */
 /* ------------------------------------------------------------------------ */
+/* bfloat16: the upper 16 bits of an IEEE binary32 (1 sign, 8 exponent, 7 mantissa bits). */
+float orc_bf16_to_float(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static void matmul_w4a16(const uint16_t *x, float (*load_x)(uint16_t), int B, const uint32_t *qweight,
+                         const uint16_t *scales, const uint32_t *qzeros, int N, int K, int g,
+                         const int *rows, int nrows, double *y, double *bound);
+
 void orc_matmul_w4a16_ref(const uint16_t *x, int B, const uint32_t *qweight,
                           const uint16_t *scales, const uint32_t *qzeros, int N, int K,
                           int g, const int *rows, int nrows, double *y, double *bound)
+{
+    matmul_w4a16(x, orc_half_to_float, B, qweight, scales, qzeros, N, K, g, rows, nrows, y, bound);
+}
+
+/* The same reference with bf16 activations. */
+void orc_matmul_w4a16_ref_bf16(const uint16_t *x, int B, const uint32_t *qweight,
+                               const uint16_t *scales, const uint32_t *qzeros, int N, int K,
+                               int g, const int *rows, int nrows, double *y, double *bound)
+{
+    matmul_w4a16(x, orc_bf16_to_float, B, qweight, scales, qzeros, N, K, g, rows, nrows, y, bound);
+}
+
+static void matmul_w4a16(const uint16_t *x, float (*load_x)(uint16_t), int B, const uint32_t *qweight,
+                         const uint16_t *scales, const uint32_t *qzeros, int N, int K, int g,
+                         const int *rows, int nrows, double *y, double *bound)
 {
     const int G = K / g;
     if (!rows) nrows = N;
@@ -290,7 +318,7 @@ void orc_matmul_w4a16_ref(const uint16_t *x, int B, const uint32_t *qweight,
                 double s = (double)orc_half_to_float(scales[(size_t)n * G + j]);
                 int q = orc_int4_code(qweight, K, n, k);
                 int z = orc_int4_zero(qzeros, K, g, n, j);
-                double t = s * (double)(q - z) * (double)orc_half_to_float(x[(size_t)b * K + k]);
+                double t = s * (double)(q - z) * (double)load_x(x[(size_t)b * K + k]);
                 acc += t;
                 bnd += fabs(t);
             }

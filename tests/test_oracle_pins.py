@@ -769,3 +769,21 @@ def test_awq_helps_with_outlier_channels():
     H = oracle.hessian(x)
     _, _, _, _, best, err = oracle.awq(w, x, H, 128)
     assert best > 0 and err[best] < 0.9 * err[0]
+
+
+def test_bf16_decode_and_reference_against_torch():
+    import torch
+    bits = np.arange(65536, dtype=np.uint32)
+    ours = np.array([oracle.bf16_to_float(int(b)) for b in bits[::7]], np.float32)
+    ref = torch.from_numpy(bits[::7].astype(np.int32).astype(np.int16)).view(torch.bfloat16).float().numpy()
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(ours), nan) and np.array_equal(ours[~nan].view(np.uint32), ref[~nan].view(np.uint32))
+    # the bf16 reference equals the fp16 one on activations exact in both formats
+    g = np.random.default_rng(71)
+    w = (g.standard_normal((20, 256)) * 0.02).astype(np.float16)
+    qw, sc, qz = oracle.quantize_group_int4(w, 128)
+    x = (g.integers(-64, 64, (2, 256)) / 8.0).astype(np.float32)         # exact in fp16 and bf16
+    xb = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    y16, b16 = oracle.matmul_w4a16_ref(x.astype(np.float16), qw, sc, qz, 256)
+    ybf, bbf = oracle.matmul_w4a16_ref_bf16(xb, qw, sc, qz, 256)
+    assert np.array_equal(y16, ybf) and np.array_equal(b16, bbf)
