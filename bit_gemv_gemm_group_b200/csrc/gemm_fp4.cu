@@ -80,29 +80,39 @@ __device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint3
 
 // Lane `lane` writes the scale factors of rows lane + 32 i (i = 0..3) of one 128-row block into
 // the G atoms at `dst`: atom g, bytes 16 lane .. 16 lane + 15 = factors 4g..4g+3 of those rows.
+// Scale factors of one stage for one lane: rows lane + 32 i (i = 0..3) of the A tile and of the
+// B tile, 16 (NVFP4) or 8 (MXFP4) bytes each.  Loaded into registers a few stages ahead of their
+// use, so the producer does not wait for the L2 round trip on every stage.
 template <bool NV>
-__device__ __forceinline__ void stage_factors(const uint8_t *__restrict__ sf, int rows, int row0, int ld, int kb,
-                                              int lane, uint32_t dst) {
-    if constexpr (NV) {  // 16 factors per row per stage: one 16-byte load per row, four groups
-        uint4 v[4];
+struct StageFactors {
+    uint4 a[4], b[4];  // MXFP4 uses .x/.y only
+};
+
+template <bool NV>
+__device__ __forceinline__ void load_factor_rows(const uint8_t *__restrict__ sf, int rows, int row0, int ld, int kb,
+                                                 int lane, uint4 (&v)[4]) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = min(row0 + lane + 32 * i, rows - 1);
-            v[i] = __ldg(reinterpret_cast<const uint4 *>(sf + (size_t)r * ld + (size_t)kb * 16));
+    for (int i = 0; i < 4; ++i) {
+        const int r = min(row0 + lane + 32 * i, rows - 1);
+        const uint8_t *p = sf + (size_t)r * ld + (size_t)kb * (NV ? 16 : 8);
+        if constexpr (NV) {
+            v[i] = __ldg(reinterpret_cast<const uint4 *>(p));
+        } else {
+            const uint2 t = __ldg(reinterpret_cast<const uint2 *>(p));
+            v[i] = make_uint4(t.x, t.y, 0u, 0u);
         }
-        sts128(dst + 0 * ATOM + lane * 16, v[0].x, v[1].x, v[2].x, v[3].x);
-        sts128(dst + 1 * ATOM + lane * 16, v[0].y, v[1].y, v[2].y, v[3].y);
+    }
+}
+
+// Lane `lane` writes its rows' factors into the G atoms at `dst`: atom g, bytes 16 lane ..
+// 16 lane + 15 = factors 4g..4g+3 of rows lane, lane + 32, lane + 64, lane + 96.
+template <bool NV>
+__device__ __forceinline__ void store_factor_rows(const uint4 (&v)[4], int lane, uint32_t dst) {
+    sts128(dst + 0 * ATOM + lane * 16, v[0].x, v[1].x, v[2].x, v[3].x);
+    sts128(dst + 1 * ATOM + lane * 16, v[0].y, v[1].y, v[2].y, v[3].y);
+    if constexpr (NV) {
         sts128(dst + 2 * ATOM + lane * 16, v[0].z, v[1].z, v[2].z, v[3].z);
         sts128(dst + 3 * ATOM + lane * 16, v[0].w, v[1].w, v[2].w, v[3].w);
-    } else {  // 8 factors per row per stage: one 8-byte load per row, two groups
-        uint2 v[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int r = min(row0 + lane + 32 * i, rows - 1);
-            v[i] = __ldg(reinterpret_cast<const uint2 *>(sf + (size_t)r * ld + (size_t)kb * 8));
-        }
-        sts128(dst + 0 * ATOM + lane * 16, v[0].x, v[1].x, v[2].x, v[3].x);
-        sts128(dst + 1 * ATOM + lane * 16, v[0].y, v[1].y, v[2].y, v[3].y);
     }
 }
 
@@ -153,29 +163,45 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         // -------------------------------------------------------------------- producer warp
+        // The CTA's stages in order: stage j is k block j % kblocks of its tile j / kblocks.
+        const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+        const int nstages = my_tiles * kblocks;
+        auto load = [&](int j, StageFactors<NV> &f) {
+            const int tile = (int)blockIdx.x + (j / kblocks) * (int)gridDim.x, kb = j % kblocks;
+            load_factor_rows<NV>(sfa, M, (tile % mt) * BM, ld_sf, kb, lane, f.a);
+            load_factor_rows<NV>(sfb, N, (tile / mt) * BN, ld_sf, kb, lane, f.b);
+        };
+        // two stages of factors in registers (f0: even stages, f1: odd ones): stage j + 2 is
+        // requested as soon as stage j has been stored
+        StageFactors<NV> f0, f1;
+        if (nstages > 0) load(0, f0);
+        if (nstages > 1) load(1, f1);
         uint32_t it = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+        auto produce = [&](int j, StageFactors<NV> &cur) -> bool {
+            const int tile = (int)blockIdx.x + (j / kblocks) * (int)gridDim.x, kb = j % kblocks;
             const int m0 = (tile % mt) * BM, n0 = (tile / mt) * BN;
-            for (int kb = 0; kb < kblocks; ++kb, ++it) {
-                const uint32_t s = it % STAGES, u = it / STAGES;
-                if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&sm->empty[s]), (u & 1) ^ 1, ctl, SITE_PRODUCER))) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t fb = smem_u32(&sm->full[s]);
-                const uint32_t st = sbase + s * F::STAGE_BYTES;
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
-                    tma_load_2d(st, &tmap_a, fb, kb * BKB, m0);
-                    tma_load_2d(st + A_BYTES, &tmap_b, fb, kb * BKB, n0);
-                }
-                const uint32_t sf_dst = st + A_BYTES + B_BYTES;
-                stage_factors<NV>(sfa, M, m0, ld_sf, kb, lane, sf_dst);
-                stage_factors<NV>(sfb, N, n0, ld_sf, kb, lane, sf_dst + F::G * ATOM);
-                fence_proxy_async_smem();  // the factors are read by tcgen05.cp (async proxy)
-                mbar_arrive(fb);
+            const uint32_t s = it % STAGES, u = it / STAGES;
+            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&sm->empty[s]), (u & 1) ^ 1, ctl, SITE_PRODUCER)))
+                return false;
+            const uint32_t fb = smem_u32(&sm->full[s]);
+            const uint32_t st = sbase + s * F::STAGE_BYTES;
+            if (lane == 0) {
+                mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
+                tma_load_2d(st, &tmap_a, fb, kb * BKB, m0);
+                tma_load_2d(st + A_BYTES, &tmap_b, fb, kb * BKB, n0);
             }
+            ++it;
+            const uint32_t sf_dst = st + A_BYTES + B_BYTES;
+            store_factor_rows<NV>(cur.a, lane, sf_dst);
+            store_factor_rows<NV>(cur.b, lane, sf_dst + F::G * ATOM);
+            fence_proxy_async_smem();  // the factors are read by tcgen05.cp (async proxy)
+            mbar_arrive(fb);
+            if (j + 2 < nstages) load(j + 2, cur);
+            return true;
+        };
+        for (int j = 0; j < nstages; j += 2) {
+            if (!produce(j, f0)) break;
+            if (j + 1 < nstages && !produce(j + 1, f1)) break;
         }
         // Every issued TMA load must land before the CTA may exit.
         if (lane == 0) {
