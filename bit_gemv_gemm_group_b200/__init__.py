@@ -20,7 +20,7 @@ __all__ = ["WQError", "lib", "quantize_group_int4", "quantize_int8_per_channel",
            "smooth", "smooth_workspace_bytes", "smooth_noalloc", "gemv_w4a16", "gemm_w4a16", "gemm_w8a8", "gemv_w8a16",
            "matmul_w4a16", "quantize_fp8_e4m3", "gemm_fp8", "outlier_columns", "gather_outliers",
            "gemm_w8a8_outliers", "llm_int8_matmul", "quantize_mxfp4", "quantize_nvfp4", "gemm_fp4",
-           "device_status", "set_wait_limit",
+           "gemv_w4a16_bf16", "gemm_w4a16_bf16", "hessian", "gptq_prepare", "gptq_quantize", "awq", "device_status", "set_wait_limit",
            "selftest_wait_timeout", "LIB_PATH"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libwq.so")
@@ -61,6 +61,12 @@ _SIGS = {
     "wq_quantize_mxfp4": [_P, _I, _I, _P, _P, _P],
     "wq_quantize_nvfp4": [_P, _I, _I, _P, _P, _P, _P],
     "wq_gemm_fp4": [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _P, _P, _P],
+    "wq_hessian": [_P, _I, _I, _P, _P],
+    "wq_gemv_w4a16_bf16": [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P],
+    "wq_gemm_w4a16_bf16": [_P, _I, _P, _P, _P, _I, _I, _I, _P, _P],
+    "wq_gptq_prepare": [_P, _I, _F, _P, _P, _P],
+    "wq_gptq_quantize": [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P],
+    "wq_awq": [_P, _I, _I, _I, _P, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P],
     "wq_device_status": [_P],
     "wq_selftest_wait_timeout": [_P],
 }
@@ -72,6 +78,10 @@ lib.wq_last_error.argtypes = []
 lib.wq_last_error.restype = ctypes.c_char_p
 lib.wq_smooth_workspace_bytes.argtypes = [_I]
 lib.wq_smooth_workspace_bytes.restype = ctypes.c_size_t
+lib.wq_gptq_workspace_bytes.argtypes = [_I]
+lib.wq_gptq_workspace_bytes.restype = ctypes.c_size_t
+lib.wq_awq_workspace_bytes.argtypes = [_I, _I]
+lib.wq_awq_workspace_bytes.restype = ctypes.c_size_t
 lib.wq_set_wait_limit.argtypes = [ctypes.c_uint64]
 lib.wq_set_wait_limit.restype = None
 
@@ -201,8 +211,8 @@ def smooth_noalloc(x: torch.Tensor, w: torch.Tensor, alpha: float = 0.5, s: torc
 # --------------------------------------------------------------------------
 # matmuls
 # --------------------------------------------------------------------------
-def _w4_args(x, qweight, scales, qzeros, group_size):
-    _cuda(x, "x", (torch.float16,), 2)
+def _w4_args(x, qweight, scales, qzeros, group_size, xdtype=torch.float16):
+    _cuda(x, "x", (xdtype,), 2)
     _cuda(qweight, "qweight", (torch.int32,), 2)
     _cuda(scales, "scales", (torch.float16,), 2)
     _cuda(qzeros, "qzeros", (torch.int32,), 2)
@@ -234,6 +244,26 @@ def gemm_w4a16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stre
     _cuda(y, "out", (torch.float16,), 2)
     _check(lib.wq_gemm_w4a16(_ptr(x), M, _ptr(qweight), _ptr(scales), _ptr(qzeros), N, K, group_size, _ptr(y),
                              _P(_stream(stream))), "wq_gemm_w4a16")
+    return y
+
+
+def gemv_w4a16_bf16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stream=None):
+    """bf16 y [B, N] = x [B, K] (bf16) @ dequant(W)^T for B = 1..8."""
+    B, N, K = _w4_args(x, qweight, scales, qzeros, group_size, torch.bfloat16)
+    y = out if out is not None else _empty((B, N), torch.bfloat16, x)
+    _cuda(y, "out", (torch.bfloat16,), 2)
+    _check(lib.wq_gemv_w4a16_bf16(_ptr(x), B, _ptr(qweight), _ptr(scales), _ptr(qzeros), N, K, group_size, _ptr(y),
+                                  _P(_stream(stream))), "wq_gemv_w4a16_bf16")
+    return y
+
+
+def gemm_w4a16_bf16(x, qweight, scales, qzeros, group_size: int = 128, out=None, stream=None):
+    """bf16 y [M, N] = x [M, K] (bf16) @ dequant(W)^T for M >= 9."""
+    M, N, K = _w4_args(x, qweight, scales, qzeros, group_size, torch.bfloat16)
+    y = out if out is not None else _empty((M, N), torch.bfloat16, x)
+    _cuda(y, "out", (torch.bfloat16,), 2)
+    _check(lib.wq_gemm_w4a16_bf16(_ptr(x), M, _ptr(qweight), _ptr(scales), _ptr(qzeros), N, K, group_size, _ptr(y),
+                                  _P(_stream(stream))), "wq_gemm_w4a16_bf16")
     return y
 
 
@@ -410,6 +440,61 @@ def gemm_fp4(a, sfa, b, sfb, ta=None, tb=None, out=None, return_acc: bool = Fals
     _check(lib.wq_gemm_fp4(1 if nv else 0, _ptr(a), _ptr(sfa), _ptr(ta), _ptr(b), _ptr(sfb), _ptr(tb), M, N, K,
                            _ptr(y), _ptr(acc), _P(_stream(stream))), "wq_gemm_fp4")
     return (y, acc) if return_acc else y
+
+
+def hessian(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """H = 2 X^T X (fp32 [K, K]) from fp16 calibration activations x [T, K]."""
+    _cuda(x, "x", (torch.float16,), 2)
+    T, K = x.shape
+    H = _empty((K, K), torch.float32, x)
+    _check(lib.wq_hessian(_ptr(x), T, K, _ptr(H), _P(_stream(stream))), "wq_hessian")
+    return H
+
+
+def gptq_prepare(H: torch.Tensor, damp: float = 0.01, stream=None) -> torch.Tensor:
+    """U (fp32 [K, K], upper) with U^T U = (H + damp * mean(diag H) I)^-1."""
+    _cuda(H, "H", (torch.float32,), 2)
+    K = H.shape[0]
+    U = _empty((K, K), torch.float32, H)
+    ws = _empty((max(16, int(lib.wq_gptq_workspace_bytes(K))),), torch.uint8, H)
+    _check(lib.wq_gptq_prepare(_ptr(H), K, float(damp), _ptr(U), _ptr(ws), _P(_stream(stream))), "wq_gptq_prepare")
+    return U
+
+
+def gptq_quantize(w: torch.Tensor, U: torch.Tensor, group_size: int = 128, stream=None):
+    """GPTQ of fp16 w [N, K] given U -> (qweight int32 [N, K/8], scales fp16 [N, K/g], qzeros int32)."""
+    _cuda(w, "w", (torch.float16,), 2)
+    _cuda(U, "U", (torch.float32,), 2)
+    N, K = w.shape
+    G = K // group_size
+    work = _empty((N * K + N * 128,), torch.float32, w)
+    qw = _empty((N, K // 8), torch.int32, w)
+    sc = _empty((N, G), torch.float16, w)
+    qz = _empty((N, (G + 7) // 8), torch.int32, w)
+    _check(lib.wq_gptq_quantize(_ptr(w), N, K, group_size, _ptr(U), _ptr(work), _ptr(qw), _ptr(sc), _ptr(qz),
+                                _P(_stream(stream))), "wq_gptq_quantize")
+    return qw, sc, qz
+
+
+def awq(w: torch.Tensor, x: torch.Tensor, grid=None, group_size: int = 128, stream=None):
+    """AWQ's scaling search -> (qweight, scales, qzeros of W diag(s), s fp32 [K], err fp64 [len(grid)], best int32 [1])."""
+    _cuda(w, "w", (torch.float16,), 2)
+    _cuda(x, "x", (torch.float16,), 2)
+    N, K = w.shape
+    T = x.shape[0]
+    g = [i / 10 for i in range(11)] if grid is None else [float(a) for a in grid]
+    garr = (ctypes.c_double * len(g))(*g)
+    G = K // group_size
+    qw = _empty((N, K // 8), torch.int32, w)
+    sc = _empty((N, G), torch.float16, w)
+    qz = _empty((N, (G + 7) // 8), torch.int32, w)
+    s = _empty((K,), torch.float32, w)
+    err = _empty((len(g),), torch.float64, w)
+    best = _empty((1,), torch.int32, w)
+    ws = _empty((max(16, int(lib.wq_awq_workspace_bytes(N, K))),), torch.uint8, w)
+    _check(lib.wq_awq(_ptr(w), N, K, group_size, _ptr(x), T, garr, len(g), _ptr(qw), _ptr(sc), _ptr(qz), _ptr(s),
+                      _ptr(err), _ptr(best), _ptr(ws), _P(_stream(stream))), "wq_awq")
+    return qw, sc, qz, s, err, best
 
 
 def device_status(stream=None) -> int:

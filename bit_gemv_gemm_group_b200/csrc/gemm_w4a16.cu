@@ -133,6 +133,28 @@ __device__ __forceinline__ uint4 dequant_word(uint32_t w, uint32_t zc, uint32_t 
     return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// bf16 tiles: q - z exactly in fp16 as above, then the product with the fp32 scale rounded once to
+// bf16 (bf16_rn(s (q - z)); s is the stored fp16 value, exact in fp32).
+__device__ __forceinline__ uint4 dequant_word_bf16(uint32_t w, uint32_t zc, float s) {
+    const uint32_t c1 = 0x2C003C00u;  // (1.0, 0.0625)
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t y = prmt(w, 0u, 0x4040u + 0x0101u * i);
+        const uint32_t h = (y & 0x00F0000Fu) | 0x64006400u;
+        const float2 d = half2_bits_to_float2(hfma2(h, c1, zc));
+        uint32_t b;
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(b) : "f"(__fmul_rn(d.y, s)), "f"(__fmul_rn(d.x, s)));
+        o[i] = b;
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+template <bool BF>
+__device__ __forceinline__ uint16_t store_bits(float v) {
+    return BF ? float_to_bf16_bits_rn(v) : float_to_half_bits_rn(v);
+}
+
 // Columns [c, c + 16) of the tile's accumulator for this warp's 32 TMEM lanes:
 // the even-stage accumulator, plus the odd-stage one (MT columns further) when
 // the second issuer ran.
@@ -152,7 +174,8 @@ __device__ __forceinline__ void load_acc16(uint32_t t_row, int c, int mt, bool t
     }
 }
 
-template <int MT, bool SB>
+// BF: bf16 activations, dequantized bf16 tiles (kind::f16 with bf16 operands) and bf16 output.
+template <int MT, bool SB, bool BF = false>
 __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     gemm_w4a16_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_x,
                       const uint16_t *__restrict__ scales, const uint32_t *__restrict__ qzeros,
@@ -171,7 +194,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     const int nkb = kb_total / splits;
     const int kb0 = rank * nkb;
     const int groups = K / gs, zwords = (groups + 7) / 8;
-    constexpr uint32_t IDESC = make_idesc(/*f32*/ 1, /*f16*/ 0, /*f16*/ 0, BMW, MT);
+    constexpr uint32_t IDESC = make_idesc(/*f32*/ 1, /*f16 or bf16*/ BF ? 1 : 0, BF ? 1 : 0, BMW, MT);
     constexpr uint32_t TMEM_COLS = 2 * MT;  // two MT-column accumulators; MT >= 16
 
     if (threadIdx.x == 0) {
@@ -293,7 +316,8 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint4 o = dequant_word(ws[j], zc, s2);
+                const uint4 o = BF ? dequant_word_bf16(ws[j], zc, half_bits_to_float((uint16_t)(s2 & 0xFFFFu)))
+                                   : dequant_word(ws[j], zc, s2);
                 const int chunk = half * 4 + j;
                 asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst + ((chunk ^ sw) << 4)), "r"(o.x),
                              "r"(o.y), "r"(o.z), "r"(o.w)
@@ -328,7 +352,8 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
                 const uint32_t ws[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    const uint4 o = dequant_word(ws[j], zc, s2);
+                    const uint4 o = BF ? dequant_word_bf16(ws[j], zc, half_bits_to_float((uint16_t)(s2 & 0xFFFFu)))
+                                   : dequant_word(ws[j], zc, s2);
                     const int chunk = half * 4 + j;
                     asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst + ((chunk ^ sw) << 4)), "r"(o.x),
                                  "r"(o.y), "r"(o.z), "r"(o.w)
@@ -425,7 +450,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
                         if (m0 + c + j < M)
-                            y[(size_t)(m0 + c + j) * N + n] = float_to_half_bits_rn(__uint_as_float(r[j]));
+                            y[(size_t)(m0 + c + j) * N + n] = store_bits<BF>(__uint_as_float(r[j]));
                 }
             }
         }
@@ -464,7 +489,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
                 if (n < N && have_acc) {
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        if (m0 + c + j < M) y[(size_t)(m0 + c + j) * N + n] = float_to_half_bits_rn(acc[j]);
+                        if (m0 + c + j < M) y[(size_t)(m0 + c + j) * N + n] = store_bits<BF>(acc[j]);
                 }
             }
         }
@@ -477,10 +502,10 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     }
 }
 
-template <int MT, bool SB>
+template <int MT, bool SB, bool BF>
 wq_status launch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t *scales, const uint32_t *qzeros,
                  uint16_t *y, int M, int N, int K, int gs, int splits, unsigned int *status, cudaStream_t st) {
-    auto kern = gemm_w4a16_kernel<MT, SB>;
+    auto kern = gemm_w4a16_kernel<MT, SB, BF>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Layout<MT>::SMEM);
     if (e != cudaSuccess) return fail(WQ_ERR_CUDA, "wq_gemm_w4a16: cudaFuncSetAttribute: %s", cudaGetErrorString(e));
@@ -525,7 +550,7 @@ int choose_splits(int tiles, int K, int MT, bool fast, bool generic, size_t pipe
     return best;
 }
 
-template <int MT>
+template <int MT, bool BF>
 wq_status dispatch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t *scales, const uint32_t *qzeros,
                    uint16_t *y, int M, int N, int K, int gs, unsigned int *status, cudaStream_t st) {
     const bool fast = gs == 128 && (K % 1024) == 0;
@@ -533,35 +558,42 @@ wq_status dispatch(const CUtensorMap &tq, const CUtensorMap &tx, const uint16_t 
     const int splits = choose_splits(tiles, K, MT, fast, gs != 128, Layout<MT>::PIPE_BYTES,
                                      Layout<MT>::CTAS_PER_SM * num_sms());
     if (fast && (K / BK / splits) % 16 == 0)
-        return launch<MT, true>(tq, tx, scales, qzeros, y, M, N, K, gs, splits, status, st);
-    return launch<MT, false>(tq, tx, scales, qzeros, y, M, N, K, gs, splits, status, st);
+        return launch<MT, true, BF>(tq, tx, scales, qzeros, y, M, N, K, gs, splits, status, st);
+    return launch<MT, false, BF>(tq, tx, scales, qzeros, y, M, N, K, gs, splits, status, st);
 }
 
 }  // namespace
 }  // namespace wq
 
-extern "C" wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
-                                   const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y, void *stream) {
-    using namespace wq;
+namespace wq {
+namespace {
+
+template <bool BF>
+wq_status gemm_w4a16_entry(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
+                           const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y, void *stream,
+                           const char *who) {
     WQ_REQUIRE_PTR(x, "x");
     WQ_REQUIRE_PTR(qweight, "qweight");
     WQ_REQUIRE_PTR(scales, "scales");
     WQ_REQUIRE_PTR(qzeros, "qzeros");
     WQ_REQUIRE_PTR(y, "y");
-    WQ_REQUIRE(M > 0 && N > 0 && K > 0, WQ_ERR_INVALID_ARG, "wq_gemm_w4a16: sizes must be positive (M=%d N=%d K=%d)",
-               M, N, K);
+    WQ_REQUIRE(M > 0 && N > 0 && K > 0, WQ_ERR_INVALID_ARG, "%s: sizes must be positive (M=%d N=%d K=%d)", who, M, N,
+               K);
     WQ_REQUIRE(group_size == 32 || group_size == 64 || group_size == 128 || group_size == 256, WQ_ERR_UNSUPPORTED,
-               "wq_gemm_w4a16: group_size must be 32, 64, 128 or 256 (got %d)", group_size);
-    WQ_REQUIRE(K % group_size == 0, WQ_ERR_INVALID_ARG, "wq_gemm_w4a16: K (%d) must be a multiple of group_size (%d)",
-               K, group_size);
-    WQ_REQUIRE(K % 128 == 0, WQ_ERR_INVALID_ARG, "wq_gemm_w4a16: K (%d) must be a multiple of 128", K);
-    WQ_REQUIRE(M >= 16 || (M >= 9 && (K % 256 == 0 || group_size != 128)), WQ_ERR_UNSUPPORTED,
-               "wq_gemm_w4a16: M (%d) below 16 needs K %% 256 == 0 (K = %d); use wq_gemv_w4a16 for M <= 8", M, K);
-    // Other group sizes below 16 rows: the CUDA-core GEMV kernel in passes of up to 8 rows.
-    if (group_size != 128 && M < 16) {
+               "%s: group_size must be 32, 64, 128 or 256 (got %d)", who, group_size);
+    WQ_REQUIRE(K % group_size == 0, WQ_ERR_INVALID_ARG, "%s: K (%d) must be a multiple of group_size (%d)", who, K,
+               group_size);
+    WQ_REQUIRE(K % 128 == 0, WQ_ERR_INVALID_ARG, "%s: K (%d) must be a multiple of 128", who, K);
+    const bool stream_ok = !BF && group_size == 128 && K % 256 == 0;  // the fp16 streaming kernel
+    WQ_REQUIRE(M >= 16 || (M >= 9 && (K % 256 == 0 || group_size != 128 || BF)), WQ_ERR_UNSUPPORTED,
+               "%s: M (%d) below 16 needs K %% 256 == 0 (K = %d); use the GEMV for M <= 8", who, M, K);
+    // Below 16 rows without the streaming kernel: the CUDA-core GEMV in passes of up to 8 rows.
+    if (M < 16 && !stream_ok) {
         for (int r0 = 0; r0 < M; r0 += 8) {
-            const wq_status e = wq_gemv_w4a16(x + (size_t)r0 * K, std::min(8, M - r0), qweight, scales, qzeros, N, K,
-                                              group_size, y + (size_t)r0 * N, stream);
+            const wq_status e = BF ? wq_gemv_w4a16_bf16(x + (size_t)r0 * K, std::min(8, M - r0), qweight, scales,
+                                                        qzeros, N, K, group_size, y + (size_t)r0 * N, stream)
+                                   : wq_gemv_w4a16(x + (size_t)r0 * K, std::min(8, M - r0), qweight, scales, qzeros,
+                                                   N, K, group_size, y + (size_t)r0 * N, stream);
             if (e != WQ_OK) return e;
         }
         return WQ_OK;
@@ -571,10 +603,10 @@ extern "C" wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qwe
     // serves 9 <= M < 16, which the tensor-core kernel below does not take) and, measured
     // on B200, beats the tensor-core kernel below at M <= 32 (2 passes at M = 32 take 0.36x its
     // time on the 28672x8192 projection; at three passes the two are even).
-    if (group_size == 128 && M <= 32 && K % 256 == 0) {
+    if (stream_ok && M <= 32) {
         for (int r0 = 0; r0 < M; r0 += 16) {
             const wq_status e = gemv_stream(x + (size_t)r0 * K, std::min(16, M - r0), qweight, scales, qzeros, N, K,
-                                            y + (size_t)r0 * N, as_stream(stream), "wq_gemm_w4a16");
+                                            y + (size_t)r0 * N, as_stream(stream), who);
             if (e != WQ_OK) return e;
         }
         return WQ_OK;
@@ -586,14 +618,29 @@ extern "C" wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qwe
     if (!encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qweight, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
                         BK / 2, BMW, CU_TENSOR_MAP_SWIZZLE_NONE))
         return WQ_ERR_CUDA;
-    if (!encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, BK,
-                        MT, CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_tmap_2d(&tx, BF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, (uint64_t)K,
+                        (uint64_t)M, (uint64_t)K * 2, BK, MT, CU_TENSOR_MAP_SWIZZLE_128B))
         return WQ_ERR_CUDA;
     cudaStream_t st = as_stream(stream);
     switch (MT) {
-        case 16: return dispatch<16>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
-        case 32: return dispatch<32>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
-        case 64: return dispatch<64>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
-        default: return dispatch<128>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
+        case 16: return dispatch<16, BF>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
+        case 32: return dispatch<32, BF>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
+        case 64: return dispatch<64, BF>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
+        default: return dispatch<128, BF>(tq, tx, scales, qzeros, y, M, N, K, group_size, status, st);
     }
+}
+
+}  // namespace
+}  // namespace wq
+
+extern "C" wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
+                                   const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y, void *stream) {
+    return wq::gemm_w4a16_entry<false>(x, M, qweight, scales, qzeros, N, K, group_size, y, stream, "wq_gemm_w4a16");
+}
+
+extern "C" wq_status wq_gemm_w4a16_bf16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
+                                        const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y,
+                                        void *stream) {
+    return wq::gemm_w4a16_entry<true>(x, M, qweight, scales, qzeros, N, K, group_size, y, stream,
+                                      "wq_gemm_w4a16_bf16");
 }

@@ -78,7 +78,12 @@ __device__ __forceinline__ Unpacked unpack_word(uint32_t w, const ZeroOffsets &o
     return r;
 }
 
-template <int B, int R>
+// Activations and output in fp16, or in bf16 (BF: x = bits << 16 as fp32, exact; y rounded to bf16).
+__device__ __forceinline__ float2 bf16x2_bits_to_float2(uint32_t b) {
+    return make_float2(__uint_as_float(b << 16), __uint_as_float(b & 0xFFFF0000u));
+}
+
+template <int B, int R, bool BF = false>
 __global__ void __launch_bounds__(kWarps * 32) gemv_w4a16_kernel(const uint16_t *__restrict__ x,
                                                                  const uint32_t *__restrict__ qweight,
                                                                  const uint16_t *__restrict__ scales,
@@ -119,10 +124,10 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_w4a16_kernel(const uint16_t 
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
                 const uint4 xv = ld_shared_ro_u4(xp + 8 * v);
-                xf[4 * v + 0] = half2_bits_to_float2(xv.x);
-                xf[4 * v + 1] = half2_bits_to_float2(xv.y);
-                xf[4 * v + 2] = half2_bits_to_float2(xv.z);
-                xf[4 * v + 3] = half2_bits_to_float2(xv.w);
+                xf[4 * v + 0] = BF ? bf16x2_bits_to_float2(xv.x) : half2_bits_to_float2(xv.x);
+                xf[4 * v + 1] = BF ? bf16x2_bits_to_float2(xv.y) : half2_bits_to_float2(xv.y);
+                xf[4 * v + 2] = BF ? bf16x2_bits_to_float2(xv.z) : half2_bits_to_float2(xv.z);
+                xf[4 * v + 3] = BF ? bf16x2_bits_to_float2(xv.w) : half2_bits_to_float2(xv.w);
             }
 #pragma unroll
             for (int r = 0; r < R; ++r) {
@@ -152,7 +157,9 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_w4a16_kernel(const uint16_t 
         for (int r = 0; r < R; ++r) {
             if (row0 + r < N) {
 #pragma unroll
-                for (int b = 0; b < B; ++b) y[(size_t)b * N + row0 + r] = float_to_half_bits_rn(acc[r][b]);
+                for (int b = 0; b < B; ++b)
+                    y[(size_t)b * N + row0 + r] =
+                        BF ? float_to_bf16_bits_rn(acc[r][b]) : float_to_half_bits_rn(acc[r][b]);
             }
         }
     }
@@ -897,22 +904,22 @@ cudaError_t launch_mma(const uint16_t *x, int B, const uint32_t *qw, const uint1
     return cudaGetLastError();
 }
 
-template <int B, int R>
+template <int B, int R, bool BF>
 cudaError_t launch_br(const uint16_t *x, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
                       int K, int g, uint16_t *y, cudaStream_t st) {
     const int rows_per_block = kWarps * R;
     const int blocks = (N + rows_per_block - 1) / rows_per_block;
-    gemv_w4a16_kernel<B, R><<<blocks, kWarps * 32, 0, st>>>(x, qw, sc, qz, N, K, g, y);
+    gemv_w4a16_kernel<B, R, BF><<<blocks, kWarps * 32, 0, st>>>(x, qw, sc, qz, N, K, g, y);
     return cudaGetLastError();
 }
 
-template <int B>
+template <int B, bool BF = false>
 cudaError_t launch_b(const uint16_t *x, const uint32_t *qw, const uint16_t *sc, const uint32_t *qz, int N,
                      int K, int g, uint16_t *y, cudaStream_t st) {
     // Two rows per warp when that still gives every SM several CTAs.
     const long long blocks2 = (N + kWarps * 2 - 1) / (kWarps * 2);
-    if (blocks2 >= 6ll * num_sms()) return launch_br<B, 2>(x, qw, sc, qz, N, K, g, y, st);
-    return launch_br<B, 1>(x, qw, sc, qz, N, K, g, y, st);
+    if (blocks2 >= 6ll * num_sms()) return launch_br<B, 2, BF>(x, qw, sc, qz, N, K, g, y, st);
+    return launch_br<B, 1, BF>(x, qw, sc, qz, N, K, g, y, st);
 }
 
 }  // namespace
@@ -955,5 +962,38 @@ extern "C" wq_status wq_gemv_w4a16(const uint16_t *x, int B, const uint32_t *qwe
         default: e = wq::launch_b<8>(x, qweight, scales, qzeros, N, K, group_size, y, st); break;
     }
     if (e != cudaSuccess) return wq::fail(WQ_ERR_CUDA, "wq_gemv_w4a16: launch failed: %s", cudaGetErrorString(e));
+    return WQ_OK;
+}
+
+// bf16 activations and output, any group size: the CUDA-core kernel (fp32 products of the exact
+// q - z and the exactly converted x, group scale applied in fp32, one rounding to bf16 at the end).
+extern "C" wq_status wq_gemv_w4a16_bf16(const uint16_t *x, int B, const uint32_t *qweight, const uint16_t *scales,
+                                        const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y,
+                                        void *stream) {
+    WQ_REQUIRE_PTR(x, "x");
+    WQ_REQUIRE_PTR(qweight, "qweight");
+    WQ_REQUIRE_PTR(scales, "scales");
+    WQ_REQUIRE_PTR(qzeros, "qzeros");
+    WQ_REQUIRE_PTR(y, "y");
+    WQ_REQUIRE(N > 0 && K > 0, WQ_ERR_INVALID_ARG, "wq_gemv_w4a16_bf16: N and K must be positive (N=%d K=%d)", N, K);
+    WQ_REQUIRE(B >= 1 && B <= 8, WQ_ERR_UNSUPPORTED, "wq_gemv_w4a16_bf16: B must be 1..8 (got %d)", B);
+    WQ_REQUIRE(group_size == 32 || group_size == 64 || group_size == 128 || group_size == 256, WQ_ERR_UNSUPPORTED,
+               "wq_gemv_w4a16_bf16: group_size must be 32, 64, 128 or 256 (got %d)", group_size);
+    WQ_REQUIRE(K % group_size == 0, WQ_ERR_INVALID_ARG,
+               "wq_gemv_w4a16_bf16: K (%d) must be a multiple of group_size (%d)", K, group_size);
+    cudaStream_t st = wq::as_stream(stream);
+    cudaError_t e;
+    switch (B) {
+        case 1: e = wq::launch_b<1, true>(x, qweight, scales, qzeros, N, K, group_size, y, st); break;
+        case 2: e = wq::launch_b<2, true>(x, qweight, scales, qzeros, N, K, group_size, y, st); break;
+        case 3: e = wq::launch_b<3, true>(x, qweight, scales, qzeros, N, K, group_size, y, st); break;
+        case 4: e = wq::launch_b<4, true>(x, qweight, scales, qzeros, N, K, group_size, y, st); break;
+        case 5: e = wq::launch_b<5, true>(x, qweight, scales, qzeros, N, K, group_size, y, st); break;
+        case 6: e = wq::launch_b<6, true>(x, qweight, scales, qzeros, N, K, group_size, y, st); break;
+        case 7: e = wq::launch_b<7, true>(x, qweight, scales, qzeros, N, K, group_size, y, st); break;
+        default: e = wq::launch_b<8, true>(x, qweight, scales, qzeros, N, K, group_size, y, st); break;
+    }
+    if (e != cudaSuccess)
+        return wq::fail(WQ_ERR_CUDA, "wq_gemv_w4a16_bf16: launch failed: %s", cudaGetErrorString(e));
     return WQ_OK;
 }

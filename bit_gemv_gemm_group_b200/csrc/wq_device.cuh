@@ -2,6 +2,7 @@
 // cache hints and fp16 bit handling.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
 
@@ -35,6 +36,10 @@ __device__ __forceinline__ float2 half2_bits_to_float2(uint32_t b) {
 
 __device__ __forceinline__ uint16_t float_to_half_bits_rn(float f) {
     return __half_as_ushort(__float2half_rn(f));
+}
+
+__device__ __forceinline__ uint16_t float_to_bf16_bits_rn(float f) {
+    return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
 __device__ __forceinline__ int clampi(int v, int lo, int hi) { return min(max(v, lo), hi); }

@@ -201,6 +201,23 @@ wq_status wq_gemm_w4a16(const uint16_t *x, int M, const uint32_t *qweight, const
                         void *stream);
 
 /*
+ * bf16 activations (the variants bf16 models call): same packed weights,
+ * arithmetic and arguments as wq_gemv_w4a16 / wq_gemm_w4a16, with x and y
+ * bf16 bit patterns instead of fp16.  The GEMV (B = 1..8, any group size)
+ * multiplies the exact q - z by the exactly converted x in fp32 and applies
+ * each group's scale in fp32; the GEMM's tensor-core path rounds each
+ * dequantized weight s (q - z) to bf16 (tcgen05 kind::f16 with bf16
+ * operands).  y is rounded to bf16 once, so the error is within
+ * 2^-8 * sum_k |w^ x| (bf16 output and, for the GEMM, bf16 weights) on top
+ * of the fp32 accumulation.  Preconditions as for the fp16 functions (the
+ * GEMM below 16 rows runs the bf16 GEMV in passes of 8 rows).
+ */
+wq_status wq_gemv_w4a16_bf16(const uint16_t *x, int B, const uint32_t *qweight, const uint16_t *scales,
+                             const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y, void *stream);
+wq_status wq_gemm_w4a16_bf16(const uint16_t *x, int M, const uint32_t *qweight, const uint16_t *scales,
+                             const uint32_t *qzeros, int N, int K, int group_size, uint16_t *y, void *stream);
+
+/*
  * W8A8 INT8 GEMM on the tensor cores with a fused dequantization epilogue.
  * Source: [P4] "How does quantized matrix multiplication actually run on the
  * GPU?" (int8 operands, exact 32-bit accumulation; symmetric scales make the
@@ -343,6 +360,53 @@ wq_status wq_quantize_nvfp4(const uint16_t *x, int R, int K, uint8_t *q, uint8_t
 wq_status wq_gemm_fp4(int nvfp4, const uint8_t *a, const uint8_t *sfa, const float *ta, const uint8_t *b,
                       const uint8_t *sfb, const float *tb, int M, int N, int K, uint16_t *y, float *acc_out,
                       void *stream);
+
+/*
+ * Calibration-driven INT4 (GPTQ and AWQ), producing the stored INT4 format of
+ * wq_quantize_group_int4 (group size 128).  Source: [P3] "GPTQ: rounding with
+ * error compensation", "AWQ: protect the channels that matter" and the
+ * gptq() / awq() routines of "Measured on two real layers"; [P2] "The
+ * Mathematics" (H = 2 X^T X).  A group's grid is the stored-format rule of
+ * wq_quantize_group_int4 applied to the fp32 values it quantizes.  These are
+ * fp32 GPU computations: their codes follow the fp64 reference closely but
+ * not bit for bit (compensation rounds differently), except where no
+ * compensation happens (U = identity gives round-to-nearest exactly).
+ *
+ * wq_hessian: H = 2 X^T X, fp32 [K][K], from fp16 calibration activations
+ * x [T][K].
+ *
+ * wq_gptq_prepare: U = upper Cholesky factor of (H + damp * mean(diag H) I)^-1,
+ * fp32 [K][K] (U^T U = that inverse), via the Cholesky factor of the
+ * index-reversed matrix and its inverse.  K % 64 == 0; damp >= 0 (the pages
+ * use 0.01); H must be symmetric and H + damping positive definite.
+ * workspace: wq_gptq_workspace_bytes(K) bytes, 16-byte aligned.
+ *
+ * wq_gptq_quantize: GPTQ of fp16 w [N][K] given U: one column at a time in
+ * blocks of 128 columns (one group), each block's grid from its compensated
+ * weights, each column's scaled error e = (w - (q - z) s) / U[i][i] pushed
+ * onto the block's later columns and, after the block, onto the columns after
+ * it.  work: fp32 scratch of N * K + N * 128 floats.  group_size == 128,
+ * K % 128 == 0.
+ *
+ * wq_awq: AWQ's scaling search.  mag_j = mean_t |x[t][j]|; for each alpha of
+ * the host array grid[0..ngrid): s_j = fp32(mag_j^alpha / sqrt(max * min))
+ * (fp64 powers), codes = round-to-nearest of the fp32 products w[n][j] * s_j,
+ * D = w - dequant / s, err[a] = 2 ||x D^T||^2 (the calibration objective
+ * sum_n D H D^T); the first alpha with the smallest err wins.  Outputs (device):
+ * qweight/scales/qzeros of W diag(s) for the winner (serve it with x / s),
+ * s fp32 [K], err fp64 [ngrid], best int [1].  workspace:
+ * wq_awq_workspace_bytes(N, K) bytes.  group_size == 128, K % 128 == 0,
+ * 1 <= ngrid <= 64.
+ */
+wq_status wq_hessian(const uint16_t *x, int T, int K, float *H, void *stream);
+size_t wq_gptq_workspace_bytes(int K);
+wq_status wq_gptq_prepare(const float *H, int K, float damp, float *U, void *workspace, void *stream);
+wq_status wq_gptq_quantize(const uint16_t *w, int N, int K, int group_size, const float *U, float *work,
+                           uint32_t *qweight, uint16_t *scales, uint32_t *qzeros, void *stream);
+size_t wq_awq_workspace_bytes(int N, int K);
+wq_status wq_awq(const uint16_t *w, int N, int K, int group_size, const uint16_t *x, int T, const double *grid,
+                 int ngrid, uint32_t *qweight, uint16_t *scales, uint32_t *qzeros, float *s, double *err, int *best,
+                 void *workspace, void *stream);
 
 /* Message describing the last error status returned on this host thread. */
 const char *wq_last_error(void);

@@ -790,3 +790,116 @@ def test_w8a8_split_last_round(wq, fp8):
         _, ry2, rb2 = oracle.gemm_w8a8_ref(xq, sx, wq8, sw, ms2, ns2)
     assert_within_bound(host(y)[np.ix_(ms2, ns2)].astype(np.float64), ry2, rb2, f"split round sample fp8={fp8}")
     assert wq.device_status() == 0
+
+
+# --------------------------------------------------------------------------
+# GPTQ and AWQ on the GPU (fp32) against the fp64 oracle: the Hessian and the
+# factor within rounding, GPTQ with U = I exactly round-to-nearest, GPTQ's
+# objective and codes close to the oracle's and below RTN, AWQ's choice,
+# scales and codes exact
+# --------------------------------------------------------------------------
+def _calib_inputs(seed, N=256, K=512, T=512, outliers=()):
+    g = np.random.default_rng(seed)
+    x = g.standard_normal((T, K)).astype(np.float32)
+    x += 0.8 * (g.standard_normal((T, 4)) @ g.standard_normal((4, K))).astype(np.float32)
+    for c in outliers:
+        x[:, c] *= 30.0
+    w = (g.standard_normal((N, K)) * 0.02).astype(np.float32)
+    return x.astype(np.float16), w.astype(np.float16)
+
+
+def _cal_objective(x, w, qw, sc, qz, K, s=None):
+    what = oracle.dequant_int4(qw, sc, qz, K, 128)
+    if s is not None:
+        what = what / s.astype(np.float64)[None, :]
+    d = w.astype(np.float64) - what
+    return float(np.sum((x.astype(np.float64) @ d.T) ** 2))
+
+
+def test_hessian_and_gptq_factor(wq):
+    x, _ = _calib_inputs(61, K=256, T=300)
+    H = wq.hessian(dev(x))
+    U = wq.gptq_prepare(H, 0.01)
+    torch.cuda.synchronize()
+    rH = oracle.hessian(x)
+    assert np.max(np.abs(host(H) - rH)) <= 1e-5 * np.max(np.abs(rH))
+    rU = oracle.gptq_hinv_chol(rH, 0.01)
+    hU = host(U).astype(np.float64)
+    assert np.allclose(np.triu(hU), hU)
+    assert np.linalg.norm(hU - rU) <= 1e-3 * np.linalg.norm(rU)
+
+
+def test_gptq_with_identity_factor_is_round_to_nearest(wq):
+    _, w = _calib_inputs(62)
+    K = w.shape[1]
+    qw, sc, qz = wq.gptq_quantize(dev(w), torch.eye(K, dtype=torch.float32, device="cuda"))
+    torch.cuda.synchronize()
+    rqw, rsc, rqz = oracle.quantize_group_int4(w, 128)
+    assert np.array_equal(host(qw, np.uint32), rqw) and np.array_equal(host(qz, np.uint32), rqz)
+    assert np.array_equal(host(sc).view(np.uint16), rsc.view(np.uint16))
+
+
+def test_gptq_matches_the_oracle_objective(wq):
+    x, w = _calib_inputs(63)
+    K = w.shape[1]
+    U = wq.gptq_prepare(wq.hessian(dev(x)), 0.01)
+    qw, sc, qz = wq.gptq_quantize(dev(w), U)
+    torch.cuda.synchronize()
+    rU = oracle.gptq_hinv_chol(oracle.hessian(x), 0.01)
+    rqw, rsc, rqz = oracle.gptq(w, rU, 128)
+    hqw, hsc, hqz = host(qw, np.uint32), host(sc), host(qz, np.uint32)
+    e_gpu = _cal_objective(x, w, hqw, hsc, hqz, K)
+    e_ref = _cal_objective(x, w, rqw, rsc, rqz, K)
+    tqw, tsc, tqz = oracle.quantize_group_int4(w, 128)
+    e_rtn = _cal_objective(x, w, tqw, tsc, tqz, K)
+    assert abs(e_gpu - e_ref) <= 0.02 * e_ref and e_gpu < 0.8 * e_rtn
+    codes_gpu, codes_ref = oracle.unpack_int4_codes(hqw, K), oracle.unpack_int4_codes(rqw, K)
+    assert np.mean(codes_gpu == codes_ref) >= 0.97
+    assert np.mean(hsc.view(np.uint16) == rsc.view(np.uint16)) >= 0.95
+
+
+def test_awq_matches_the_oracle(wq):
+    x, w = _calib_inputs(64, outliers=(3, 70, 200, 301))
+    K = w.shape[1]
+    qw, sc, qz, s, err, best = wq.awq(dev(w), dev(x))
+    torch.cuda.synchronize()
+    rqw, rsc, rqz, rs, rbest, rerr = oracle.awq(w, x, oracle.hessian(x), 128)
+    assert int(host(best)[0]) == rbest
+    assert np.allclose(host(err), rerr, rtol=1e-4)
+    assert np.array_equal(host(s), rs)
+    assert np.array_equal(host(qw, np.uint32), rqw) and np.array_equal(host(qz, np.uint32), rqz)
+    assert np.array_equal(host(sc).view(np.uint16), rsc.view(np.uint16))
+    assert rbest > 0 and rerr[rbest] < rerr[0]
+
+
+# --------------------------------------------------------------------------
+# bf16 activations: the W4A16 GEMV (any group size) and GEMM (tensor cores with bf16 tiles)
+# against the oracle with bf16 x; bf16 outputs, so the bound is 2^-8 sum |w^ x| + 1e-5
+# (bf16 rounding of the output and, in the GEMM, of each dequantized weight)
+# --------------------------------------------------------------------------
+BF16_RTOL = 2.0 ** -8
+
+BF16_CASES = [  # (kind, M, N, K, g)
+    ("gemv", 1, 300, 1024, 128), ("gemv", 8, 520, 2048, 32), ("gemv", 5, 129, 768, 64), ("gemv", 3, 77, 512, 256),
+    ("gemm", 16, 300, 1024, 128), ("gemm", 64, 1000, 4096, 128), ("gemm", 100, 384, 3072, 64),
+    ("gemm", 12, 300, 1280, 128), ("gemm", 130, 260, 2048, 32), ("gemm", 48, 640, 16384, 256),
+]
+
+
+@pytest.mark.parametrize("kind,M,N,K,g", BF16_CASES)
+def test_w4a16_bf16_activations(wq, kind, M, N, K, g):
+    w = _special_weights(N, K, seed=M + N + K + 7)
+    rqw, rsc, rqz = oracle.quantize_group_int4(w, g)
+    x = workloads.activations(M, K, 0.01, 50.0, seed=M + 1, tensor_id=N).astype(np.float32)
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    xbits = xt.view(torch.int16).numpy().view(np.uint16)
+    f = wq.gemv_w4a16_bf16 if kind == "gemv" else wq.gemm_w4a16_bf16
+    y = f(xt.cuda(), dev(rqw.view(np.int32)), dev(rsc), dev(rqz.view(np.int32)), g)
+    torch.cuda.synchronize()
+    rows = sample_rows(N, 300, seed=K)
+    y_ref, bound = oracle.matmul_w4a16_ref_bf16(xbits, rqw, rsc, rqz, K, g, rows=rows)
+    hy = y.float().cpu().numpy().astype(np.float64)[:, rows]
+    err = np.abs(hy - y_ref)
+    lim = BF16_RTOL * bound + ATOL
+    assert not (err > lim).any(), f"bf16 {kind} M={M} N={N} K={K} g={g}: worst excess {(err - lim).max():.3e}"
+    assert wq.device_status() == 0
