@@ -17,8 +17,10 @@
 // weight: 2 (fp16 in) + 0.5 + 2.5/G (out).  The codes rne(w / s) are decided
 // from w * RN(1/s) with an exact near-tie fallback (rne_quotient), which gives
 // the same integers as the IEEE division at a third of its instructions.
+#include <algorithm>
 #include <type_traits>
 
+#include "sm100.cuh"
 #include "wq_device.cuh"
 #include "wq_host.h"
 
@@ -148,16 +150,17 @@ __device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
 
 // rne(w * rs) + z of an fp16 pair as int16x2, with magic = 1.5 * 2^23 + z: one fused
 // multiply-add rounds w * rs + magic to an integer, which is magic + rne(w * rs) away from a
-// tie (at a tie the parity of z decides, and the guard band below catches it); `bad`
-// collects the sign bit of (1/2 - 2^-16)^2 - d^2 (set when a lane lies in the guard band).
-__device__ __forceinline__ uint32_t pair_rne(uint32_t h2, float rs, float magic, uint32_t &bad) {
+// tie (at a tie the parity of z decides, and the guard band below catches it).  magic - r is
+// exact (Sterbenz), so d = w * rs + (magic - r) is the remainder rounded once; `ok` keeps the
+// sign bit of d^2 - (1/2 - 2^-16)^2, which stays set while no lane lies in the guard band.
+__device__ __forceinline__ uint32_t pair_rne(uint32_t h2, float rs, float magic, uint32_t &ok) {
     constexpr float kGuardSq = (0.5f - 0x1p-16f) * (0.5f - 0x1p-16f);
     const float2 f = half2_bits_to_float2(h2);
     const float2 r = __ffma2_rn(f, make_float2(rs, rs), make_float2(magic, magic));
-    const float2 n = __fadd2_rn(r, make_float2(-magic, -magic));
-    const float2 d = __ffma2_rn(f, make_float2(rs, rs), make_float2(-n.x, -n.y));
-    const float2 e = __ffma2_rn(d, make_float2(-d.x, -d.y), make_float2(kGuardSq, kGuardSq));
-    bad |= __float_as_uint(e.x) | __float_as_uint(e.y);
+    const float2 m = __ffma2_rn(r, make_float2(-1.0f, -1.0f), make_float2(magic, magic));
+    const float2 d = __ffma2_rn(f, make_float2(rs, rs), m);
+    const float2 e = __ffma2_rn(d, d, make_float2(-kGuardSq, -kGuardSq));
+    ok &= __float_as_uint(e.x) & __float_as_uint(e.y);
     return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);  // low 16 bits: rne(t) + z
 }
 
@@ -224,11 +227,11 @@ __global__ void __launch_bounds__(256) quant_int4_group_f16_kernel(const uint16_
         // z = round(-lo / s) in [0, 15]; |-lo / s| and |w / s| stay below 32 (E = 4)
         const int z = clampi(rne_quotient<4>(-lo, s, rs), 0, 15);
         if (j < groups) {
-            uint32_t bad = 0;
+            uint32_t ok = ~0u;
             const float magic = 12582912.0f + (float)z;  // 1.5 * 2^23 + z
-            uint32_t p0 = pair_rne(c.x, rs, magic, bad), p1 = pair_rne(c.y, rs, magic, bad);
-            uint32_t p2 = pair_rne(c.z, rs, magic, bad), p3 = pair_rne(c.w, rs, magic, bad);
-            if (bad >> 31) {  // a near-tie: the IEEE quotient decides every code of this lane
+            uint32_t p0 = pair_rne(c.x, rs, magic, ok), p1 = pair_rne(c.y, rs, magic, ok);
+            uint32_t p2 = pair_rne(c.z, rs, magic, ok), p3 = pair_rne(c.w, rs, magic, ok);
+            if (!(ok >> 31)) {  // a near-tie: the IEEE quotient decides every code of this lane
                 const uint32_t h[4] = {c.x, c.y, c.z, c.w};
                 uint32_t pp[4];
 #pragma unroll
@@ -255,111 +258,244 @@ __global__ void __launch_bounds__(256) quant_int4_group_f16_kernel(const uint16_
     if (lane == 0) qzeros[(size_t)n * zwords + zw] = zword;
 }
 
-// G >= 64: 16 elements (two 16-byte loads) per lane, so the range butterfly,
-// which a warp pays once for all its lanes, is spread over twice the elements;
-// the range travels as one fp16x2 value (-lo, hi) (negation and max are exact
-// in fp16), one shuffle and one max per butterfly step.  The scale and zero
-// point of the warp's 8 groups are then computed once, on lanes 0..7 (one
-// group each), and shuffled to the group's lanes: measured 5% faster on B200
-// than every lane computing its own group's values in each iteration.
+// G >= 64: one warp per (row, unit of 32 E consecutive elements), E = 32
+// elements per lane (E = 64 for G = 256), so a group spans LPG = G / E lanes
+// (2 or 4) and a unit holds whole zero words (one, or two for G = 64).  Each
+// lane loads its E elements with E / 8 16-byte loads issued before any
+// arithmetic, and computes the scale and zero point of its own group itself:
+// nothing is distributed by shuffles and no scalar step runs more than once
+// per unit.  The range is one fp16x2 value (-lo, hi) (negation and max are
+// exact in fp16), reduced over the group's lanes with one shuffle and one max
+// per step.  The grid is (row blocks of 8, units), so no index is divided.
 template <int G>
-__global__ void __launch_bounds__(256) quant_int4_group_f16x16_kernel(const uint16_t *__restrict__ w, int N, int K,
-                                                                      uint32_t *__restrict__ qweight,
-                                                                      uint16_t *__restrict__ scales,
-                                                                      uint32_t *__restrict__ qzeros) {
-    constexpr int LPG = G / 16;      // lanes per group
-    constexpr int GPI = 32 / LPG;    // groups per warp iteration
-    constexpr int ITERS = 8 / GPI;   // iterations per zero word (8 groups)
-    static_assert(ITERS >= 1, "G >= 64");
-    const int groups = K / G;
-    const int zwords = (groups + 7) / 8;
-    const int lane = threadIdx.x & 31;
-    const long long unit = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (unit >= (long long)N * zwords) return;
-    const int n = (int)(unit / zwords);
-    const int zw = (int)(unit % zwords);
-    const int sub = lane / LPG;  // group slot within an iteration
-    const int li = lane % LPG;   // lane within the group
+struct Wide {
+    static constexpr int E = G >= 256 ? 64 : 32;  // elements per lane
+    static constexpr int V = E / 8;               // 16-byte loads (and code words) per lane
+    static constexpr int LPG = G / E;             // lanes per group
+    static constexpr int UE = 32 * E;             // elements per unit
+    static constexpr int ZPU = UE / (8 * G);      // zero words per unit
+    static_assert(G >= 64 && LPG >= 2 && ZPU >= 1, "G in {64, 128, 256}");
+};
 
-    // Issue every load of this warp first.
-    uint4 raw[ITERS][2];
-#pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-        const int j = zw * 8 + it * GPI + sub;
-        const uint16_t *p = w + (size_t)n * K + (size_t)j * G + li * 16;
-        raw[it][0] = j < groups ? ld_stream_u4(p) : make_uint4(0u, 0u, 0u, 0u);
-        raw[it][1] = j < groups ? ld_stream_u4(p + 8) : make_uint4(0u, 0u, 0u, 0u);
-    }
+// RN(d / 15) for a finite fp32 d >= 0 (the scale's quotient (hi - lo) / 15).
+// With d = m 2^e (m a 24-bit integer), m / 15 is either exact or k + r / 15
+// with r in 1..14, whose binary fraction repeats r's four bits forever; the
+// part below an fp32 ulp is then c / 15 of an ulp with c in 1..14, so the
+// quotient is never a tie and stays at least ulp / 30 away from one.  The
+// fp64 product d * RN64(1/15) is within 2^-52 relative (well under 2^-28 ulp)
+// of d / 15, so rounding it to fp32 gives the correctly rounded quotient.
+__device__ __forceinline__ float div15_rn(float d) {
+    return __double2float_rn(__dmul_rn((double)d, 0x1.1111111111111p-4));
+}
 
-    // Range of every group: (-lo, hi) with lo = min(0, min w), hi = max(0, max w), as fp16x2.
-    uint32_t rr[ITERS];
+// One lane's share of a unit: its E weights (raw fp16, zeros past the end) -> its V code
+// words, and the scale and zero point of its group.  Every lane of the warp must call it
+// (the range is reduced across the group's lanes).
+template <int G>
+__device__ __forceinline__ void quantize_lane(const uint4 (&raw)[Wide<G>::V], uint32_t (&words)[Wide<G>::V],
+                                              uint16_t &s16_out, int &z_out) {
+    using P = Wide<G>;
+    // Range of the group, widened to contain 0, as fp16x2 (-lo, hi).
+    uint32_t mn = hmin2_bits(hmin2_bits(raw[0].x, raw[0].y), hmin2_bits(raw[0].z, raw[0].w));
+    uint32_t mx = hmax2_bits(hmax2_bits(raw[0].x, raw[0].y), hmax2_bits(raw[0].z, raw[0].w));
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-        const uint4 c0 = raw[it][0], c1 = raw[it][1];
-        const uint32_t mn = hmin2_bits(hmin2_bits(hmin2_bits(c0.x, c0.y), hmin2_bits(c0.z, c0.w)),
-                                       hmin2_bits(hmin2_bits(c1.x, c1.y), hmin2_bits(c1.z, c1.w)));
-        const uint32_t mx = hmax2_bits(hmax2_bits(hmax2_bits(c0.x, c0.y), hmax2_bits(c0.z, c0.w)),
-                                       hmax2_bits(hmax2_bits(c1.x, c1.y), hmax2_bits(c1.z, c1.w)));
-        uint32_t r = hmax2_bits(__byte_perm(mn, mx, 0x5410) ^ 0x00008000u, __byte_perm(mn, mx, 0x7632) ^ 0x00008000u);
-        r = hmax2_bits(r, 0u);
-#pragma unroll
-        for (int off = LPG / 2; off >= 1; off >>= 1) r = hmax2_bits(r, __shfl_xor_sync(0xffffffffu, r, off));
-        rr[it] = r;
+    for (int v = 1; v < P::V; ++v) {
+        mn = hmin2_bits(mn, hmin2_bits(hmin2_bits(raw[v].x, raw[v].y), hmin2_bits(raw[v].z, raw[v].w)));
+        mx = hmax2_bits(mx, hmax2_bits(hmax2_bits(raw[v].x, raw[v].y), hmax2_bits(raw[v].z, raw[v].w)));
     }
-    // Scale and zero point once per group: lane g (and its copies g + 8, g + 16, g + 24)
-    // takes group g of the zero word, so the scalar work runs once, not once per iteration.
-    const int gl = lane & 7;
-    uint32_t mine = 0;
+    uint32_t r = hmax2_bits(__byte_perm(mn, mx, 0x5410) ^ 0x00008000u, __byte_perm(mn, mx, 0x7632) ^ 0x00008000u);
+    r = hmax2_bits(r, 0u);
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-        const uint32_t t = __shfl_sync(0xffffffffu, rr[it], (gl % GPI) * LPG);
-        if (gl / GPI == it) mine = t;
-    }
-    const float2 rf = half2_bits_to_float2(mine);
+    for (int off = 1; off < P::LPG; off <<= 1) r = hmax2_bits(r, __shfl_xor_sync(0xffffffffu, r, off));
+
+    const float2 rf = half2_bits_to_float2(r);
     const float lo = -rf.x, hi = rf.y;
     // s = fp16((hi - lo) / 15); a zero scale becomes 1.
-    uint16_t s16 = float_to_half_bits_rn(__fdiv_rn(hi - lo, 15.0f));
+    uint16_t s16 = float_to_half_bits_rn(div15_rn(hi - lo));
     if (s16 == 0) s16 = 0x3c00;
     const float s = half_bits_to_float(s16);
     const float rs = __frcp_rn(s);
     // z = round(-lo / s) in [0, 15]; |-lo / s| and |w / s| stay below 32 (E = 4)
     const int z = clampi(rne_quotient<4>(-lo, s, rs), 0, 15);
-    const float magic_g = 12582912.0f + (float)z;  // 1.5 * 2^23 + z
-    // groups past the end have w = 0: s = 1, z = 0, nothing stored
-    if (lane < 8 && zw * 8 + lane < groups) scales[(size_t)n * groups + zw * 8 + lane] = s16;
-    const uint32_t zword = __reduce_or_sync(0xffffffffu, lane < 8 ? (uint32_t)z << (4 * lane) : 0u);
+    const float magic = 12582912.0f + (float)z;  // 1.5 * 2^23 + z
 
+    uint32_t ok = ~0u;
 #pragma unroll
-    for (int it = 0; it < ITERS; ++it) {
-        const int j = zw * 8 + it * GPI + sub;
-        const int owner = it * GPI + sub;  // lane holding this group's scale and zero point
-        const float rs_g = __shfl_sync(0xffffffffu, rs, owner);
-        const float mg = __shfl_sync(0xffffffffu, magic_g, owner);
-        const float s_g = __shfl_sync(0xffffffffu, s, owner);
-        if (j < groups) {
-            const uint4 c0 = raw[it][0], c1 = raw[it][1];
-            const uint32_t h[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-            uint32_t p[8];
-            uint32_t bad = 0;
+    for (int v = 0; v < P::V; ++v)
+        words[v] = pack8(clamp15x2(pair_rne(raw[v].x, rs, magic, ok)), clamp15x2(pair_rne(raw[v].y, rs, magic, ok)),
+                         clamp15x2(pair_rne(raw[v].z, rs, magic, ok)), clamp15x2(pair_rne(raw[v].w, rs, magic, ok)));
+    if (!(ok >> 31)) {  // a near-tie: the IEEE quotient decides every code of this lane
 #pragma unroll
-            for (int e = 0; e < 8; ++e) p[e] = pair_rne(h[e], rs_g, mg, bad);
-            if (bad >> 31) {  // a near-tie: the IEEE quotient decides every code of this lane
-                const int zg = (int)(mg - 12582912.0f);
+        for (int v = 0; v < P::V; ++v) {
+            const uint32_t h[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
+            uint32_t pp[4];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float2 f = half2_bits_to_float2(h[e]);
-                    const uint32_t a = (uint32_t)(__float2int_rn(__fdiv_rn(f.x, s_g)) + zg) & 0xFFFFu;
-                    const uint32_t b = (uint32_t)(__float2int_rn(__fdiv_rn(f.y, s_g)) + zg) & 0xFFFFu;
-                    p[e] = a | (b << 16);
-                }
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = half2_bits_to_float2(h[e]);
+                const uint32_t a = (uint32_t)(__float2int_rn(__fdiv_rn(f.x, s)) + z) & 0xFFFFu;
+                const uint32_t b = (uint32_t)(__float2int_rn(__fdiv_rn(f.y, s)) + z) & 0xFFFFu;
+                pp[e] = clamp15x2(a | (b << 16));
             }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) p[e] = clamp15x2(p[e]);
-            *reinterpret_cast<uint2 *>(qweight + (size_t)n * (K / 8) + (size_t)j * (G / 8) + li * 2) =
-                make_uint2(pack8(p[0], p[1], p[2], p[3]), pack8(p[4], p[5], p[6], p[7]));
+            words[v] = pack8(pp[0], pp[1], pp[2], pp[3]);
         }
     }
-    if (lane == 0) qzeros[(size_t)n * zwords + zw] = zword;
+    s16_out = s16;
+    z_out = z;
+}
+
+// The unit's zero words (nibble j mod 8 of a word from each group's first lane, j the group's
+// index in its row) -> zw(q, word) for each of the unit's ZPU words.
+template <int G, typename Store>
+__device__ __forceinline__ void store_zero_words(int lane, int j, int z, Store zw) {
+    using P = Wide<G>;
+    const uint32_t zbits = lane % P::LPG == 0 ? (uint32_t)z << (4 * (j & 7)) : 0u;
+    constexpr int kLanesPerWord = 32 / P::ZPU;
+#pragma unroll
+    for (int q = 0; q < P::ZPU; ++q) {
+        const uint32_t word = __reduce_or_sync(0xffffffffu, lane / kLanesPerWord == q ? zbits : 0u);
+        if (lane == q * kLanesPerWord) zw(q, word);
+    }
+}
+
+// Any K (a multiple of G): grid (row blocks of 8, units of a row), one warp per (row, unit).
+template <int G>
+__global__ void __launch_bounds__(256, G >= 256 ? 2 : 4) quant_int4_group_f16w_kernel(const uint16_t *__restrict__ w, int N, int K,
+                                                                       uint32_t *__restrict__ qweight,
+                                                                       uint16_t *__restrict__ scales,
+                                                                       uint32_t *__restrict__ qzeros) {
+    using P = Wide<G>;
+    const int lane = threadIdx.x & 31;
+    const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (n >= N) return;
+    const int k0 = blockIdx.y * P::UE + lane * P::E;  // this lane's first element
+    const bool in = k0 < K;                           // K % G == 0: a lane is wholly in or out
+    const uint16_t *src = w + (size_t)n * K + k0;
+
+    uint4 raw[P::V];
+#pragma unroll
+    for (int v = 0; v < P::V; ++v) raw[v] = in ? ld_stream_u4(src + 8 * v) : make_uint4(0u, 0u, 0u, 0u);
+    uint32_t words[P::V];
+    uint16_t s16;
+    int z;
+    quantize_lane<G>(raw, words, s16, z);
+
+    const int j = k0 / G;  // this lane's group
+    if (in) {
+        uint32_t *dst = qweight + (size_t)n * (K / 8) + k0 / 8;
+#pragma unroll
+        for (int v = 0; v < P::V; v += 4)
+            *reinterpret_cast<uint4 *>(dst + v) = make_uint4(words[v], words[v + 1], words[v + 2], words[v + 3]);
+        if (lane % P::LPG == 0) scales[(size_t)n * (K / G) + j] = s16;
+    }
+    const int zwords = (K / G + 7) / 8;
+    store_zero_words<G>(lane, j, z, [&](int q, uint32_t word) {
+        const int zw = blockIdx.y * P::ZPU + q;
+        if (zw < zwords) qzeros[(size_t)n * zwords + zw] = word;
+    });
+}
+
+// K a multiple of the unit (every decode shape): the matrix is one run of N K / UE units, and
+// the codes, scales and zero words of unit u start at u's element offset divided by 8, G and
+// 8 G.  A persistent CTA of 8 quantizing warps and one copy warp walks stages of 8
+// consecutive units (16 KB of fp16; 32 KB for G = 256), stages blockIdx.x + i gridDim.x;
+// the copy warp keeps the CTA's next S stages in flight with 1-D bulk copies into a ring of
+// shared-memory slots, so the loads never wait for the arithmetic, and each quantizing warp
+// takes one unit of a stage, frees the slot as soon as its data is in registers and writes
+// its results straight to global memory.
+constexpr unsigned kQ4RingSite = 0x2000;
+
+template <int G>
+struct Q4Ring {
+    static constexpr uint32_t STAGE = 8u * Wide<G>::UE * 2u;  // bytes per stage
+    static constexpr int S = G >= 256 ? 2 : 4;                // slots: three CTAs per SM
+    static constexpr uint32_t OFF_BAR = S * STAGE;
+    static constexpr uint32_t SMEM = 128 + OFF_BAR + 16u * S + 16u;
+};
+
+template <int G>
+__global__ void __launch_bounds__(288, G >= 256 ? 2 : 3)
+    quant_int4_group_ring_kernel(const uint16_t *__restrict__ w, long long units, uint32_t *__restrict__ qweight,
+                                 uint16_t *__restrict__ scales, uint32_t *__restrict__ qzeros, unsigned int *status,
+                                 uint64_t limit_ns) {
+    using namespace sm100;
+    using P = Wide<G>;
+    using RL = Q4Ring<G>;
+    extern __shared__ uint8_t q4_ring_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q4_ring_raw) + 127) & ~uintptr_t(127));
+    uint64_t *full = reinterpret_cast<uint64_t *>(base + RL::OFF_BAR);
+    uint64_t *empty = full + RL::S;
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + RL::S);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long stages = (units + 7) / 8;
+    const long long mine = (long long)blockIdx.x < stages ? (stages - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < RL::S; ++i) {
+            mbar_init(smem_u32(&full[i]), 1);
+            mbar_init(smem_u32(&empty[i]), 8);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const WaitCtl ctl{abort_flag, status, limit_ns};
+
+    long long issued = 0;  // copy warp, lane 0: stages handed to the copy engine
+    if (warp == 8) {
+        // ------------------------------------------------------------ copy warp
+        if (lane == 0) {
+            for (; issued < mine; ++issued) {
+                const int slot = (int)(issued % RL::S);
+                const uint32_t u = (uint32_t)(issued / RL::S);
+                if (!wait_parity(smem_u32(&empty[slot]), (u & 1u) ^ 1u, ctl, kQ4RingSite | 0x1)) break;
+                const long long u0 = (blockIdx.x + issued * gridDim.x) * 8;
+                const uint32_t bytes = (uint32_t)(min(8ll, units - u0) * P::UE * 2);
+                const uint32_t fb = smem_u32(&full[slot]);
+                mbar_arrive_expect_tx(fb, bytes);
+                bulk_load(smem_u32(base + (uint32_t)slot * RL::STAGE), w + u0 * P::UE, bytes, fb);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ quantizing warps
+        for (long long i = 0; i < mine; ++i) {
+            const int slot = (int)(i % RL::S);
+            const uint32_t u = (uint32_t)(i / RL::S);
+            // warp-uniform: the lanes leave together (the shuffles below need the whole warp)
+            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&full[slot]), u & 1u, ctl, kQ4RingSite))) break;
+            const long long unit = (blockIdx.x + i * gridDim.x) * 8 + warp;
+            uint4 raw[P::V];
+            const uint4 *src = reinterpret_cast<const uint4 *>(base + (uint32_t)slot * RL::STAGE +
+                                                               (uint32_t)warp * P::UE * 2 + (uint32_t)lane * P::E * 2);
+#pragma unroll
+            for (int v = 0; v < P::V; ++v) raw[v] = src[v];
+            // Every lane orders its reads of the slot before the copy engine's next write into it
+            // (generic -> async proxy), then the warp releases the slot.
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty[slot]));
+            if (unit >= units) continue;  // past the end of the last stage (warp-uniform)
+            uint32_t words[P::V];
+            uint16_t s16;
+            int z;
+            quantize_lane<G>(raw, words, s16, z);
+            const size_t e0 = (size_t)unit * P::UE + (size_t)lane * P::E;  // this lane's first element
+            uint32_t *dst = qweight + e0 / 8;
+#pragma unroll
+            for (int v = 0; v < P::V; v += 4)
+                *reinterpret_cast<uint4 *>(dst + v) = make_uint4(words[v], words[v + 1], words[v + 2], words[v + 3]);
+            if (lane % P::LPG == 0) scales[e0 / G] = s16;
+            store_zero_words<G>(lane, (int)((e0 / G) & 7), z,
+                                [&](int q, uint32_t word) { qzeros[(size_t)unit * P::ZPU + q] = word; });
+        }
+    }
+    // Every warp is done with the ring.  After a timeout the copies still in flight (at most the
+    // last S issued) land before the CTA exits.
+    __syncthreads();
+    if (warp == 8 && lane == 0 && *abort_flag) {
+        for (long long j = issued > RL::S ? issued - RL::S : 0; j < issued; ++j)
+            drain_parity(smem_u32(&full[j % RL::S]), (uint32_t)(j / RL::S) & 1u, 2000000000ull, status,
+                         kQ4RingSite | 0x2);
+    }
 }
 
 template <typename TIn, int G>
@@ -368,11 +504,32 @@ cudaError_t launch(const void *w, int N, int K, uint32_t *qweight, uint16_t *sca
     const int zwords = (K / G + 7) / 8;
     const long long units = (long long)N * zwords;
     const int warps_per_block = 8;
+    if (std::is_same<TIn, __half>::value && G >= 64) {
+        constexpr int GW = G < 64 ? 64 : G;
+        if (K % Wide<GW>::UE == 0) {
+            using RL = Q4Ring<GW>;
+            unsigned int *status = device_status_word();
+            if (!status) return cudaErrorUnknown;
+            auto kern = quant_int4_group_ring_kernel<GW>;
+            cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)RL::SMEM);
+            if (e != cudaSuccess) return e;
+            int per_sm = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 288, RL::SMEM);
+            if (e != cudaSuccess) return e;
+            const long long total = (long long)N * (K / Wide<GW>::UE);
+            const long long stages = (total + 7) / 8;
+            const int grid = (int)std::min<long long>(stages, (long long)num_sms() * std::max(per_sm, 1));
+            kern<<<grid, 288, RL::SMEM, stream>>>(static_cast<const uint16_t *>(w), total, qweight, scales, qzeros,
+                                                  status, wait_limit());
+            return cudaGetLastError();
+        }
+        const dim3 grid((unsigned)((N + 7) / 8), (unsigned)((K + Wide<GW>::UE - 1) / Wide<GW>::UE));
+        quant_int4_group_f16w_kernel<GW><<<grid, 256, 0, stream>>>(static_cast<const uint16_t *>(w), N, K, qweight,
+                                                                   scales, qzeros);
+        return cudaGetLastError();
+    }
     const long long blocks = (units + warps_per_block - 1) / warps_per_block;
-    if (std::is_same<TIn, __half>::value && G >= 64)
-        quant_int4_group_f16x16_kernel<G < 64 ? 64 : G><<<(unsigned)blocks, warps_per_block * 32, 0, stream>>>(
-            static_cast<const uint16_t *>(w), N, K, qweight, scales, qzeros);
-    else if (std::is_same<TIn, __half>::value)
+    if (std::is_same<TIn, __half>::value)
         quant_int4_group_f16_kernel<G><<<(unsigned)blocks, warps_per_block * 32, 0, stream>>>(
             static_cast<const uint16_t *>(w), N, K, qweight, scales, qzeros);
     else
@@ -400,6 +557,9 @@ extern "C" wq_status wq_quantize_group_int4(const void *w, wq_dtype w_dtype, int
                group_size);
     const long long units = (long long)N * ((K / group_size + 7) / 8);
     WQ_REQUIRE(units / 8 < (1ll << 31), WQ_ERR_UNSUPPORTED, "matrix too large");
+    // fp16 with g >= 64: a grid of (ceil(N / 8), ceil(K / 1024)) blocks (K / 2048 for g = 256)
+    WQ_REQUIRE(!(w_dtype == WQ_F16 && group_size >= 64) || (K + 1023) / 1024 <= 65535, WQ_ERR_UNSUPPORTED,
+               "K (%d) too large for the fp16 quantizer (at most 65535 * 1024)", K);
     cudaStream_t st = wq::as_stream(stream);
     cudaError_t e;
     const bool f16 = w_dtype == WQ_F16;

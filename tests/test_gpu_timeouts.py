@@ -37,6 +37,7 @@ def _cases(wq):
         "streaming GEMV": lambda: wq.gemv_w4a16(x1, qw, sc, qz, 128),
         "tcgen05 W4A16 GEMM": lambda: wq.gemm_w4a16(x64, qw, sc, qz, 128),
         "tcgen05 W8A8 GEMM": lambda: wq.gemm_w8a8(xq, sx, w8, sw),
+        "bulk-copy ring INT4 quantizer": lambda: wq.quantize_group_int4(w, 128)[0].view(torch.int16),
     }
 
 
