@@ -17,19 +17,26 @@
 //
 // Swap-AB: the MMA's M dimension is 128 weight rows (TMEM lanes) and its N
 // dimension is the activation tile (16..128 rows of x), so small batches still
-// use full 128-row MMAs.  Per CTA (512 threads):
+// use full 128-row MMAs.  The dequantized weight tile never touches shared
+// memory: the dequantizers write it into tensor memory (tcgen05.st), and the
+// MMAs read their A operand from there, so shared memory holds only the TMA
+// rings and the packed-code ring can be deep enough to keep HBM busy.  Per CTA
+// (512 threads):
 //   warp 0      TMA: packed weight tiles (128 rows x 32 bytes = 64 codes) into
-//               a 6- or 12-deep ring (two or one CTAs per SM, see Layout)
+//               a 16- or 24-deep ring (two or one CTAs per SM, see Layout)
 //   warp 1      TMA: x tiles (MT rows x 64 fp16, 128-byte swizzle)
-//   warps 2, 15 tcgen05.mma issue (4 x K=16 per stage), warp 2 for the even
-//               stages and warp 15 for the odd ones, each into its own fp32
-//               accumulator in TMEM (warp 2 also allocates it); one thread
-//               issues a tcgen05.mma only every ~50 cycles, so a second issuer
-//               measured 6% (64 rows) to 16% (100-128 rows) faster on B200
-//   warps 3-10  dequantize: each thread turns 32 codes of one row into fp16
+//   warps 2, 15 tcgen05.mma issue (4 x K=16 per stage, A from tensor memory),
+//               warp 2 for the even stages and warp 15 for the odd ones, each
+//               into its own fp32 accumulator in TMEM (warp 2 also allocates
+//               it); one thread issues a tcgen05.mma only every ~50 cycles, so
+//               a second issuer measured 6% (64 rows) to 16% (100-128 rows)
+//               faster on B200
+//   warps 3-10  dequantize: thread (warp w, lane l) owns weight row
+//               32 (w mod 4) + l (the TMEM lanes its warp may access) and one
+//               half of each 64-code stage; it turns its 32 codes into fp16
 //               with PRMT/LOP3 (code -> 1024 + q), one exact fp16x2 fma
-//               (-> q - z) and one fp16x2 multiply by the scale, and stores
-//               them into the 128-byte-swizzled K-major A tile
+//               (-> q - z) and one fp16x2 multiply by the scale, and writes
+//               them to the stage's 16 TMEM columns of its lane
 //   warps 11-14 epilogue: tcgen05.ld of the two 128 x MT fp32 accumulators,
 //               summed
 // K is split over the S CTAs of a thread-block cluster when the weight tiles
@@ -48,10 +55,10 @@ namespace {
 using namespace sm100;
 
 constexpr int BMW = 128;                    // weight rows per tile (MMA M)
-constexpr int BK = 64;                      // k per stage: one 128-byte fp16 row
-constexpr int MAX_STAGES = 4;               // dequantized A stages (barrier arrays)
-constexpr int MAX_PSTAGES = 12;             // packed-tile ring (barrier arrays)
-constexpr uint32_t A_BYTES = BMW * BK * 2;  // 16 KB
+constexpr int BK = 64;                      // k per stage: 32 TMEM columns of fp16 pairs
+constexpr int MAX_STAGES = 8;               // dequantized A stages in TMEM (barrier arrays)
+constexpr int MAX_PSTAGES = 24;             // packed-tile ring (barrier arrays)
+constexpr uint32_t A_COLS = BK / 2;         // TMEM columns per A stage
 constexpr uint32_t P_BYTES = BMW * BK / 2;  // 4 KB of packed codes
 constexpr int THREADS = 512;
 constexpr int DQ_THREADS = 256;
@@ -59,32 +66,34 @@ constexpr uint64_t DRAIN_NS = 2000000000ull;
 constexpr unsigned SITE_PRODUCER = 0x201, SITE_MMA = 0x202, SITE_DEQUANT = 0x204, SITE_EPILOGUE = 0x208,
                    SITE_DRAIN = 0x210;
 
-// Activation tiles of up to 64 rows run two CTAs per SM (smaller rings, at most
-// 64 registers per thread): measured on B200 that halves the time of the
-// 64-row GEMM on the 28672x8192 projection, because a CTA's stage loop is
-// bound by handoff latency rather than by any unit's throughput.  128-row
-// tiles need the deeper activation ring and keep one CTA per SM.
+// Activation tiles of up to 64 rows run two CTAs per SM (each CTA half of tensor memory, at
+// most 64 registers per thread): measured on B200 that halves the time of the 64-row GEMM on
+// the 28672x8192 projection against one CTA per SM, because a CTA's stage loop is bound by
+// handoff latency rather than by any unit's throughput.  128-row tiles keep one CTA per SM.
+// Tensor memory: two MT-column accumulators, then the A stages (32 columns each).
 template <int MT>
 struct Layout {
     static constexpr int CTAS_PER_SM = MT <= 64 ? 2 : 1;
-    static constexpr int STAGES = MT <= 64 ? 3 : 4;
-    static constexpr int PSTAGES = MT <= 64 ? 6 : 12;
+    static constexpr uint32_t TMEM_COLS = MT <= 64 ? 256 : 512;
+    static constexpr int STAGES = (int)((TMEM_COLS - 2 * MT) / A_COLS) < MAX_STAGES
+                                      ? (int)((TMEM_COLS - 2 * MT) / A_COLS) : MAX_STAGES;
+    static constexpr int PSTAGES = MT <= 64 ? 16 : 24;
     static constexpr uint32_t B_BYTES = MT * 128;
     // activation tiles get their own ring, deep enough that a tile is requested
     // well before the MMA needs it (x comes from L2; its latency would otherwise
     // stall the MMA warp every few stages)
     static constexpr int XSTAGES = MT <= 32 ? 6 : 4;
-    static constexpr uint32_t OFF_A = 0;
-    static constexpr uint32_t OFF_B = OFF_A + STAGES * A_BYTES;
+    static constexpr uint32_t OFF_B = 0;
     static constexpr uint32_t OFF_P = OFF_B + XSTAGES * B_BYTES;
     static constexpr uint32_t PIPE_BYTES = OFF_P + PSTAGES * P_BYTES;  // reused for split-K partials
     static constexpr size_t SMEM = 1024 + PIPE_BYTES + 1024;  // alignment slack + barriers
+    static_assert(STAGES >= 2, "tensor memory holds at least two A stages");
 };
 
 struct Bars {
     uint64_t pk_full[MAX_PSTAGES];
     uint64_t pk_empty[MAX_PSTAGES];
-    uint64_t a_full[MAX_STAGES];   // dequantized weight tile written (256 arrivals)
+    uint64_t a_full[MAX_STAGES];   // dequantized weight stage written to TMEM (256 arrivals)
     uint64_t st_empty[MAX_STAGES]; // A stage consumed by the MMAs
     uint64_t x_full[12];       // activation tile landed (TMA transaction count)
     uint64_t x_empty[12];      // activation tile consumed by the MMAs
@@ -185,7 +194,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     Bars *bar = reinterpret_cast<Bars *>(base + L::PIPE_BYTES);
-    const uint32_t sA = smem_u32(base + L::OFF_A), sB = smem_u32(base + L::OFF_B), sP = smem_u32(base + L::OFF_P);
+    const uint32_t sB = smem_u32(base + L::OFF_B), sP = smem_u32(base + L::OFF_P);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int rank = (int)blockIdx.x;  // cluster dims (splits, 1, 1)
@@ -195,7 +204,8 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
     const int kb0 = rank * nkb;
     const int groups = K / gs, zwords = (groups + 7) / 8;
     constexpr uint32_t IDESC = make_idesc(/*f32*/ 1, /*f16 or bf16*/ BF ? 1 : 0, BF ? 1 : 0, BMW, MT);
-    constexpr uint32_t TMEM_COLS = 2 * MT;  // two MT-column accumulators; MT >= 16
+    constexpr uint32_t TMEM_COLS = L::TMEM_COLS;
+    constexpr uint32_t A_COL0 = 2 * MT;  // first A stage column, after the two accumulators
 
     if (threadIdx.x == 0) {
         for (int p = 0; p < L::PSTAGES; ++p) {
@@ -278,11 +288,11 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t a_addr = sA + s * A_BYTES, b_addr = sB + xs * L::B_BYTES;
+                const uint32_t a_tm = tmem_base + A_COL0 + (uint32_t)s * A_COLS, b_addr = sB + xs * L::B_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < BK / 16; ++kk)
-                    mma_f16(acc, umma_desc_sw128_kmajor(a_addr + kk * 32), umma_desc_sw128_kmajor(b_addr + kk * 32),
-                            IDESC, i != j || kk != 0);
+                    mma_f16_tmem_a(acc, a_tm + kk * 8, umma_desc_sw128_kmajor(b_addr + kk * 32), IDESC,
+                                   i != j || kk != 0);
                 tc_commit(smem_u32(&bar->st_empty[s]));
                 tc_commit(smem_u32(&bar->x_empty[xs]));
             }
@@ -293,83 +303,49 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
         __syncwarp();
     } else if (warp < 11) {
         // -------------------------------------------------------------------- dequantizers
-        const int d = threadIdx.x - 96;
-        // Thread pairs take the two 16-byte halves of one row, so a warp's code load reads 512
-        // contiguous bytes (16 rows) without bank conflicts; the swizzled stores stay conflict-free.
-        const int row = d >> 1, half = d & 1;
+        // Warp w may access TMEM lanes 32 (w mod 4) .. + 31: thread (w, l) owns weight row
+        // 32 (w mod 4) + l and half (w - 3) / 4 of each stage's 64 codes.
+        const int row = 32 * (warp & 3) + lane, half = (warp - 3) >> 2;
         const int n = min(n0 + row, N - 1);
-        const uint32_t a_row = sA + row * 128;
-        const int sw = row & 7;
+        const uint32_t t_a = tmem_base + ((uint32_t)(32 * (warp & 3)) << 16) + A_COL0 + (uint32_t)half * (A_COLS / 2);
         const uint16_t *srow = scales + (size_t)n * groups;
         const uint32_t *zrow = qzeros + (size_t)n * zwords;
         bool ok = true;
         auto stage = [&](int i, uint32_t zc, uint32_t s2) -> bool {
             const int p = i % L::PSTAGES, up = i / L::PSTAGES;
             const int s = i % L::STAGES, u = i / L::STAGES;
-            if (!wait_parity(smem_u32(&bar->pk_full[p]), up & 1, ctl, SITE_DEQUANT)) return false;
+            // Waits are warp-uniform: tcgen05.st and tcgen05.wait are warp-collective.
+            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&bar->pk_full[p]), up & 1, ctl, SITE_DEQUANT)))
+                return false;
             uint4 w;
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                          : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
                          : "r"(sP + p * P_BYTES + row * 32 + half * 16));
-            if (!wait_parity(smem_u32(&bar->st_empty[s]), (u & 1) ^ 1, ctl, SITE_DEQUANT)) return false;
-            const uint32_t dst = a_row + s * A_BYTES;
+            // The codes are in registers: the packed slot goes back to the producer (the proxy
+            // fence orders this read before the next TMA write into the slot).
+            fence_proxy_async_smem();
+            mbar_arrive(smem_u32(&bar->pk_empty[p]));
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+            uint32_t o[16];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const uint4 o = BF ? dequant_word_bf16(ws[j], zc, half_bits_to_float((uint16_t)(s2 & 0xFFFFu)))
+                const uint4 v = BF ? dequant_word_bf16(ws[j], zc, half_bits_to_float((uint16_t)(s2 & 0xFFFFu)))
                                    : dequant_word(ws[j], zc, s2);
-                const int chunk = half * 4 + j;
-                asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst + ((chunk ^ sw) << 4)), "r"(o.x),
-                             "r"(o.y), "r"(o.z), "r"(o.w)
-                             : "memory");
+                o[4 * j] = v.x;
+                o[4 * j + 1] = v.y;
+                o[4 * j + 2] = v.z;
+                o[4 * j + 3] = v.w;
             }
-            fence_proxy_async_smem();
+            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&bar->st_empty[s]), (u & 1) ^ 1, ctl, SITE_DEQUANT)))
+                return false;
+            tc_fence_after();
+            tmem_st_32x32b_x16(t_a + (uint32_t)s * A_COLS, o);
+            tmem_st_wait();
+            tc_fence_before();
             mbar_arrive(smem_u32(&bar->a_full[s]));
-            // The packed slot is released only now: its codes have been consumed and the
-            // proxy fence above orders this thread's read of it before the next TMA write.
-            mbar_arrive(smem_u32(&bar->pk_empty[p]));
-            return true;
-        };
-        // Two stages per proxy fence: measured 3-8% faster with 128-row activation
-        // tiles (four A stages, one CTA per SM), 6-10% slower with the three-stage
-        // two-CTA layout of smaller tiles, so only the former pairs.  nkb is even
-        // (K is a multiple of 128, and split-K parts a multiple of 16 stages).
-        auto stage2 = [&](int i, uint32_t zc, uint32_t s2) -> bool {
-            uint4 w[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int p = (i + e) % L::PSTAGES, up = (i + e) / L::PSTAGES;
-                if (!wait_parity(smem_u32(&bar->pk_full[p]), up & 1, ctl, SITE_DEQUANT)) return false;
-                asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                             : "=r"(w[e].x), "=r"(w[e].y), "=r"(w[e].z), "=r"(w[e].w)
-                             : "r"(sP + p * P_BYTES + row * 32 + half * 16));
-            }
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                const int s = (i + e) % L::STAGES, u = (i + e) / L::STAGES;
-                if (!wait_parity(smem_u32(&bar->st_empty[s]), (u & 1) ^ 1, ctl, SITE_DEQUANT)) return false;
-                const uint32_t dst = a_row + s * A_BYTES;
-                const uint32_t ws[4] = {w[e].x, w[e].y, w[e].z, w[e].w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 o = BF ? dequant_word_bf16(ws[j], zc, half_bits_to_float((uint16_t)(s2 & 0xFFFFu)))
-                                   : dequant_word(ws[j], zc, s2);
-                    const int chunk = half * 4 + j;
-                    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(dst + ((chunk ^ sw) << 4)), "r"(o.x),
-                                 "r"(o.y), "r"(o.z), "r"(o.w)
-                                 : "memory");
-                }
-            }
-            fence_proxy_async_smem();
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                mbar_arrive(smem_u32(&bar->a_full[(i + e) % L::STAGES]));
-                mbar_arrive(smem_u32(&bar->pk_empty[(i + e) % L::PSTAGES]));
-            }
             return true;
         };
         auto two_stages = [&](int i, uint32_t zc, uint32_t s2) -> bool {
-            if (MT > 64 && i + 1 < nkb) return stage2(i, zc, s2);
             return stage(i, zc, s2) && (i + 1 >= nkb || stage(i + 1, zc, s2));
         };
         if (SB) {
