@@ -80,6 +80,8 @@ lib.wq_smooth_workspace_bytes.argtypes = [_I]
 lib.wq_smooth_workspace_bytes.restype = ctypes.c_size_t
 lib.wq_gptq_workspace_bytes.argtypes = [_I]
 lib.wq_gptq_workspace_bytes.restype = ctypes.c_size_t
+lib.wq_fp4_scale_bytes.argtypes = [_I, _I, _I]
+lib.wq_fp4_scale_bytes.restype = ctypes.c_size_t
 lib.wq_awq_workspace_bytes.argtypes = [_I, _I]
 lib.wq_awq_workspace_bytes.restype = ctypes.c_size_t
 lib.wq_set_wait_limit.argtypes = [ctypes.c_uint64]
@@ -398,22 +400,28 @@ def llm_int8_matmul(x, wq, sw, threshold: float = 6.0, cap: int = 64, stream=Non
     return gemm_w8a8_outliers(xq, sx, wq, sw, x16, w16, stream=stream), count
 
 
+def fp4_scale_bytes(R: int, K: int, nvfp4: bool) -> int:
+    """Bytes of the scale-factor buffer of an R x K FP4 tensor (the tensor-core atom layout)."""
+    return int(lib.wq_fp4_scale_bytes(int(R), int(K), 1 if nvfp4 else 0))
+
+
 def quantize_mxfp4(x: torch.Tensor, stream=None):
-    """MXFP4 of fp16 x [R, K]: (packed E2M1 codes uint8 [R, K/2], E8M0 scales uint8 [R, K/32])."""
+    """MXFP4 of fp16 x [R, K]: (packed E2M1 codes uint8 [R, K/2], E8M0 scales uint8 in the atom layout)."""
     _cuda(x, "x", (torch.float16,), 2)
     R, K = x.shape
     q = _empty((R, K // 2), torch.uint8, x)
-    s = _empty((R, K // 32), torch.uint8, x)
+    s = _empty((fp4_scale_bytes(R, K, False),), torch.uint8, x)
     _check(lib.wq_quantize_mxfp4(_ptr(x), R, K, _ptr(q), _ptr(s), _P(_stream(stream))), "wq_quantize_mxfp4")
     return q, s
 
 
 def quantize_nvfp4(x: torch.Tensor, stream=None):
-    """NVFP4 of fp16 x [R, K]: (packed E2M1 uint8 [R, K/2], E4M3 scales uint8 [R, K/16], fp32 tensor scale [1])."""
+    """NVFP4 of fp16 x [R, K]: (packed E2M1 uint8 [R, K/2], E4M3 scales uint8 in the atom layout,
+    fp32 tensor scale [1])."""
     _cuda(x, "x", (torch.float16,), 2)
     R, K = x.shape
     q = _empty((R, K // 2), torch.uint8, x)
-    s = _empty((R, K // 16), torch.uint8, x)
+    s = _empty((fp4_scale_bytes(R, K, True),), torch.uint8, x)
     t = _empty((1,), torch.float32, x)
     _check(lib.wq_quantize_nvfp4(_ptr(x), R, K, _ptr(q), _ptr(s), _ptr(t), _P(_stream(stream))),
            "wq_quantize_nvfp4")
@@ -422,18 +430,19 @@ def quantize_nvfp4(x: torch.Tensor, stream=None):
 
 def gemm_fp4(a, sfa, b, sfb, ta=None, tb=None, out=None, return_acc: bool = False, stream=None):
     """Block-scaled FP4 GEMM: NVFP4 when the tensor scales ta/tb are given, MXFP4 otherwise.
-    a [M, K/2], sfa [M, K/bs], b [N, K/2], sfb [N, K/bs] -> y fp16 [M, N]."""
+    a [M, K/2], b [N, K/2] codes; sfa, sfb scale bytes in the atom layout -> y fp16 [M, N]."""
     nv = ta is not None
-    for t, n in ((a, "a"), (sfa, "sfa"), (b, "b"), (sfb, "sfb")):
+    for t, n in ((a, "a"), (b, "b")):
         _cuda(t, n, (torch.uint8,), 2)
+    for t, n in ((sfa, "sfa"), (sfb, "sfb")):
+        _cuda(t, n, (torch.uint8,), 1)
     if nv:
         _cuda(ta, "ta", (torch.float32,), 1)
         _cuda(tb, "tb", (torch.float32,), 1)
     M, K = a.shape[0], a.shape[1] * 2
     N = b.shape[0]
-    bs = 16 if nv else 32
-    if b.shape[1] * 2 != K or tuple(sfa.shape) != (M, K // bs) or tuple(sfb.shape) != (N, K // bs):
-        raise ValueError("shape mismatch: a [M,K/2], b [N,K/2], sfa [M,K/bs], sfb [N,K/bs]")
+    if b.shape[1] * 2 != K or sfa.numel() != fp4_scale_bytes(M, K, nv) or sfb.numel() != fp4_scale_bytes(N, K, nv):
+        raise ValueError("shape mismatch: a [M,K/2], b [N,K/2], sfa/sfb of fp4_scale_bytes(M or N, K) bytes")
     y = out if out is not None else _empty((M, N), torch.float16, a)
     _cuda(y, "out", (torch.float16,), 2)
     acc = _empty((M, N), torch.float32, a) if return_acc else None

@@ -13,12 +13,12 @@
 //
 // Persistent, warp-specialized CTA (one per SM, 192 threads), 128 x 128 tiles,
 // 256 K (128 bytes of codes per row) per stage:
-//   warp 0   lane 0 loads the A and B code tiles with TMA (128-byte swizzle);
-//            all 32 lanes load the stage's scale factors with plain loads and
-//            store them in the 512-byte atoms that tcgen05.cp expects (row r
-//            of a 128-row block at byte 16 (r % 32) + 4 (r / 32) + j for its
-//            j-th factor of a group of four), then fence them for the async
-//            proxy; the stage's full barrier counts the TMA bytes and 32 lanes
+//   warp 0   lane 0 loads the A and B code tiles with TMA (128-byte swizzle) and
+//            the stage's scale factors with two 1-D bulk copies: the quantizers
+//            store them in the 512-byte atoms tcgen05.cp expects (row r of a
+//            128-row block at byte 16 (r % 32) + 4 (r / 32) + j for its j-th
+//            factor of a group of four, atoms row-block-major), so a tile's
+//            factors for one stage are G contiguous atoms per operand
 //   warp 1   allocates 512 TMEM columns (two 128-column accumulators and a
 //            ring of scale-factor slots), copies a stage's factors into its
 //            slot with tcgen05.cp (each 512-byte atom fills 4 columns, one
@@ -74,48 +74,6 @@ struct Smem {
     int abort;
 };
 
-__device__ __forceinline__ void sts128(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-    asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(a), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
-}
-
-// Lane `lane` writes the scale factors of rows lane + 32 i (i = 0..3) of one 128-row block into
-// the G atoms at `dst`: atom g, bytes 16 lane .. 16 lane + 15 = factors 4g..4g+3 of those rows.
-// Scale factors of one stage for one lane: rows lane + 32 i (i = 0..3) of the A tile and of the
-// B tile, 16 (NVFP4) or 8 (MXFP4) bytes each.  Loaded into registers a few stages ahead of their
-// use, so the producer does not wait for the L2 round trip on every stage.
-template <bool NV>
-struct StageFactors {
-    uint4 a[4], b[4];  // MXFP4 uses .x/.y only
-};
-
-template <bool NV>
-__device__ __forceinline__ void load_factor_rows(const uint8_t *__restrict__ sf, int rows, int row0, int ld, int kb,
-                                                 int lane, uint4 (&v)[4]) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int r = min(row0 + lane + 32 * i, rows - 1);
-        const uint8_t *p = sf + (size_t)r * ld + (size_t)kb * (NV ? 16 : 8);
-        if constexpr (NV) {
-            v[i] = __ldg(reinterpret_cast<const uint4 *>(p));
-        } else {
-            const uint2 t = __ldg(reinterpret_cast<const uint2 *>(p));
-            v[i] = make_uint4(t.x, t.y, 0u, 0u);
-        }
-    }
-}
-
-// Lane `lane` writes its rows' factors into the G atoms at `dst`: atom g, bytes 16 lane ..
-// 16 lane + 15 = factors 4g..4g+3 of rows lane, lane + 32, lane + 64, lane + 96.
-template <bool NV>
-__device__ __forceinline__ void store_factor_rows(const uint4 (&v)[4], int lane, uint32_t dst) {
-    sts128(dst + 0 * ATOM + lane * 16, v[0].x, v[1].x, v[2].x, v[3].x);
-    sts128(dst + 1 * ATOM + lane * 16, v[0].y, v[1].y, v[2].y, v[3].y);
-    if constexpr (NV) {
-        sts128(dst + 2 * ATOM + lane * 16, v[0].z, v[1].z, v[2].z, v[3].z);
-        sts128(dst + 3 * ATOM + lane * 16, v[0].w, v[1].w, v[2].w, v[3].w);
-    }
-}
-
 template <bool NV>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -132,11 +90,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
     const int tiles = mt * nt;
     const int kblocks = K / 256;
-    const int ld_sf = K / F::BS;  // scale factors per row
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&sm->full[s]), 1 + 32);  // TMA transaction + the 32 factor-storing lanes
+            mbar_init(smem_u32(&sm->full[s]), 1);
             mbar_init(smem_u32(&sm->empty[s]), 1);
         }
         for (int a = 0; a < 2; ++a) {
@@ -162,49 +119,31 @@ __global__ void __launch_bounds__(THREADS, 1)
     const WaitCtl ctl{&sm->abort, status, limit_ns};
 
     if (warp == 0) {
-        // -------------------------------------------------------------------- producer warp
-        // The CTA's stages in order: stage j is k block j % kblocks of its tile j / kblocks.
-        const int my_tiles = tiles > (int)blockIdx.x ? (tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
-        const int nstages = my_tiles * kblocks;
-        auto load = [&](int j, StageFactors<NV> &f) {
-            const int tile = (int)blockIdx.x + (j / kblocks) * (int)gridDim.x, kb = j % kblocks;
-            load_factor_rows<NV>(sfa, M, (tile % mt) * BM, ld_sf, kb, lane, f.a);
-            load_factor_rows<NV>(sfb, N, (tile / mt) * BN, ld_sf, kb, lane, f.b);
-        };
-        // two stages of factors in registers (f0: even stages, f1: odd ones): stage j + 2 is
-        // requested as soon as stage j has been stored
-        StageFactors<NV> f0, f1;
-        if (nstages > 0) load(0, f0);
-        if (nstages > 1) load(1, f1);
-        uint32_t it = 0;
-        auto produce = [&](int j, StageFactors<NV> &cur) -> bool {
-            const int tile = (int)blockIdx.x + (j / kblocks) * (int)gridDim.x, kb = j % kblocks;
-            const int m0 = (tile % mt) * BM, n0 = (tile / mt) * BN;
-            const uint32_t s = it % STAGES, u = it / STAGES;
-            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&sm->empty[s]), (u & 1) ^ 1, ctl, SITE_PRODUCER)))
-                return false;
-            const uint32_t fb = smem_u32(&sm->full[s]);
-            const uint32_t st = sbase + s * F::STAGE_BYTES;
-            if (lane == 0) {
-                mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
-                tma_load_2d(st, &tmap_a, fb, kb * BKB, m0);
-                tma_load_2d(st + A_BYTES, &tmap_b, fb, kb * BKB, n0);
-            }
-            ++it;
-            const uint32_t sf_dst = st + A_BYTES + B_BYTES;
-            store_factor_rows<NV>(cur.a, lane, sf_dst);
-            store_factor_rows<NV>(cur.b, lane, sf_dst + F::G * ATOM);
-            fence_proxy_async_smem();  // the factors are read by tcgen05.cp (async proxy)
-            mbar_arrive(fb);
-            if (j + 2 < nstages) load(j + 2, cur);
-            return true;
-        };
-        for (int j = 0; j < nstages; j += 2) {
-            if (!produce(j, f0)) break;
-            if (j + 1 < nstages && !produce(j + 1, f1)) break;
-        }
-        // Every issued TMA load must land before the CTA may exit.
         if (lane == 0) {
+            // ---------------------------------------------------------------- producer
+            const int fg = K / F::BS / 4;  // atoms per 128-row block
+            uint32_t it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; ok && tile < tiles; tile += gridDim.x) {
+                const int m0 = (tile % mt) * BM, n0 = (tile / mt) * BN;
+                const uint8_t *sfa_t = sfa + ((size_t)(m0 / BM) * fg) * ATOM;
+                const uint8_t *sfb_t = sfb + ((size_t)(n0 / BN) * fg) * ATOM;
+                for (int kb = 0; kb < kblocks; ++kb, ++it) {
+                    const uint32_t s = it % STAGES, u = it / STAGES;
+                    if (!wait_parity(smem_u32(&sm->empty[s]), (u & 1) ^ 1, ctl, SITE_PRODUCER)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&sm->full[s]);
+                    const uint32_t st = sbase + s * F::STAGE_BYTES;
+                    mbar_arrive_expect_tx(fb, F::STAGE_BYTES);
+                    tma_load_2d(st, &tmap_a, fb, kb * BKB, m0);
+                    tma_load_2d(st + A_BYTES, &tmap_b, fb, kb * BKB, n0);
+                    bulk_load(st + A_BYTES + B_BYTES, sfa_t + (size_t)kb * F::G * ATOM, F::G * ATOM, fb);
+                    bulk_load(st + A_BYTES + B_BYTES + F::G * ATOM, sfb_t + (size_t)kb * F::G * ATOM, F::G * ATOM, fb);
+                }
+            }
+            // Every issued copy must land before the CTA may exit.
             for (uint32_t s = 0; s < STAGES; ++s) {
                 const uint32_t issued = it > s ? (it - s - 1) / STAGES + 1 : 0;
                 if (issued) drain_parity(smem_u32(&sm->full[s]), (issued - 1) & 1, DRAIN_NS, status, SITE_DRAIN);

@@ -19,6 +19,13 @@
 // One thread per block: 64 (MX) or 32 (NV) bytes in, 16 or 8 bytes of packed
 // codes (element 2i in the low nibble of byte i) and one scale byte out; HBM
 // traffic is 2 B in + 0.5 B + one scale byte per block out, per element.
+//
+// The scale bytes are written in the layout the tensor cores read them in
+// (tcgen05.cp of 512-byte atoms into tensor memory for the block-scaled MMA):
+// rows in blocks of 128, a row's factors in groups of 4, one atom per (row
+// block, group), atoms in row-block-major order; factor f of row r is byte
+// 16 (r % 32) + 4 ((r / 32) % 4) + f % 4 of atom (r / 128, f / 4).  A GEMM
+// stage then fetches its factors with one contiguous bulk copy per operand.
 #include "wq_device.cuh"
 #include "wq_host.h"
 
@@ -28,6 +35,26 @@ namespace wq {
 namespace {
 
 constexpr int kThreads = 256;
+
+// Byte offset of factor f of row r in the atom layout; fg = groups of 4 factors per row.
+__device__ __forceinline__ size_t sf_offset(int r, int f, int fg) {
+    return ((size_t)(r >> 7) * fg + (f >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (f & 3);
+}
+
+// (row, factor) of block b = r F + f along a grid-stride loop, without a division per step.
+struct BlockPos {
+    int r, f, dr, df, F;
+    __device__ BlockPos(size_t b0, size_t stride, int F_)
+        : r((int)(b0 / F_)), f((int)(b0 % F_)), dr((int)(stride / F_)), df((int)(stride % F_)), F(F_) {}
+    __device__ void advance() {
+        r += dr;
+        f += df;
+        if (f >= F) {
+            f -= F;
+            ++r;
+        }
+    }
+};
 
 // Eight fp32 values to eight E2M1 codes (round to nearest even, saturating at +-6), element 0 in
 // the low nibble.  cvt ... e2m1x2 puts its first operand in the high nibble of the byte.
@@ -58,9 +85,12 @@ __device__ __forceinline__ float amax8(const float (&v)[8], float m) {
     return m;
 }
 
-__global__ void __launch_bounds__(kThreads) quant_mxfp4_kernel(const uint16_t *__restrict__ x, size_t nblocks,
+__global__ void __launch_bounds__(kThreads) quant_mxfp4_kernel(const uint16_t *__restrict__ x, size_t nblocks, int F,
                                                                uint8_t *__restrict__ q, uint8_t *__restrict__ scales) {
-    for (size_t b = (size_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += (size_t)gridDim.x * kThreads) {
+    const int fg = (F + 3) / 4;
+    const size_t stride = (size_t)gridDim.x * kThreads;
+    BlockPos pos((size_t)blockIdx.x * kThreads + threadIdx.x, stride, F);
+    for (size_t b = (size_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += stride, pos.advance()) {
         float v[4][8];
         float a = 0.0f;
 #pragma unroll
@@ -80,7 +110,7 @@ __global__ void __launch_bounds__(kThreads) quant_mxfp4_kernel(const uint16_t *_
             c[i] = cvt_e2m1x8(t);
         }
         *reinterpret_cast<uint4 *>(q + 16 * b) = make_uint4(c[0], c[1], c[2], c[3]);
-        scales[b] = (uint8_t)(e + 127);
+        scales[sf_offset(pos.r, pos.f, fg)] = (uint8_t)(e + 127);
     }
 }
 
@@ -122,12 +152,15 @@ __device__ __forceinline__ uint32_t float_to_e4m3(float v) {
     return r & 0xFFu;
 }
 
-__global__ void __launch_bounds__(kThreads) quant_nvfp4_kernel(const uint16_t *__restrict__ x, size_t nblocks,
+__global__ void __launch_bounds__(kThreads) quant_nvfp4_kernel(const uint16_t *__restrict__ x, size_t nblocks, int F,
                                                                const unsigned int *__restrict__ tensor_amax,
                                                                uint8_t *__restrict__ q, uint8_t *__restrict__ scales) {
+    const int fg = (F + 3) / 4;
     const float S = __fdiv_rn(fmaxf(__uint_as_float(*tensor_amax), 1e-8f), 2688.0f);
     constexpr float kDown = 1.0f - 0x1p-20f, kUp = 1.0f + 0x1p-20f;
-    for (size_t b = (size_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += (size_t)gridDim.x * kThreads) {
+    const size_t stride = (size_t)gridDim.x * kThreads;
+    BlockPos pos((size_t)blockIdx.x * kThreads + threadIdx.x, stride, F);
+    for (size_t b = (size_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += stride, pos.advance()) {
         float v[2][8];
         load8h(x + 16 * b, v[0]);
         load8h(x + 16 * b + 8, v[1]);
@@ -163,7 +196,7 @@ __global__ void __launch_bounds__(kThreads) quant_nvfp4_kernel(const uint16_t *_
             }
         }
         *reinterpret_cast<uint2 *>(q + 8 * b) = make_uint2(c[0], c[1]);
-        scales[b] = (uint8_t)sb;
+        scales[sf_offset(pos.r, pos.f, fg)] = (uint8_t)sb;
     }
 }
 
@@ -185,8 +218,9 @@ extern "C" wq_status wq_quantize_mxfp4(const uint16_t *x, int R, int K, uint8_t 
     WQ_REQUIRE_PTR(scales, "scales");
     WQ_REQUIRE(R > 0 && K > 0, WQ_ERR_INVALID_ARG, "wq_quantize_mxfp4: sizes must be positive (rows=%d K=%d)", R, K);
     WQ_REQUIRE(K % 32 == 0, WQ_ERR_UNSUPPORTED, "wq_quantize_mxfp4: K (%d) must be a multiple of 32", K);
+    WQ_REQUIRE(R < (1 << 30), WQ_ERR_UNSUPPORTED, "wq_quantize_mxfp4: too many rows");
     const size_t nblocks = (size_t)R * (K / 32);
-    quant_mxfp4_kernel<<<grid_for(nblocks), kThreads, 0, as_stream(stream)>>>(x, nblocks, q, scales);
+    quant_mxfp4_kernel<<<grid_for(nblocks), kThreads, 0, as_stream(stream)>>>(x, nblocks, K / 32, q, scales);
     return check_launch("wq_quantize_mxfp4");
 }
 
@@ -199,6 +233,7 @@ extern "C" wq_status wq_quantize_nvfp4(const uint16_t *x, int R, int K, uint8_t 
     WQ_REQUIRE_PTR(tensor_scale, "tensor_scale");
     WQ_REQUIRE(R > 0 && K > 0, WQ_ERR_INVALID_ARG, "wq_quantize_nvfp4: sizes must be positive (rows=%d K=%d)", R, K);
     WQ_REQUIRE(K % 16 == 0, WQ_ERR_UNSUPPORTED, "wq_quantize_nvfp4: K (%d) must be a multiple of 16", K);
+    WQ_REQUIRE(R < (1 << 30), WQ_ERR_UNSUPPORTED, "wq_quantize_nvfp4: too many rows");
     cudaStream_t st = as_stream(stream);
     unsigned int *amax = reinterpret_cast<unsigned int *>(tensor_scale);
     cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(unsigned int), st);
@@ -207,9 +242,15 @@ extern "C" wq_status wq_quantize_nvfp4(const uint16_t *x, int R, int K, uint8_t 
     tensor_absmax_fp4_kernel<<<grid_for(n8), kThreads, 0, st>>>(x, n8, amax);
     if ((e = cudaGetLastError()) != cudaSuccess)
         return fail(WQ_ERR_CUDA, "wq_quantize_nvfp4: launch failed: %s", cudaGetErrorString(e));
-    quant_nvfp4_kernel<<<grid_for(nblocks), kThreads, 0, st>>>(x, nblocks, amax, q, scales);
+    quant_nvfp4_kernel<<<grid_for(nblocks), kThreads, 0, st>>>(x, nblocks, K / 16, amax, q, scales);
     if ((e = cudaGetLastError()) != cudaSuccess)
         return fail(WQ_ERR_CUDA, "wq_quantize_nvfp4: launch failed: %s", cudaGetErrorString(e));
     finish_nvfp4_scale_kernel<<<1, 1, 0, st>>>(tensor_scale);
     return check_launch("wq_quantize_nvfp4");
+}
+
+extern "C" size_t wq_fp4_scale_bytes(int R, int K, int nvfp4) {
+    if (R <= 0 || K <= 0) return 0;
+    const long long F = K / (nvfp4 ? 16 : 32);
+    return (size_t)((R + 127) / 128) * (size_t)((F + 3) / 4) * 512;
 }

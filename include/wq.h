@@ -337,13 +337,21 @@ wq_status wq_gemm_w8a8_outliers(const int8_t *xq, const float *sx, const int8_t 
  *   written to *tensor_scale); per block of 16, scale byte
  *   b = e4m3_rn((max|v| / 6) / S) (two fp32 divisions), d = e4m3(b) * S,
  *   q = e2m1_rn(v / d) (fp32 IEEE division; all zero when b == 0).
- * x: fp16 [R][K];  q: out [R][K/2];  scales: out [R][K/32] (MX) or [R][K/16]
- * (NV);  tensor_scale: out fp32 [1] (also the call's reduction word).
+ * x: fp16 [R][K];  q: out [R][K/2];  tensor_scale: out fp32 [1] (also the
+ * call's reduction word);  scales: out, wq_fp4_scale_bytes(R, K, nvfp4) bytes
+ * in the tensor-core atom layout: with F = K/32 (MX) or K/16 (NV) factors per
+ * row, rows in blocks of 128 and factors in groups of 4, one 512-byte atom per
+ * (row block, group), atoms ordered row block major; factor f of row r is
+ *   byte ((r/128) * ceil(F/4) + f/4) * 512 + 16 (r % 32) + 4 ((r/32) % 4) + f % 4.
+ * Bytes of rows past R (and of factors past F) are not written.
  * K % 32 == 0 (MX) or K % 16 == 0 (NV).  Inputs must be finite.
  */
 wq_status wq_quantize_mxfp4(const uint16_t *x, int R, int K, uint8_t *q, uint8_t *scales, void *stream);
 wq_status wq_quantize_nvfp4(const uint16_t *x, int R, int K, uint8_t *q, uint8_t *scales, float *tensor_scale,
                             void *stream);
+
+/* Size in bytes of the scale-factor buffer of an R x K FP4 tensor (0 for non-positive sizes). */
+size_t wq_fp4_scale_bytes(int R, int K, int nvfp4);
 
 /*
  * Block-scaled FP4 GEMM on the tensor cores (tcgen05 kind::mxf4 for MXFP4,
@@ -353,9 +361,10 @@ wq_status wq_quantize_nvfp4(const uint16_t *x, int R, int K, uint8_t *q, uint8_t
  *   y[m][n] = fp16_rn( ta * tb * sum_k e2m1(a[m][k]) sa(m, k/bs) e2m1(b[n][k]) sb(n, k/bs) )
  * nvfp4 = 0: MXFP4 (bs = 32, E8M0 scales, ta = tb = 1, both may be NULL);
  * nvfp4 = 1: NVFP4 (bs = 16, E4M3 scales, ta/tb: device fp32 [1] tensor
- * scales).  a: [M][K/2], sfa: [M][K/bs], b: [N][K/2], sfb: [N][K/bs] in the
- * layouts the quantizers write;  y: out fp16 [M][N];  acc_out: nullable,
- * out fp32 [M][N] (the block-scaled sums before ta * tb).  K % 256 == 0.
+ * scales).  a: [M][K/2], b: [N][K/2] packed codes; sfa, sfb: the scale
+ * factors of a and b in the atom layout above (wq_fp4_scale_bytes(M or N, K,
+ * nvfp4) bytes each);  y: out fp16 [M][N];  acc_out: nullable, out fp32
+ * [M][N] (the block-scaled sums before ta * tb).  K % 256 == 0.
  */
 wq_status wq_gemm_fp4(int nvfp4, const uint8_t *a, const uint8_t *sfa, const float *ta, const uint8_t *b,
                       const uint8_t *sfb, const float *tb, int M, int N, int K, uint16_t *y, float *acc_out,

@@ -62,6 +62,11 @@ def _special_weights(N, K, seed, dtype=np.float16):
         w[3, 256:384] = np.abs(w[3, 256:384]) + 0.01
         w[4, 384:512] = -np.abs(w[4, 384:512]) - 0.01
         w[5, ::7] = 0.0
+    if N > 8 and K >= 640:
+        # s = 1/16 exactly and every other weight at (k + 1/2) / 16: w / s lands on ties
+        tie = (np.arange(128) % 14 + 0.5) / 16.0
+        tie[0], tie[1] = 0.0, 15.0 / 16.0
+        w[6, 512:640] = tie
     return w.astype(dtype)
 
 
@@ -69,6 +74,8 @@ SMALL_INT4 = [  # (N, K, g, dtype)
     (1, 128, 128, np.float16), (17, 384, 128, np.float16), (33, 1024, 128, np.float16),
     (64, 1536, 128, np.float16), (9, 96, 32, np.float16), (40, 640, 64, np.float16),
     (13, 2048, 256, np.float16), (24, 512, 128, np.float32), (300, 4096, 128, np.float16),
+    (11, 768, 256, np.float16), (13, 4096, 64, np.float16), (9, 8320, 128, np.float16),
+    (10, 1280, 128, np.float16),
 ]
 
 
@@ -95,6 +102,25 @@ def test_int4_quantizer_bit_exact_configs(wq, cfg, shape_index):
     assert np.array_equal(host(qw, np.uint32)[rows], rqw)
     assert np.array_equal(host(sc).view(np.uint16)[rows], rsc.view(np.uint16))
     assert np.array_equal(host(qz, np.uint32)[rows], rqz)
+
+
+def test_int4_quantizer_repeatable(wq):
+    # The bulk-copy ring reuses shared-memory slots; repeated runs must give the same bits, and
+    # the rows of every CTA's first stages (whose slots are refilled) must match the oracle.
+    g = np.random.default_rng(7)
+    w = (g.standard_normal((4096, 4096)) * 0.02).astype(np.float16)
+    wd = dev(w)
+    runs = []
+    for _ in range(5):
+        qw, sc, qz = wq.quantize_group_int4(wd, 128)
+        torch.cuda.synchronize()
+        runs.append((host(qw, np.uint32), host(sc).view(np.uint16), host(qz, np.uint32)))
+    for r in runs[1:]:
+        assert all(np.array_equal(a, b) for a, b in zip(runs[0], r))
+    rqw, rsc, rqz = oracle.quantize_group_int4(w[:1024], 128)
+    assert np.array_equal(runs[0][0][:1024], rqw)
+    assert np.array_equal(runs[0][1][:1024], rsc.view(np.uint16))
+    assert np.array_equal(runs[0][2][:1024], rqz)
 
 
 # --------------------------------------------------------------------------
@@ -199,6 +225,26 @@ def test_gemv_w4a16_configs(wq, cfg):
             torch.cuda.synchronize()
             y_ref, bound = oracle.matmul_w4a16_ref(x, hqw, hsc, hqz, K, 128, rows=rows)
             assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"{cfg} {N}x{K} B={B}")
+
+
+@pytest.mark.parametrize("N,K,B", [(40000, 2048, 1), (30000, 4096, 8), (9000, 14336, 3)])
+def test_gemv_w4a16_large_shapes_tile_boundaries(wq, N, K, B):
+    # Larger streaming-GEMV shapes (several tiles, K splits over clusters of 1, 2 and 7 CTAs);
+    # sampled rows include the rows next to the boundaries of 224- and 128-row tiles and of
+    # near-equal row blocks.
+    g = np.random.default_rng(N + K)
+    w = (g.standard_normal((N, K)) * 0.02).astype(np.float16)
+    qw, sc, qz = wq.quantize_group_int4(dev(w), 128)
+    bounds = {int(p * N // P) + d for s in range(1, 9) for P in [296 // s] for p in range(1, P)
+              for d in (-1, 0)}
+    bounds |= {t * r + d for r in (224, 128) for t in range(1, N // r + 1) for d in (-1, 0)}
+    rows = np.unique(np.concatenate([sample_rows(N, 256, seed=N), np.array(sorted(bounds), np.int32)]))
+    rows = rows[(rows >= 0) & (rows < N)].astype(np.int32)
+    x = workloads.activations(B, K, 0.01, 50.0, seed=B, tensor_id=N)
+    y = wq.gemv_w4a16(dev(x), qw, sc, qz, 128)
+    torch.cuda.synchronize()
+    y_ref, bound = oracle.matmul_w4a16_ref(x, host(qw, np.uint32), host(sc), host(qz, np.uint32), K, 128, rows=rows)
+    assert_within_bound(host(y).astype(np.float64)[:, rows], y_ref, bound, f"{N}x{K} B={B}")
 
 
 # --------------------------------------------------------------------------
@@ -634,6 +680,36 @@ def test_llm_int8_full_size(wq):
 FP4_Q_SMALL = [(1, 32), (7, 64), (33, 2048), (5, 2080), (64, 4096), (3, 16384), (300, 1024)]
 
 
+def _sf_offsets(R, F):
+    # byte offset of factor f of row r in the tensor-core atom layout (see wq.h)
+    r = np.arange(R)[:, None]
+    f = np.arange(F)[None, :]
+    fg = -(-F // 4)
+    return ((r >> 7) * fg + (f >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (f & 3)
+
+
+def sf_to_atoms(sf):
+    """Row-major scale factors [R][F] -> the atom-layout buffer the GPU kernels use."""
+    R, F = sf.shape
+    out = np.zeros(-(-R // 128) * -(-F // 4) * 512, np.uint8)
+    out[_sf_offsets(R, F)] = sf
+    return out
+
+
+def sf_from_atoms(buf, R, F):
+    """The atom-layout buffer -> row-major scale factors [R][F]."""
+    return np.asarray(buf)[_sf_offsets(R, F)]
+
+
+def test_sf_atom_layout_helpers_round_trip():
+    g = np.random.default_rng(3)
+    sf = g.integers(0, 256, (300, 37), dtype=np.uint8)
+    buf = sf_to_atoms(sf)
+    assert buf.size == 3 * 10 * 512 and np.array_equal(sf_from_atoms(buf, 300, 37), sf)
+    offs = _sf_offsets(300, 37).ravel()
+    assert np.unique(offs).size == offs.size  # a bijection onto its image
+
+
 def _fp4_inputs(R, K, seed):
     g = np.random.default_rng(seed)
     a = (g.standard_normal((R, K)) * np.exp(g.uniform(-3, 3, (R, 1)))).astype(np.float32)
@@ -650,7 +726,8 @@ def test_mxfp4_quantizer_bit_exact(wq, R, K):
     q, s = wq.quantize_mxfp4(dev(a))
     torch.cuda.synchronize()
     rq, rs = oracle.quantize_mxfp4(a)
-    assert np.array_equal(host(s), rs) and np.array_equal(host(q), rq)
+    assert host(s).size == wq.fp4_scale_bytes(R, K, False)
+    assert np.array_equal(sf_from_atoms(host(s), R, K // 32), rs) and np.array_equal(host(q), rq)
 
 
 @pytest.mark.parametrize("R,K", [rk for rk in FP4_Q_SMALL if rk[1] % 16 == 0])
@@ -660,7 +737,8 @@ def test_nvfp4_quantizer_bit_exact(wq, R, K):
     torch.cuda.synchronize()
     rq, rs, rt = oracle.quantize_nvfp4(a)
     assert np.array_equal(host(t), rt)
-    assert np.array_equal(host(s), rs) and np.array_equal(host(q), rq)
+    assert host(s).size == wq.fp4_scale_bytes(R, K, True)
+    assert np.array_equal(sf_from_atoms(host(s), R, K // 16), rs) and np.array_equal(host(q), rq)
 
 
 def test_fp4_quantizers_every_e2m1_midpoint(wq):
@@ -671,10 +749,11 @@ def test_fp4_quantizers_every_e2m1_midpoint(wq):
     a = np.stack([row[:32], -row[:32]]).astype(np.float16)
     q, s = wq.quantize_mxfp4(dev(a))
     rq, rs = oracle.quantize_mxfp4(a)
-    assert np.array_equal(host(s), rs) and np.array_equal(host(q), rq)
+    assert np.array_equal(sf_from_atoms(host(s), 2, 1), rs) and np.array_equal(host(q), rq)
     q, s, t = wq.quantize_nvfp4(dev(a))
     rq, rs, rt = oracle.quantize_nvfp4(a)
-    assert np.array_equal(host(t), rt) and np.array_equal(host(s), rs) and np.array_equal(host(q), rq)
+    assert np.array_equal(host(t), rt) and np.array_equal(sf_from_atoms(host(s), 2, 2), rs)
+    assert np.array_equal(host(q), rq)
 
 
 FP4_GEMM_SMALL = [(1, 1, 256), (128, 128, 256), (130, 300, 512), (64, 40, 1024), (257, 513, 256),
@@ -689,12 +768,12 @@ def test_gemm_fp4_small(wq, M, N, K, nv):
     if nv:
         qa, sa, ta = oracle.quantize_nvfp4(a)
         qb, sb, tb = oracle.quantize_nvfp4(b)
-        y = wq.gemm_fp4(dev(qa), dev(sa), dev(qb), dev(sb), dev(ta), dev(tb))
+        y = wq.gemm_fp4(dev(qa), dev(sf_to_atoms(sa)), dev(qb), dev(sf_to_atoms(sb)), dev(ta), dev(tb))
         tav, tbv = float(ta[0]), float(tb[0])
     else:
         qa, sa = oracle.quantize_mxfp4(a)
         qb, sb = oracle.quantize_mxfp4(b)
-        y = wq.gemm_fp4(dev(qa), dev(sa), dev(qb), dev(sb))
+        y = wq.gemm_fp4(dev(qa), dev(sf_to_atoms(sa)), dev(qb), dev(sf_to_atoms(sb)))
         tav = tbv = 1.0
     torch.cuda.synchronize()
     ms, ns = sample_rows(M, 64, seed=1), sample_rows(N, 96, seed=2)
@@ -717,11 +796,12 @@ def test_gemm_fp4_scale_factor_placement(wq, nv):
         sa = ((g.integers(-3, 4, (M, K // bs)) + 7) << 3).astype(np.uint8)
         sb = np.full((N, K // bs), 7 << 3, np.uint8)                # 1.0
         one = np.ones(1, np.float32)
-        y, acc = wq.gemm_fp4(dev(qa), dev(sa), dev(qb), dev(sb), dev(one), dev(one), return_acc=True)
+        y, acc = wq.gemm_fp4(dev(qa), dev(sf_to_atoms(sa)), dev(qb), dev(sf_to_atoms(sb)), dev(one), dev(one),
+                             return_acc=True)
     else:
         sa = (g.integers(-3, 4, (M, K // bs)) + 127).astype(np.uint8)
         sb = np.full((N, K // bs), 127, np.uint8)
-        y, acc = wq.gemm_fp4(dev(qa), dev(sa), dev(qb), dev(sb), return_acc=True)
+        y, acc = wq.gemm_fp4(dev(qa), dev(sf_to_atoms(sa)), dev(qb), dev(sf_to_atoms(sb)), return_acc=True)
     torch.cuda.synchronize()
     ry, _ = oracle.gemm_fp4_ref(nv, qa, sa, 1.0, qb, sb, 1.0, K)
     assert np.array_equal(host(acc).astype(np.float64), ry)
@@ -750,7 +830,9 @@ def test_fp4_w4a4_full_size(wq):
             rqx, rsx = oracle.quantize_mxfp4(X[ms])
             tv = (1.0, 1.0)
         torch.cuda.synchronize()
-        hqx, hsx, hqw, hsw = host(qx), host(sx), host(qw), host(sw)
+        F = K // (16 if nv else 32)
+        hqx, hqw = host(qx), host(qw)
+        hsx, hsw = sf_from_atoms(host(sx), M, F), sf_from_atoms(host(sw), N, F)
         assert np.array_equal(hqx[ms], rqx[ms] if nv else rqx) and np.array_equal(hsx[ms], rsx[ms] if nv else rsx)
         ry, rb = oracle.gemm_fp4_ref(nv, hqx, hsx, tv[0], hqw, hsw, tv[1], K, ms, ns)
         assert_within_bound(host(y)[np.ix_(ms, ns)].astype(np.float64), ry, rb, f"fp4 full nv={nv}")
