@@ -62,6 +62,8 @@ struct Fmt {
     static constexpr uint32_t SF_COLS = 2 * G * 4;    // TMEM columns of one stage's factors
     static constexpr uint32_t IDESC = make_idesc_fp4(NV ? 0u : 1u, BM, BN);
     static constexpr size_t SMEM = 1024 + STAGES * STAGE_BYTES + 256;
+    static_assert(SF_TMEM0 + STAGES * SF_COLS <= TMEM_COLS, "scale-factor slots fit in tensor memory");
+    static_assert(SMEM <= 232448, "fits the 227 KB of shared memory a CTA may use");
 };
 
 struct Smem {

@@ -481,8 +481,17 @@ __global__ void __launch_bounds__(THREADS, 1)
                         r[j + e] = FP8 ? __float_as_uint(__uint_as_float(r[j + e]) + __uint_as_float(o[e]))
                                        : r[j + e] + o[e];
                 }
-                if (m < M && nb + c * 32 < N)
+                if (OUTL) {
+                    if (nb + c * 32 < N) {  // warp-uniform: the whole warp runs the outlier MMAs
+                        float o16[32];
+                        float *tr = reinterpret_cast<float *>(base + STAGES * STAGE_BYTES + 256) +
+                                    (warp - 2) * 32 * TR_PITCH;
+                        outlier_chunk(ol, M, N, m - row + q * 32, nb + c * 32, lane, tr, o16);
+                        if (m < M) store_chunk_outliers(y, m, nb + c * 32, N, sxm, sw, r, o16, vec_ok);
+                    }
+                } else if (m < M && nb + c * 32 < N) {
                     store_chunk<FP8>(y, acc_out, m, nb + c * 32, N, sxm, sw, sw_stride, r, vec_ok);
+                }
             }
         }
     }
@@ -502,10 +511,11 @@ namespace {
 // CTA pairs (clusters of 2, one CTA per SM) that can be resident at once, at most half the SMs;
 // 0 if the query fails.  Cached per device.
 int split_pairs(const void *kern, size_t smem, int sms) {
-    static int cached[64] = {};
+    static int cached[64][2] = {};  // per device, per shared-memory size (plain / LLM.int8())
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-    if (cached[dev]) return cached[dev] > 0 ? cached[dev] : 0;
+    int &slot = cached[dev][smem > SMEM_BYTES ? 1 : 0];
+    if (slot) return slot > 0 ? slot : 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (sms / 2));
     cfg.blockDim = dim3(THREADS);
@@ -523,7 +533,7 @@ int split_pairs(const void *kern, size_t smem, int sms) {
         clusters = -1;
     }
     const int pairs = clusters > 0 ? std::min(clusters, sms / 2) : -1;
-    cached[dev] = pairs;
+    slot = pairs;
     return pairs > 0 ? pairs : 0;
 }
 
@@ -551,8 +561,8 @@ wq_status launch_gemm(const void *xq, const float *sx, int sx_stride, const void
     const int kblocks = (K + BK - 1) / BK;
     // Split schedule when the tiles left after whole rounds fit one per CTA pair: the last
     // round then takes half a tile's time instead of a whole one.
-    if (!OUTL && kblocks >= 2 && tiles > sms) {
-        auto kern = gemm_w8a8_kernel<FP8, false, true>;
+    if (kblocks >= 2 && tiles > sms) {
+        auto kern = gemm_w8a8_kernel<FP8, OUTL, true>;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess)
             return fail(WQ_ERR_CUDA, "%s: cudaFuncSetAttribute failed: %s", who, cudaGetErrorString(e));

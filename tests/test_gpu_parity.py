@@ -655,6 +655,26 @@ def test_llm_int8_small(wq, M, N, K, planted, cap):
     assert wq.device_status() == 0
 
 
+def test_llm_int8_split_last_round(wq):
+    # 160 tiles of 128 x 256 on 148 SMs: the last 12 are shared by CTA pairs (each half of K, the
+    # halves summed through distributed shared memory), and their epilogue adds the outlier product.
+    M, N, K = 1280, 4096, 512
+    x, wq8, sw = _llm_inputs(M, N, K, tuple(range(5, K, 37)), seed=23)
+    xd, wd, sd = dev(x), dev(wq8), dev(sw)
+    y, count = wq.llm_int8_matmul(xd, wd, sd, 6.0, 16)
+    torch.cuda.synchronize()
+    ridx, total = oracle.outlier_columns(x, 6.0, 16)
+    assert int(host(count)[0]) == total
+    ms = np.arange(M, dtype=np.int32)
+    ns = np.arange(14 * 256, 16 * 256, dtype=np.int32)
+    ry, rb, _, _ = oracle.llm_int8_ref(x, wq8, sw, ridx, ms, ns)
+    assert_within_bound(host(y)[:, ns].astype(np.float64), ry, rb, "llm.int8 split round")
+    ms2, ns2 = sample_rows(M, 64, seed=5), sample_rows(N, 64, seed=6)
+    ry2, rb2, _, _ = oracle.llm_int8_ref(x, wq8, sw, ridx, ms2, ns2)
+    assert_within_bound(host(y)[np.ix_(ms2, ns2)].astype(np.float64), ry2, rb2, "llm.int8 split sample")
+    assert wq.device_status() == 0
+
+
 def test_llm_int8_full_size(wq):
     # The W8A8 layer's activations (64 outlier channels x60) through the whole sequence at
     # threshold 6: the 64 planted columns are carved out; sampled rows checked one by one.
