@@ -403,6 +403,9 @@ __global__ void __launch_bounds__(256, G >= 256 ? 2 : 4) quant_int4_group_f16w_k
 // takes one unit of a stage, frees the slot as soon as its data is in registers and writes
 // its results straight to global memory.
 constexpr unsigned kQ4RingSite = 0x2000;
+// Waiting threads sleep inside mbarrier.try_wait (up to this long per test) instead of polling:
+// the kernel is issue-bound, and the polling took issue slots (measured 2% faster).
+constexpr uint32_t kQ4SleepNs = 20000;
 
 template <int G>
 struct Q4Ring {
@@ -447,7 +450,7 @@ __global__ void __launch_bounds__(288, G >= 256 ? 2 : 3)
             for (; issued < mine; ++issued) {
                 const int slot = (int)(issued % RL::S);
                 const uint32_t u = (uint32_t)(issued / RL::S);
-                if (!wait_parity(smem_u32(&empty[slot]), (u & 1u) ^ 1u, ctl, kQ4RingSite | 0x1)) break;
+                if (!wait_parity(smem_u32(&empty[slot]), (u & 1u) ^ 1u, ctl, kQ4RingSite | 0x1, kQ4SleepNs)) break;
                 const long long u0 = (blockIdx.x + issued * gridDim.x) * 8;
                 const uint32_t bytes = (uint32_t)(min(8ll, units - u0) * P::UE * 2);
                 const uint32_t fb = smem_u32(&full[slot]);
@@ -461,7 +464,7 @@ __global__ void __launch_bounds__(288, G >= 256 ? 2 : 3)
             const int slot = (int)(i % RL::S);
             const uint32_t u = (uint32_t)(i / RL::S);
             // warp-uniform: the lanes leave together (the shuffles below need the whole warp)
-            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&full[slot]), u & 1u, ctl, kQ4RingSite))) break;
+            if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&full[slot]), u & 1u, ctl, kQ4RingSite, kQ4SleepNs))) break;
             const long long unit = (blockIdx.x + i * gridDim.x) * 8 + warp;
             uint4 raw[P::V];
             const uint4 *src = reinterpret_cast<const uint4 *>(base + (uint32_t)slot * RL::STAGE +

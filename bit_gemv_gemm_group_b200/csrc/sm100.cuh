@@ -54,6 +54,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test, letting the thread sleep until the phase completes or about `hint_ns`
+// passes, so that a waiting thread does not spend issue slots polling.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Abort/timeout bookkeeping shared by the roles of one CTA.
 struct WaitCtl {
     volatile int *abort;    // shared-memory flag, nonzero once any role gave up
@@ -63,12 +77,14 @@ struct WaitCtl {
 
 // Waits for the phase of `bar` with parity `parity` to complete.  Returns
 // false (after recording `site`) if the limit runs out or another role of the
-// CTA has already given up.
-__device__ __forceinline__ bool wait_parity(uint32_t bar, uint32_t parity, const WaitCtl &c, unsigned site) {
+// CTA has already given up.  sleep_hint_ns > 0 lets each test suspend the
+// thread for up to that long instead of returning at once.
+__device__ __forceinline__ bool wait_parity(uint32_t bar, uint32_t parity, const WaitCtl &c, unsigned site,
+                                            uint32_t sleep_hint_ns = 0) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (sleep_hint_ns ? mbar_try_wait_sleep(bar, parity, sleep_hint_ns) : mbar_try_wait(bar, parity)) return true;
         if (*c.abort) return false;
         if (globaltimer() - t0 > c.limit_ns) {
             *c.abort = 1;
