@@ -148,20 +148,31 @@ __device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
     return d;
 }
 
-// rne(w * rs) + z of an fp16 pair as int16x2, with magic = 1.5 * 2^23 + z: one fused
-// multiply-add rounds w * rs + magic to an integer, which is magic + rne(w * rs) away from a
-// tie (at a tie the parity of z decides, and the guard band below catches it).  magic - r is
-// exact (Sterbenz), so d = w * rs + (magic - r) is the remainder rounded once; `ok` keeps the
-// sign bit of d^2 - (1/2 - 2^-16)^2, which stays set while no lane lies in the guard band.
-__device__ __forceinline__ uint32_t pair_rne(uint32_t h2, float rs, float magic, uint32_t &ok) {
-    constexpr float kGuardSq = (0.5f - 0x1p-16f) * (0.5f - 0x1p-16f);
+// rne(w / s) + z of an fp16 pair as int16x2, exactly, without a division: rs_lo and rs_hi are
+// RN(1/s) one ulp down and one ulp up (so rs_lo < 1/s < rs_hi), magic = 1.5 * 2^23 + z.
+//  - For fp16 w and s with |w / s| < 32, w / s is either exactly a half-integer or at least
+//    2^-13 away from every half-integer (w / s = M_w 2^c / M_s with 11-bit M_w, M_s; a
+//    nonzero distance is at least 1 / (2 M_s 2^max(-c, 0)) >= 1/8190).  w rs_lo and w rs_hi
+//    are within 1.5 2^-23 |w / s| < 2^-17 of w / s, so off a tie both round (one fused
+//    multiply-add each, rounding w rs + magic to an integer) to rne(w / s) + z, which is also
+//    rne(fl(w / s)) + z (fl(w / s) is within 2^-19).
+//  - At an exact tie k + 1/2 the two products lie strictly on either side of it (rs_lo <
+//    1/s < rs_hi), so one gives k + z and the other k + 1 + z; fl(w / s) = k + 1/2 exactly
+//    and rounds to the even of k, k + 1, which is the candidate whose code - z is even.
+//  - The fused sums never sit exactly on a half-integer themselves: that would need rs_lo or
+//    rs_hi to have at most 6 significant bits, and a float within 1.5 ulp of 1/s has that few
+//    only if s is a power of two, whose RN(1/s) -+ 1 ulp have 24.
+// zz holds z mod 2 in both 16-bit lanes.
+__device__ __forceinline__ uint32_t pair_code(uint32_t h2, float rs_lo, float rs_hi, float magic, uint32_t zz) {
     const float2 f = half2_bits_to_float2(h2);
-    const float2 r = __ffma2_rn(f, make_float2(rs, rs), make_float2(magic, magic));
-    const float2 m = __ffma2_rn(r, make_float2(-1.0f, -1.0f), make_float2(magic, magic));
-    const float2 d = __ffma2_rn(f, make_float2(rs, rs), m);
-    const float2 e = __ffma2_rn(d, d, make_float2(-kGuardSq, -kGuardSq));
-    ok &= __float_as_uint(e.x) & __float_as_uint(e.y);
-    return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);  // low 16 bits: rne(t) + z
+    const float2 rl = __ffma2_rn(f, make_float2(rs_lo, rs_lo), make_float2(magic, magic));
+    const float2 rh = __ffma2_rn(f, make_float2(rs_hi, rs_hi), make_float2(magic, magic));
+    const uint32_t pl = __byte_perm(__float_as_uint(rl.x), __float_as_uint(rl.y), 0x5410);
+    const uint32_t ph = __byte_perm(__float_as_uint(rh.x), __float_as_uint(rh.y), 0x5410);
+    // take ph in a lane where the candidates differ and pl's code - z is odd
+    const uint32_t sel = (pl ^ ph) & (pl ^ zz) & 0x00010001u;
+    const uint32_t mask = sel * 0xFFFFu;
+    return (ph & mask) | (pl & ~mask);
 }
 
 // int16x2 -> each half clamped to [0, 15] in one instruction
@@ -227,22 +238,12 @@ __global__ void __launch_bounds__(256) quant_int4_group_f16_kernel(const uint16_
         // z = round(-lo / s) in [0, 15]; |-lo / s| and |w / s| stay below 32 (E = 4)
         const int z = clampi(rne_quotient<4>(-lo, s, rs), 0, 15);
         if (j < groups) {
-            uint32_t ok = ~0u;
             const float magic = 12582912.0f + (float)z;  // 1.5 * 2^23 + z
-            uint32_t p0 = pair_rne(c.x, rs, magic, ok), p1 = pair_rne(c.y, rs, magic, ok);
-            uint32_t p2 = pair_rne(c.z, rs, magic, ok), p3 = pair_rne(c.w, rs, magic, ok);
-            if (!(ok >> 31)) {  // a near-tie: the IEEE quotient decides every code of this lane
-                const uint32_t h[4] = {c.x, c.y, c.z, c.w};
-                uint32_t pp[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = half2_bits_to_float2(h[e]);
-                    const uint32_t a = (uint32_t)(__float2int_rn(__fdiv_rn(f.x, s)) + z) & 0xFFFFu;
-                    const uint32_t b = (uint32_t)(__float2int_rn(__fdiv_rn(f.y, s)) + z) & 0xFFFFu;
-                    pp[e] = a | (b << 16);
-                }
-                p0 = pp[0]; p1 = pp[1]; p2 = pp[2]; p3 = pp[3];
-            }
+            const float rs_lo = __uint_as_float(__float_as_uint(rs) - 1u);
+            const float rs_hi = __uint_as_float(__float_as_uint(rs) + 1u);
+            const uint32_t zz = (uint32_t)(z & 1) * 0x00010001u;
+            uint32_t p0 = pair_code(c.x, rs_lo, rs_hi, magic, zz), p1 = pair_code(c.y, rs_lo, rs_hi, magic, zz);
+            uint32_t p2 = pair_code(c.z, rs_lo, rs_hi, magic, zz), p3 = pair_code(c.w, rs_lo, rs_hi, magic, zz);
             p0 = clamp15x2(p0);
             p1 = clamp15x2(p1);
             p2 = clamp15x2(p2);
@@ -319,26 +320,14 @@ __device__ __forceinline__ void quantize_lane(const uint4 (&raw)[Wide<G>::V], ui
     const int z = clampi(rne_quotient<4>(-lo, s, rs), 0, 15);
     const float magic = 12582912.0f + (float)z;  // 1.5 * 2^23 + z
 
-    uint32_t ok = ~0u;
+    const float rs_lo = __uint_as_float(__float_as_uint(rs) - 1u), rs_hi = __uint_as_float(__float_as_uint(rs) + 1u);
+    const uint32_t zz = (uint32_t)(z & 1) * 0x00010001u;
 #pragma unroll
     for (int v = 0; v < P::V; ++v)
-        words[v] = pack8(clamp15x2(pair_rne(raw[v].x, rs, magic, ok)), clamp15x2(pair_rne(raw[v].y, rs, magic, ok)),
-                         clamp15x2(pair_rne(raw[v].z, rs, magic, ok)), clamp15x2(pair_rne(raw[v].w, rs, magic, ok)));
-    if (!(ok >> 31)) {  // a near-tie: the IEEE quotient decides every code of this lane
-#pragma unroll
-        for (int v = 0; v < P::V; ++v) {
-            const uint32_t h[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
-            uint32_t pp[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = half2_bits_to_float2(h[e]);
-                const uint32_t a = (uint32_t)(__float2int_rn(__fdiv_rn(f.x, s)) + z) & 0xFFFFu;
-                const uint32_t b = (uint32_t)(__float2int_rn(__fdiv_rn(f.y, s)) + z) & 0xFFFFu;
-                pp[e] = clamp15x2(a | (b << 16));
-            }
-            words[v] = pack8(pp[0], pp[1], pp[2], pp[3]);
-        }
-    }
+        words[v] = pack8(clamp15x2(pair_code(raw[v].x, rs_lo, rs_hi, magic, zz)),
+                         clamp15x2(pair_code(raw[v].y, rs_lo, rs_hi, magic, zz)),
+                         clamp15x2(pair_code(raw[v].z, rs_lo, rs_hi, magic, zz)),
+                         clamp15x2(pair_code(raw[v].w, rs_lo, rs_hi, magic, zz)));
     s16_out = s16;
     z_out = z;
 }

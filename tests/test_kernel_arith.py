@@ -22,3 +22,40 @@ def test_div15_by_fp64_product_is_correctly_rounded():
     d32 = np.arange(0, 1 << 12, dtype=np.float32)
     assert np.array_equal((d32 / np.float32(15.0)).view(np.uint32),
                           (d32.astype(np.float64) * inv15).astype(np.float32).view(np.uint32))
+
+
+def _round_pair_rule(w, s):
+    """The fp16 INT4 quantizer's division-free rounding: candidates from RN(1/s) one ulp down
+    and one ulp up, the even one where they differ.  Returns (codes, any exact half-integer
+    products); products are exact in fp64 (11-bit x 24-bit significands)."""
+    rs = (np.float32(1.0) / np.float32(s)).astype(np.float32)
+    bits = rs.view(np.uint32)
+    rs_lo = (bits - np.uint32(1)).view(np.float32).astype(np.float64)
+    rs_hi = (bits + np.uint32(1)).view(np.float32).astype(np.float64)
+    x_lo, x_hi = w * rs_lo, w * rs_hi
+    half = np.any(np.abs(x_lo - np.floor(x_lo)) == 0.5) or np.any(np.abs(x_hi - np.floor(x_hi)) == 0.5)
+    n_lo, n_hi = np.rint(x_lo), np.rint(x_hi)
+    pick_hi = (n_lo != n_hi) & (np.mod(n_lo, 2) != 0)
+    return np.where(pick_hi, n_hi, n_lo), half
+
+
+def test_int4_division_free_rounding_is_exact():
+    # For fp16 weights w and fp16 scales s with |w / s| < 32 the rule must give rne(fl32(w / s))
+    # for every w, and no fused sum may land exactly on a half-integer (where the hardware's
+    # own tie-break would decide).  All finite fp16 w; every power-of-two s and 3000 others.
+    hw = np.arange(0x10000, dtype=np.uint32).astype(np.uint16)
+    w16 = hw.view(np.float16)
+    w16 = w16[np.isfinite(w16)]
+    w = w16.astype(np.float64)
+    g = np.random.default_rng(11)
+    pos = np.arange(1, 0x7C00, dtype=np.uint16)
+    pow2 = pos[(pos & 0x3FF) == 0]
+    sub_pow2 = np.array([1 << i for i in range(10)], np.uint16)
+    pick = np.concatenate([pow2, sub_pow2, g.choice(pos, 3000, replace=False)])
+    for sb in pick:
+        s = np.float64(np.array([sb], np.uint16).view(np.float16)[0])
+        ww = w[np.abs(w / s) < 32]
+        got, half = _round_pair_rule(ww, s)
+        ref = np.rint((ww.astype(np.float32) / np.float32(s)).astype(np.float64))
+        assert not half, sb
+        assert np.array_equal(got, ref), (sb, ww[got != ref][:4])
