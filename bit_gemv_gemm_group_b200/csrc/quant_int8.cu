@@ -53,6 +53,13 @@ __device__ __forceinline__ void smooth8(float (&v)[8], const float *__restrict__
     }
 }
 
+__device__ __forceinline__ void unpack8(const uint4 r, float (&v)[8]) {
+    const float2 a = half2_bits_to_float2(r.x), b = half2_bits_to_float2(r.y);
+    const float2 c = half2_bits_to_float2(r.z), d = half2_bits_to_float2(r.w);
+    v[0] = a.x; v[1] = a.y; v[2] = b.x; v[3] = b.y;
+    v[4] = c.x; v[5] = c.y; v[6] = d.x; v[7] = d.y;
+}
+
 __device__ __forceinline__ void load8(const uint16_t *p, float (&v)[8]) {
     const uint4 r = ld_stream_u4(p);
     const float2 a = half2_bits_to_float2(r.x), b = half2_bits_to_float2(r.y);
@@ -168,7 +175,41 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
     int8_t *qr = q + row * K;
     const int t0 = threadIdx.x * kChunk;
     float amax = 0.0f;
-    if (NCH > 0) {
+    if (NCH > 0 && MODE != kDiv) {
+        // The row stays in registers as fp16 (half the registers of fp32, so more rows are in
+        // flight per SM); the conversion (and W * s) is redone in the second pass.
+        uint4 raw[NCH > 0 ? NCH : 1];
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int k = c * kRowStep + t0;
+            raw[c] = k < K ? ld_stream_u4(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int k = c * kRowStep + t0;
+            if (k < K) {
+                float v[8];
+                unpack8(raw[c], v);
+                smooth8<MODE>(v, smooth, k);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
+            }
+        }
+        const float a = fmaxf(tensor_amax ? __uint_as_float(*tensor_amax) : block_max(amax, red), 1e-8f);
+        const float s = __fdiv_rn(a, F::kMax);
+        const float rs = __frcp_rn(s);
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int k = c * kRowStep + t0;
+            if (k < K) {
+                float v[8];
+                unpack8(raw[c], v);
+                smooth8<MODE>(v, smooth, k);
+                *reinterpret_cast<uint2 *>(qr + k) = F::chunk(v, s, rs);
+            }
+        }
+        if (threadIdx.x == 0 && !tensor_amax) scales[row] = s;
+    } else if (NCH > 0) {
         float v[NCH > 0 ? NCH : 1][8];
 #pragma unroll
         for (int c = 0; c < NCH; ++c) {
