@@ -147,6 +147,7 @@ struct FormatTraits<kE4M3> {
     __device__ static uint2 chunk(const float (&v)[8], float s, float rs) { return quant8_e4m3(v, s, rs); }
 };
 
+template <int T = kThreads>
 __device__ __forceinline__ float block_max(float a, float *red) {
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, off));
@@ -155,21 +156,24 @@ __device__ __forceinline__ float block_max(float a, float *red) {
     __syncthreads();
     float m = red[0];
 #pragma unroll
-    for (int i = 1; i < kThreads / 32; ++i) m = fmaxf(m, red[i]);
+    for (int i = 1; i < T / 32; ++i) m = fmaxf(m, red[i]);
     return m;
 }
 
 // NCH > 0: the row is kept in registers (K <= NCH * 2048).  NCH == 0: two passes.
 // tensor_amax (FP8 per tensor): the tensor's max |x| (float bits), used instead of the
 // row's; the scale is then written by finish_tensor_scale_kernel, not here.
-template <int NCH, int MODE, int FMT = kInt8>
-__global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_t *__restrict__ x, int K,
+// T threads per row (256, or 512 for the X / s rows of 4096 < K <= 8192: measured on B200,
+// twice the threads per row hide the IEEE division better there and nowhere else).
+template <int NCH, int MODE, int FMT = kInt8, int T = kThreads>
+__global__ void __launch_bounds__(T) quant_int8_rows_kernel(const uint16_t *__restrict__ x, int K,
                                                                    const float *__restrict__ smooth,
                                                                    int8_t *__restrict__ q,
                                                                    float *__restrict__ scales,
                                                                    const unsigned int *__restrict__ tensor_amax = nullptr) {
     using F = FormatTraits<FMT>;
-    __shared__ float red[kThreads / 32];
+    constexpr int kRowStep = T * kChunk;
+    __shared__ float red[T / 32];
     const size_t row = blockIdx.x;
     const uint16_t *xr = x + row * K;
     int8_t *qr = q + row * K;
@@ -195,7 +199,7 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
                 for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
             }
         }
-        const float a = fmaxf(tensor_amax ? __uint_as_float(*tensor_amax) : block_max(amax, red), 1e-8f);
+        const float a = fmaxf(tensor_amax ? __uint_as_float(*tensor_amax) : block_max<T>(amax, red), 1e-8f);
         const float s = __fdiv_rn(a, F::kMax);
         const float rs = __frcp_rn(s);
 #pragma unroll
@@ -221,7 +225,7 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
                 for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[c][e]));
             }
         }
-        const float a = fmaxf(tensor_amax ? __uint_as_float(*tensor_amax) : block_max(amax, red), 1e-8f);
+        const float a = fmaxf(tensor_amax ? __uint_as_float(*tensor_amax) : block_max<T>(amax, red), 1e-8f);
         const float s = __fdiv_rn(a, F::kMax);
         const float rs = __frcp_rn(s);
 #pragma unroll
@@ -252,7 +256,7 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_kernel(const uint16_
 #pragma unroll
             for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[e]));
         }
-        const float a = fmaxf(tensor_amax ? __uint_as_float(*tensor_amax) : block_max(amax, red), 1e-8f);
+        const float a = fmaxf(tensor_amax ? __uint_as_float(*tensor_amax) : block_max<T>(amax, red), 1e-8f);
         const float s = __fdiv_rn(a, F::kMax);
         const float rs = __frcp_rn(s);
         for (int k = t0; k < K; k += kRowStep) {
@@ -350,6 +354,10 @@ cudaError_t launch_mode(const uint16_t *x, int R, int K, const float *smooth, in
     if (!tensor_amax && nch > 4 && nch <= 8 && R < 65536 && K % 16 == 0)
         return launch_cluster<2, MODE, FMT>(x, R, K, smooth, q, scales, st);
     dim3 grid(R), block(kThreads);
+    if (MODE == kDiv && !tensor_amax && K > 4096 && K <= 8192) {
+        quant_int8_rows_kernel<2, MODE, FMT, 512><<<grid, dim3(512), 0, st>>>(x, K, smooth, q, scales, tensor_amax);
+        return cudaGetLastError();
+    }
     if (nch <= 1)
         quant_int8_rows_kernel<1, MODE, FMT><<<grid, block, 0, st>>>(x, K, smooth, q, scales, tensor_amax);
     else if (nch <= 2)

@@ -250,8 +250,8 @@ def test_gemv_w4a16_large_shapes_tile_boundaries(wq, N, K, B):
 # --------------------------------------------------------------------------
 # INT8 quantizers and smoothing
 # --------------------------------------------------------------------------
-INT8_SMALL = [(1, 16), (7, 48), (33, 2048), (5, 2064), (64, 4096), (3, 16384), (2, 16400), (4, 40960),
-              (5, 28672), (3, 32768), (2, 24592)]
+INT8_SMALL = [(1, 16), (7, 48), (33, 2048), (5, 2064), (64, 4096), (3, 4112), (6, 6000), (9, 8192), (3, 16384),
+              (2, 16400), (4, 40960), (5, 28672), (3, 32768), (2, 24592)]
 
 
 @pytest.mark.parametrize("R,K", INT8_SMALL)
