@@ -387,10 +387,14 @@ __global__ void __launch_bounds__(256, G >= 256 ? 2 : 4) quant_int4_group_f16w_k
 // the codes, scales and zero words of unit u start at u's element offset divided by 8, G and
 // 8 G.  A persistent CTA of 8 quantizing warps and one copy warp walks stages of 8
 // consecutive units (16 KB of fp16; 32 KB for G = 256), stages blockIdx.x + i gridDim.x;
-// the copy warp keeps the CTA's next S stages in flight with 1-D bulk copies into a ring of
-// shared-memory slots, so the loads never wait for the arithmetic, and each quantizing warp
-// takes one unit of a stage, frees the slot as soon as its data is in registers and writes
-// its results straight to global memory.
+// the copy warp keeps the CTA's next S stages in flight in a ring of shared-memory slots, so
+// the loads never wait for the arithmetic, and each quantizing warp takes one unit of a
+// stage, frees the slot as soon as its data is in registers and writes its results straight
+// to global memory.  A stage arrives by one 2-D TMA copy of the matrix seen as rows of 128
+// bytes, with the 128-byte swizzle (16-byte chunk c of row r lands at chunk c ^ (r mod 8)):
+// a lane's E contiguous weights start 64 or 128 bytes after its neighbour's, so unswizzled
+// its 16-byte loads would meet on the same banks (16- or 32-way); swizzled, a warp's load
+// spreads over all 32 banks.
 constexpr unsigned kQ4RingSite = 0x2000;
 // Waiting threads sleep inside mbarrier.try_wait (up to this long per test) instead of polling:
 // the kernel is issue-bound, and the polling took issue slots (measured 2% faster).
@@ -400,20 +404,23 @@ template <int G>
 struct Q4Ring {
     static constexpr uint32_t STAGE = 8u * Wide<G>::UE * 2u;  // bytes per stage
     static constexpr int S = G >= 256 ? 2 : 4;                // slots: three CTAs per SM
+    static constexpr uint32_t ROWS = STAGE / 128;                // 128-byte rows per stage (TMA box)
     static constexpr uint32_t OFF_BAR = S * STAGE;
-    static constexpr uint32_t SMEM = 128 + OFF_BAR + 16u * S + 16u;
+    static constexpr uint32_t SMEM = 1024 + OFF_BAR + 16u * S + 16u;  // slots 1024-byte aligned (swizzle)
+    static_assert(ROWS <= 256, "TMA box height");
 };
 
 template <int G>
 __global__ void __launch_bounds__(288, G >= 256 ? 2 : 3)
-    quant_int4_group_ring_kernel(const uint16_t *__restrict__ w, long long units, uint32_t *__restrict__ qweight,
+    quant_int4_group_ring_kernel(const __grid_constant__ CUtensorMap tmap_w, long long units,
+                                 uint32_t *__restrict__ qweight,
                                  uint16_t *__restrict__ scales, uint32_t *__restrict__ qzeros, unsigned int *status,
                                  uint64_t limit_ns) {
     using namespace sm100;
     using P = Wide<G>;
     using RL = Q4Ring<G>;
     extern __shared__ uint8_t q4_ring_raw[];
-    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q4_ring_raw) + 127) & ~uintptr_t(127));
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(q4_ring_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(base + RL::OFF_BAR);
     uint64_t *empty = full + RL::S;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(empty + RL::S);
@@ -436,15 +443,17 @@ __global__ void __launch_bounds__(288, G >= 256 ? 2 : 3)
     if (warp == 8) {
         // ------------------------------------------------------------ copy warp
         if (lane == 0) {
+            prefetch_tmap(&tmap_w);
             for (; issued < mine; ++issued) {
                 const int slot = (int)(issued % RL::S);
                 const uint32_t u = (uint32_t)(issued / RL::S);
                 if (!wait_parity(smem_u32(&empty[slot]), (u & 1u) ^ 1u, ctl, kQ4RingSite | 0x1, kQ4SleepNs)) break;
                 const long long u0 = (blockIdx.x + issued * gridDim.x) * 8;
-                const uint32_t bytes = (uint32_t)(min(8ll, units - u0) * P::UE * 2);
                 const uint32_t fb = smem_u32(&full[slot]);
-                mbar_arrive_expect_tx(fb, bytes);
-                bulk_load(smem_u32(base + (uint32_t)slot * RL::STAGE), w + u0 * P::UE, bytes, fb);
+                // rows past the matrix (a last, partial stage) arrive as zeros and count in full
+                mbar_arrive_expect_tx(fb, RL::STAGE);
+                tma_load_2d(smem_u32(base + (uint32_t)slot * RL::STAGE), &tmap_w, fb, 0,
+                            (int)(u0 * (P::UE * 2 / 128)));
             }
         }
     } else {
@@ -456,10 +465,13 @@ __global__ void __launch_bounds__(288, G >= 256 ? 2 : 3)
             if (!__all_sync(0xffffffffu, wait_parity(smem_u32(&full[slot]), u & 1u, ctl, kQ4RingSite, kQ4SleepNs))) break;
             const long long unit = (blockIdx.x + i * gridDim.x) * 8 + warp;
             uint4 raw[P::V];
-            const uint4 *src = reinterpret_cast<const uint4 *>(base + (uint32_t)slot * RL::STAGE +
-                                                               (uint32_t)warp * P::UE * 2 + (uint32_t)lane * P::E * 2);
+            // this lane's E weights: row r of the stage, chunks c0 .. c0 + V - 1, stored swizzled
+            const uint32_t pos = (uint32_t)warp * P::UE * 2 + (uint32_t)lane * P::E * 2;
+            const uint32_t row = pos >> 7, c0 = (pos & 127u) >> 4;
+            const uint8_t *rp = base + (uint32_t)slot * RL::STAGE + row * 128u;
 #pragma unroll
-            for (int v = 0; v < P::V; ++v) raw[v] = src[v];
+            for (int v = 0; v < P::V; ++v)
+                raw[v] = *reinterpret_cast<const uint4 *>(rp + (((c0 + (uint32_t)v) ^ (row & 7u)) << 4));
             // Every lane orders its reads of the slot before the copy engine's next write into it
             // (generic -> async proxy), then the warp releases the slot.
             fence_proxy_async_smem();
@@ -511,8 +523,11 @@ cudaError_t launch(const void *w, int N, int K, uint32_t *qweight, uint16_t *sca
             const long long total = (long long)N * (K / Wide<GW>::UE);
             const long long stages = (total + 7) / 8;
             const int grid = (int)std::min<long long>(stages, (long long)num_sms() * std::max(per_sm, 1));
-            kern<<<grid, 288, RL::SMEM, stream>>>(static_cast<const uint16_t *>(w), total, qweight, scales, qzeros,
-                                                  status, wait_limit());
+            CUtensorMap tmap;
+            if (!encode_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, w, 64, (uint64_t)total * (Wide<GW>::UE / 64),
+                                128, 64, RL::ROWS, CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+            kern<<<grid, 288, RL::SMEM, stream>>>(tmap, total, qweight, scales, qzeros, status, wait_limit());
             return cudaGetLastError();
         }
         const dim3 grid((unsigned)((N + 7) / 8), (unsigned)((K + Wide<GW>::UE - 1) / Wide<GW>::UE));
