@@ -88,6 +88,7 @@ struct Layout {
     static constexpr uint32_t PIPE_BYTES = OFF_P + PSTAGES * P_BYTES;  // reused for split-K partials
     static constexpr size_t SMEM = 1024 + PIPE_BYTES + 1024;  // alignment slack + barriers
     static_assert(STAGES >= 2, "tensor memory holds at least two A stages");
+    static_assert(OFF_P % 256 == 0, "packed tiles keep the 32-byte swizzle's 256-byte period");
 };
 
 struct Bars {
@@ -320,7 +321,7 @@ __global__ void __launch_bounds__(THREADS, Layout<MT>::CTAS_PER_SM)
             uint4 w;
             asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                          : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
-                         : "r"(sP + p * P_BYTES + row * 32 + half * 16));
+                         : "r"(sP + p * P_BYTES + row * 32 + ((half ^ ((row >> 2) & 1)) << 4)));
             // The codes are in registers: the packed slot goes back to the producer (the proxy
             // fence orders this read before the next TMA write into the slot).
             fence_proxy_async_smem();
@@ -591,8 +592,10 @@ wq_status gemm_w4a16_entry(const uint16_t *x, int M, const uint32_t *qweight, co
     if (!status) return WQ_ERR_CUDA;
     const int MT = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
     CUtensorMap tq, tx;
+    // 32-byte swizzle: half h of row r lands at h ^ ((r / 4) mod 2), so the dequantizers' 16-byte loads
+    // (one row per lane, rows 32 bytes apart) spread over all 32 banks.
     if (!encode_tmap_2d(&tq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, qweight, (uint64_t)K / 2, (uint64_t)N, (uint64_t)K / 2,
-                        BK / 2, BMW, CU_TENSOR_MAP_SWIZZLE_NONE))
+                        BK / 2, BMW, CU_TENSOR_MAP_SWIZZLE_32B))
         return WQ_ERR_CUDA;
     if (!encode_tmap_2d(&tx, BF ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, x, (uint64_t)K,
                         (uint64_t)M, (uint64_t)K * 2, BK, MT, CU_TENSOR_MAP_SWIZZLE_128B))
