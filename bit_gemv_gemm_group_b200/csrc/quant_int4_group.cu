@@ -128,13 +128,10 @@ __global__ void __launch_bounds__(256) quant_int4_group_kernel(const TIn *__rest
 // ---------------------------------------------------------------------------
 // fp16 input: the same decomposition with packed arithmetic.  The range comes
 // from fp16x2 min/max on the raw bits (exact); a pair of codes is decided with
-// f32x2 fused operations on the exact product w * RN(1/s):
-//   r = RN(w * RN(1/s) + (1.5*2^23 + z))   (rne + z lands in r's low mantissa bits),
-//   d = RN(w * RN(1/s) - (r - (1.5*2^23 + z)))   (within 2^-25 of the true remainder).
-// w * RN(1/s) is within 2^-19 of w/s (|w/s| < 32), so the pair is exact unless
-// |d| comes within 2^-16 of 1/2, in which case the lane recomputes its codes
-// with the IEEE quotient.  Clamping (one min.relu.s16x2 per pair) and nibble
-// packing run on 16-bit SIMD lanes.
+// f32x2 fused operations on the products of w with RN(1/s) one ulp down and
+// one ulp up (pair_code below: exact without a division, ties to even).
+// Clamping (one min.relu.s16x2 per pair) and nibble packing run on 16-bit SIMD
+// lanes.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t hmin2_bits(uint32_t a, uint32_t b) {
     uint32_t d;
@@ -149,30 +146,32 @@ __device__ __forceinline__ uint32_t hmax2_bits(uint32_t a, uint32_t b) {
 }
 
 // rne(w / s) + z of an fp16 pair as int16x2, exactly, without a division: rs_lo and rs_hi are
-// RN(1/s) one ulp down and one ulp up (so rs_lo < 1/s < rs_hi), magic = 1.5 * 2^23 + z.
+// RN(1/s) one ulp down and one ulp up (so rs_lo < 1/s < rs_hi).
 //  - For fp16 w and s with |w / s| < 32, w / s is either exactly a half-integer or at least
 //    2^-13 away from every half-integer (w / s = M_w 2^c / M_s with 11-bit M_w, M_s; a
 //    nonzero distance is at least 1 / (2 M_s 2^max(-c, 0)) >= 1/8190).  w rs_lo and w rs_hi
 //    are within 1.5 2^-23 |w / s| < 2^-17 of w / s, so off a tie both round (one fused
-//    multiply-add each, rounding w rs + magic to an integer) to rne(w / s) + z, which is also
-//    rne(fl(w / s)) + z (fl(w / s) is within 2^-19).
+//    multiply-add each, rounding w rs + M, M = 1.5 * 2^23, to an integer) to rne(w / s),
+//    which is also rne(fl(w / s)) (fl(w / s) is within 2^-19).
 //  - At an exact tie k + 1/2 the two products lie strictly on either side of it (rs_lo <
-//    1/s < rs_hi), so one gives k + z and the other k + 1 + z; fl(w / s) = k + 1/2 exactly
-//    and rounds to the even of k, k + 1, which is the candidate whose code - z is even.
+//    1/s < rs_hi), so one gives M + k and the other M + k + 1; fl(w / s) = k + 1/2 exactly
+//    and rounds to the even of k, k + 1.  The mean of the two candidates, rounded once
+//    (a fused multiply-add), is M + k + 1/2 there and rounds to the even one (M is even,
+//    the ulp is 1, ties go to even); off a tie it is the common candidate itself.
 //  - The fused sums never sit exactly on a half-integer themselves: that would need rs_lo or
 //    rs_hi to have at most 6 significant bits, and a float within 1.5 ulp of 1/s has that few
 //    only if s is a power of two, whose RN(1/s) -+ 1 ulp have 24.
-// zz holds z mod 2 in both 16-bit lanes.
-__device__ __forceinline__ uint32_t pair_code(uint32_t h2, float rs_lo, float rs_hi, float magic, uint32_t zz) {
+// Adding z (an integer below 16) is exact; the low 16 bits of M + j are j as an int16.
+// All of it runs on the fp32 pipe (f32x2); the one integer instruction gathers the halves.
+__device__ __forceinline__ uint32_t pair_code(uint32_t h2, float rs_lo, float rs_hi, float zf) {
+    constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
     const float2 f = half2_bits_to_float2(h2);
-    const float2 rl = __ffma2_rn(f, make_float2(rs_lo, rs_lo), make_float2(magic, magic));
-    const float2 rh = __ffma2_rn(f, make_float2(rs_hi, rs_hi), make_float2(magic, magic));
-    const uint32_t pl = __byte_perm(__float_as_uint(rl.x), __float_as_uint(rl.y), 0x5410);
-    const uint32_t ph = __byte_perm(__float_as_uint(rh.x), __float_as_uint(rh.y), 0x5410);
-    // take ph in a lane where the candidates differ and pl's code - z is odd
-    const uint32_t sel = (pl ^ ph) & (pl ^ zz) & 0x00010001u;
-    const uint32_t mask = sel * 0xFFFFu;
-    return (ph & mask) | (pl & ~mask);
+    const float2 rl = __ffma2_rn(f, make_float2(rs_lo, rs_lo), make_float2(kMagic, kMagic));
+    const float2 rh = __ffma2_rn(f, make_float2(rs_hi, rs_hi), make_float2(kMagic, kMagic));
+    const float2 half_rh = __fmul2_rn(rh, make_float2(0.5f, 0.5f));                   // exact
+    const float2 mean = __ffma2_rn(rl, make_float2(0.5f, 0.5f), half_rh);             // M + rne(w / s)
+    const float2 r = __fadd2_rn(mean, make_float2(zf, zf));                           // + z, exact
+    return __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x5410);
 }
 
 // int16x2 -> each half clamped to [0, 15] in one instruction
@@ -238,12 +237,11 @@ __global__ void __launch_bounds__(256) quant_int4_group_f16_kernel(const uint16_
         // z = round(-lo / s) in [0, 15]; |-lo / s| and |w / s| stay below 32 (E = 4)
         const int z = clampi(rne_quotient<4>(-lo, s, rs), 0, 15);
         if (j < groups) {
-            const float magic = 12582912.0f + (float)z;  // 1.5 * 2^23 + z
+            const float zf = (float)z;
             const float rs_lo = __uint_as_float(__float_as_uint(rs) - 1u);
             const float rs_hi = __uint_as_float(__float_as_uint(rs) + 1u);
-            const uint32_t zz = (uint32_t)(z & 1) * 0x00010001u;
-            uint32_t p0 = pair_code(c.x, rs_lo, rs_hi, magic, zz), p1 = pair_code(c.y, rs_lo, rs_hi, magic, zz);
-            uint32_t p2 = pair_code(c.z, rs_lo, rs_hi, magic, zz), p3 = pair_code(c.w, rs_lo, rs_hi, magic, zz);
+            uint32_t p0 = pair_code(c.x, rs_lo, rs_hi, zf), p1 = pair_code(c.y, rs_lo, rs_hi, zf);
+            uint32_t p2 = pair_code(c.z, rs_lo, rs_hi, zf), p3 = pair_code(c.w, rs_lo, rs_hi, zf);
             p0 = clamp15x2(p0);
             p1 = clamp15x2(p1);
             p2 = clamp15x2(p2);
@@ -318,16 +316,15 @@ __device__ __forceinline__ void quantize_lane(const uint4 (&raw)[Wide<G>::V], ui
     const float rs = __frcp_rn(s);
     // z = round(-lo / s) in [0, 15]; |-lo / s| and |w / s| stay below 32 (E = 4)
     const int z = clampi(rne_quotient<4>(-lo, s, rs), 0, 15);
-    const float magic = 12582912.0f + (float)z;  // 1.5 * 2^23 + z
+    const float zf = (float)z;
 
     const float rs_lo = __uint_as_float(__float_as_uint(rs) - 1u), rs_hi = __uint_as_float(__float_as_uint(rs) + 1u);
-    const uint32_t zz = (uint32_t)(z & 1) * 0x00010001u;
 #pragma unroll
     for (int v = 0; v < P::V; ++v)
-        words[v] = pack8(clamp15x2(pair_code(raw[v].x, rs_lo, rs_hi, magic, zz)),
-                         clamp15x2(pair_code(raw[v].y, rs_lo, rs_hi, magic, zz)),
-                         clamp15x2(pair_code(raw[v].z, rs_lo, rs_hi, magic, zz)),
-                         clamp15x2(pair_code(raw[v].w, rs_lo, rs_hi, magic, zz)));
+        words[v] = pack8(clamp15x2(pair_code(raw[v].x, rs_lo, rs_hi, zf)),
+                         clamp15x2(pair_code(raw[v].y, rs_lo, rs_hi, zf)),
+                         clamp15x2(pair_code(raw[v].z, rs_lo, rs_hi, zf)),
+                         clamp15x2(pair_code(raw[v].w, rs_lo, rs_hi, zf)));
     s16_out = s16;
     z_out = z;
 }

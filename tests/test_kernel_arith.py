@@ -36,7 +36,20 @@ def _round_pair_rule(w, s):
     half = np.any(np.abs(x_lo - np.floor(x_lo)) == 0.5) or np.any(np.abs(x_hi - np.floor(x_hi)) == 0.5)
     n_lo, n_hi = np.rint(x_lo), np.rint(x_hi)
     pick_hi = (n_lo != n_hi) & (np.mod(n_lo, 2) != 0)
-    return np.where(pick_hi, n_hi, n_lo), half
+    return np.where(pick_hi, n_hi, n_lo), half, n_lo, n_hi
+
+
+def _mean_rule(n_lo, n_hi):
+    """The kernel's tie-break on the fp32 pipe: the candidates as M + n (M = 1.5 * 2^23), the
+    exact half of one plus the other times 1/2 rounded once (a fused multiply-add), minus M.
+    The fp64 sum is exact (integers and halves near 2^23), so one conversion to fp32 is the
+    fused rounding."""
+    M = np.float64(1.5 * 2.0 ** 23)
+    rl = (M + n_lo).astype(np.float32)
+    half_rh = ((M + n_hi).astype(np.float32) * np.float32(0.5)).astype(np.float32)
+    assert np.array_equal(half_rh.astype(np.float64) * 2, M + n_hi)  # the halving is exact
+    mean = (rl.astype(np.float64) * 0.5 + half_rh.astype(np.float64)).astype(np.float32)
+    return mean.astype(np.float64) - M
 
 
 def test_int4_division_free_rounding_is_exact():
@@ -55,7 +68,10 @@ def test_int4_division_free_rounding_is_exact():
     for sb in pick:
         s = np.float64(np.array([sb], np.uint16).view(np.float16)[0])
         ww = w[np.abs(w / s) < 32]
-        got, half = _round_pair_rule(ww, s)
+        got, half, n_lo, n_hi = _round_pair_rule(ww, s)
         ref = np.rint((ww.astype(np.float32) / np.float32(s)).astype(np.float64))
         assert not half, sb
         assert np.array_equal(got, ref), (sb, ww[got != ref][:4])
+        # the candidates differ by at most one, and the rounded mean picks the same code
+        assert np.all(np.abs(n_lo - n_hi) <= 1), sb
+        assert np.array_equal(_mean_rule(n_lo, n_hi), got), sb
