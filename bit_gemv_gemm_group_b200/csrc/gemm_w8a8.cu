@@ -213,6 +213,73 @@ __device__ __forceinline__ void outlier_chunk(const Outliers &ol, int M, int N, 
     for (int j = 0; j < 32; ++j) o[j] = tr[lane * TR_PITCH + j];
 }
 
+// Up to 64 carved columns (four k-steps): the epilogue keeps a warp's X_16 fragments for the
+// whole tile and fetches the W_16 fragments of the next 32-column chunk while the current one
+// is multiplied, so the chunks no longer wait for an L2 round trip each.  Fragments of k-steps
+// at or past cap are zero.
+__device__ __forceinline__ void outlier_x_frags(const Outliers &ol, int M, int r0, int lane, uint32_t (&a)[4][2][4]) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        const uint16_t *p0 = ol.x16 + (size_t)min(r0 + 16 * mt + g, M - 1) * ol.cap + 2 * t;
+        const uint16_t *p1 = ol.x16 + (size_t)min(r0 + 16 * mt + 8 + g, M - 1) * ol.cap + 2 * t;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const bool in = 16 * ks < ol.cap;
+            a[ks][mt][0] = in ? ldg_u32(p0 + 16 * ks) : 0u;
+            a[ks][mt][1] = in ? ldg_u32(p1 + 16 * ks) : 0u;
+            a[ks][mt][2] = in ? ldg_u32(p0 + 16 * ks + 8) : 0u;
+            a[ks][mt][3] = in ? ldg_u32(p1 + 16 * ks + 8) : 0u;
+        }
+    }
+}
+
+__device__ __forceinline__ void outlier_w_frags(const Outliers &ol, int N, int n0, int lane, uint32_t (&b)[4][4][2]) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+        const uint16_t *p = ol.w16 + (size_t)min(n0 + 8 * nt + g, N - 1) * ol.cap + 2 * t;
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const bool in = 16 * ks < ol.cap;
+            b[ks][nt][0] = in ? ldg_u32(p + 16 * ks) : 0u;
+            b[ks][nt][1] = in ? ldg_u32(p + 16 * ks + 8) : 0u;
+        }
+    }
+}
+
+// o[j] = sum_i X_16[row of lane][i] W_16[chunk column j][i] from fragments already in registers
+// (the same MMA tiling and transpose as outlier_chunk).
+__device__ __forceinline__ void outlier_mma64(const uint32_t (&a)[4][2][4], const uint32_t (&b)[4][4][2], int lane,
+                                              float *__restrict__ tr, float (&o)[32]) {
+    const int g = lane >> 2, t = lane & 3;
+    float cf[2][4][4];
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) cf[mt][nt][0] = cf[mt][nt][1] = cf[mt][nt][2] = cf[mt][nt][3] = 0.0f;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) mma_16816_f16(cf[mt][nt], a[ks][mt], b[ks][nt][0], b[ks][nt][1]);
+    __syncwarp();  // the previous chunk's readers are done with tr
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            float *p = tr + (16 * mt + g) * TR_PITCH + 8 * nt + 2 * t;
+            p[0] = cf[mt][nt][0];
+            p[1] = cf[mt][nt][1];
+            p[8 * TR_PITCH] = cf[mt][nt][2];
+            p[8 * TR_PITCH + 1] = cf[mt][nt][3];
+        }
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) o[j] = tr[lane * TR_PITCH + j];
+}
+
 // y = fp16((acc * s_x + o) * s_w) for one row's 32-column chunk (INT8 accumulators).
 __device__ __forceinline__ void store_chunk_outliers(uint16_t *__restrict__ y, int m, int n0, int N, float sxm,
                                                      const float *__restrict__ sw, const uint32_t (&r)[32],
@@ -414,6 +481,33 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int m = (tile % mt) * BM + row;
             const int nb = (tile / mt) * BN;
             const float sxm = m < M ? __ldg(sx + m * sx_stride) : 0.0f;
+            if (OUTL && ol.cap <= 64) {
+                float *tr = reinterpret_cast<float *>(base + STAGES * STAGE_BYTES + 256) + (warp - 2) * 32 * TR_PITCH;
+                const int r0 = m - row + q * 32;
+                uint32_t xa[4][2][4], wb0[4][4][2], wb1[4][4][2];
+                outlier_x_frags(ol, M, r0, lane, xa);
+                outlier_w_frags(ol, N, nb, lane, wb0);
+                // chunks in pairs so that each W_16 buffer has a fixed register home
+#pragma unroll 1
+                for (int c = 0; c < BN / 32; c += 2) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int cc = c + h;
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + a * BN + cc * 32, r);
+                        if (cc + 1 < BN / 32) outlier_w_frags(ol, N, nb + (cc + 1) * 32, lane, h ? wb0 : wb1);
+                        tmem_ld_wait();
+                        if (nb + cc * 32 < N) {  // warp-uniform: the whole warp runs the outlier MMAs
+                            float o[32];
+                            outlier_mma64(xa, h ? wb1 : wb0, lane, tr, o);
+                            if (m < M) store_chunk_outliers(y, m, nb + cc * 32, N, sxm, sw, r, o, vec_ok);
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&sm->tmem_empty[a]));
+                continue;
+            }
 #pragma unroll 1
             for (int c = 0; c < BN / 32; ++c) {
                 uint32_t r[32];
@@ -437,16 +531,22 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (SPLIT) {
         // Every CTA of the pair is past its last wait: the MMAs of the shared tile are complete
-        // (the epilogue warps waited for them) and every TMA load has landed, so the leading CTA's
-        // pipeline buffers are free to receive the second CTA's partial accumulator.
+        // (the epilogue warps waited for them) and every TMA load has landed, so both CTAs'
+        // pipeline buffers are free.  The leading CTA stores the shared tile's columns 0..127 and
+        // the second CTA columns 128..255: each first sends the other, through distributed shared
+        // memory, the half of its partial accumulator that the other stores, so the two halves of
+        // this last, unhidden epilogue run side by side.
         cluster_sync();
         const bool epi = warp >= 2;
         const int q = warp & 3, row = q * 32 + lane;
-        uint32_t *part = reinterpret_cast<uint32_t *>(base);  // [BM][PART_PITCH] in the leading CTA
-        if (epi && split_acc >= 0 && (blockIdx.x & 1)) {
-            const uint32_t dst = mapa_shared(smem_u32(part + row * PART_PITCH), 0);
+        const uint32_t second = blockIdx.x & 1;
+        constexpr int HALF = BN / 64;                 // 32-column chunks per half
+        const int c_mine = second ? HALF : 0, c_send = second ? 0 : HALF;
+        uint32_t *part = reinterpret_cast<uint32_t *>(base);  // [BM][PART_PITCH] in each CTA of the pair
+        if (epi && split_acc >= 0) {
+            const uint32_t dst = mapa_shared(smem_u32(part + row * PART_PITCH), second ^ 1u);
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int c = c_send; c < c_send + HALF; ++c) {
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + split_acc * BN + c * 32, r);
                 tmem_ld_wait();
@@ -458,15 +558,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
         cluster_sync();
-        if (epi && split_acc >= 0 && !(blockIdx.x & 1) && !sm->abort) {
+        if (epi && split_acc >= 0 && !sm->abort) {
             const int m = (split_tile % mt) * BM + row;
             const int nb = (split_tile / mt) * BN;
             const float sxm = m < M ? __ldg(sx + m * sx_stride) : 0.0f;
             const bool vec_ok = (N % 8) == 0;
             const uint32_t src = smem_u32(part + row * PART_PITCH);
-#pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
-                uint32_t r[32];
+            float *tr = reinterpret_cast<float *>(base + STAGES * STAGE_BYTES + 256) + (warp - 2) * 32 * TR_PITCH;
+            // this CTA's partial of chunk c plus the other CTA's, which arrived in `part`
+            auto summed = [&](int c, uint32_t (&r)[32]) {
                 tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + split_acc * BN + c * 32, r);
                 tmem_ld_wait();
 #pragma unroll
@@ -481,16 +581,40 @@ __global__ void __launch_bounds__(THREADS, 1)
                         r[j + e] = FP8 ? __float_as_uint(__uint_as_float(r[j + e]) + __uint_as_float(o[e]))
                                        : r[j + e] + o[e];
                 }
-                if (OUTL) {
-                    if (nb + c * 32 < N) {  // warp-uniform: the whole warp runs the outlier MMAs
-                        float o16[32];
-                        float *tr = reinterpret_cast<float *>(base + STAGES * STAGE_BYTES + 256) +
-                                    (warp - 2) * 32 * TR_PITCH;
-                        outlier_chunk(ol, M, N, m - row + q * 32, nb + c * 32, lane, tr, o16);
-                        if (m < M) store_chunk_outliers(y, m, nb + c * 32, N, sxm, sw, r, o16, vec_ok);
+            };
+            if (OUTL && ol.cap <= 64) {
+                uint32_t xa[4][2][4], wb0[4][4][2], wb1[4][4][2];
+                outlier_x_frags(ol, M, m - row + q * 32, lane, xa);
+                outlier_w_frags(ol, N, nb + c_mine * 32, lane, wb0);
+#pragma unroll 1
+                for (int c = c_mine; c < c_mine + HALF; c += 2) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int cc = c + h;
+                        if (cc + 1 < c_mine + HALF) outlier_w_frags(ol, N, nb + (cc + 1) * 32, lane, h ? wb0 : wb1);
+                        uint32_t r[32];
+                        summed(cc, r);
+                        if (nb + cc * 32 < N) {  // warp-uniform
+                            float o16[32];
+                            outlier_mma64(xa, h ? wb1 : wb0, lane, tr, o16);
+                            if (m < M) store_chunk_outliers(y, m, nb + cc * 32, N, sxm, sw, r, o16, vec_ok);
+                        }
                     }
-                } else if (m < M && nb + c * 32 < N) {
-                    store_chunk<FP8>(y, acc_out, m, nb + c * 32, N, sxm, sw, sw_stride, r, vec_ok);
+                }
+            } else {
+#pragma unroll 1
+                for (int c = c_mine; c < c_mine + HALF; ++c) {
+                    uint32_t r[32];
+                    summed(c, r);
+                    if (OUTL) {
+                        if (nb + c * 32 < N) {  // warp-uniform: the whole warp runs the outlier MMAs
+                            float o16[32];
+                            outlier_chunk(ol, M, N, m - row + q * 32, nb + c * 32, lane, tr, o16);
+                            if (m < M) store_chunk_outliers(y, m, nb + c * 32, N, sxm, sw, r, o16, vec_ok);
+                        }
+                    } else if (m < M && nb + c * 32 < N) {
+                        store_chunk<FP8>(y, acc_out, m, nb + c * 32, N, sxm, sw, sw_stride, r, vec_ok);
+                    }
                 }
             }
         }
