@@ -44,6 +44,10 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_w8a16_kernel(const uint16_t 
 #pragma unroll
         for (int b = 0; b < B; ++b) acc[r][b] = make_float2(0.0f, 0.0f);
 
+    // Two rows per warp: four chunk steps unrolled keep more 16-byte loads in flight per lane
+    // (measured on B200: 28672x8192 batch 1 51.8 -> 49.6 us, batch 4 111 -> 99 us); one row per
+    // warp (the shapes with few rows) measured slower unrolled.
+#pragma unroll (R == 2 ? 4 : 1)
     for (int c = lane; c < chunks; c += 32) {
         const int k0 = c << 4;
         float2 wf[R][8];
