@@ -348,7 +348,7 @@ def outlier_columns(x: torch.Tensor, threshold: float = 6.0, cap: int = 64, stre
     idx[:min(count, cap)] are the carved columns (lowest first); keep is 0 there and 1 elsewhere."""
     _cuda(x, "x", (torch.float16,), 2)
     M, K = x.shape
-    idx = torch.zeros((cap,), dtype=torch.int32, device=x.device)
+    idx = _empty((cap,), torch.int32, x)  # the call writes every entry (0 past the carved ones)
     count = _empty((1,), torch.int32, x)
     keep = _empty((K,), torch.float32, x)
     _check(lib.wq_outlier_columns(_ptr(x), M, K, float(threshold), int(cap), _ptr(idx), _ptr(count), _ptr(keep),

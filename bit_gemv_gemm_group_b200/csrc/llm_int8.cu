@@ -42,7 +42,21 @@ __global__ void __launch_bounds__(kThreads) column_absmax_kernel(const uint16_t 
     const int r0 = blockIdx.y * rows_per_share, r1 = min(M, r0 + rows_per_share);
     uint32_t m[4] = {0u, 0u, 0u, 0u};  // |x| as fp16 bit pairs
     if (col < K) {
-        for (int r = r0 + warp; r < r1; r += kThreads / 32) {
+        constexpr int W = kThreads / 32;
+        int r = r0 + warp;
+        for (; r + 3 * W < r1; r += 4 * W) {  // four rows per step: four loads in flight per lane
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) v[u] = ld_stream_u4(x + (size_t)(r + u * W) * K + col);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                m[0] = __vmaxu2(m[0], v[u].x & 0x7fff7fffu);
+                m[1] = __vmaxu2(m[1], v[u].y & 0x7fff7fffu);
+                m[2] = __vmaxu2(m[2], v[u].z & 0x7fff7fffu);
+                m[3] = __vmaxu2(m[3], v[u].w & 0x7fff7fffu);
+            }
+        }
+        for (; r < r1; r += W) {
             const uint4 v = ld_stream_u4(x + (size_t)r * K + col);
             m[0] = __vmaxu2(m[0], v.x & 0x7fff7fffu);
             m[1] = __vmaxu2(m[1], v.y & 0x7fff7fffu);
@@ -63,19 +77,23 @@ __global__ void __launch_bounds__(kThreads) column_absmax_kernel(const uint16_t 
     }
 }
 
-// One CTA: thread t owns columns [t*per, (t+1)*per).  Flags (max >= threshold) are counted,
-// exclusive-scanned over the CTA, and the first `cap` flagged columns (lowest index first)
-// become the carved set: idx gets their indices, keep gets 0 there and 1 elsewhere (in place
-// of the maxima), count gets the number of flagged columns.
+// One CTA: thread t owns columns [t*per, (t+1)*per), per a multiple of 4 (K is a multiple of
+// 8), read and written as float4.  Flags (max >= threshold) are counted, exclusive-scanned over
+// the CTA, and the first `cap` flagged columns (lowest index first) become the carved set: idx
+// gets their indices (0 in its unused entries), keep gets 0 there and 1 elsewhere (in place of
+// the maxima), count gets the number of flagged columns.
 __global__ void __launch_bounds__(kScanThreads) compact_outliers_kernel(int K, float threshold, int cap,
                                                                         float *__restrict__ keep,
                                                                         int32_t *__restrict__ idx,
                                                                         int32_t *__restrict__ count) {
     __shared__ int warp_sum[kScanThreads / 32];
-    const int per = (K + kScanThreads - 1) / kScanThreads;
+    const int per = (K + 4 * kScanThreads - 1) / (4 * kScanThreads) * 4;
     const int c0 = threadIdx.x * per, c1 = min(K, c0 + per);
     int n = 0;
-    for (int c = c0; c < c1; ++c) n += keep[c] >= threshold;
+    for (int c = c0; c < c1; c += 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(keep + c);
+        n += (v.x >= threshold) + (v.y >= threshold) + (v.z >= threshold) + (v.w >= threshold);
+    }
     // inclusive scan of n over the CTA
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int s = n;
@@ -97,13 +115,26 @@ __global__ void __launch_bounds__(kScanThreads) compact_outliers_kernel(int K, f
     }
     __syncthreads();
     int pos = s - n + (warp > 0 ? warp_sum[warp - 1] : 0);  // exclusive prefix of this thread
-    for (int c = c0; c < c1; ++c) {
-        const bool out = keep[c] >= threshold;
-        if (out && pos < cap) idx[pos] = c;
-        keep[c] = (out && pos < cap) ? 0.0f : 1.0f;
-        pos += out;
+    for (int c = c0; c < c1; c += 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(keep + c);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+        float kv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const bool out = vv[e] >= threshold;
+            if (out && pos < cap) idx[pos] = c + e;
+            kv[e] = (out && pos < cap) ? 0.0f : 1.0f;
+            pos += out;
+        }
+        *reinterpret_cast<float4 *>(keep + c) = make_float4(kv[0], kv[1], kv[2], kv[3]);
     }
-    if (threadIdx.x == kScanThreads - 1) *count = pos;
+    __shared__ int total;
+    if (threadIdx.x == kScanThreads - 1) {
+        *count = pos;
+        total = pos;
+    }
+    __syncthreads();
+    for (int j = min(total, cap) + threadIdx.x; j < cap; j += kScanThreads) idx[j] = 0;  // unused entries
 }
 
 // Row r < M: X_16[r][i] = x[r][idx[i]]; row r >= M: W_16[r - M][i] = (fp16) wq[r - M][idx[i]];
@@ -116,14 +147,30 @@ __global__ void __launch_bounds__(kThreads) gather_outliers_kernel(const uint16_
                                                                    uint16_t *__restrict__ w16) {
     const int n_out = min(*count, cap);
     const size_t total = (size_t)(M + N) * cap;
-    for (size_t e = (size_t)blockIdx.x * kThreads + threadIdx.x; e < total; e += (size_t)gridDim.x * kThreads) {
-        const int r = (int)(e / cap), i = (int)(e % cap);
-        if (r < M) {
-            x16[e] = i < n_out ? x[(size_t)r * K + idx[i]] : (uint16_t)0;
-        } else {
-            const int n = r - M;
-            const float v = i < n_out ? (float)wq[(size_t)n * K + idx[i]] : 0.0f;
-            w16[(size_t)n * cap + i] = float_to_half_bits_rn(v);  // |code| <= 128: exact
+    const size_t stride = (size_t)gridDim.x * kThreads;
+    // four elements per thread and step, every load issued before the first store (the loads
+    // are scattered single elements, so only their number in flight sets the speed)
+    for (size_t e0 = (size_t)blockIdx.x * kThreads + threadIdx.x; e0 < total; e0 += 4 * stride) {
+        uint32_t v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const size_t e = e0 + u * stride;
+            v[u] = 0u;
+            if (e < total) {
+                const int r = (int)(e / cap), i = (int)(e % cap);
+                if (i < n_out)
+                    v[u] = r < M ? (uint32_t)x[(size_t)r * K + idx[i]]
+                                 : (uint32_t)float_to_half_bits_rn((float)wq[(size_t)(r - M) * K + idx[i]]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const size_t e = e0 + u * stride;
+            if (e < total) {
+                // rows < M: X_16 (fp16 bits as read); rows >= M: W_16 (|code| <= 128 is exact in fp16)
+                if (e < (size_t)M * cap) x16[e] = (uint16_t)v[u];
+                else w16[e - (size_t)M * cap] = (uint16_t)v[u];
+            }
         }
     }
 }
@@ -147,8 +194,8 @@ extern "C" wq_status wq_outlier_columns(const uint16_t *x, int M, int K, float t
     if (e != cudaSuccess)
         return fail(WQ_ERR_CUDA, "wq_outlier_columns: clearing keep failed: %s", cudaGetErrorString(e));
     const int tiles = (K + kTileCols - 1) / kTileCols;
-    // row shares: about two CTAs per SM over the whole grid, at least 8 rows each
-    const int shares = std::max(1, std::min((M + 7) / 8, (2 * num_sms() + tiles - 1) / tiles));
+    // row shares: about eight CTAs per SM over the whole grid, at least 8 rows each
+    const int shares = std::max(1, std::min((M + 7) / 8, (8 * num_sms() + tiles - 1) / tiles));
     const int rows_per_share = (M + shares - 1) / shares;
     column_absmax_kernel<<<dim3(tiles, (M + rows_per_share - 1) / rows_per_share), kThreads, 0, st>>>(
         x, M, K, rows_per_share, reinterpret_cast<unsigned int *>(keep));

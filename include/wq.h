@@ -291,7 +291,8 @@ wq_status wq_gemm_fp8(const uint8_t *xq, const float *sx, int sx_per_row, const 
  *
  * wq_outlier_columns: an outlier column is a column j of x [M][K] (fp16) with
  * max_m |x[m][j]| >= threshold.  idx (int32 [cap]) receives the first
- * min(total, cap) of them in increasing order (the ones carved out), *count
+ * min(total, cap) of them in increasing order (the ones carved out) and 0 in
+ * its remaining entries, *count
  * (int32, device) the total that qualify, keep (fp32 [K]) 0 for the carved
  * columns and 1 elsewhere (keep also serves as the call's reduction buffer).
  * K % 8 == 0; 1 <= cap <= K; threshold > 0.

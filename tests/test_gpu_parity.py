@@ -645,6 +645,7 @@ def test_llm_int8_small(wq, M, N, K, planted, cap):
     ridx, total = oracle.outlier_columns(x, 6.0, cap)
     assert int(host(count)[0]) == total
     assert np.array_equal(host(idx)[: ridx.size], ridx)
+    assert np.all(host(idx)[ridx.size:] == 0)  # the unused entries are written too
     assert np.array_equal(host(keep) == 0, np.isin(np.arange(K), ridx))
     ry, rb, rxq, rsx = oracle.llm_int8_ref(x, wq8, sw, ridx)
     assert np.array_equal(host(xq), rxq) and np.array_equal(host(sx), rsx)
