@@ -275,19 +275,23 @@ __global__ void __launch_bounds__(T) quant_int8_rows_kernel(const uint16_t *__re
     }
 }
 
-// 8192 < K <= 16384: a row is split over a cluster of C = 2 CTAs (at most
-// 8192 columns each), each keeping its (smoothed) part in registers
-// with at most 4 chunks per thread (few registers, four CTAs per SM); the
-// partial maxima are exchanged through distributed shared memory, so HBM still
-// sees each element once.
+// 8192 < K <= 16384: a row is split over a cluster of C = 2 CTAs (at most 8192
+// columns each), each keeping its part in registers with at most 4 chunks per thread (as fp16
+// bits, converted and smoothed again for the codes; fp32 for X / s, whose division is not worth
+// doing twice); the partial maxima are exchanged through distributed shared memory, so HBM
+// sees each element once.  Every CTA signals the cluster barrier on entry and waits on it
+// before its first store into a peer's shared memory, so no store reaches a CTA that has not
+// started.
 template <int C, int MODE, int FMT = kInt8>
 __global__ void __launch_bounds__(kThreads) quant_int8_rows_cluster_kernel(const uint16_t *__restrict__ x, int K,
                                                                            const float *__restrict__ smooth,
                                                                            int8_t *__restrict__ q,
                                                                            float *__restrict__ scales) {
     constexpr int NCH = 4;
+    constexpr bool RAW = MODE != kDiv;
     __shared__ float red[kThreads / 32];
     __shared__ float part_max[C];
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
     const size_t row = blockIdx.y;
     const uint32_t rank = sm100::cluster_ctarank();  // cluster (C, 1, 1) along x
     const int part = K / C;                          // K % (8 C) == 0: whole chunks per CTA
@@ -296,18 +300,39 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_cluster_kernel(const
     int8_t *qr = q + row * K + kb;
     const int t0 = threadIdx.x * kChunk;
     float amax = 0.0f;
-    float v[NCH][8];
+    uint4 raw[RAW ? NCH : 1];
+    float v[RAW ? 1 : NCH][8];
+    if (RAW) {
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) {
-        const int k = c * kRowStep + t0;
-        if (k < part) {
-            load8(xr + k, v[c]);
-            smooth8<MODE>(v[c], smooth, kb + k);
+        for (int c = 0; c < NCH; ++c) {
+            const int k = c * kRowStep + t0;
+            raw[c] = k < part ? ld_stream_u4(xr + k) : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
-            for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[c][e]));
+        for (int c = 0; c < NCH; ++c) {
+            const int k = c * kRowStep + t0;
+            if (k < part) {
+                float w[8];
+                unpack8(raw[c], w);
+                smooth8<MODE>(w, smooth, kb + k);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(w[e]));
+            }
+        }
+    } else {
+#pragma unroll
+        for (int c = 0; c < NCH; ++c) {
+            const int k = c * kRowStep + t0;
+            if (k < part) {
+                load8(xr + k, v[c]);
+                smooth8<MODE>(v[c], smooth, kb + k);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(v[c][e]));
+            }
         }
     }
     const float mine = block_max(amax, red);
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");  // every CTA of the cluster has started
     if (threadIdx.x < C) {  // this CTA's maximum into slot `rank` of every CTA of the cluster
         const uint32_t slot = sm100::smem_u32(&part_max[rank]);
         asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(sm100::mapa_shared(slot, threadIdx.x)), "f"(mine)
@@ -323,7 +348,16 @@ __global__ void __launch_bounds__(kThreads) quant_int8_rows_cluster_kernel(const
 #pragma unroll
     for (int c = 0; c < NCH; ++c) {
         const int k = c * kRowStep + t0;
-        if (k < part) *reinterpret_cast<uint2 *>(qr + k) = FormatTraits<FMT>::chunk(v[c], s, rs);
+        if (k < part) {
+            if (RAW) {
+                float w[8];
+                unpack8(raw[c], w);
+                smooth8<MODE>(w, smooth, kb + k);
+                *reinterpret_cast<uint2 *>(qr + k) = FormatTraits<FMT>::chunk(w, s, rs);
+            } else {
+                *reinterpret_cast<uint2 *>(qr + k) = FormatTraits<FMT>::chunk(v[RAW ? 0 : c], s, rs);
+            }
+        }
     }
     if (threadIdx.x == 0 && rank == 0) scales[row] = s;
 }
@@ -349,8 +383,9 @@ template <int MODE, int FMT = kInt8>
 cudaError_t launch_mode(const uint16_t *x, int R, int K, const float *smooth, int8_t *q, float *scales,
                         cudaStream_t st, const unsigned int *tensor_amax = nullptr) {
     const int nch = (K + kRowStep - 1) / kRowStep;
-    // Measured on B200: pairs beat the 8-chunk single CTA; for longer rows the
-    // two-pass kernel (second read from L2) beats clusters of 4 or 8.
+    // Measured on B200: pairs beat the 8-chunk single CTA (4096x16384: 59.7 -> 45.6 us with the
+    // pair's rows kept as fp16); for longer rows the two-pass kernel (second read from L2) beats
+    // clusters of 4 (8192x28672: 129.5 against 155.9 us) or 8.
     if (!tensor_amax && nch > 4 && nch <= 8 && R < 65536 && K % 16 == 0)
         return launch_cluster<2, MODE, FMT>(x, R, K, smooth, q, scales, st);
     dim3 grid(R), block(kThreads);
