@@ -152,35 +152,58 @@ __device__ __forceinline__ uint32_t float_to_e4m3(float v) {
     return r & 0xFFu;
 }
 
+// RN(a / 6) for an fp16 value a >= 0 (a block's max |v|): a = m 2^e with an 11-bit integer m,
+// and m / 3 is either exact or k + r / 3 (r = 1, 2), whose binary tail repeats 01 or 10, so the
+// quotient never lies within an fp32 ulp / 6 of a rounding boundary; the fp64 product with
+// RN64(1/6) is within 2^-52 relative of it and rounds to the same fp32 value.
+__device__ __forceinline__ float div6_rn(float a) {
+    return __double2float_rn(__dmul_rn((double)a, 0x1.5555555555555p-3));
+}
+
 __global__ void __launch_bounds__(kThreads) quant_nvfp4_kernel(const uint16_t *__restrict__ x, size_t nblocks, int F,
                                                                const unsigned int *__restrict__ tensor_amax,
                                                                uint8_t *__restrict__ q, uint8_t *__restrict__ scales) {
     const int fg = (F + 3) / 4;
     const float S = __fdiv_rn(fmaxf(__uint_as_float(*tensor_amax), 1e-8f), 2688.0f);
+    const float rS = __frcp_rn(S);
     constexpr float kDown = 1.0f - 0x1p-20f, kUp = 1.0f + 0x1p-20f;
     const size_t stride = (size_t)gridDim.x * kThreads;
     BlockPos pos((size_t)blockIdx.x * kThreads + threadIdx.x, stride, F);
     for (size_t b = (size_t)blockIdx.x * kThreads + threadIdx.x; b < nblocks; b += stride, pos.advance()) {
-        float v[2][8];
-        load8h(x + 16 * b, v[0]);
-        load8h(x + 16 * b + 8, v[1]);
-        const float a = amax8(v[1], amax8(v[0], 0.0f));
-        const uint32_t sb = float_to_e4m3(__fdiv_rn(__fdiv_rn(a, 6.0f), S));
+        const uint4 r0 = ld_stream_u4(x + 16 * b), r1 = ld_stream_u4(x + 16 * b + 8);
+        // max |v| on the fp16 bits (non-negative fp16 order like their bit patterns)
+        uint32_t m = __vmaxu2(__vmaxu2(r0.x & 0x7fff7fffu, r0.y & 0x7fff7fffu),
+                              __vmaxu2(r0.z & 0x7fff7fffu, r0.w & 0x7fff7fffu));
+        m = __vmaxu2(m, __vmaxu2(__vmaxu2(r1.x & 0x7fff7fffu, r1.y & 0x7fff7fffu),
+                                 __vmaxu2(r1.z & 0x7fff7fffu, r1.w & 0x7fff7fffu)));
+        const float a = half_bits_to_float((uint16_t)max(m & 0xffffu, m >> 16));
+        // b = e4m3_rn(fl(fl(a / 6) / S)): t = RN(fl(a / 6) RN(1/S)) is within 1.5 2^-23 |t| of the
+        // quotient, so fl(quotient) lies between t (1 -+ 2^-20); E4M3 rounding is monotone, so
+        // where both ends give one code it is the code, else the IEEE quotient decides.
+        const float a6 = div6_rn(a);
+        const float t = __fmul_rn(a6, rS);
+        uint32_t sb = float_to_e4m3(__fmul_rn(t, kDown));
+        if (sb != float_to_e4m3(__fmul_rn(t, kUp))) sb = float_to_e4m3(__fdiv_rn(a6, S));
         const float d = __fmul_rn(e4m3_to_float(sb), S);
         uint32_t c[2] = {0u, 0u};
         if (sb != 0u) {
             // e2m1_rn(fl(v / d)): t = RN(v * RN(1/d)) and both t (1 -+ 2^-20) round to the same code
             // unless fl(v / d) sits next to an E2M1 midpoint; then the IEEE quotient decides.
             const float rd = __frcp_rn(d);
+            const float2 rd2 = make_float2(rd, rd), dn = make_float2(kDown, kDown), up = make_float2(kUp, kUp);
+            const uint32_t w[8] = {r0.x, r0.y, r0.z, r0.w, r1.x, r1.y, r1.z, r1.w};
             uint32_t bad = 0;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 float lo[8], hi[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const float t = __fmul_rn(v[i][k], rd);
-                    lo[k] = __fmul_rn(t, kDown);
-                    hi[k] = __fmul_rn(t, kUp);
+                for (int k = 0; k < 4; ++k) {
+                    const float2 tv = __fmul2_rn(half2_bits_to_float2(w[4 * i + k]), rd2);
+                    const float2 l = __fmul2_rn(tv, dn), h = __fmul2_rn(tv, up);
+                    lo[2 * k] = l.x;
+                    lo[2 * k + 1] = l.y;
+                    hi[2 * k] = h.x;
+                    hi[2 * k + 1] = h.y;
                 }
                 c[i] = cvt_e2m1x8(lo);
                 bad |= c[i] ^ cvt_e2m1x8(hi);
@@ -188,10 +211,14 @@ __global__ void __launch_bounds__(kThreads) quant_nvfp4_kernel(const uint16_t *_
             if (bad) {
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    float t[8];
+                    float tq[8];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k) t[k] = __fdiv_rn(v[i][k], d);
-                    c[i] = cvt_e2m1x8(t);
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 v = half2_bits_to_float2(w[4 * i + k]);
+                        tq[2 * k] = __fdiv_rn(v.x, d);
+                        tq[2 * k + 1] = __fdiv_rn(v.y, d);
+                    }
+                    c[i] = cvt_e2m1x8(tq);
                 }
             }
         }

@@ -75,3 +75,15 @@ def test_int4_division_free_rounding_is_exact():
         # the candidates differ by at most one, and the rounded mean picks the same code
         assert np.all(np.abs(n_lo - n_hi) <= 1), sb
         assert np.array_equal(_mean_rule(n_lo, n_hi), got), sb
+
+
+def test_div6_by_fp64_product_is_correctly_rounded():
+    # The NVFP4 quantizer takes a block's max |v| / 6 as the fp64 product with RN64(1/6) rounded to
+    # fp32.  The dividend is an fp16 value, so every case is checked: all finite non-negative fp16.
+    inv6 = np.float64(1.0) / np.float64(6.0)
+    assert inv6.view(np.uint64) == 0x3FC5555555555555
+    h = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16)
+    a32 = h.astype(np.float32)
+    ieee = a32 / np.float32(6.0)
+    fast = (a32.astype(np.float64) * inv6).astype(np.float32)
+    assert np.array_equal(ieee.view(np.uint32), fast.view(np.uint32))
