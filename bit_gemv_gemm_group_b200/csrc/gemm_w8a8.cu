@@ -368,7 +368,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int mt = (M + BM - 1) / BM, nt = (N + BN - 1) / BN;
-    const int tiles = mt * nt;
     const int kblocks = (K + BK - 1) / BK;
 
     if (threadIdx.x == 0) {
