@@ -94,6 +94,16 @@ def test_workspace_size(wq):
     assert wq.smooth_workspace_bytes(0) == 0
 
 
+def test_fp4_scale_bytes(wq):
+    # 512-byte atoms: one per (128-row block, group of four factors); a factor per 32 (MXFP4) or 16 (NVFP4) values
+    assert wq.fp4_scale_bytes(128, 256, False) == 1 * 2 * 512
+    assert wq.fp4_scale_bytes(128, 256, True) == 1 * 4 * 512
+    assert wq.fp4_scale_bytes(2048, 8192, True) == 16 * 128 * 512
+    assert wq.fp4_scale_bytes(129, 160, False) == 2 * 2 * 512     # 5 factors -> 2 groups; 2 row blocks
+    assert wq.fp4_scale_bytes(1, 16, True) == 512
+    assert wq.fp4_scale_bytes(0, 256, True) == 0 and wq.fp4_scale_bytes(4, 0, False) == 0
+
+
 def test_binding_rejects_cpu_tensors(wq):
     import torch
     with pytest.raises(ValueError, match="CUDA"):
